@@ -1,0 +1,398 @@
+#!/usr/bin/env python
+"""Benchmark of the TT-gather training step on B200 (one process per GPU).
+
+A step is the whole hot path over one batch: index validation and key
+extraction, radix sort, unique + prefix grouping, the fused gather with
+in-kernel pooling, the backward into the cores and the SGD update.  The
+default workload is the 26-table, rank-64 training step at batch 32768
+(pooling Poisson(20)+1, Zipf(1.1) indices); ``--config`` picks another of the
+five workloads.  Inputs (indices 143 MB, upstream gradient 436 MB, cores
+221 MB) are larger than the 126 MB L2, so no flush is needed between steps.
+
+Prints ONE JSON line on rank 0.  ``--impl reference`` times the fp64 CPU
+oracle instead, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "pooled TT lookups/sec fwd and fwd+bwd at batch 32768; % of roofline"
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # FFMA lanes x 2 flops x max SM clock
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--config", type=int, default=4)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0,
+                   help="target CPU time of the oracle sample")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# workload arithmetic (counts only; the TT arithmetic runs in the kernels)
+# ---------------------------------------------------------------------------
+def macs_per_prefix(d, r):
+    """MACs of the shared prefix chain of one group (first k-1 slices)."""
+    k, rows, m = len(d), d[0], 0
+    for j in range(1, k - 1):
+        m += rows * r[j] * d[j] * r[j + 1]
+        rows *= d[j]
+    return m
+
+
+def macs_per_suffix(d, r):
+    k = len(d)
+    return int(np.prod(d[:-1])) * r[k - 1] * d[k - 1]
+
+
+def algorithmic(w, U, G):
+    """Algorithmic FLOPs (method's own work) and compulsory HBM bytes."""
+    d, r = w.d, w.r
+    L, D, T, B = w.num_lookups, w.dim, w.num_tables, w.batch
+    Mp, Ms = macs_per_prefix(d, r), macs_per_suffix(d, r)
+    f_fwd = 2.0 * (G * Mp + U * Ms) + L * D
+    f_bwd = 2.0 * (2 * U * Ms + 2 * G * Mp) + L * D
+    core_bytes = 4.0 * sum(c.size for tab in w.cores for c in tab)
+    io = 8.0 * L + 8.0 * (T * B + 1)
+    out_bytes = 4.0 * B * T * D
+    b_fwd = io + out_bytes + core_bytes
+    b_train = b_fwd + out_bytes + core_bytes + 3 * core_bytes
+    return {"f_fwd": f_fwd, "f_bwd": f_bwd, "f_sgd": 2.0 * core_bytes / 4, "b_fwd": b_fwd,
+            "b_train": b_train, "Mp": Mp, "Ms": Ms}
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(x[0]) for x in rows if x[0].replace(".", "").isdigit()]
+        mx = [float(x[1]) for x in rows if x[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for x in rows for i in range(4) if x[4 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_init(n):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, x):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def kernel_traffic(name):
+    """Per-launch DRAM bytes from a committed ncu summary, if it matches the current source."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        rec = json.load(open(path)).get(name)
+    except (OSError, ValueError):
+        return None
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "tensor_train_compressed_mixed_b200", "csrc", rec["source"])
+    if not os.path.exists(src):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return rec["dram_bytes_per_launch"] if sha == rec.get("source_sha") else None
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle on a bounded sample (the reported CPU baseline / reference arm)
+# ---------------------------------------------------------------------------
+def oracle_step(w_sample, threads):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.workload_forward(w_sample, threads=threads)
+    grads = oracle.workload_backward(w_sample, threads=threads) if w_sample.grad_out is not None else None
+    if grads is not None:
+        oracle.sgd(w_sample.cores, grads, w_sample.lr)
+    return time.perf_counter() - t0
+
+
+def cpu_sample(w, target_s, threads):
+    """Pick the number of samples whose oracle step takes about target_s seconds."""
+    from workloads import sub_batch
+    probe = sub_batch(w, np.arange(1))
+    t1 = oracle_step(probe, threads)
+    per_lookup = t1 / max(probe.num_lookups, 1)
+    avg = w.num_lookups / w.batch
+    S = int(max(1, min(w.batch, target_s / max(per_lookup * avg, 1e-9))))
+    return sub_batch(w, np.arange(S)), S
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from workloads import config_workload
+    w = config_workload(args.config, with_grad=True)
+    threads = len(os.sched_getaffinity(0))
+    per_step = max(0.5, min(6.0, 150.0 / max(args.steps + args.warmup, 1)))
+    sample, S = cpu_sample(w, per_step, threads)
+    for _ in range(args.warmup):
+        oracle_step(sample, threads)
+    total = 0.0
+    for _ in range(args.steps):
+        total += oracle_step(sample, threads)
+    v = sample.num_lookups * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "lookups/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "tables": w.num_tables,
+                   "sample_samples": S, "step": "fwd+bwd+sgd" if w.grad_out is not None else "fwd"},
+        "cpu_baseline": {"value": v, "unit": "lookups/s", "cores": threads, "kind": "oracle",
+                         "sample": f"first {S} of {w.batch} samples, all {w.num_tables} tables "
+                                   f"({sample.num_lookups} lookups) per step"},
+        "e2e": {"value": v, "unit": "lookups/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+PHASE_SOURCE = {"fwd_fused": "fused_generic.cu", "bwd_fused": "fused_generic.cu",
+                "fwd_sort": "grouping.cu", "fwd_keys": "grouping.cu", "fwd_segment": "grouping.cu",
+                "bwd_reduce": "elementwise.cu", "sgd": "elementwise.cu"}
+
+
+def run_ours(args):
+    import torch
+    from tensor_train_compressed_mixed_b200 import abi, from_workload
+    from workloads import config_workload
+
+    world, rank, local = dist_init(args.gpus)
+    dev = torch.device("cuda", local)
+    w = config_workload(args.config, with_grad=True)
+    train = w.grad_out is not None and args.config in (4, 5)
+    emb, cores, idx, off = from_workload(w, device=dev, with_grads=True)
+    g = torch.from_numpy(w.grad_out).to(dev)
+    L, B, T, D = w.num_lookups, w.batch, w.num_tables, w.dim
+    out = torch.empty(B, T * D, dtype=torch.float32, device=dev)
+    emb.reserve(L, B)
+
+    def step():
+        emb.forward(idx, off, B, out)
+        if train:
+            emb.backward(g)
+            if args.config == 4:
+                emb.sgd_update(w.lr)
+
+    def timed(fn, K):
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(K):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        emb.sync()
+        barrier(world)
+        return max_over_ranks(world, e0.elapsed_time(e1))
+
+    for _ in range(args.warmup):
+        step()
+    emb.sync()
+    seg = emb.segmentation()
+    U, G = seg["num_unique"], seg["num_groups"]
+    alg = algorithmic(w, U, G)
+
+    # --- the timed training steps (phase events on, clocks sampled) ---
+    abi.tt_emb_enable_timing(emb.handle, True)
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    ms_total = timed(step, args.steps)
+    clk = clocks.stop()
+    ph, launches = abi.tt_emb_phase_times(emb.handle)
+    abi.tt_emb_enable_timing(emb.handle, False)
+    ms_step = ms_total / args.steps
+    value = world * L * args.steps / (ms_total / 1e3)
+
+    # --- forward only ---
+    ms_fwd = timed(lambda: emb.forward(idx, off, B, out), args.steps) / args.steps
+
+    # --- dominant kernel roofline (device times from the timed region) ---
+    per_step = {k: v / args.steps for k, v in ph.items()}
+    dom = max(per_step, key=per_step.get)
+    flops = {"fwd_fused": alg["f_fwd"], "bwd_fused": alg["f_bwd"]}
+    if dom in flops:
+        achieved = flops[dom] / (per_step[dom] / 1e3) / 1e12
+        roof = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": FP32_PEAK_TFLOPS,
+                "unit": "TFLOP/s", "frac": achieved / FP32_PEAK_TFLOPS,
+                "traffic": kernel_traffic(dom), "peak_source": "derived: 148 SM x 128 FP32 lanes x 2 x 1.965 GHz"}
+    else:
+        roof = {"bound": "hbm", "kernel": dom, "achieved": None, "peak": None, "unit": "GB/s",
+                "frac": None, "traffic": kernel_traffic(dom)}
+    t_roof_step = max((alg["f_fwd"] + (alg["f_bwd"] if train else 0)) / (FP32_PEAK_TFLOPS * 1e12),
+                      (alg["b_train"] if train else alg["b_fwd"]) / 6550.4e9)
+    t_roof_fwd = max(alg["f_fwd"] / (FP32_PEAK_TFLOPS * 1e12), alg["b_fwd"] / 6550.4e9)
+
+    # --- end to end through the public API with host buffers ---
+    e2e = None
+    if not args.no_e2e:
+        h_idx = torch.from_numpy(w.indices).pin_memory()
+        h_off = torch.from_numpy(w.offsets).pin_memory()
+        h_g = torch.from_numpy(w.grad_out).pin_memory()
+        h_out = torch.empty(B, T * D, dtype=torch.float32).pin_memory()
+        d_idx, d_off, d_g = torch.empty_like(idx), torch.empty_like(off), torch.empty_like(g)
+
+        def e2e_step():
+            d_idx.copy_(h_idx, non_blocking=True)
+            d_off.copy_(h_off, non_blocking=True)
+            if train:
+                d_g.copy_(h_g, non_blocking=True)
+            emb.forward(d_idx, d_off, B, out)
+            if train:
+                emb.backward(d_g)
+                if args.config == 4:
+                    emb.sgd_update(w.lr)
+            h_out.copy_(out, non_blocking=True)
+
+        e2e_step()
+        ms_e2e = timed(e2e_step, max(2, args.steps // 2)) / max(2, args.steps // 2)
+        h2d = 8 * L + 8 * (T * B + 1) + (4 * B * T * D if train else 0)
+        e2e = {"value": world * L / (ms_e2e / 1e3), "unit": "lookups/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": 4 * B * T * D, "ms_per_step": ms_e2e}
+
+    # --- CPU oracle on a bounded sample (rank 0, one GPU only) ---
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = len(os.sched_getaffinity(0))
+        sample, S = cpu_sample(w, args.cpu_seconds, threads)
+        sec = oracle_step(sample, threads)
+        cpu = {"value": sample.num_lookups / sec, "unit": "lookups/s", "cores": threads,
+               "kind": "oracle",
+               "sample": f"first {S} of {B} samples, all {T} tables ({sample.num_lookups} lookups), "
+                         f"fwd+bwd+sgd in fp64, {sec:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "lookups/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": w.name, "batch": B, "tables": T, "lookups": L,
+                       "unique_rows": U, "prefix_groups": G,
+                       "step": "fwd+bwd+sgd" if train else "fwd",
+                       "l2": "inputs larger than L2 (indices+grad+cores ~800 MB), no flush",
+                       "parallelism": f"replicas{world}" if world > 1 else "single"},
+            "fwd": {"value": world * L / (ms_fwd / 1e3), "unit": "lookups/s", "ms": ms_fwd,
+                    "roofline_frac": t_roof_fwd / (ms_fwd / 1e3)},
+            "step_roofline_frac": t_roof_step / (ms_step / 1e3),
+            "phases_ms": per_step,
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    emb.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

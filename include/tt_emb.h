@@ -1,0 +1,240 @@
+/*
+ * tt_emb.h -- C ABI of the B200 Tensor-Train embedding gather library (libttemb.so).
+ *
+ * The operation (FlowTT: Exploiting Computation Flow Reuse in Irregular
+ * Tensor-Train Embedding -- Abstract, section 2.4 "Problem Definition",
+ * section 3.2 "Flow-Aware Fused TT Embedding Execution", section 3.3
+ * "Flow-Aligned Prefix-Based Index Grouping"):
+ *
+ *   A virtual table of N rows and D = d_1*...*d_k columns is held as k TT
+ *   cores G_j, each a row-major float32 array of shape [r_{j-1}][n_j][d_j][r_j]
+ *   with r_0 = r_k = 1 and N <= n_1*...*n_k.  Row i is split into mixed-radix
+ *   digits (i_1..i_k) over (n_1..n_k), i_1 the most significant; the row is
+ *   the chained product G_1[:, i_1] . G_2[:, i_2] ... G_k[:, i_k], column
+ *   (a_1..a_k) flattened row-major.  Lookups are sum-pooled into bags.  Rows
+ *   that share their first k-1 digits (the prefix) share the intermediate
+ *   product of the first k-1 slices; the library groups a batch by prefix
+ *   (sort, unique, run-length encoding) and computes each shared intermediate
+ *   once.  Training adds dL/dG_j for L = sum_b <grad_out_b, out_b> and a plain
+ *   SGD step.
+ *
+ * Conventions shared by every entry point
+ *   - One handle holds T tables that share k, d and r; each table has its own
+ *     (n_1..n_k) and its own valid row count N_t.  Limits: 1 <= T <=
+ *     TT_EMB_MAX_TABLES, 1 <= k <= TT_EMB_MAX_CORES, N_t < 2^31 * ... see
+ *     tt_emb_create.
+ *   - "device" pointers are CUDA global-memory pointers of the current device;
+ *     "host" pointers are ordinary CPU memory.  The library never frees memory
+ *     it did not allocate; it only allocates the handle (host) and, in
+ *     tt_emb_create, one small device status block (freed by tt_emb_destroy).
+ *   - Bags are table-major: bag (t, b) holds indices[offsets[t*B+b] ..
+ *     offsets[t*B+b+1]), and its pooled row goes to out[b][t*D .. (t+1)*D).
+ *   - Calls that take a stream only enqueue work on it and never synchronise
+ *     the host.  Errors found on the host (bad arguments, shapes, state) are
+ *     returned at once.  Errors found on the device (an index outside
+ *     [0, N_t), offsets that are not a valid partition of [0, L), a bounded
+ *     wait that ran out) are recorded in the handle's device status block;
+ *     every later kernel of the handle then does nothing, the outputs of the
+ *     failed call are unspecified, and the code surfaces at the next
+ *     tt_emb_sync().  No error ever crosses the ABI as an exception.
+ *   - Calls on one handle must be ordered (same stream, or ordered streams);
+ *     two handles are independent.
+ */
+#ifndef TT_EMB_H
+#define TT_EMB_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TT_EMB_MAX_TABLES 64
+#define TT_EMB_MAX_CORES 4
+#define TT_EMB_ABI_VERSION 1
+
+typedef struct tt_emb_handle* tt_emb_t;
+/* A cudaStream_t passed as an opaque pointer (NULL = the legacy default stream). */
+typedef void* tt_stream_t;
+
+typedef enum {
+    TT_OK = 0,
+    TT_ERR_ARG = 1,          /* a null pointer, a negative size or an unknown option */
+    TT_ERR_SHAPE = 2,        /* table / core shapes outside the supported set */
+    TT_ERR_INDEX_RANGE = 3,  /* (device) an index outside [0, N_t) */
+    TT_ERR_OFFSETS = 4,      /* (device) offsets not monotone, offsets[0] != 0 or offsets[T*B] != L */
+    TT_ERR_WORKSPACE = 5,    /* no workspace, or one smaller than tt_emb_workspace_size() asked for */
+    TT_ERR_STATE = 6,        /* cores not set, backward without a forward, grads not registered */
+    TT_ERR_CUDA = 7,         /* a CUDA runtime call failed (launch, memset, copy) */
+    TT_ERR_TIMEOUT = 8,      /* (device) a bounded wait ran out of iterations */
+    TT_ERR_UNSUPPORTED = 9   /* a valid request this build does not implement */
+} tt_status;
+
+/* Scheduling of the fused kernels (FlowTT section 3.4 and the ablation in section 4). */
+typedef enum {
+    TT_SCHED_STATIC = 0,     /* each block takes a fixed, precomputed share of the prefix groups */
+    TT_SCHED_STEAL = 1,      /* persistent blocks: own share first, then steal chunks of unfinished groups */
+    TT_SCHED_STEAL_L2 = 2    /* as STEAL, and shared intermediates of split groups are checkpointed in L2 */
+} tt_sched_mode;
+
+/* Grouping depth (FlowTT section 4, "Prefix-Based Reuse over Exact Deduplication"). */
+typedef enum {
+    TT_GROUP_PREFIX = 0,     /* deduplicate rows and share each prefix intermediate */
+    TT_GROUP_UNIQUE_ONLY = 1 /* deduplicate rows only: every distinct row is contracted on its own */
+} tt_group_mode;
+
+typedef struct {
+    int32_t sched;           /* tt_sched_mode, default TT_SCHED_STEAL_L2 */
+    int32_t grouping;        /* tt_group_mode, default TT_GROUP_PREFIX */
+    int32_t chunk;           /* rows per stealable chunk of a prefix group; 0 = library default */
+    int32_t grid;            /* persistent blocks; 0 = one wave on the current device */
+    int32_t reserved[12];    /* must be zero */
+} tt_emb_options;
+
+/* Fills *opt with the defaults. */
+void tt_emb_default_options(tt_emb_options* opt);
+
+/*
+ * Creates a handle for T tables sharing k, d and r (host call, no device work
+ * besides allocating the 256-byte device status block).
+ *   num_tables   T, 1..TT_EMB_MAX_TABLES
+ *   num_cores    k, 1..TT_EMB_MAX_CORES
+ *   n_factors    host int64 [T][k]: n_j of each table, each >= 1; the product of
+ *                a table's factors must be < 2^40
+ *   n_rows       host int64 [T]: valid rows N_t, 1 <= N_t <= prod_j n_j and N_t < 2^32
+ *   d_factors    host int32 [k]: d_j >= 1, D = prod d_j <= 1024
+ *   ranks        host int32 [k+1]: r_0 = r_k = 1, 1 <= r_j <= 128
+ *   opt          host, may be NULL (defaults)
+ *   out          host: receives the handle
+ * Returns TT_OK, TT_ERR_ARG, TT_ERR_SHAPE or TT_ERR_CUDA.
+ */
+int tt_emb_create(int32_t num_tables, int32_t num_cores, const int64_t* n_factors,
+                  const int64_t* n_rows, const int32_t* d_factors, const int32_t* ranks,
+                  const tt_emb_options* opt, tt_emb_t* out);
+
+/*
+ * Registers the cores (and optionally the gradient buffers) by borrowing
+ * device pointers.  Host arrays of T*k device pointers, table-major
+ * (entry t*k + j is core j of table t, float32 [r_{j-1}][n_j][d_j][r_j],
+ * 16-byte aligned).  core_grads may be NULL for inference; when given, each
+ * buffer has the shape of its core and is overwritten by tt_emb_backward.
+ * The caller keeps ownership and must keep the memory alive while the handle
+ * uses it.  Returns TT_OK or TT_ERR_ARG.
+ */
+int tt_emb_set_cores(tt_emb_t h, float* const* cores, float* const* core_grads);
+
+/*
+ * Device workspace needed for batches of at most max_lookups lookups and
+ * batch bags per table (host call).  *bytes receives the size.
+ */
+int tt_emb_workspace_size(tt_emb_t h, int64_t max_lookups, int64_t batch, size_t* bytes);
+
+/*
+ * Registers caller-owned device workspace (256-byte aligned) of `bytes` bytes,
+ * sized for (max_lookups, batch) by tt_emb_workspace_size.  The workspace
+ * holds the segmentation between a forward and its backward; it must not be
+ * shared by two handles that run at the same time.
+ */
+int tt_emb_set_workspace(tt_emb_t h, void* workspace, size_t bytes, int64_t max_lookups,
+                         int64_t batch);
+
+/*
+ * Forward pass: out[b][t*D + c] = sum over bag (t, b) of row_t(i)[c] (float32,
+ * fp32 accumulation).  Enqueues on `stream`: index validation, digit/key
+ * extraction, radix sort, unique + prefix run-length grouping, and the fused
+ * gather + pooling kernel.
+ *   indices   device int64 [num_lookups], each in [0, N_t) of its table
+ *   offsets   device int64 [T*batch + 1], non-decreasing, offsets[0] = 0,
+ *             offsets[T*batch] = num_lookups
+ *   out       device float32 [batch][T*D], overwritten (empty bags give 0)
+ * num_lookups and batch must not exceed the workspace's sizes.  The
+ * segmentation is kept in the workspace for tt_emb_backward.
+ */
+int tt_emb_forward(tt_emb_t h, const int64_t* indices, const int64_t* offsets,
+                   int64_t num_lookups, int64_t batch, float* out, tt_stream_t stream);
+
+/*
+ * Backward pass of the last forward on this handle: overwrites the registered
+ * core_grads with dL/dG_j for L = sum <grad_out, out> (zero for slices no
+ * lookup touched).  grad_out: device float32 [batch][T*D] of the last forward's
+ * batch.  Reuses the forward's segmentation (no re-sort).  Returns
+ * TT_ERR_STATE without a preceding forward or without registered core_grads.
+ */
+int tt_emb_backward(tt_emb_t h, const float* grad_out, tt_stream_t stream);
+
+/* SGD step on every registered core: G <- G - lr * dG (float32, elementwise). */
+int tt_emb_sgd_update(tt_emb_t h, float lr, tt_stream_t stream);
+
+/*
+ * Test and inspection hook: device views of the last forward's segmentation,
+ * valid until the next forward on the handle.  Synchronises the stream of the
+ * last call to read the counts.
+ */
+typedef struct {
+    int64_t num_lookups;        /* L */
+    int64_t num_unique;         /* U: distinct (table, row) pairs */
+    int64_t num_groups;         /* G: distinct (table, prefix) pairs */
+    int32_t key_bits;           /* bits of the row field in a sort key */
+    int32_t key_bytes;          /* 4 or 8 */
+    const void* sorted_keys;    /* device [L]: (table << key_bits) | row, ascending */
+    const int32_t* perm;        /* device [L]: input position of each sorted lookup (stable) */
+    const void* uniq_keys;      /* device [U]: the distinct keys */
+    const int32_t* uniq_start;  /* device [U+1]: first sorted lookup of each distinct key */
+    const int32_t* grp_start;   /* device [G+1]: first distinct key of each prefix group */
+    const int32_t* bag_sorted;  /* device [L]: bag t*B + b of each sorted lookup */
+} tt_seg_view;
+
+int tt_emb_get_segmentation(tt_emb_t h, tt_seg_view* view);
+
+/*
+ * Copies the last forward's segmentation arrays (see tt_seg_view for shapes)
+ * into caller buffers, host or device (any pointer may be NULL to skip it).
+ * Synchronous.  Test and inspection hook.
+ */
+int tt_emb_copy_segmentation(tt_emb_t h, void* sorted_keys, int32_t* perm, void* uniq_keys,
+                             int32_t* uniq_start, int32_t* grp_start, int32_t* bag_sorted);
+
+/*
+ * Waits for the handle's work on the stream of its last call and returns the
+ * first device-side error recorded since the last tt_emb_sync (then clears it),
+ * or TT_ERR_CUDA if the stream itself failed.
+ */
+int tt_emb_sync(tt_emb_t h);
+
+/* Message for a status code (static storage). */
+const char* tt_emb_error_string(int code);
+
+/* Destroys the handle (host + its status block).  NULL is ignored. */
+void tt_emb_destroy(tt_emb_t h);
+
+/*
+ * Per-phase device timing, for benchmarks.  While enabled, every call records
+ * CUDA events on its stream around each phase below; tt_emb_sync() folds the
+ * finished intervals into per-phase totals.  tt_emb_phase_times copies the
+ * totals (milliseconds, host double [TT_EMB_NUM_PHASES]) and the number of
+ * kernels the handle has launched since timing was last enabled (host int64,
+ * may be NULL).  Enabling resets both.  The launch count is kept whether or
+ * not timing is on.
+ */
+typedef enum {
+    TT_PHASE_FWD_KEYS = 0,   /* offsets/index validation and key extraction */
+    TT_PHASE_FWD_SORT = 1,   /* radix sort of the keys */
+    TT_PHASE_FWD_SEGMENT = 2,/* unique + prefix run-length segmentation */
+    TT_PHASE_FWD_FUSED = 3,  /* fused gather + pooling (includes zeroing out) */
+    TT_PHASE_BWD_FUSED = 4,  /* fused backward kernels */
+    TT_PHASE_BWD_REDUCE = 5, /* segmented reductions and gradient write-out */
+    TT_PHASE_SGD = 6,        /* SGD update */
+    TT_EMB_NUM_PHASES = 7
+} tt_phase;
+
+int tt_emb_enable_timing(tt_emb_t h, int enable);
+int tt_emb_phase_times(tt_emb_t h, double* ms, int64_t* launches);
+
+/* ABI version of the loaded library (TT_EMB_ABI_VERSION). */
+int tt_emb_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TT_EMB_H */

@@ -1,0 +1,540 @@
+// C ABI of libttemb: handle, argument and shape validation, workspace layout,
+// stream-ordered launch sequences and the device status block.
+#include <new>
+#include <string.h>
+#include <vector>
+
+#include "tt_common.cuh"
+
+using namespace tt;
+
+namespace {
+
+struct Layout {
+    size_t counters, keys[2], vals[2], bag_of_pos, hist, digit_total, partials, uniq_keys,
+        uniq_start, grp_start, bag_sorted, total;
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+Layout make_layout(int key_bytes, int64_t L, int64_t B)
+{
+    (void)B;
+    Layout y;
+    size_t p = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = p;
+        p = align_up(p + bytes, 256);
+        return at;
+    };
+    const size_t Lz = (size_t)(L > 0 ? L : 1);
+    const size_t tiles = (size_t)ceil_div((int64_t)Lz, kSortTile);
+    y.counters = take(sizeof(WsCounters));
+    y.keys[0] = take(Lz * key_bytes);
+    y.keys[1] = take(Lz * key_bytes);
+    y.vals[0] = take(Lz * 4);
+    y.vals[1] = take(Lz * 4);
+    y.bag_of_pos = take(Lz * 4);
+    y.hist = take(256 * tiles * 4);
+    y.digit_total = take(256 * 4);
+    y.partials = take((size_t)ceil_div((int64_t)Lz, kScanTile) * 8);
+    y.uniq_keys = take(Lz * key_bytes);
+    y.uniq_start = take((Lz + 1) * 4);
+    y.grp_start = take((Lz + 1) * 4);
+    y.bag_sorted = take(Lz * 4);
+    y.total = p;
+    return y;
+}
+
+int bits_for(uint64_t v)  // bits needed to hold values 0..v
+{
+    int b = 0;
+    while (b < 64 && (v >> b) != 0) ++b;
+    return b;
+}
+
+}  // namespace
+
+struct tt_emb_handle {
+    int32_t T = 0, k = 0, D = 0, P = 0;
+    int64_t n[kMaxT][kMaxK] = {};
+    int64_t n_rows[kMaxT] = {};
+    int32_t d[kMaxK] = {};
+    int32_t r[kMaxK + 1] = {};
+    tt_emb_options opt{};
+    int ibits = 0, tbits = 0;
+    bool key64 = false;
+    float* cores[kMaxT * kMaxK] = {};
+    float* grads[kMaxT * kMaxK] = {};
+    bool have_cores = false, have_grads = false;
+    char* ws = nullptr;
+    size_t ws_bytes = 0;
+    int64_t ws_L = 0, ws_B = 0;
+    Layout lay{};
+    int32_t* d_status = nullptr;
+    cudaStream_t last_stream = nullptr;
+    bool used_stream = false;
+    bool have_fwd = false;
+    int64_t fwd_L = 0, fwd_B = 0;
+    int fwd_which = 0;
+    int device = 0, num_sms = 148;
+    // timing and launch accounting
+    bool timing = false;
+    double phase_ms[TT_EMB_NUM_PHASES] = {};
+    int64_t launches = 0;
+    struct Interval { int phase; cudaEvent_t a, b; };
+    std::vector<Interval> pending;
+    std::vector<cudaEvent_t> pool;
+    int open_phase = -1;
+    cudaEvent_t open_event = nullptr;
+
+    cudaEvent_t take_event()
+    {
+        if (!pool.empty()) {
+            cudaEvent_t e = pool.back();
+            pool.pop_back();
+            return e;
+        }
+        cudaEvent_t e = nullptr;
+        if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+        return e;
+    }
+    void begin(int phase, cudaStream_t s)
+    {
+        if (!timing) return;
+        open_phase = phase;
+        open_event = take_event();
+        if (open_event) cudaEventRecord(open_event, s);
+    }
+    void end(cudaStream_t s)
+    {
+        if (!timing || open_phase < 0) return;
+        cudaEvent_t b = take_event();
+        if (open_event && b) {
+            cudaEventRecord(b, s);
+            pending.push_back({open_phase, open_event, b});
+        }
+        open_phase = -1;
+        open_event = nullptr;
+    }
+    void fold()
+    {
+        for (const Interval& iv : pending) {
+            float ms = 0.f;
+            if (cudaEventSynchronize(iv.b) == cudaSuccess && cudaEventElapsedTime(&ms, iv.a, iv.b) == cudaSuccess)
+                phase_ms[iv.phase] += ms;
+            pool.push_back(iv.a);
+            pool.push_back(iv.b);
+        }
+        pending.clear();
+    }
+
+    int key_bytes() const { return key64 ? 8 : 4; }
+    int64_t core_floats(int t, int j) const { return (int64_t)r[j] * n[t][j] * d[j] * r[j + 1]; }
+
+    CoreParams core_params() const
+    {
+        CoreParams cp;
+        memset(&cp, 0, sizeof(cp));
+        cp.T = T; cp.k = k; cp.D = D; cp.P = P;
+        for (int j = 0; j < k; ++j) cp.d[j] = d[j];
+        for (int j = 0; j <= k; ++j) cp.r[j] = r[j];
+        cp.ibits = ibits;
+        cp.unique_only = opt.grouping == TT_GROUP_UNIQUE_ONLY;
+        cp.B = fwd_B;
+        for (int t = 0; t < T; ++t)
+            for (int j = 0; j < k; ++j) {
+                cp.n[t][j] = (uint32_t)n[t][j];
+                cp.cores[t][j] = cores[t * k + j];
+            }
+        return cp;
+    }
+
+    BufferList buffers(bool with_grads_as_b, bool grads_as_a) const
+    {
+        BufferList bl;
+        memset(&bl, 0, sizeof(bl));
+        bl.count = T * k;
+        int64_t c = 0;
+        for (int q = 0; q < T * k; ++q) {
+            const int64_t sz = core_floats(q / k, q % k);
+            bl.chunk_start[q] = c;
+            bl.size[q] = sz;
+            bl.a[q] = grads_as_a ? grads[q] : cores[q];
+            bl.b[q] = with_grads_as_b ? grads[q] : nullptr;
+            c += ceil_div(sz, kElemChunk);
+        }
+        bl.chunk_start[T * k] = c;
+        return bl;
+    }
+
+    char* at(size_t off) const { return ws + off; }
+};
+
+static int cuda_status(cudaError_t e) { return e == cudaSuccess ? TT_OK : TT_ERR_CUDA; }
+
+extern "C" {
+
+int tt_emb_abi_version(void) { return TT_EMB_ABI_VERSION; }
+
+void tt_emb_default_options(tt_emb_options* opt)
+{
+    if (!opt) return;
+    memset(opt, 0, sizeof(*opt));
+    opt->sched = TT_SCHED_STEAL_L2;
+    opt->grouping = TT_GROUP_PREFIX;
+    opt->chunk = 0;
+    opt->grid = 0;
+}
+
+const char* tt_emb_error_string(int code)
+{
+    switch (code) {
+    case TT_OK: return "ok";
+    case TT_ERR_ARG: return "invalid argument";
+    case TT_ERR_SHAPE: return "unsupported table or core shape";
+    case TT_ERR_INDEX_RANGE: return "an index is outside [0, N) of its table";
+    case TT_ERR_OFFSETS: return "offsets are not a monotone partition of [0, num_lookups)";
+    case TT_ERR_WORKSPACE: return "workspace missing or too small";
+    case TT_ERR_STATE: return "call out of order (cores, gradients or forward missing)";
+    case TT_ERR_CUDA: return "a CUDA runtime call failed";
+    case TT_ERR_TIMEOUT: return "a bounded device wait ran out";
+    case TT_ERR_UNSUPPORTED: return "not supported by this build";
+    default: return "unknown status code";
+    }
+}
+
+int tt_emb_create(int32_t num_tables, int32_t num_cores, const int64_t* n_factors,
+                  const int64_t* n_rows, const int32_t* d_factors, const int32_t* ranks,
+                  const tt_emb_options* opt, tt_emb_t* out)
+{
+    if (!out || !n_factors || !n_rows || !d_factors || !ranks) return TT_ERR_ARG;
+    *out = nullptr;
+    if (num_tables < 1 || num_tables > kMaxT || num_cores < 1 || num_cores > kMaxK) return TT_ERR_SHAPE;
+    tt_emb_options o;
+    tt_emb_default_options(&o);
+    if (opt) {
+        o = *opt;
+        for (int i = 0; i < 12; ++i)
+            if (o.reserved[i] != 0) return TT_ERR_ARG;
+        if (o.sched < TT_SCHED_STATIC || o.sched > TT_SCHED_STEAL_L2) return TT_ERR_ARG;
+        if (o.grouping < TT_GROUP_PREFIX || o.grouping > TT_GROUP_UNIQUE_ONLY) return TT_ERR_ARG;
+        if (o.chunk < 0 || o.grid < 0) return TT_ERR_ARG;
+    }
+    const int k = num_cores;
+    if (ranks[0] != 1 || ranks[k] != 1) return TT_ERR_SHAPE;
+    int64_t D = 1;
+    for (int j = 0; j < k; ++j) {
+        if (d_factors[j] < 1 || ranks[j] < 1 || ranks[j] > 128) return TT_ERR_SHAPE;
+        D *= d_factors[j];
+    }
+    if (D > 1024) return TT_ERR_SHAPE;
+    uint64_t max_rows = 1;
+    for (int t = 0; t < num_tables; ++t) {
+        long double prod = 1;
+        for (int j = 0; j < k; ++j) {
+            const int64_t nj = n_factors[(int64_t)t * k + j];
+            if (nj < 1 || nj > 0xffffffffLL) return TT_ERR_SHAPE;
+            prod *= (long double)nj;
+        }
+        if (prod >= (long double)(1ULL << 40)) return TT_ERR_SHAPE;
+        if (n_rows[t] < 1 || (long double)n_rows[t] > prod || n_rows[t] > 0xffffffffLL) return TT_ERR_SHAPE;
+        if ((uint64_t)n_rows[t] > max_rows) max_rows = (uint64_t)n_rows[t];
+    }
+
+    tt_emb_handle* h = new (std::nothrow) tt_emb_handle();
+    if (!h) return TT_ERR_ARG;
+    h->T = num_tables;
+    h->k = k;
+    h->D = (int32_t)D;
+    h->P = (int32_t)(D / d_factors[k - 1]);
+    for (int j = 0; j < k; ++j) h->d[j] = d_factors[j];
+    for (int j = 0; j <= k; ++j) h->r[j] = ranks[j];
+    for (int t = 0; t < num_tables; ++t) {
+        h->n_rows[t] = n_rows[t];
+        for (int j = 0; j < k; ++j) h->n[t][j] = n_factors[(int64_t)t * k + j];
+    }
+    h->opt = o;
+    h->ibits = bits_for(max_rows - 1);
+    if (h->ibits < 1) h->ibits = 1;
+    h->tbits = bits_for((uint64_t)num_tables - 1);
+    h->key64 = h->ibits + h->tbits > 32;
+
+    const CoreParams cp = h->core_params();
+    if (generic_backward_smem_floats(cp) * 4 > 200 * 1024 ||
+        generic_forward_smem_floats(cp) * 4 > 200 * 1024) {
+        delete h;
+        return TT_ERR_SHAPE;
+    }
+    if (cudaGetDevice(&h->device) != cudaSuccess ||
+        cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess ||
+        cudaMalloc((void**)&h->d_status, 256) != cudaSuccess) {
+        delete h;
+        return TT_ERR_CUDA;
+    }
+    if (cudaMemset(h->d_status, 0, 256) != cudaSuccess) {
+        cudaFree(h->d_status);
+        delete h;
+        return TT_ERR_CUDA;
+    }
+    *out = h;
+    return TT_OK;
+}
+
+int tt_emb_set_cores(tt_emb_t h, float* const* cores, float* const* core_grads)
+{
+    if (!h || !cores) return TT_ERR_ARG;
+    const int n = h->T * h->k;
+    for (int q = 0; q < n; ++q) {
+        if (!cores[q] || ((uintptr_t)cores[q] & 15)) return TT_ERR_ARG;
+        if (core_grads && (!core_grads[q] || ((uintptr_t)core_grads[q] & 15))) return TT_ERR_ARG;
+    }
+    for (int q = 0; q < n; ++q) {
+        h->cores[q] = cores[q];
+        h->grads[q] = core_grads ? core_grads[q] : nullptr;
+    }
+    h->have_cores = true;
+    h->have_grads = core_grads != nullptr;
+    return TT_OK;
+}
+
+int tt_emb_workspace_size(tt_emb_t h, int64_t max_lookups, int64_t batch, size_t* bytes)
+{
+    if (!h || !bytes || max_lookups < 0 || batch < 1) return TT_ERR_ARG;
+    if (max_lookups >= (int64_t)INT32_MAX) return TT_ERR_ARG;
+    *bytes = make_layout(h->key_bytes(), max_lookups, batch).total;
+    return TT_OK;
+}
+
+int tt_emb_set_workspace(tt_emb_t h, void* workspace, size_t bytes, int64_t max_lookups,
+                         int64_t batch)
+{
+    if (!h || !workspace || max_lookups < 0 || batch < 1) return TT_ERR_ARG;
+    if (((uintptr_t)workspace & 255) != 0) return TT_ERR_ARG;
+    if (max_lookups >= (int64_t)INT32_MAX) return TT_ERR_ARG;
+    const Layout lay = make_layout(h->key_bytes(), max_lookups, batch);
+    if (bytes < lay.total) return TT_ERR_WORKSPACE;
+    h->ws = (char*)workspace;
+    h->ws_bytes = bytes;
+    h->ws_L = max_lookups;
+    h->ws_B = batch;
+    h->lay = lay;
+    h->have_fwd = false;
+    return TT_OK;
+}
+
+int tt_emb_forward(tt_emb_t h, const int64_t* indices, const int64_t* offsets, int64_t num_lookups,
+                   int64_t batch, float* out, tt_stream_t stream)
+{
+    if (!h || !offsets || !out || num_lookups < 0 || batch < 1) return TT_ERR_ARG;
+    if (num_lookups > 0 && !indices) return TT_ERR_ARG;
+    if (!h->have_cores) return TT_ERR_STATE;
+    if (!h->ws || num_lookups > h->ws_L || batch > h->ws_B) return TT_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    h->last_stream = s;
+    h->used_stream = true;
+    h->have_fwd = false;
+    const Layout& y = h->lay;
+    WsCounters* counters = (WsCounters*)h->at(y.counters);
+    const int64_t L = num_lookups;
+
+    cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)batch * h->T * h->D, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(counters, 0, sizeof(WsCounters), s);
+    if (e != cudaSuccess) return TT_ERR_CUDA;
+
+    KeyParams kp;
+    memset(&kp, 0, sizeof(kp));
+    kp.T = h->T;
+    kp.ibits = h->ibits;
+    kp.B = batch;
+    kp.L = L;
+    kp.unique_only = h->opt.grouping == TT_GROUP_UNIQUE_ONLY;
+    for (int t = 0; t < h->T; ++t) {
+        kp.nrows[t] = (uint32_t)h->n_rows[t];
+        kp.nlast[t] = (uint32_t)h->n[t][h->k - 1];
+    }
+    int32_t* bag_of_pos = (int32_t*)h->at(y.bag_of_pos);
+    SortBuffers sb;
+    sb.keys[0] = h->at(y.keys[0]);
+    sb.keys[1] = h->at(y.keys[1]);
+    sb.vals[0] = (int32_t*)h->at(y.vals[0]);
+    sb.vals[1] = (int32_t*)h->at(y.vals[1]);
+    sb.hist = (uint32_t*)h->at(y.hist);
+    sb.digit_total = (uint32_t*)h->at(y.digit_total);
+
+    int nl = 0;
+    h->begin(TT_PHASE_FWD_KEYS, s);
+    e = launch_make_keys(kp, h->key64, indices, offsets, sb.keys[0], sb.vals[0], bag_of_pos,
+                         h->d_status, s, &nl);
+    h->end(s);
+    h->launches += nl;
+    if (e != cudaSuccess) return TT_ERR_CUDA;
+    h->fwd_L = L;
+    h->fwd_B = batch;
+    if (L == 0) {
+        h->fwd_which = 0;
+        h->have_fwd = true;
+        return TT_OK;
+    }
+    int which = 0;
+    nl = 0;
+    h->begin(TT_PHASE_FWD_SORT, s);
+    e = radix_sort_pairs(h->key64, L, h->ibits + h->tbits, sb, &which, h->d_status, s, &nl);
+    h->end(s);
+    if (e != cudaSuccess) return TT_ERR_CUDA;
+    h->begin(TT_PHASE_FWD_SEGMENT, s);
+    e = launch_segment(kp, h->key64, sb.keys[which], sb.vals[which], bag_of_pos,
+                       h->at(y.uniq_keys), (int32_t*)h->at(y.uniq_start),
+                       (int32_t*)h->at(y.grp_start), (int32_t*)h->at(y.bag_sorted),
+                       (uint64_t*)h->at(y.partials), counters, h->d_status, s, &nl);
+    h->end(s);
+    if (e != cudaSuccess) return TT_ERR_CUDA;
+    const CoreParams cp = h->core_params();
+    const int grid = h->opt.grid > 0 ? h->opt.grid : h->num_sms * 8;
+    h->begin(TT_PHASE_FWD_FUSED, s);
+    e = launch_forward_generic(cp, h->key64, h->at(y.uniq_keys), (const int32_t*)h->at(y.uniq_start),
+                               (const int32_t*)h->at(y.grp_start), (const int32_t*)h->at(y.bag_sorted),
+                               counters, L, out, h->d_status, s, grid, &nl);
+    h->end(s);
+    h->launches += nl;
+    if (e != cudaSuccess) return TT_ERR_CUDA;
+    h->fwd_which = which;
+    h->have_fwd = true;
+    return TT_OK;
+}
+
+int tt_emb_backward(tt_emb_t h, const float* grad_out, tt_stream_t stream)
+{
+    if (!h || !grad_out) return TT_ERR_ARG;
+    if (!h->have_fwd || !h->have_grads || !h->have_cores) return TT_ERR_STATE;
+    cudaStream_t s = (cudaStream_t)stream;
+    h->last_stream = s;
+    h->used_stream = true;
+    int nl = 0;
+    h->begin(TT_PHASE_BWD_REDUCE, s);
+    cudaError_t e = launch_fill_zero(h->buffers(false, true), h->d_status, s, &nl);
+    h->end(s);
+    h->launches += nl;
+    if (e != cudaSuccess) return TT_ERR_CUDA;
+    if (h->fwd_L == 0) return TT_OK;
+    const Layout& y = h->lay;
+    GradPtrs gp;
+    memset(&gp, 0, sizeof(gp));
+    for (int t = 0; t < h->T; ++t)
+        for (int j = 0; j < h->k; ++j) gp.g[t][j] = h->grads[t * h->k + j];
+    const CoreParams cp = h->core_params();
+    const int grid = h->opt.grid > 0 ? h->opt.grid : h->num_sms * 8;
+    nl = 0;
+    h->begin(TT_PHASE_BWD_FUSED, s);
+    e = launch_backward_generic(cp, gp, h->key64, h->at(y.uniq_keys),
+                                (const int32_t*)h->at(y.uniq_start), (const int32_t*)h->at(y.grp_start),
+                                (const int32_t*)h->at(y.bag_sorted), (const WsCounters*)h->at(y.counters),
+                                h->fwd_L, grad_out, h->d_status, s, grid, &nl);
+    h->end(s);
+    h->launches += nl;
+    return cuda_status(e);
+}
+
+int tt_emb_sgd_update(tt_emb_t h, float lr, tt_stream_t stream)
+{
+    if (!h) return TT_ERR_ARG;
+    if (!h->have_cores || !h->have_grads) return TT_ERR_STATE;
+    cudaStream_t s = (cudaStream_t)stream;
+    h->last_stream = s;
+    h->used_stream = true;
+    int nl = 0;
+    h->begin(TT_PHASE_SGD, s);
+    const cudaError_t e = launch_sgd(h->buffers(true, false), lr, h->d_status, s, &nl);
+    h->end(s);
+    h->launches += nl;
+    return cuda_status(e);
+}
+
+int tt_emb_sync(tt_emb_t h)
+{
+    if (!h) return TT_ERR_ARG;
+    cudaStream_t s = h->used_stream ? h->last_stream : (cudaStream_t)0;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return TT_ERR_CUDA;
+    h->fold();
+    int32_t st[2] = {0, 0};
+    if (cudaMemcpyAsync(st, h->d_status, sizeof(st), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return TT_ERR_CUDA;
+    if (st[0] != 0) {
+        if (cudaMemsetAsync(h->d_status, 0, 256, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+            return TT_ERR_CUDA;
+        return st[0];
+    }
+    return TT_OK;
+}
+
+int tt_emb_get_segmentation(tt_emb_t h, tt_seg_view* v)
+{
+    if (!h || !v) return TT_ERR_ARG;
+    if (!h->have_fwd) return TT_ERR_STATE;
+    cudaStream_t s = h->used_stream ? h->last_stream : (cudaStream_t)0;
+    WsCounters c;
+    if (cudaMemcpyAsync(&c, h->at(h->lay.counters), sizeof(c), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return TT_ERR_CUDA;
+    const Layout& y = h->lay;
+    v->num_lookups = h->fwd_L;
+    v->num_unique = c.num_unique;
+    v->num_groups = c.num_groups;
+    v->key_bits = h->ibits;
+    v->key_bytes = h->key_bytes();
+    v->sorted_keys = h->at(y.keys[h->fwd_which]);
+    v->perm = (const int32_t*)h->at(y.vals[h->fwd_which]);
+    v->uniq_keys = h->at(y.uniq_keys);
+    v->uniq_start = (const int32_t*)h->at(y.uniq_start);
+    v->grp_start = (const int32_t*)h->at(y.grp_start);
+    v->bag_sorted = (const int32_t*)h->at(y.bag_sorted);
+    return TT_OK;
+}
+
+int tt_emb_copy_segmentation(tt_emb_t h, void* sorted_keys, int32_t* perm, void* uniq_keys,
+                             int32_t* uniq_start, int32_t* grp_start, int32_t* bag_sorted)
+{
+    tt_seg_view v;
+    int rc = tt_emb_get_segmentation(h, &v);
+    if (rc != TT_OK) return rc;
+    const size_t L = (size_t)v.num_lookups, U = (size_t)v.num_unique, G = (size_t)v.num_groups;
+    const size_t kb = (size_t)v.key_bytes;
+    cudaError_t e = cudaSuccess;
+    if (sorted_keys && L) e = cudaMemcpy(sorted_keys, v.sorted_keys, L * kb, cudaMemcpyDefault);
+    if (e == cudaSuccess && perm && L) e = cudaMemcpy(perm, v.perm, L * 4, cudaMemcpyDefault);
+    if (e == cudaSuccess && uniq_keys && U) e = cudaMemcpy(uniq_keys, v.uniq_keys, U * kb, cudaMemcpyDefault);
+    if (e == cudaSuccess && uniq_start && U) e = cudaMemcpy(uniq_start, v.uniq_start, (U + 1) * 4, cudaMemcpyDefault);
+    if (e == cudaSuccess && grp_start && G) e = cudaMemcpy(grp_start, v.grp_start, (G + 1) * 4, cudaMemcpyDefault);
+    if (e == cudaSuccess && bag_sorted && L) e = cudaMemcpy(bag_sorted, v.bag_sorted, L * 4, cudaMemcpyDefault);
+    return cuda_status(e);
+}
+
+int tt_emb_enable_timing(tt_emb_t h, int enable)
+{
+    if (!h) return TT_ERR_ARG;
+    h->fold();
+    h->timing = enable != 0;
+    for (int i = 0; i < TT_EMB_NUM_PHASES; ++i) h->phase_ms[i] = 0.0;
+    h->launches = 0;
+    return TT_OK;
+}
+
+int tt_emb_phase_times(tt_emb_t h, double* ms, int64_t* launches)
+{
+    if (!h || !ms) return TT_ERR_ARG;
+    for (int i = 0; i < TT_EMB_NUM_PHASES; ++i) ms[i] = h->phase_ms[i];
+    if (launches) *launches = h->launches;
+    return TT_OK;
+}
+
+void tt_emb_destroy(tt_emb_t h)
+{
+    if (!h) return;
+    h->fold();
+    for (cudaEvent_t e : h->pool) cudaEventDestroy(e);
+    if (h->d_status) cudaFree(h->d_status);
+    delete h;
+}
+
+}  // extern "C"

@@ -1,0 +1,163 @@
+// Internal declarations shared by the kernels and the C ABI of libttemb.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tt_emb.h"
+
+namespace tt {
+
+constexpr int kMaxT = TT_EMB_MAX_TABLES;
+constexpr int kMaxK = TT_EMB_MAX_CORES;
+constexpr unsigned kFull = 0xffffffffu;
+
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+// ---------------------------------------------------------------------------
+// Device status block (one per handle, 256 bytes): word 0 holds the first
+// error code raised by any kernel, word 1 a detail (e.g. the bad position).
+// Every kernel returns at once when word 0 is set, so one bad input stops the
+// rest of the call without touching memory it was not given.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void raise_error(int32_t* st, int code, int info)
+{
+    if (atomicCAS(st, 0, code) == 0) st[1] = info;
+}
+
+__device__ __forceinline__ bool has_error(const int32_t* st)
+{
+    return *reinterpret_cast<const volatile int32_t*>(st) != 0;
+}
+
+// Counters that the grouping kernels leave in the workspace header.
+struct WsCounters {
+    int64_t num_unique;  // U: distinct (table, row) keys
+    int64_t num_groups;  // G: prefix groups
+    int64_t pad[30];
+};
+
+// Parameters of the key / grouping kernels.
+struct KeyParams {
+    int32_t T;
+    int32_t ibits;        // bits of the row field of a key
+    int64_t B;            // bags per table
+    int64_t L;            // lookups
+    int32_t unique_only;  // 1: every distinct row is its own group
+    int32_t pad;
+    uint32_t nrows[kMaxT];  // valid rows per table
+    uint32_t nlast[kMaxT];  // n_k per table (prefix = row / n_k)
+};
+
+// Shapes and cores of the fused kernels.
+struct CoreParams {
+    int32_t T, k, D;
+    int32_t P;            // rows of the prefix intermediate, D / d_k
+    int32_t d[kMaxK];
+    int32_t r[kMaxK + 1];
+    int32_t ibits;
+    int32_t unique_only;
+    int64_t B;
+    uint32_t n[kMaxT][kMaxK];
+    const float* cores[kMaxT][kMaxK];
+};
+
+struct GradPtrs {
+    float* g[kMaxT][kMaxK];
+};
+
+// Up to T*k float buffers handled by one elementwise launch (zero fill, SGD).
+struct BufferList {
+    int32_t count;
+    int32_t pad;
+    int64_t chunk_start[kMaxT * kMaxK + 1];  // prefix sums of per-buffer chunk counts
+    int64_t size[kMaxT * kMaxK];             // floats per buffer
+    float* a[kMaxT * kMaxK];                 // updated buffers (16-byte aligned)
+    const float* b[kMaxT * kMaxK];           // second operand (gradients), may be null
+};
+constexpr int kElemChunk = 8192;             // floats per block of an elementwise launch
+
+// ---------------------------------------------------------------------------
+// Block-wide exclusive scan for 256-thread blocks (8 warps).  All threads
+// must call it; `total` receives the block sum.  s_tmp: 8 elements of smem.
+// ---------------------------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ T block256_exclusive_scan(T v, T* total, T* s_tmp)
+{
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    T x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        T y = __shfl_up_sync(kFull, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_tmp[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+        T w = lane < 8 ? s_tmp[lane] : T(0);
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) {
+            T y = __shfl_up_sync(kFull, w, o);
+            if (lane >= o) w += y;
+        }
+        if (lane < 8) s_tmp[lane] = w;
+    }
+    __syncthreads();
+    const T before = wid ? s_tmp[wid - 1] : T(0);
+    *total = s_tmp[7];
+    __syncthreads();
+    return before + x - v;
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launchers (stream-ordered, no host synchronisation).
+// ---------------------------------------------------------------------------
+struct SortBuffers {
+    void* keys[2];        // ping-pong key arrays (uint32 or uint64)
+    int32_t* vals[2];     // ping-pong positions
+    uint32_t* hist;       // [256 * tiles]
+    uint32_t* digit_total;// [256]
+};
+
+constexpr int kSortItems = 8;
+constexpr int kSortTile = 256 * kSortItems;
+constexpr int kScanTile = 256 * 16;
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+cudaError_t launch_make_keys(const KeyParams& kp, bool key64, const int64_t* indices,
+                             const int64_t* offsets, void* keys, int32_t* vals,
+                             int32_t* bag_of_pos, int32_t* status, cudaStream_t s, int* nl);
+
+// Sorts (keys, vals) by the low `bits` bits of the key; returns in *which the
+// buffer index (0 or 1) that holds the result.
+cudaError_t radix_sort_pairs(bool key64, int64_t n, int bits, SortBuffers& sb, int* which,
+                             int32_t* status, cudaStream_t s, int* nl);
+
+cudaError_t launch_segment(const KeyParams& kp, bool key64, const void* sorted_keys,
+                           const int32_t* perm, const int32_t* bag_of_pos, void* uniq_keys,
+                           int32_t* uniq_start, int32_t* grp_start, int32_t* bag_sorted,
+                           uint64_t* partials, WsCounters* counters, int32_t* status,
+                           cudaStream_t s, int* nl);
+
+cudaError_t launch_forward_generic(const CoreParams& cp, bool key64, const void* uniq_keys,
+                                   const int32_t* uniq_start, const int32_t* grp_start,
+                                   const int32_t* bag_sorted, const WsCounters* counters,
+                                   int64_t max_groups, float* out, int32_t* status,
+                                   cudaStream_t s, int grid, int* nl);
+
+cudaError_t launch_backward_generic(const CoreParams& cp, const GradPtrs& gp, bool key64,
+                                    const void* uniq_keys, const int32_t* uniq_start,
+                                    const int32_t* grp_start, const int32_t* bag_sorted,
+                                    const WsCounters* counters, int64_t max_groups,
+                                    const float* grad_out, int32_t* status, cudaStream_t s,
+                                    int grid, int* nl);
+
+cudaError_t launch_fill_zero(const BufferList& bl, int32_t* status, cudaStream_t s, int* nl);
+cudaError_t launch_sgd(const BufferList& bl, float lr, int32_t* status, cudaStream_t s, int* nl);
+
+// Shared-memory floats the generic fused kernels need for these shapes.
+int64_t generic_forward_smem_floats(const CoreParams& cp);
+int64_t generic_backward_smem_floats(const CoreParams& cp);
+
+}  // namespace tt
