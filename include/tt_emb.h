@@ -231,6 +231,40 @@ typedef enum {
 int tt_emb_enable_timing(tt_emb_t h, int enable);
 int tt_emb_phase_times(tt_emb_t h, double* ms, int64_t* launches);
 
+/*
+ * tt_emb_forward_noalloc -- the forward pass (same contract and result as
+ * tt_emb_forward) for callers that cannot allocate device memory.  The paper
+ * has no counterpart; this is a deployment variant of this library.
+ *
+ * Who needs it: hosts that give an embedded library neither an allocator nor
+ * a workspace (plugin interfaces with fixed buffers), processes that forbid
+ * device allocation once they are serving so that memory use and latency stay
+ * fixed, and C callers that do not link PyTorch or any other allocator.  None
+ * of them can provide the workspace that tt_emb_set_workspace expects.
+ *
+ * Instead, the sort buffers, histograms and segmentation arrays live in one
+ * fixed device array of TT_EMB_NOALLOC_SCRATCH_BYTES (16 MiB) that is part of
+ * the library: every GPU on which the library is used holds it until the
+ * process exits.  The call itself allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library routine); the caller still passes inputs and outputs, and
+ * the handle (created beforehand) supplies cores and its status block.
+ *   - num_lookups above TT_EMB_NOALLOC_MAX_LOOKUPS (262144) is rejected with
+ *     TT_ERR_WORKSPACE before any work is enqueued.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and keeps it; make that
+ *     first call before any stream capture.
+ *   - Every call, on every handle and stream, shares the one array, which keeps
+ *     the previous call's contents (the call clears what must start at zero).
+ *     Calls that overlap on the GPU race: order them (one stream, or events).
+ *   - The segmentation of this call is not kept for tt_emb_backward; a backward
+ *     after it returns TT_ERR_STATE until the next tt_emb_forward.
+ */
+#define TT_EMB_NOALLOC_MAX_LOOKUPS 262144
+#define TT_EMB_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+int tt_emb_forward_noalloc(tt_emb_t h, const int64_t* indices, const int64_t* offsets,
+                           int64_t num_lookups, int64_t batch, float* out, tt_stream_t stream);
+
 /* ABI version of the loaded library (TT_EMB_ABI_VERSION). */
 int tt_emb_abi_version(void);
 

@@ -69,8 +69,12 @@ _SIGS = {
     "tt_emb_enable_timing": ([ctypes.c_void_p, ctypes.c_int], ctypes.c_int),
     "tt_emb_phase_times": ([ctypes.c_void_p, ctypes.POINTER(ctypes.c_double),
                             ctypes.POINTER(ctypes.c_int64)], ctypes.c_int),
+    "tt_emb_forward_noalloc": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
     "tt_emb_destroy": ([ctypes.c_void_p], None),
 }
+
+NOALLOC_MAX_LOOKUPS = 262144
 
 PHASES = ("fwd_keys", "fwd_sort", "fwd_segment", "fwd_fused", "bwd_fused", "bwd_reduce", "sgd")
 
@@ -220,6 +224,16 @@ def tt_emb_copy_segmentation(h) -> dict:
         out["grp_start"][:] = 0
     out.update(num_lookups=L, num_unique=U, num_groups=G, key_bits=v.key_bits)
     return out
+
+
+def tt_emb_forward_noalloc(h, indices, offsets, batch: int, out, stream=None):
+    """Forward pass using the library's fixed device scratch instead of a workspace."""
+    import torch
+    _check(lib().tt_emb_forward_noalloc(h, _dev_ptr(indices, torch.int64, "indices"),
+                                        _dev_ptr(offsets, torch.int64, "offsets"), indices.numel(),
+                                        int(batch), _dev_ptr(out, torch.float32, "out"),
+                                        _stream(stream)),
+           "tt_emb_forward_noalloc")
 
 
 def tt_emb_enable_timing(h, enable: bool = True):

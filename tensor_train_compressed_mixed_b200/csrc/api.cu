@@ -538,3 +538,79 @@ void tt_emb_destroy(tt_emb_t h)
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Forward into caller-provided scratch (used by tt_emb_forward_noalloc in
+// noalloc.cu).  Same launch sequence as tt_emb_forward, laid out for exactly
+// num_lookups in `scratch`; no event recording, no allocation, and the
+// segmentation is not kept for a backward pass.
+// ---------------------------------------------------------------------------
+namespace tt {
+
+size_t scratch_bytes_for(tt_emb_t h, int64_t num_lookups)
+{
+    return make_layout(h->key_bytes(), num_lookups, 1).total;
+}
+
+int forward_with_scratch(tt_emb_t h, char* scratch, size_t scratch_bytes, const int64_t* indices,
+                         const int64_t* offsets, int64_t num_lookups, int64_t batch, float* out,
+                         cudaStream_t s)
+{
+    if (!h || !scratch || !offsets || !out || num_lookups < 0 || batch < 1) return TT_ERR_ARG;
+    if (num_lookups > 0 && !indices) return TT_ERR_ARG;
+    if (!h->have_cores) return TT_ERR_STATE;
+    const Layout y = make_layout(h->key_bytes(), num_lookups, batch);
+    if (y.total > scratch_bytes) return TT_ERR_WORKSPACE;
+    h->last_stream = s;
+    h->used_stream = true;
+    h->have_fwd = false;
+    auto at = [&](size_t off) { return scratch + off; };
+    WsCounters* counters = (WsCounters*)at(y.counters);
+    const int64_t L = num_lookups;
+    cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)batch * h->T * h->D, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(counters, 0, sizeof(WsCounters), s);
+    if (e != cudaSuccess) return TT_ERR_CUDA;
+    KeyParams kp;
+    memset(&kp, 0, sizeof(kp));
+    kp.T = h->T;
+    kp.ibits = h->ibits;
+    kp.B = batch;
+    kp.L = L;
+    kp.unique_only = h->opt.grouping == TT_GROUP_UNIQUE_ONLY;
+    for (int t = 0; t < h->T; ++t) {
+        kp.nrows[t] = (uint32_t)h->n_rows[t];
+        kp.nlast[t] = (uint32_t)h->n[t][h->k - 1];
+    }
+    int32_t* bag_of_pos = (int32_t*)at(y.bag_of_pos);
+    SortBuffers sb;
+    sb.keys[0] = at(y.keys[0]);
+    sb.keys[1] = at(y.keys[1]);
+    sb.vals[0] = (int32_t*)at(y.vals[0]);
+    sb.vals[1] = (int32_t*)at(y.vals[1]);
+    sb.hist = (uint32_t*)at(y.hist);
+    sb.digit_total = (uint32_t*)at(y.digit_total);
+    int nl = 0;
+    e = launch_make_keys(kp, h->key64, indices, offsets, sb.keys[0], sb.vals[0], bag_of_pos,
+                         h->d_status, s, &nl);
+    if (e == cudaSuccess && L > 0) {
+        int which = 0;
+        e = radix_sort_pairs(h->key64, L, h->ibits + h->tbits, sb, &which, h->d_status, s, &nl);
+        if (e == cudaSuccess)
+            e = launch_segment(kp, h->key64, sb.keys[which], sb.vals[which], bag_of_pos,
+                               at(y.uniq_keys), (int32_t*)at(y.uniq_start), (int32_t*)at(y.grp_start),
+                               (int32_t*)at(y.bag_sorted), (uint64_t*)at(y.partials), counters,
+                               h->d_status, s, &nl);
+        if (e == cudaSuccess) {
+            CoreParams cp = h->core_params();
+            cp.B = batch;
+            const int grid = h->opt.grid > 0 ? h->opt.grid : h->num_sms * 8;
+            e = launch_forward_generic(cp, h->key64, at(y.uniq_keys), (const int32_t*)at(y.uniq_start),
+                                       (const int32_t*)at(y.grp_start), (const int32_t*)at(y.bag_sorted),
+                                       counters, L, out, h->d_status, s, grid, &nl);
+        }
+    }
+    h->launches += nl;
+    return cuda_status(e);
+}
+
+}  // namespace tt
