@@ -41,6 +41,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--config", type=int, default=4)
+    p.add_argument("--batch", type=int, default=None, help="smaller batch (profiling runs)")
+    p.add_argument("--tables", type=int, default=None, help="fewer tables (profiling runs)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -214,7 +216,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     from workloads import config_workload
-    w = config_workload(args.config, with_grad=True)
+    w = config_workload(args.config, batch=args.batch, tables=args.tables, with_grad=True)
     threads = len(os.sched_getaffinity(0))
     per_step = max(0.5, min(6.0, 150.0 / max(args.steps + args.warmup, 1)))
     sample, S = cpu_sample(w, per_step, threads)
@@ -255,7 +257,7 @@ def run_ours(args):
 
     world, rank, local = dist_init(args.gpus)
     dev = torch.device("cuda", local)
-    w = config_workload(args.config, with_grad=True)
+    w = config_workload(args.config, batch=args.batch, tables=args.tables, with_grad=True)
     train = w.grad_out is not None and args.config in (4, 5)
     emb, cores, idx, off = from_workload(w, device=dev, with_grads=True)
     g = torch.from_numpy(w.grad_out).to(dev)

@@ -12,15 +12,26 @@ namespace {
 
 struct Layout {
     size_t counters, keys[2], vals[2], bag_of_pos, hist, digit_total, partials, uniq_keys,
-        uniq_start, grp_start, bag_sorted, total;
+        uniq_start, grp_start, bag_sorted;
+    // specialised path only (zero when unused)
+    size_t uid_at_pos, uid_sorted, rowbuf, pkeys[2], pvals[2], col_count, col_start, chunk_base,
+        hdr, chunks, tasks;
+    int64_t chunk_cap, task_cap;
+    size_t total;
+};
+
+// Sizes the specialised path adds (filled from the handle).
+struct FastDims {
+    bool on;
+    int D, ncols, MP, T;
 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-Layout make_layout(int key_bytes, int64_t L, int64_t B)
+Layout make_layout(int key_bytes, int64_t L, int64_t B, const FastDims& f)
 {
-    (void)B;
     Layout y;
+    memset(&y, 0, sizeof(y));
     size_t p = 0;
     auto take = [&](size_t bytes) {
         const size_t at = p;
@@ -42,6 +53,23 @@ Layout make_layout(int key_bytes, int64_t L, int64_t B)
     y.uniq_start = take((Lz + 1) * 4);
     y.grp_start = take((Lz + 1) * 4);
     y.bag_sorted = take(Lz * 4);
+    if (f.on) {
+        y.uid_at_pos = take(Lz * 4);
+        y.uid_sorted = take(Lz * 4);
+        y.rowbuf = take(Lz * (size_t)f.D * 4);
+        y.pkeys[0] = take(Lz * 4);
+        y.pkeys[1] = take(Lz * 4);
+        y.pvals[0] = take(Lz * 4);
+        y.pvals[1] = take(Lz * 4);
+        y.col_count = take(((size_t)f.ncols + 1) * 4);
+        y.col_start = take(((size_t)f.ncols + 1) * 4);
+        y.chunk_base = take(((size_t)f.ncols + 1) * 4);
+        y.hdr = take(sizeof(PlanHeader));
+        y.chunk_cap = (int64_t)f.ncols + ceil_div((int64_t)Lz, f.MP) + 1;
+        y.chunks = take((size_t)y.chunk_cap * sizeof(int4));
+        y.task_cap = y.chunk_cap + (int64_t)f.T * ceil_div(B, kPoolBags);
+        y.tasks = take((size_t)y.task_cap * 4);
+    }
     y.total = p;
     return y;
 }
@@ -78,6 +106,10 @@ struct tt_emb_handle {
     int64_t fwd_L = 0, fwd_B = 0;
     int fwd_which = 0;
     int device = 0, num_sms = 148;
+    // specialised three-core path
+    bool fast = false;
+    int ncols = 0;
+    int col_base[kMaxT + 1] = {};
     // timing and launch accounting
     bool timing = false;
     double phase_ms[TT_EMB_NUM_PHASES] = {};
@@ -130,6 +162,34 @@ struct tt_emb_handle {
     }
 
     int key_bytes() const { return key64 ? 8 : 4; }
+    FastDims fast_dims() const
+    {
+        FastDims f;
+        f.on = fast;
+        f.D = D;
+        f.ncols = ncols;
+        f.MP = fast ? k3_plan_mp(core_params()) : 1;
+        f.T = T;
+        return f;
+    }
+    PlanParams plan_params(int64_t batch) const
+    {
+        PlanParams pp;
+        memset(&pp, 0, sizeof(pp));
+        pp.T = T;
+        pp.k = k;
+        pp.ibits = ibits;
+        pp.col_digit = 1;
+        pp.B = batch;
+        pp.MP = k3_plan_mp(core_params());
+        pp.NB = kPoolBags;
+        pp.ncols = ncols;
+        pp.sched = opt.sched;
+        for (int t = 0; t < T; ++t)
+            for (int j = 0; j < k; ++j) pp.n[t][j] = (uint32_t)n[t][j];
+        for (int t = 0; t <= T; ++t) pp.col_base[t] = col_base[t];
+        return pp;
+    }
     int64_t core_floats(int t, int j) const { return (int64_t)r[j] * n[t][j] * d[j] * r[j + 1]; }
 
     CoreParams core_params() const
@@ -169,6 +229,51 @@ struct tt_emb_handle {
     }
 
     char* at(size_t off) const { return ws + off; }
+
+    int32_t* plan_sorted_groups = nullptr;  // set by the last forward's plan
+
+    PlanBuffers plan_buffers(const SortBuffers& lookup_sort)
+    {
+        PlanBuffers pb;
+        memset(&pb, 0, sizeof(pb));
+        pb.sort.keys[0] = at(lay.pkeys[0]);
+        pb.sort.keys[1] = at(lay.pkeys[1]);
+        pb.sort.vals[0] = (int32_t*)at(lay.pvals[0]);
+        pb.sort.vals[1] = (int32_t*)at(lay.pvals[1]);
+        pb.sort.hist = lookup_sort.hist ? lookup_sort.hist : (uint32_t*)at(lay.hist);
+        pb.sort.digit_total = lookup_sort.digit_total ? lookup_sort.digit_total : (uint32_t*)at(lay.digit_total);
+        pb.col_count = (int32_t*)at(lay.col_count);
+        pb.col_start = (int32_t*)at(lay.col_start);
+        pb.chunk_base = (int32_t*)at(lay.chunk_base);
+        pb.hdr = (PlanHeader*)at(lay.hdr);
+        pb.chunks = (int4*)at(lay.chunks);
+        pb.tasks = (int32_t*)at(lay.tasks);
+        return pb;
+    }
+
+    K3Args k3_args(const CoreParams* cp, const PlanParams* pp, const PlanBuffers* pb,
+                   const int64_t* offsets, int64_t L, bool backward) const
+    {
+        K3Args a;
+        memset(&a, 0, sizeof(a));
+        a.cp = cp;
+        a.pp = pp;
+        a.key64 = key64;
+        a.uniq_keys = at(lay.uniq_keys);
+        a.uniq_start = (const int32_t*)at(lay.uniq_start);
+        a.grp_start = (const int32_t*)at(lay.grp_start);
+        a.bag_sorted = (const int32_t*)at(lay.bag_sorted);
+        a.uid_at_pos = (const int32_t*)at(lay.uid_at_pos);
+        a.uid_sorted = (const int32_t*)at(lay.uid_sorted);
+        a.counters = (const WsCounters*)at(lay.counters);
+        a.pb = pb;
+        a.offsets = offsets;
+        a.rowbuf = (float*)at(lay.rowbuf);
+        a.L = L;
+        a.grid = opt.grid > 0 ? opt.grid : num_sms * k3_blocks_per_sm(*cp, backward);
+        a.status = d_status;
+        return a;
+    }
 };
 
 static int cuda_status(cudaError_t e) { return e == cudaSuccess ? TT_OK : TT_ERR_CUDA; }
@@ -261,6 +366,17 @@ int tt_emb_create(int32_t num_tables, int32_t num_cores, const int64_t* n_factor
     h->key64 = h->ibits + h->tbits > 32;
 
     const CoreParams cp = h->core_params();
+    h->fast = k3_supported(cp);
+    if (h->fast) {
+        int64_t nc = 0;
+        for (int t = 0; t < num_tables; ++t) {
+            h->col_base[t] = (int)nc;
+            nc += h->n[t][1];
+        }
+        h->col_base[num_tables] = (int)nc;
+        if (nc >= (1LL << 24)) h->fast = false;
+        h->ncols = (int)nc;
+    }
     if (generic_backward_smem_floats(cp) * 4 > 200 * 1024 ||
         generic_forward_smem_floats(cp) * 4 > 200 * 1024) {
         delete h;
@@ -302,7 +418,7 @@ int tt_emb_workspace_size(tt_emb_t h, int64_t max_lookups, int64_t batch, size_t
 {
     if (!h || !bytes || max_lookups < 0 || batch < 1) return TT_ERR_ARG;
     if (max_lookups >= (int64_t)INT32_MAX) return TT_ERR_ARG;
-    *bytes = make_layout(h->key_bytes(), max_lookups, batch).total;
+    *bytes = make_layout(h->key_bytes(), max_lookups, batch, h->fast_dims()).total;
     return TT_OK;
 }
 
@@ -312,7 +428,7 @@ int tt_emb_set_workspace(tt_emb_t h, void* workspace, size_t bytes, int64_t max_
     if (!h || !workspace || max_lookups < 0 || batch < 1) return TT_ERR_ARG;
     if (((uintptr_t)workspace & 255) != 0) return TT_ERR_ARG;
     if (max_lookups >= (int64_t)INT32_MAX) return TT_ERR_ARG;
-    const Layout lay = make_layout(h->key_bytes(), max_lookups, batch);
+    const Layout lay = make_layout(h->key_bytes(), max_lookups, batch, h->fast_dims());
     if (bytes < lay.total) return TT_ERR_WORKSPACE;
     h->ws = (char*)workspace;
     h->ws_bytes = bytes;
@@ -338,7 +454,8 @@ int tt_emb_forward(tt_emb_t h, const int64_t* indices, const int64_t* offsets, i
     WsCounters* counters = (WsCounters*)h->at(y.counters);
     const int64_t L = num_lookups;
 
-    cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)batch * h->T * h->D, s);
+    cudaError_t e = cudaSuccess;
+    if (!h->fast || L == 0) e = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)batch * h->T * h->D, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(counters, 0, sizeof(WsCounters), s);
     if (e != cudaSuccess) return TT_ERR_CUDA;
 
@@ -386,15 +503,32 @@ int tt_emb_forward(tt_emb_t h, const int64_t* indices, const int64_t* offsets, i
     e = launch_segment(kp, h->key64, sb.keys[which], sb.vals[which], bag_of_pos,
                        h->at(y.uniq_keys), (int32_t*)h->at(y.uniq_start),
                        (int32_t*)h->at(y.grp_start), (int32_t*)h->at(y.bag_sorted),
-                       (uint64_t*)h->at(y.partials), counters, h->d_status, s, &nl);
+                       (uint64_t*)h->at(y.partials), counters,
+                       h->fast ? (int32_t*)h->at(y.uid_at_pos) : nullptr,
+                       h->fast ? (int32_t*)h->at(y.uid_sorted) : nullptr, h->d_status, s, &nl);
+    PlanBuffers pb;
+    PlanParams pp;
+    CoreParams cp = h->core_params();
+    cp.B = batch;
+    if (e == cudaSuccess && h->fast) {
+        pp = h->plan_params(batch);
+        pb = h->plan_buffers(sb);
+        e = launch_plan(pp, h->key64, h->at(y.uniq_keys), (const int32_t*)h->at(y.grp_start), counters, L,
+                        pb, h->d_status, s, &nl);
+        h->plan_sorted_groups = pb.sorted_groups;
+    }
     h->end(s);
     if (e != cudaSuccess) return TT_ERR_CUDA;
-    const CoreParams cp = h->core_params();
-    const int grid = h->opt.grid > 0 ? h->opt.grid : h->num_sms * 8;
     h->begin(TT_PHASE_FWD_FUSED, s);
-    e = launch_forward_generic(cp, h->key64, h->at(y.uniq_keys), (const int32_t*)h->at(y.uniq_start),
-                               (const int32_t*)h->at(y.grp_start), (const int32_t*)h->at(y.bag_sorted),
-                               counters, L, out, h->d_status, s, grid, &nl);
+    if (h->fast) {
+        K3Args a = h->k3_args(&cp, &pp, &pb, offsets, L, false);
+        e = k3_forward(a, out, s, &nl);
+    } else {
+        const int grid = h->opt.grid > 0 ? h->opt.grid : h->num_sms * 8;
+        e = launch_forward_generic(cp, h->key64, h->at(y.uniq_keys), (const int32_t*)h->at(y.uniq_start),
+                                   (const int32_t*)h->at(y.grp_start), (const int32_t*)h->at(y.bag_sorted),
+                                   counters, L, out, h->d_status, s, grid, &nl);
+    }
     h->end(s);
     h->launches += nl;
     if (e != cudaSuccess) return TT_ERR_CUDA;
@@ -423,13 +557,26 @@ int tt_emb_backward(tt_emb_t h, const float* grad_out, tt_stream_t stream)
     for (int t = 0; t < h->T; ++t)
         for (int j = 0; j < h->k; ++j) gp.g[t][j] = h->grads[t * h->k + j];
     const CoreParams cp = h->core_params();
-    const int grid = h->opt.grid > 0 ? h->opt.grid : h->num_sms * 8;
     nl = 0;
     h->begin(TT_PHASE_BWD_FUSED, s);
-    e = launch_backward_generic(cp, gp, h->key64, h->at(y.uniq_keys),
-                                (const int32_t*)h->at(y.uniq_start), (const int32_t*)h->at(y.grp_start),
-                                (const int32_t*)h->at(y.bag_sorted), (const WsCounters*)h->at(y.counters),
-                                h->fwd_L, grad_out, h->d_status, s, grid, &nl);
+    if (h->fast) {
+        PlanParams pp = h->plan_params(h->fwd_B);
+        SortBuffers sb;
+        memset(&sb, 0, sizeof(sb));
+        PlanBuffers pb = h->plan_buffers(sb);
+        pb.sorted_groups = h->plan_sorted_groups;
+        e = cudaMemsetAsync(&pb.hdr->col_head, 0, sizeof(int32_t), s);
+        if (e == cudaSuccess) {
+            K3Args a = h->k3_args(&cp, &pp, &pb, nullptr, h->fwd_L, true);
+            e = k3_backward(a, gp, grad_out, s, &nl);
+        }
+    } else {
+        const int grid = h->opt.grid > 0 ? h->opt.grid : h->num_sms * 8;
+        e = launch_backward_generic(cp, gp, h->key64, h->at(y.uniq_keys),
+                                    (const int32_t*)h->at(y.uniq_start), (const int32_t*)h->at(y.grp_start),
+                                    (const int32_t*)h->at(y.bag_sorted), (const WsCounters*)h->at(y.counters),
+                                    h->fwd_L, grad_out, h->d_status, s, grid, &nl);
+    }
     h->end(s);
     h->launches += nl;
     return cuda_status(e);
@@ -549,7 +696,9 @@ namespace tt {
 
 size_t scratch_bytes_for(tt_emb_t h, int64_t num_lookups)
 {
-    return make_layout(h->key_bytes(), num_lookups, 1).total;
+    FastDims off;
+    memset(&off, 0, sizeof(off));
+    return make_layout(h->key_bytes(), num_lookups, 1, off).total;
 }
 
 int forward_with_scratch(tt_emb_t h, char* scratch, size_t scratch_bytes, const int64_t* indices,
@@ -559,7 +708,9 @@ int forward_with_scratch(tt_emb_t h, char* scratch, size_t scratch_bytes, const 
     if (!h || !scratch || !offsets || !out || num_lookups < 0 || batch < 1) return TT_ERR_ARG;
     if (num_lookups > 0 && !indices) return TT_ERR_ARG;
     if (!h->have_cores) return TT_ERR_STATE;
-    const Layout y = make_layout(h->key_bytes(), num_lookups, batch);
+    FastDims off;
+    memset(&off, 0, sizeof(off));
+    const Layout y = make_layout(h->key_bytes(), num_lookups, batch, off);
     if (y.total > scratch_bytes) return TT_ERR_WORKSPACE;
     h->last_stream = s;
     h->used_stream = true;
@@ -599,7 +750,7 @@ int forward_with_scratch(tt_emb_t h, char* scratch, size_t scratch_bytes, const 
             e = launch_segment(kp, h->key64, sb.keys[which], sb.vals[which], bag_of_pos,
                                at(y.uniq_keys), (int32_t*)at(y.uniq_start), (int32_t*)at(y.grp_start),
                                (int32_t*)at(y.bag_sorted), (uint64_t*)at(y.partials), counters,
-                               h->d_status, s, &nl);
+                               nullptr, nullptr, h->d_status, s, &nl);
         if (e == cudaSuccess) {
             CoreParams cp = h->core_params();
             cp.B = batch;

@@ -100,12 +100,14 @@ cudaError_t launch_make_keys(const KeyParams& kp, bool key64, const int64_t* ind
 // the tile, visited in (item, lane) order, which is input order.
 // ---------------------------------------------------------------------------
 template <typename K>
-__global__ void __launch_bounds__(256) k_radix_hist(const K* __restrict__ kin, int64_t n, int shift,
+__global__ void __launch_bounds__(256) k_radix_hist(const K* __restrict__ kin, int64_t n,
+                                                    const int64_t* __restrict__ dev_n, int shift,
                                                     uint32_t* __restrict__ hist, int tiles,
                                                     const int32_t* status)
 {
     __shared__ uint32_t s_cnt[256];
     if (has_error(status)) return;
+    if (dev_n) n = min64(n, *dev_n);
     s_cnt[threadIdx.x] = 0;
     __syncthreads();
     const int64_t base = (int64_t)blockIdx.x * kSortTile;
@@ -158,7 +160,8 @@ template <typename K>
 __global__ void __launch_bounds__(256) k_radix_scatter(const K* __restrict__ kin,
                                                        const int32_t* __restrict__ vin,
                                                        K* __restrict__ kout, int32_t* __restrict__ vout,
-                                                       int64_t n, int shift,
+                                                       int64_t n, const int64_t* __restrict__ dev_n,
+                                                       int shift,
                                                        const uint32_t* __restrict__ hist,
                                                        const uint32_t* __restrict__ digit_total,
                                                        int tiles, const int32_t* status)
@@ -172,8 +175,10 @@ __global__ void __launch_bounds__(256) k_radix_scatter(const K* __restrict__ kin
     if (has_error(status)) return;
 
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    if (dev_n) n = min64(n, *dev_n);
     const int64_t base = (int64_t)blockIdx.x * kSortTile;
     const int cnt = (int)min64(kSortTile, n - base);
+    if (cnt <= 0) return;
     for (int i = tid; i < 8 * 256; i += 256) (&s_wcnt[0][0])[i] = 0;
     {
         uint32_t tot;
@@ -235,16 +240,16 @@ __global__ void __launch_bounds__(256) k_radix_scatter(const K* __restrict__ kin
 
 template <typename K>
 static cudaError_t radix_sort_t(int64_t n, int bits, SortBuffers& sb, int* which, int32_t* status,
-                                cudaStream_t s, int* nl)
+                                cudaStream_t s, int* nl, const int64_t* dev_n)
 {
     const int tiles = (int)ceil_div(n, kSortTile);
     int cur = 0;
     for (int shift = 0; shift < bits; shift += 8) {
         const K* kin = (const K*)sb.keys[cur];
-        k_radix_hist<K><<<tiles, 256, 0, s>>>(kin, n, shift, sb.hist, tiles, status);
+        k_radix_hist<K><<<tiles, 256, 0, s>>>(kin, n, dev_n, shift, sb.hist, tiles, status);
         k_radix_colscan<<<256, 1024, 0, s>>>(sb.hist, tiles, sb.digit_total, status);
         k_radix_scatter<K><<<tiles, 256, 0, s>>>(kin, sb.vals[cur], (K*)sb.keys[cur ^ 1],
-                                                 sb.vals[cur ^ 1], n, shift, sb.hist,
+                                                 sb.vals[cur ^ 1], n, dev_n, shift, sb.hist,
                                                  sb.digit_total, tiles, status);
         cur ^= 1;
         *nl += 3;
@@ -254,14 +259,14 @@ static cudaError_t radix_sort_t(int64_t n, int bits, SortBuffers& sb, int* which
 }
 
 cudaError_t radix_sort_pairs(bool key64, int64_t n, int bits, SortBuffers& sb, int* which,
-                             int32_t* status, cudaStream_t s, int* nl)
+                             int32_t* status, cudaStream_t s, int* nl, const int64_t* dev_n)
 {
     if (n <= 0) {
         *which = 0;
         return cudaSuccess;
     }
-    return key64 ? radix_sort_t<uint64_t>(n, bits, sb, which, status, s, nl)
-                 : radix_sort_t<uint32_t>(n, bits, sb, which, status, s, nl);
+    return key64 ? radix_sort_t<uint64_t>(n, bits, sb, which, status, s, nl, dev_n)
+                 : radix_sort_t<uint32_t>(n, bits, sb, which, status, s, nl, dev_n);
 }
 
 // ---------------------------------------------------------------------------
@@ -356,6 +361,8 @@ __global__ void __launch_bounds__(256) k_seg_write(KeyParams kp, const K* __rest
                                                    int32_t* __restrict__ uniq_start,
                                                    int32_t* __restrict__ grp_start,
                                                    int32_t* __restrict__ bag_sorted,
+                                                   int32_t* __restrict__ uid_at_pos,
+                                                   int32_t* __restrict__ uid_sorted,
                                                    const int32_t* status)
 {
     __shared__ uint64_t s_tmp[8];
@@ -382,7 +389,11 @@ __global__ void __launch_bounds__(256) k_seg_write(KeyParams kp, const K* __rest
             if (f[j] >> 32) grp_start[gid] = (int32_t)uid;
         }
         run += f[j];
-        bag_sorted[l] = bag_of_pos[perm[l]];
+        const int32_t pl = perm[l];
+        bag_sorted[l] = bag_of_pos[pl];
+        const int32_t my_uid = (int32_t)(run & 0xffffffffull) - 1;  // inclusive count - 1
+        if (uid_at_pos) uid_at_pos[pl] = my_uid;
+        if (uid_sorted) uid_sorted[l] = my_uid;
         if (l == kp.L - 1) {
             uniq_start[(uint32_t)(run & 0xffffffffull)] = (int32_t)kp.L;
             grp_start[(uint32_t)(run >> 32)] = (int32_t)(run & 0xffffffffull);
@@ -393,8 +404,8 @@ __global__ void __launch_bounds__(256) k_seg_write(KeyParams kp, const K* __rest
 cudaError_t launch_segment(const KeyParams& kp, bool key64, const void* sorted_keys,
                            const int32_t* perm, const int32_t* bag_of_pos, void* uniq_keys,
                            int32_t* uniq_start, int32_t* grp_start, int32_t* bag_sorted,
-                           uint64_t* partials, WsCounters* counters, int32_t* status,
-                           cudaStream_t s, int* nl)
+                           uint64_t* partials, WsCounters* counters, int32_t* uid_at_pos,
+                           int32_t* uid_sorted, int32_t* status, cudaStream_t s, int* nl)
 {
     const int nb = (int)ceil_div(kp.L, kScanTile);
     if (nb == 0) return cudaSuccess;
@@ -403,13 +414,15 @@ cudaError_t launch_segment(const KeyParams& kp, bool key64, const void* sorted_k
         k_seg_partials<<<1, 1024, 0, s>>>(partials, nb, counters, status);
         k_seg_write<uint64_t><<<nb, 256, 0, s>>>(kp, (const uint64_t*)sorted_keys, perm, bag_of_pos,
                                                  partials, (uint64_t*)uniq_keys, uniq_start,
-                                                 grp_start, bag_sorted, status);
+                                                 grp_start, bag_sorted, uid_at_pos, uid_sorted,
+                                                 status);
     } else {
         k_seg_reduce<uint32_t><<<nb, 256, 0, s>>>(kp, (const uint32_t*)sorted_keys, partials, status);
         k_seg_partials<<<1, 1024, 0, s>>>(partials, nb, counters, status);
         k_seg_write<uint32_t><<<nb, 256, 0, s>>>(kp, (const uint32_t*)sorted_keys, perm, bag_of_pos,
                                                  partials, (uint32_t*)uniq_keys, uniq_start,
-                                                 grp_start, bag_sorted, status);
+                                                 grp_start, bag_sorted, uid_at_pos, uid_sorted,
+                                                 status);
     }
     *nl += 3;
     return cudaGetLastError();

@@ -1,0 +1,212 @@
+// Work planning for the shape-specialised fused kernels.
+//
+// FlowTT section 3.4 ("Dynamic Load Balancing via Persistent Threads and Work
+// Stealing"): prefix groups become block-level work units, long runs are cut
+// into chunks, and persistent blocks take chunks dynamically.  Here a work
+// unit is a *column group*: all prefix groups of one table that share the
+// digit of the largest prefix slice (i_2 for three cores), so that slice is
+// staged in shared memory once and reused by every prefix of the unit.  The
+// plan
+//   1. keys every prefix group by its column (table, i_c) and counts columns,
+//   2. stable-sorts the groups by column (so each column's groups stay in
+//      canonical order and results do not depend on the schedule),
+//   3. scans the column counts into column starts and chunk bases,
+//   4. writes one record per chunk (at most MP groups of one column) and the
+//      task queue: compute chunks and pooling tasks, table-major, with each
+//      table's pooling placed after the next table's compute chunks so the
+//      pooled rows are still in L2 when they are gathered (TT_SCHED_STEAL_L2),
+//      or all pooling after all compute (other modes).
+#include "tt_common.cuh"
+
+namespace tt {
+
+__device__ __forceinline__ void group_col(const PlanParams& pp, uint64_t key, int* t_out,
+                                          uint32_t* ic_out, uint32_t* i1_out)
+{
+    const int t = (int)(key >> pp.ibits);
+    uint32_t row = (uint32_t)(key & ((uint64_t(1) << pp.ibits) - 1));
+    uint32_t dig[kMaxK];
+    for (int j = pp.k - 1; j >= 0; --j) {
+        const uint32_t nj = pp.n[t][j];
+        dig[j] = row % nj;
+        row /= nj;
+    }
+    *t_out = t;
+    *ic_out = dig[pp.col_digit];
+    *i1_out = dig[0];
+}
+
+template <typename K>
+__global__ void __launch_bounds__(256) k_plan_keys(PlanParams pp, const K* __restrict__ uniq_keys,
+                                                   const int32_t* __restrict__ grp_start,
+                                                   const WsCounters* __restrict__ counters,
+                                                   uint32_t* __restrict__ pkeys,
+                                                   int32_t* __restrict__ pvals,
+                                                   int32_t* __restrict__ col_count,
+                                                   const int32_t* status)
+{
+    if (has_error(status)) return;
+    const int64_t G = counters->num_groups;
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < G;
+         g += (int64_t)gridDim.x * blockDim.x) {
+        int t;
+        uint32_t ic, i1;
+        group_col(pp, (uint64_t)uniq_keys[grp_start[g]], &t, &ic, &i1);
+        const uint32_t col = (uint32_t)pp.col_base[t] + ic;
+        pkeys[g] = col;
+        pvals[g] = (int32_t)g;
+        atomicAdd(&col_count[col], 1);
+    }
+}
+
+// One block: column starts, chunk bases and the task layout.
+__global__ void __launch_bounds__(1024) k_plan_cols(PlanParams pp,
+                                                   const int32_t* __restrict__ col_count,
+                                                   int32_t* __restrict__ col_start,
+                                                   int32_t* __restrict__ chunk_base,
+                                                   PlanHeader* __restrict__ hdr,
+                                                   const int32_t* status)
+{
+    __shared__ int32_t s_w[2][32];
+    __shared__ int32_t s_carry[2];
+    if (has_error(status)) return;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    if (threadIdx.x == 0) s_carry[0] = s_carry[1] = 0;
+    __syncthreads();
+    for (int b0 = 0; b0 < pp.ncols; b0 += 1024) {
+        const int c = b0 + threadIdx.x;
+        const int cnt = c < pp.ncols ? col_count[c] : 0;
+        const int v[2] = {cnt, (cnt + pp.MP - 1) / pp.MP};
+        int x[2] = {v[0], v[1]};
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(kFull, x[q], o);
+                if (lane >= o) x[q] += y;
+            }
+            if (lane == 31) s_w[q][wid] = x[q];
+        }
+        __syncthreads();
+        if (wid == 0) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                int w = s_w[q][lane];
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(kFull, w, o);
+                    if (lane >= o) w += y;
+                }
+                s_w[q][lane] = w;
+            }
+        }
+        __syncthreads();
+        if (c < pp.ncols) {
+            col_start[c] = s_carry[0] + (wid ? s_w[0][wid - 1] : 0) + x[0] - v[0];
+            chunk_base[c] = s_carry[1] + (wid ? s_w[1][wid - 1] : 0) + x[1] - v[1];
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            s_carry[0] += s_w[0][31];
+            s_carry[1] += s_w[1][31];
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        col_start[pp.ncols] = s_carry[0];
+        chunk_base[pp.ncols] = s_carry[1];
+        const int nP = (int)((pp.B + pp.NB - 1) / pp.NB);
+        int q = 0;
+        // task layout: C(t) chunks, then (interleaved mode) P(t-1) after C(t)
+        for (int t = 0; t < pp.T; ++t) {
+            const int c0 = chunk_base[pp.col_base[t]], c1 = chunk_base[pp.col_base[t + 1]];
+            hdr->chunk_first[t] = c0;
+            hdr->nC[t] = c1 - c0;
+            hdr->task_base_C[t] = q;
+            q += c1 - c0;
+            if (pp.sched == TT_SCHED_STEAL_L2 && t >= 1) {
+                hdr->task_base_P[t - 1] = q;
+                q += nP;
+            }
+        }
+        if (pp.sched == TT_SCHED_STEAL_L2) {
+            hdr->task_base_P[pp.T - 1] = q;
+            q += nP;
+        } else {
+            for (int t = 0; t < pp.T; ++t) {
+                hdr->task_base_P[t] = q;
+                q += nP;
+            }
+        }
+        hdr->nP = nP;
+        hdr->ntasks = q;
+        hdr->nchunks = s_carry[1];
+        hdr->queue_head = 0;
+        hdr->col_head = 0;
+    }
+    if (threadIdx.x < pp.T) hdr->done[threadIdx.x] = 0;
+}
+
+__global__ void __launch_bounds__(256) k_plan_chunks(PlanParams pp, const WsCounters* __restrict__ counters,
+                                                     const uint32_t* __restrict__ sorted_cols,
+                                                     const int32_t* __restrict__ col_count,
+                                                     const int32_t* __restrict__ col_start,
+                                                     const int32_t* __restrict__ chunk_base,
+                                                     const PlanHeader* __restrict__ hdr,
+                                                     int4* __restrict__ chunks,
+                                                     int32_t* __restrict__ tasks,
+                                                     const int32_t* status)
+{
+    if (has_error(status)) return;
+    const int64_t G = counters->num_groups;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < G; i += stride) {
+        const uint32_t c = sorted_cols[i];
+        const int r = (int)(i - col_start[c]);
+        if (r % pp.MP != 0) continue;
+        // table of column c: last t with col_base[t] <= c
+        int t = 0;
+        while (t + 1 < pp.T && (uint32_t)pp.col_base[t + 1] <= c) ++t;
+        const int cid = chunk_base[c] + r / pp.MP;
+        const int cnt = min(pp.MP, col_count[c] - r);
+        chunks[cid] = make_int4((int)i, cnt, t, (int)(c - (uint32_t)pp.col_base[t]));
+        tasks[hdr->task_base_C[t] + (cid - hdr->chunk_first[t])] = cid;
+    }
+    const int nP = hdr->nP;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)pp.T * nP; i += stride) {
+        const int t = (int)(i / nP), j = (int)(i % nP);
+        tasks[hdr->task_base_P[t] + j] = -1 - (t * nP + j);
+    }
+}
+
+cudaError_t launch_plan(const PlanParams& pp, bool key64, const void* uniq_keys,
+                        const int32_t* grp_start, const WsCounters* counters, int64_t max_groups,
+                        PlanBuffers& pb, int32_t* status, cudaStream_t s, int* nl)
+{
+    cudaError_t e = cudaMemsetAsync(pb.col_count, 0, sizeof(int32_t) * (size_t)pp.ncols, s);
+    if (e != cudaSuccess) return e;
+    const int grid = 148 * 4;
+    if (key64)
+        k_plan_keys<uint64_t><<<grid, 256, 0, s>>>(pp, (const uint64_t*)uniq_keys, grp_start, counters,
+                                                   (uint32_t*)pb.sort.keys[0], pb.sort.vals[0],
+                                                   pb.col_count, status);
+    else
+        k_plan_keys<uint32_t><<<grid, 256, 0, s>>>(pp, (const uint32_t*)uniq_keys, grp_start, counters,
+                                                   (uint32_t*)pb.sort.keys[0], pb.sort.vals[0],
+                                                   pb.col_count, status);
+    *nl += 1;
+    int bits = 1;
+    while ((1u << bits) < (uint32_t)pp.ncols) ++bits;
+    int which = 0;
+    e = radix_sort_pairs(false, max_groups, bits, pb.sort, &which, status, s, nl,
+                         &counters->num_groups);
+    if (e != cudaSuccess) return e;
+    pb.sorted_groups = pb.sort.vals[which];
+    k_plan_cols<<<1, 1024, 0, s>>>(pp, pb.col_count, pb.col_start, pb.chunk_base, pb.hdr, status);
+    k_plan_chunks<<<grid, 256, 0, s>>>(pp, counters, (const uint32_t*)pb.sort.keys[which], pb.col_count,
+                                       pb.col_start, pb.chunk_base, pb.hdr, pb.chunks, pb.tasks, status);
+    *nl += 2;
+    return cudaGetLastError();
+}
+
+}  // namespace tt

@@ -77,6 +77,48 @@ struct BufferList {
 };
 constexpr int kElemChunk = 8192;             // floats per block of an elementwise launch
 
+struct SortBuffers {
+    void* keys[2];        // ping-pong key arrays (uint32 or uint64)
+    int32_t* vals[2];     // ping-pong positions
+    uint32_t* hist;       // [256 * tiles]
+    uint32_t* digit_total;// [256]
+};
+
+// Parameters of the column-group planner and of the specialised kernels.
+struct PlanParams {
+    int32_t T, k, ibits, col_digit;  // col_digit: prefix digit that names a column (1 = i_2)
+    int64_t B;
+    int32_t MP;                      // prefix groups per forward chunk
+    int32_t NB;                      // bags per pooling task
+    int32_t ncols;                   // sum over tables of n_{col_digit}
+    int32_t sched;                   // tt_sched_mode
+    uint32_t n[kMaxT][kMaxK];
+    int32_t col_base[kMaxT + 1];     // first column of each table
+};
+
+// Device-side plan header (workspace).  Queue cursors and per-table
+// completion counters are reset by the planner on every forward.
+struct PlanHeader {
+    int32_t ntasks, nchunks, nP, pad0;
+    int32_t queue_head, col_head, pad1, pad2;
+    int32_t nC[kMaxT];             // compute chunks per table
+    int32_t chunk_first[kMaxT];    // first chunk id of each table
+    int32_t task_base_C[kMaxT];    // queue position of each table's first chunk
+    int32_t task_base_P[kMaxT];    // queue position of each table's first pooling task
+    int32_t done[kMaxT];           // finished compute chunks per table
+};
+
+struct PlanBuffers {
+    SortBuffers sort;              // uint32 column keys / group ids, ping-pong
+    int32_t* sorted_groups;        // set by launch_plan: group ids in column order
+    int32_t* col_count;            // [ncols]
+    int32_t* col_start;            // [ncols + 1]
+    int32_t* chunk_base;           // [ncols + 1]
+    PlanHeader* hdr;
+    int4* chunks;                  // (first sorted position, groups, table, column digit)
+    int32_t* tasks;                // >= 0: chunk id; < 0: pooling task -1 - (t * nP + j)
+};
+
 // ---------------------------------------------------------------------------
 // Block-wide exclusive scan for 256-thread blocks (8 warps).  All threads
 // must call it; `total` receives the block sum.  s_tmp: 8 elements of smem.
@@ -112,18 +154,12 @@ __device__ __forceinline__ T block256_exclusive_scan(T v, T* total, T* s_tmp)
 // ---------------------------------------------------------------------------
 // Host-side launchers (stream-ordered, no host synchronisation).
 // ---------------------------------------------------------------------------
-struct SortBuffers {
-    void* keys[2];        // ping-pong key arrays (uint32 or uint64)
-    int32_t* vals[2];     // ping-pong positions
-    uint32_t* hist;       // [256 * tiles]
-    uint32_t* digit_total;// [256]
-};
 
 constexpr int kSortItems = 8;
 constexpr int kSortTile = 256 * kSortItems;
 constexpr int kScanTile = 256 * 16;
 
-inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+__host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 cudaError_t launch_make_keys(const KeyParams& kp, bool key64, const int64_t* indices,
                              const int64_t* offsets, void* keys, int32_t* vals,
@@ -131,14 +167,16 @@ cudaError_t launch_make_keys(const KeyParams& kp, bool key64, const int64_t* ind
 
 // Sorts (keys, vals) by the low `bits` bits of the key; returns in *which the
 // buffer index (0 or 1) that holds the result.
+// `dev_n` (may be null): a device count that caps n, for counts known only on the device.
 cudaError_t radix_sort_pairs(bool key64, int64_t n, int bits, SortBuffers& sb, int* which,
-                             int32_t* status, cudaStream_t s, int* nl);
+                             int32_t* status, cudaStream_t s, int* nl,
+                             const int64_t* dev_n = nullptr);
 
 cudaError_t launch_segment(const KeyParams& kp, bool key64, const void* sorted_keys,
                            const int32_t* perm, const int32_t* bag_of_pos, void* uniq_keys,
                            int32_t* uniq_start, int32_t* grp_start, int32_t* bag_sorted,
-                           uint64_t* partials, WsCounters* counters, int32_t* status,
-                           cudaStream_t s, int* nl);
+                           uint64_t* partials, WsCounters* counters, int32_t* uid_at_pos,
+                           int32_t* uid_sorted, int32_t* status, cudaStream_t s, int* nl);
 
 cudaError_t launch_forward_generic(const CoreParams& cp, bool key64, const void* uniq_keys,
                                    const int32_t* uniq_start, const int32_t* grp_start,
@@ -152,6 +190,37 @@ cudaError_t launch_backward_generic(const CoreParams& cp, const GradPtrs& gp, bo
                                     const WsCounters* counters, int64_t max_groups,
                                     const float* grad_out, int32_t* status, cudaStream_t s,
                                     int grid, int* nl);
+
+cudaError_t launch_plan(const PlanParams& pp, bool key64, const void* uniq_keys,
+                        const int32_t* grp_start, const WsCounters* counters, int64_t max_groups,
+                        PlanBuffers& pb, int32_t* status, cudaStream_t s, int* nl);
+
+// Shape-specialised three-core kernels (fused_k3.cu).
+struct K3Args {
+    const CoreParams* cp;
+    const PlanParams* pp;
+    bool key64;
+    const void* uniq_keys;
+    const int32_t* uniq_start;
+    const int32_t* grp_start;
+    const int32_t* bag_sorted;
+    const int32_t* uid_at_pos;
+    const int32_t* uid_sorted;
+    const WsCounters* counters;
+    const PlanBuffers* pb;
+    const int64_t* offsets;
+    float* rowbuf;                 // [U][D]: pooled-row checkpoint (forward), upstream sums (backward)
+    int64_t L;
+    int grid;
+    int32_t* status;
+};
+constexpr int kPoolBags = 64;     // bags per pooling task of the specialised forward
+bool k3_supported(const CoreParams& cp);
+int k3_plan_mp(const CoreParams& cp);
+int k3_blocks_per_sm(const CoreParams& cp, bool backward);
+cudaError_t k3_forward(const K3Args& a, float* out, cudaStream_t s, int* nl);
+cudaError_t k3_backward(const K3Args& a, const GradPtrs& gp, const float* grad_out, cudaStream_t s,
+                        int* nl);
 
 cudaError_t launch_fill_zero(const BufferList& bl, int32_t* status, cudaStream_t s, int* nl);
 cudaError_t launch_sgd(const BufferList& bl, float lr, int32_t* status, cudaStream_t s, int* nl);

@@ -118,3 +118,58 @@ def test_all_bags_empty_and_single_lookup():
                          pooling={"kind": "explicit", "sizes": [1]})
     emb1, _, out1 = gpu_forward(w1)
     np.testing.assert_allclose(out1.cpu().numpy(), oracle.workload_forward(w1), rtol=1e-5, atol=1e-6)
+
+
+def _forward_with(w, sched, grid):
+    from tensor_train_compressed_mixed_b200 import abi
+    o = abi.tt_emb_default_options()
+    o.sched = sched
+    o.grid = grid
+    emb, cores, out = gpu_forward(w, options=o)
+    return out.cpu().numpy()
+
+
+@pytest.mark.parametrize("cfg", [2, 3, 4])
+def test_scheduler_modes_and_grids_give_identical_rows(cfg):
+    """Pooling sums each bag in bag order, so every schedule yields the same bits."""
+    from tensor_train_compressed_mixed_b200 import abi
+    w = config_workload(cfg, batch=96, tables=3, with_grad=False)
+    ref = _forward_with(w, abi.TT_SCHED_STEAL_L2, 0)
+    assert output_err(ref, oracle.workload_forward(w), w.dim) <= FP32_TOL
+    for sched in (abi.TT_SCHED_STATIC, abi.TT_SCHED_STEAL, abi.TT_SCHED_STEAL_L2):
+        for grid in (1, 2, 5, 0):
+            got = _forward_with(w, sched, grid)
+            assert np.array_equal(got, ref), (sched, grid)
+
+
+@pytest.mark.parametrize("sched", [0, 1, 2])
+def test_scheduler_modes_backward(sched):
+    from tensor_train_compressed_mixed_b200 import abi
+    w = config_workload(4, batch=32, tables=2, with_grad=True)
+    o = abi.tt_emb_default_options()
+    o.sched = sched
+    o.grid = 3
+    emb, out, grads, new = gpu_train_step(w, options=o)
+    want = oracle.workload_backward(w)
+    for t in range(w.num_tables):
+        for j in range(w.num_cores):
+            assert core_grad_err(grads[t][j], want[t][j]) <= FP32_TOL, (t, j)
+
+
+def test_single_hot_row_batch():
+    """Every lookup hits one row: one group, one distinct row, ~5000 lookups split across warps."""
+    from workloads.gen import Workload
+    base = config_workload(4, batch=256, tables=1, with_grad=True)
+    rng = np.random.default_rng(9)
+    sizes = rng.integers(1, 40, size=base.batch)
+    offsets = np.zeros(base.batch + 1, dtype=np.int64)
+    np.cumsum(sizes, out=offsets[1:])
+    hot = int(rng.integers(0, base.n_rows[0]))
+    w = Workload(name="hot", d=base.d, r=base.r, n=base.n, n_rows=base.n_rows, batch=base.batch,
+                 indices=np.full(offsets[-1], hot, dtype=np.int64), offsets=offsets,
+                 cores=base.cores, grad_out=base.grad_out, train=True)
+    emb, out, grads, new = gpu_train_step(w)
+    assert output_err(out, oracle.workload_forward(w), w.dim) <= FP32_TOL
+    want = oracle.workload_backward(w)
+    for j in range(w.num_cores):
+        assert core_grad_err(grads[0][j], want[0][j]) <= FP32_TOL, j
