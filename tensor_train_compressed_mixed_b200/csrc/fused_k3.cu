@@ -30,6 +30,29 @@
     X(4, 4, 4, 32)           \
     X(4, 4, 4, 16)
 
+// Optional phase timing (build with -DTT_PROFILE_PHASES): thread 0 of every
+// block adds the clock64 cycles it spent in each phase to a device array that
+// tt_emb_debug_phase_cycles() reads and clears.  Off in normal builds.
+#ifdef TT_PROFILE_PHASES
+__device__ unsigned long long g_tt_phase_cycles[32];
+#define TT_PH_START() long long tt_ph_t0 = clock64()
+#define TT_PH(i)                                                             \
+    do {                                                                     \
+        if (threadIdx.x == 0) {                                              \
+            const long long tt_ph_t = clock64();                             \
+            atomicAdd(&g_tt_phase_cycles[i], (unsigned long long)(tt_ph_t - tt_ph_t0)); \
+            tt_ph_t0 = tt_ph_t;                                              \
+        }                                                                    \
+    } while (0)
+#else
+#define TT_PH_START() \
+    do {              \
+    } while (0)
+#define TT_PH(i) \
+    do {         \
+    } while (0)
+#endif
+
 namespace tt {
 namespace {
 
@@ -49,11 +72,15 @@ struct S3 {
     static constexpr int MPF = MF / D1;       // prefixes per forward chunk
     static constexpr int TPU = D1 * (D3 / 4); // threads per distinct row in the suffix step
     static constexpr int NUF = kThreads / TPU;
-    static constexpr int SU = R * D3 + 4;     // padded stride of one staged last slice
+    static constexpr int SU = R * D3 + 8;     // padded stride of one staged last slice
+    static constexpr size_t FWD_FIXED = (size_t)R * N + (size_t)MF * R + (size_t)MF * N;
+    static constexpr int FBUF = (FWD_FIXED + 2 * (size_t)NUF * SU) * 4 <= 220 * 1024 ? 2 : 1;
     // backward: MB x N per chunk
     static constexpr int MB = 2048 / R;
     static constexpr int MPB = MB / D1;
-    static constexpr int NUB = 16;            // distinct rows per backward batch
+    static constexpr int TPUB = (R / 4) * (D3 / 4);   // dS tiles per distinct row
+    static constexpr int NUB = kThreads / TPUB;      // distinct rows per backward batch
+    static constexpr int SR = D3 + 4;                // padded row of a staged last slice (backward)
     static constexpr int DBR = (R * N) / (kThreads * 4) >= 16 ? 8 : ((R * N) / (kThreads * 4) >= 4 ? 4 : 1);
     static constexpr int DBC = (R * N) / (kThreads * DBR);   // dB columns per thread
     static_assert(D2 == 4, "specialised path needs d_2 = 4");
@@ -62,15 +89,13 @@ struct S3 {
     static_assert(N >= 32 && N % 32 == 0, "swizzle needs N >= 32");
     static_assert(MF % 8 == 0 && (MF / 8) * (N / 8) == kThreads, "forward GEMM tiling");
     static_assert(DBC % 4 == 0, "dB columns in float4 chunks");
+    static_assert(NUB >= 1 && NUB * TPUB == kThreads, "backward batch tiling");
 
-    static constexpr size_t fwd_smem_floats()
-    {
-        return (size_t)R * N + (size_t)R * MF + (size_t)MF * N + (size_t)NUF * SU;
-    }
+    static constexpr size_t fwd_smem_floats() { return FWD_FIXED + (size_t)FBUF * NUF * SU; }
     static constexpr size_t bwd_smem_floats()
     {
         return (size_t)R * N + 2 * (size_t)MB * R + 2 * (size_t)MB * N + 2 * (size_t)NUB * P * D3 +
-               (size_t)NUB * (D3 * R + 4);
+               2 * (size_t)NUB * R * SR;
     }
 };
 
@@ -86,6 +111,11 @@ __device__ __forceinline__ int swz_m(int row, int col)  // key: row mod 8
 {
     return row * W + ((((col >> 2) ^ (row & 7))) << 2) + (col & 3);
 }
+template <int W>
+__device__ __forceinline__ int swz_a(int row, int col)  // key: (row / 4) mod (W / 4)
+{
+    return row * W + ((((col >> 2) ^ ((row >> 2) & (W / 4 - 1)))) << 2) + (col & 3);
+}
 
 __device__ __forceinline__ void red_add_v4(float* p, float4 v)
 {
@@ -98,6 +128,22 @@ __device__ __forceinline__ float4 f4add(float4 a, float4 b)
 {
     return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
 }
+
+__device__ __forceinline__ float f4get(const float4& v, int i)
+{
+    return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+// 16-byte asynchronous global -> shared copies (L2 only), grouped and awaited
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
+{
+    const unsigned a = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(a), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 template <typename K>
 __device__ __forceinline__ uint32_t key_row(K key, int ibits)
@@ -114,174 +160,204 @@ __device__ __forceinline__ int next_task(int sched, int* head, int iter)
 // ---------------------------------------------------------------------------
 // forward
 // ---------------------------------------------------------------------------
+template <class S>
+struct FwdSmem {
+    float* Bs;   // [R][N]        B = G_2[:, i_2], swizzled
+    float* As;   // [MF][R]       A_j = G_1[0, i1_j] rows, swizzled
+    float* Cn;   // [MF][N]       C_all, swizzled
+    float* Ss;   // [FBUF][NUF][SU] last slices of a batch of distinct rows
+};
+
+template <class S>
+struct FwdMeta {   // shared-memory metadata of a chunk (double buffered)
+    int u0[2][S::MPF];
+    int ucum[2][S::MPF + 1];
+    int i1[2][S::MPF];
+    int cnt[2], t[2], i2[2];
+    int bu[2][S::NUF], bp[2][S::NUF], bi3[2][S::NUF];
+    int task[2];
+    int flag;
+};
+
+// metadata of chunk `cid` into buffer mb (all threads call; ends with a barrier)
 template <class S, typename K>
-__device__ void fwd_chunk(const CoreParams& cp, int task, const K* __restrict__ uniq_keys,
-                          const int32_t* __restrict__ grp_start, const int32_t* __restrict__ sorted_groups,
-                          const int4* __restrict__ chunks, PlanHeader* hdr, float* __restrict__ rowbuf,
-                          float* sm, int* si)
+__device__ __forceinline__ void fwd_meta(const CoreParams& cp, int cid, int mb, const K* __restrict__ uniq_keys,
+                                         const int32_t* __restrict__ grp_start,
+                                         const int32_t* __restrict__ sorted_groups,
+                                         const int4* __restrict__ chunks, FwdMeta<S>& M)
 {
-    constexpr int R = S::R, N = S::N, MF = S::MF, MPF = S::MPF, D1 = S::D1, D2 = S::D2, D3 = S::D3;
-    float* Bs = sm;
-    float* AsT = Bs + R * N;
-    float* Cn = AsT + R * MF;
-    float* Ss = Cn + MF * N;
-    int* s_u0 = si;
-    int* s_ucum = s_u0 + MPF;
-    int* s_i1 = s_ucum + MPF + 1;
-    int* s_bu = s_i1 + MPF;
-    int* s_bp = s_bu + S::NUF;
-    int* s_bi3 = s_bp + S::NUF;
-    int* s_cur = s_bi3 + S::NUF;   // [0] table, [1] column digit of the staged B, [2] scratch
     const int tid = threadIdx.x;
-
-    const int4 ch = chunks[task];
-    const int start = ch.x, cnt = ch.y, t = ch.z, i2 = ch.w;
-    const uint32_t n2 = cp.n[t][1], n3 = cp.n[t][2];
-    const float* __restrict__ G1 = cp.cores[t][0];
-    const float* __restrict__ G2 = cp.cores[t][1];
-    const float* __restrict__ G3 = cp.cores[t][2];
-
-    if (tid < MPF) {
+    const int4 ch = chunks[cid];
+    const int t = ch.z;
+    if (tid < S::MPF) {
         int u0 = 0, nu = 0, i1 = 0;
-        if (tid < cnt) {
-            const int g = sorted_groups[start + tid];
+        if (tid < ch.y) {
+            const int g = sorted_groups[ch.x + tid];
             u0 = grp_start[g];
             nu = grp_start[g + 1] - u0;
-            i1 = (int)(key_row(uniq_keys[u0], cp.ibits) / n3 / n2);
+            i1 = (int)(key_row(uniq_keys[u0], cp.ibits) / cp.n[t][2] / cp.n[t][1]);
         }
-        s_u0[tid] = u0;
-        s_ucum[tid] = nu;
-        s_i1[tid] = i1;
+        M.u0[mb][tid] = u0;
+        M.ucum[mb][tid] = nu;
+        M.i1[mb][tid] = i1;
     }
-    const bool need_b = !(s_cur[0] == t && s_cur[1] == i2);
+    if (tid == 0) {
+        M.cnt[mb] = ch.y;
+        M.t[mb] = t;
+        M.i2[mb] = ch.w;
+    }
     __syncthreads();
     if (tid == 0) {
         int run = 0;
-        for (int j = 0; j < MPF; ++j) {
-            const int v = s_ucum[j];
-            s_ucum[j] = run;
+        for (int j = 0; j < S::MPF; ++j) {
+            const int v = M.ucum[mb][j];
+            M.ucum[mb][j] = run;
             run += v;
         }
-        s_ucum[MPF] = run;
-        s_cur[0] = t;
-        s_cur[1] = i2;
+        M.ucum[mb][S::MPF] = run;
     }
-    // stage B = G_2[:, i_2] (rows of N floats at stride n_2 * N), swizzled
-    if (need_b) {
+    __syncthreads();
+}
+
+// asynchronous copies of the chunk's A rows (and B when its column changes); one commit group
+template <class S>
+__device__ __forceinline__ void fwd_issue_ab(const CoreParams& cp, int mb, const FwdMeta<S>& M,
+                                             const FwdSmem<S>& sm, int& cur_t, int& cur_i2)
+{
+    constexpr int R = S::R, N = S::N, MF = S::MF, D1 = S::D1;
+    const int tid = threadIdx.x;
+    const int t = M.t[mb], i2 = M.i2[mb], cnt = M.cnt[mb];
+    if (t != cur_t || i2 != cur_i2) {
+        const float* G2 = cp.cores[t][1] + (int64_t)i2 * N;
+        const int64_t rs = (int64_t)cp.n[t][1] * N;
         for (int q = tid; q < R * N / 4; q += kThreads) {
             const int rho = q / (N / 4), c4 = q % (N / 4);
-            const float4 v = __ldg(reinterpret_cast<const float4*>(G2 + ((int64_t)rho * n2 + i2) * N) + c4);
-            *reinterpret_cast<float4*>(&Bs[swz_b<N>(rho, c4 * 4)]) = v;
+            cp_async16(&sm.Bs[swz_b<N>(rho, c4 * 4)], G2 + rho * rs + c4 * 4);
         }
+        cur_t = t;
+        cur_i2 = i2;
     }
-    // stage A^T: AsT[rho][m], m = j * D1 + a1, A_j = G_1[0, i1_j] (D1 x R)
-    for (int q = tid; q < R * MF; q += kThreads) {
-        const int rho = q / MF, m = q % MF;
+    const float* G1 = cp.cores[t][0];
+    for (int q = tid; q < MF * (R / 4); q += kThreads) {
+        const int m = q / (R / 4), c4 = q % (R / 4);
         const int j = m / D1, a1 = m % D1;
-        float v = 0.f;
-        if (j < cnt) v = __ldg(G1 + ((int64_t)s_i1[j] * D1 + a1) * R + rho);
-        AsT[rho * MF + m] = v;
+        float* dst = &sm.As[swz_a<R>(m, c4 * 4)];
+        if (j < cnt) cp_async16(dst, G1 + ((int64_t)M.i1[mb][j] * D1 + a1) * R + c4 * 4);
+        else *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    __syncthreads();
+    cp_async_commit();
+}
 
-    // C_all[m][n] = sum_rho A[m][rho] B[rho][n]; thread: rows {4tm+i, MF/2+4tm+i}, cols {4tn+j, N/2+4tn+j}
-    {
-        constexpr int TN = N / 8;
-        const int tn = tid % TN, tm = tid / TN;
-        float acc[8][8];
+// C_all = A . B into Cn; thread tile rows {4tm+i, MF/2+4tm+i} x cols {4tn+j, N/2+4tn+j}
+template <class S>
+__device__ __forceinline__ void fwd_gemm(const FwdSmem<S>& sm)
+{
+    constexpr int R = S::R, N = S::N, MF = S::MF;
+    constexpr int TN = N / 8;
+    const int tn = threadIdx.x % TN, tm = threadIdx.x / TN;
+    int rows[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < 8; ++i) rows[i] = (i < 4) ? tm * 4 + i : MF / 2 + tm * 4 + (i - 4);
+    float acc[8][8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-#pragma unroll 2
-        for (int rho = 0; rho < R; ++rho) {
-            const float4 a0 = *reinterpret_cast<const float4*>(&AsT[rho * MF + tm * 4]);
-            const float4 a1 = *reinterpret_cast<const float4*>(&AsT[rho * MF + MF / 2 + tm * 4]);
-            const float4 b0 = *reinterpret_cast<const float4*>(&Bs[swz_b<N>(rho, tn * 4)]);
-            const float4 b1 = *reinterpret_cast<const float4*>(&Bs[swz_b<N>(rho, N / 2 + tn * 4)]);
-            const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+#pragma unroll 1
+    for (int rho = 0; rho < R; rho += 4) {
+        float4 a[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a[i] = *reinterpret_cast<const float4*>(&sm.As[swz_a<R>(rows[i], rho)]);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const float4 b0 = *reinterpret_cast<const float4*>(&sm.Bs[swz_b<N>(rho + r, tn * 4)]);
+            const float4 b1 = *reinterpret_cast<const float4*>(&sm.Bs[swz_b<N>(rho + r, N / 2 + tn * 4)]);
             const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
+            for (int i = 0; i < 8; ++i) {
+                const float av = f4get(a[i], r);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int m = (i < 4) ? tm * 4 + i : MF / 2 + tm * 4 + (i - 4);
-            *reinterpret_cast<float4*>(&Cn[swz_m<N>(m, tn * 4)]) =
-                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-            *reinterpret_cast<float4*>(&Cn[swz_m<N>(m, N / 2 + tn * 4)]) =
-                make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
-        }
-    }
-    __syncthreads();
-
-    // suffix step: E_u = C_p (P x R) . S_u (R x D3), for the chunk's distinct rows
-    const int total = s_ucum[MPF];
-    const uint64_t rmask = (uint64_t(1) << cp.ibits) - 1;
-    for (int k0 = 0; k0 < total; k0 += S::NUF) {
-        const int nb = min(S::NUF, total - k0);
-        if (tid < nb) {
-            const int kq = k0 + tid;
-            int j = 0;
-            while (j + 1 < cnt && s_ucum[j + 1] <= kq) ++j;
-            const int u = s_u0[j] + (kq - s_ucum[j]);
-            s_bu[tid] = u;
-            s_bp[tid] = j;
-            s_bi3[tid] = (int)((uint32_t)((uint64_t)uniq_keys[u] & rmask) % n3);
-        }
-        __syncthreads();
-        for (int q = tid; q < nb * R * (D3 / 4); q += kThreads) {
-            const int uu = q / (R * (D3 / 4)), rem = q % (R * (D3 / 4));
-            const int rho = rem / (D3 / 4), c4 = rem % (D3 / 4);
-            const float4 v = __ldg(reinterpret_cast<const float4*>(
-                G3 + ((int64_t)rho * n3 + s_bi3[uu]) * D3) + c4);
-            *reinterpret_cast<float4*>(&Ss[uu * S::SU + rho * D3 + c4 * 4]) = v;
-        }
-        __syncthreads();
-        {
-            const int uu = tid / S::TPU;
-            const int a1 = (tid % S::TPU) / (D3 / 4), cg = tid % (D3 / 4);
-            if (uu < nb) {
-                const int p = s_bp[uu];
-                const int m = p * D1 + a1;
-                const float* srow = &Ss[uu * S::SU + cg * 4];
-                float4 e[4];
-#pragma unroll
-                for (int a2 = 0; a2 < 4; ++a2) e[a2] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 2
-                for (int rho = 0; rho < R; rho += 4) {
-                    float4 c[4];
-#pragma unroll
-                    for (int a2 = 0; a2 < 4; ++a2)
-                        c[a2] = *reinterpret_cast<const float4*>(&Cn[swz_m<N>(m, a2 * R + rho)]);
-                    float4 s[4];
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) s[r] = *reinterpret_cast<const float4*>(srow + (rho + r) * D3);
-#pragma unroll
-                    for (int a2 = 0; a2 < 4; ++a2) {
-                        const float cv[4] = {c[a2].x, c[a2].y, c[a2].z, c[a2].w};
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) {
-                            e[a2].x = fmaf(cv[r], s[r].x, e[a2].x);
-                            e[a2].y = fmaf(cv[r], s[r].y, e[a2].y);
-                            e[a2].z = fmaf(cv[r], s[r].z, e[a2].z);
-                            e[a2].w = fmaf(cv[r], s[r].w, e[a2].w);
-                        }
-                    }
-                }
-                float* dst = rowbuf + (int64_t)s_bu[uu] * S::D + cg * 4;
-#pragma unroll
-                for (int a2 = 0; a2 < 4; ++a2)
-                    *reinterpret_cast<float4*>(dst + (a1 * D2 + a2) * D3) = e[a2];
+                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av, b[j], acc[i][j]);
             }
         }
-        __syncthreads();
     }
-    __threadfence();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        *reinterpret_cast<float4*>(&sm.Cn[swz_m<N>(rows[i], tn * 4)]) =
+            make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        *reinterpret_cast<float4*>(&sm.Cn[swz_m<N>(rows[i], N / 2 + tn * 4)]) =
+            make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
+    }
+}
+
+// distinct rows k0..k0+nb of the chunk into batch buffer bb; issues their last slices (one commit group)
+template <class S, typename K>
+__device__ __forceinline__ void fwd_issue_batch(const CoreParams& cp, int mb, int k0, int bb,
+                                                const K* __restrict__ uniq_keys, FwdMeta<S>& M,
+                                                const FwdSmem<S>& sm)
+{
+    constexpr int R = S::R, D3 = S::D3;
+    const int tid = threadIdx.x;
+    const int total = M.ucum[mb][S::MPF];
+    const int nb = min(S::NUF, total - k0);
+    const int t = M.t[mb];
+    const uint32_t n3 = cp.n[t][2];
+    if (tid < nb) {
+        const int kq = k0 + tid;
+        int j = 0;
+        while (j + 1 < M.cnt[mb] && M.ucum[mb][j + 1] <= kq) ++j;
+        const int u = M.u0[mb][j] + (kq - M.ucum[mb][j]);
+        M.bu[bb][tid] = u;
+        M.bp[bb][tid] = j;
+        M.bi3[bb][tid] = (int)(key_row(uniq_keys[u], cp.ibits) % n3);
+    }
     __syncthreads();
-    if (tid == 0) atomicAdd(&hdr->done[t], 1);
+    const float* G3 = cp.cores[t][2];
+    float* Ss = sm.Ss + (size_t)bb * S::NUF * S::SU;
+    for (int q = tid; q < nb * R * (D3 / 4); q += kThreads) {
+        const int uu = q / (R * (D3 / 4)), rem = q % (R * (D3 / 4));
+        const int rho = rem / (D3 / 4), c4 = rem % (D3 / 4);
+        cp_async16(&Ss[uu * S::SU + rho * D3 + c4 * 4], G3 + ((int64_t)rho * n3 + M.bi3[bb][uu]) * D3 + c4 * 4);
+    }
+    cp_async_commit();
+}
+
+// E_u = C_p . S_u for the batch in buffer bb; tile: rows (a1, a2 = 0..3) x 4 columns of a3
+template <class S>
+__device__ __forceinline__ void fwd_batch_compute(int nb, int bb, const FwdMeta<S>& M, const FwdSmem<S>& sm,
+                                                  float* __restrict__ rowbuf)
+{
+    constexpr int R = S::R, N = S::N, D1 = S::D1, D2 = S::D2, D3 = S::D3;
+    const int tid = threadIdx.x;
+    const int uu = tid / S::TPU;
+    if (uu >= nb) return;
+    const int a1 = (tid % S::TPU) / (D3 / 4), cg = tid % (D3 / 4);
+    const int m = M.bp[bb][uu] * D1 + a1;
+    const float* srow = sm.Ss + (size_t)bb * S::NUF * S::SU + uu * S::SU + cg * 4;
+    float4 e[4];
+#pragma unroll
+    for (int a2 = 0; a2 < 4; ++a2) e[a2] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+    for (int rho = 0; rho < R; rho += 4) {
+        float4 c[4], s4[4];
+#pragma unroll
+        for (int a2 = 0; a2 < 4; ++a2) c[a2] = *reinterpret_cast<const float4*>(&sm.Cn[swz_m<N>(m, a2 * R + rho)]);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) s4[r] = *reinterpret_cast<const float4*>(srow + (rho + r) * D3);
+#pragma unroll
+        for (int a2 = 0; a2 < 4; ++a2)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const float cv = f4get(c[a2], r);
+                e[a2].x = fmaf(cv, s4[r].x, e[a2].x);
+                e[a2].y = fmaf(cv, s4[r].y, e[a2].y);
+                e[a2].z = fmaf(cv, s4[r].z, e[a2].z);
+                e[a2].w = fmaf(cv, s4[r].w, e[a2].w);
+            }
+    }
+    float* dst = rowbuf + (int64_t)M.bu[bb][uu] * S::D + cg * 4;
+#pragma unroll
+    for (int a2 = 0; a2 < 4; ++a2) *reinterpret_cast<float4*>(dst + (a1 * D2 + a2) * D3) = e[a2];
 }
 
 template <class S>
@@ -293,6 +369,7 @@ __device__ void fwd_pool(const CoreParams& cp, int ptask, int nP, const int32_t*
     constexpr int D = S::D, LB = D / 4, BPW = 32 / LB;
     const int t = ptask / nP, jb = ptask % nP;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    TT_PH_START();
     if (tid == 0) {
         const int want = hdr->nC[t];
         int it = 0, ok = 1;
@@ -308,22 +385,45 @@ __device__ void fwd_pool(const CoreParams& cp, int ptask, int nP, const int32_t*
         s_flag[0] = ok;
     }
     __syncthreads();
+    TT_PH(4);
     if (!s_flag[0]) return;
     const int64_t B = cp.B, TD = (int64_t)cp.T * D;
-    const int sub = lane / LB, col = (lane % LB) * 4;
+    const int sub = lane / LB, sl = lane % LB, col = sl * 4;
+    const unsigned smask = LB == 32 ? kFull : (((1u << LB) - 1u) << (sub * LB));
     const int b_lo = jb * kNB, b_hi = (int)min64((int64_t)b_lo + kNB, B);
+    const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+    // one sub-warp of LB lanes per bag; every lane owns 4 columns
     for (int b = b_lo + wid * BPW + sub; b < b_hi; b += (kThreads / 32) * BPW) {
         const int64_t g = (int64_t)t * B + b;
         const int64_t l0 = offsets[g], l1 = offsets[g + 1];
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int64_t l = l0; l < l1; ++l) {
-            const int u = uid_at_pos[l];
-            acc = f4add(acc, __ldcg(reinterpret_cast<const float4*>(rowbuf + (int64_t)u * D + col)));
+        float4 acc = zero;
+        for (int64_t base = l0; base < l1; base += LB) {
+            const int n = (int)min64(LB, l1 - base);
+            const int myu = sl < n ? uid_at_pos[base + sl] : 0;   // row ids of up to LB lookups
+            for (int k = 0; k < n; k += 16) {
+                float4 v[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int u = __shfl_sync(smask, myu, (k + q) & (LB - 1), LB);
+                    v[q] = (k + q < n) ? __ldcg(reinterpret_cast<const float4*>(rowbuf + (int64_t)u * D + col))
+                                       : zero;
+                }
+#pragma unroll
+                for (int q = 0; q < 16; ++q)   // lookup order: the sum is the same for every schedule
+                    if (k + q < n) acc = f4add(acc, v[q]);
+            }
         }
         *reinterpret_cast<float4*>(out + (int64_t)b * TD + (int64_t)t * D + col) = acc;
     }
+    __syncthreads();
+    TT_PH(5);
 }
 
+// Persistent forward.  Software pipeline per chunk: wait for its A/B copies,
+// GEMM, then fetch the next task and, if it is a chunk, prefetch its
+// metadata and A/B rows (As and Bs are free once the GEMM is done) while this
+// chunk's distinct rows are contracted batch by batch (double-buffered last
+// slices when shared memory allows).
 template <class S, typename K>
 __global__ void __launch_bounds__(kThreads, 1)
 k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
@@ -332,29 +432,92 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
               const int4* __restrict__ chunks, const int32_t* __restrict__ tasks, PlanHeader* hdr,
               float* __restrict__ rowbuf, float* __restrict__ out, int32_t* status)
 {
-    extern __shared__ __align__(16) float sm[];
-    int* si = reinterpret_cast<int*>(sm + S::fwd_smem_floats());
-    __shared__ int s_task[2];
+    extern __shared__ __align__(16) float smem_f[];
+    __shared__ FwdMeta<S> M;
     if (has_error(status)) return;
-    int* s_cur = si + S::MPF * 3 + 1 + S::NUF * 3;
-    if (threadIdx.x == 0) {
-        s_cur[0] = -1;
-        s_cur[1] = -1;
-    }
+    FwdSmem<S> sm;
+    sm.Bs = smem_f;
+    sm.As = sm.Bs + S::R * S::N;
+    sm.Cn = sm.As + S::MF * S::R;
+    sm.Ss = sm.Cn + S::MF * S::N;
+    const int tid = threadIdx.x;
     const int ntasks = hdr->ntasks, nP = hdr->nP;
+    int iter = 0;
+    int cur_t = -1, cur_i2 = -1;   // column of the B now in (or on its way to) Bs
+    int mb = 0;
+    bool staged = false;
+    if (tid == 0) M.task[0] = next_task(sched, &hdr->queue_head, iter);
+    ++iter;
     __syncthreads();
-    for (int iter = 0;; ++iter) {
-        if (threadIdx.x == 0) s_task[0] = next_task(sched, &hdr->queue_head, iter);
+    int q = M.task[0];
+    while (q < ntasks) {
+        const int tv = tasks[q];
+        if (tv < 0) {
+            fwd_pool<S>(cp, -1 - tv, nP, uid_at_pos, offsets, hdr, rowbuf, out, status, &M.flag);
+            __syncthreads();
+            if (tid == 0) M.task[0] = next_task(sched, &hdr->queue_head, iter);
+            ++iter;
+            __syncthreads();
+            q = M.task[0];
+            staged = false;
+            continue;
+        }
+        TT_PH_START();
+        if (!staged) {
+            fwd_meta<S, K>(cp, tv, mb, uniq_keys, grp_start, sorted_groups, chunks, M);
+            fwd_issue_ab<S>(cp, mb, M, sm, cur_t, cur_i2);
+        }
+        if (tid == 0) M.task[1] = next_task(sched, &hdr->queue_head, iter);   // result used after the GEMM
+        ++iter;
+        cp_async_wait_all();
         __syncthreads();
-        const int q = s_task[0];
-        if (q >= ntasks) break;
-        const int task = tasks[q];
-        if (task >= 0)
-            fwd_chunk<S, K>(cp, task, uniq_keys, grp_start, sorted_groups, chunks, hdr, rowbuf, sm, si);
-        else
-            fwd_pool<S>(cp, -1 - task, nP, uid_at_pos, offsets, hdr, rowbuf, out, status, &s_task[1]);
+        TT_PH(0);
+        fwd_gemm<S>(sm);
         __syncthreads();
+        TT_PH(1);
+        const int qn = M.task[1];
+        const bool next_chunk = qn < ntasks && tasks[qn] >= 0;
+        if (next_chunk) {
+            fwd_meta<S, K>(cp, tasks[qn], mb ^ 1, uniq_keys, grp_start, sorted_groups, chunks, M);
+            fwd_issue_ab<S>(cp, mb ^ 1, M, sm, cur_t, cur_i2);
+        }
+        // distinct rows of this chunk, in batches of NUF
+        const int total = M.ucum[mb][S::MPF];
+        if (S::FBUF == 2) {
+            if (total > 0) fwd_issue_batch<S, K>(cp, mb, 0, 0, uniq_keys, M, sm);
+            for (int k0 = 0, b = 0; k0 < total; k0 += S::NUF, b ^= 1) {
+                const bool more = k0 + S::NUF < total;
+                if (more) {
+                    fwd_issue_batch<S, K>(cp, mb, k0 + S::NUF, b ^ 1, uniq_keys, M, sm);
+                    cp_async_wait<1>();
+                } else {
+                    cp_async_wait_all();
+                }
+                __syncthreads();
+                TT_PH(2);
+                fwd_batch_compute<S>(min(S::NUF, total - k0), b, M, sm, rowbuf);
+                __syncthreads();
+                TT_PH(3);
+            }
+        } else {
+            for (int k0 = 0; k0 < total; k0 += S::NUF) {
+                fwd_issue_batch<S, K>(cp, mb, k0, 0, uniq_keys, M, sm);
+                cp_async_wait_all();
+                __syncthreads();
+                TT_PH(2);
+                fwd_batch_compute<S>(min(S::NUF, total - k0), 0, M, sm, rowbuf);
+                __syncthreads();
+                TT_PH(3);
+            }
+        }
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) atomicAdd(&hdr->done[M.t[mb]], 1);
+        q = qn;
+        staged = next_chunk;
+        if (next_chunk) mb ^= 1;
     }
+    cp_async_wait_all();
 }
 
 // ---------------------------------------------------------------------------
@@ -391,32 +554,150 @@ __global__ void __launch_bounds__(256) k3_hsum(const int32_t* __restrict__ uid_s
     const int lane = threadIdx.x & 31;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t c0 = warp * kHChunk;
-    if (c0 >= L || lane >= LB) return;
+    if (c0 >= L) return;
     const int64_t c1 = min64(L, c0 + kHChunk);
     const int64_t TD = (int64_t)T * D;
+    const bool active = lane < LB;
+    const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
     int cur = uid_sorted[c0];
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int64_t l = c0; l <= c1; ++l) {
-        const int u = l < c1 ? uid_sorted[l] : -1;
-        if (u != cur) {
-            float* dst = rowbuf + (int64_t)cur * D + lane * 4;
-            const bool whole = uniq_start[cur] >= c0 && uniq_start[cur + 1] <= c1;
-            if (whole) *reinterpret_cast<float4*>(dst) = acc;
-            else red_add_v4(dst, acc);
-            if (l == c1) break;
-            cur = u;
-            acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 acc = zero;
+    auto flush = [&](int u, float4 a) {
+        if (!active) return;
+        float* dst = rowbuf + (int64_t)u * D + lane * 4;
+        if (uniq_start[u] >= c0 && uniq_start[u + 1] <= c1) *reinterpret_cast<float4*>(dst) = a;
+        else red_add_v4(dst, a);
+    };
+    for (int64_t base = c0; base < c1; base += 32) {
+        const int n = (int)min64(32, c1 - base);
+        const int myu = lane < n ? uid_sorted[base + lane] : -1;
+        const int myb = lane < n ? bag_sorted[base + lane] : 0;
+        for (int k = 0; k < n; k += 8) {
+            float4 v[8];
+            int uq[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                uq[q] = __shfl_sync(kFull, myu, k + q);
+                const int bag = __shfl_sync(kFull, myb, k + q);
+                const int t = (int)(bag / B);
+                const int64_t b = bag - (int64_t)t * B;
+                v[q] = (active && k + q < n)
+                           ? __ldg(reinterpret_cast<const float4*>(grad_out + b * TD + (int64_t)t * D) + lane)
+                           : zero;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                if (k + q >= n) break;
+                if (uq[q] != cur) {
+                    flush(cur, acc);
+                    cur = uq[q];
+                    acc = zero;
+                }
+                acc = f4add(acc, v[q]);
+            }
         }
-        const int bag = bag_sorted[l];
-        const int t = (int)(bag / B);
-        const int64_t b = bag - (int64_t)t * B;
-        acc = f4add(acc, __ldg(reinterpret_cast<const float4*>(grad_out + b * TD + (int64_t)t * D) + lane));
     }
+    flush(cur, acc);
 }
 
 // ---------------------------------------------------------------------------
 // backward over column groups
 // ---------------------------------------------------------------------------
+template <class S>
+struct BwdMeta {
+    int u0[2][S::MPB];
+    int ucum[2][S::MPB + 1];
+    int i1[2][S::MPB];
+    int cnt[2];
+    int bu[2][S::NUB], bp[2][S::NUB], bi3[2][S::NUB];
+    int task;
+};
+
+// chunk metadata (groups cfirst+j0 .. +MPB of the column) into buffer mb; ends with a barrier
+template <class S, typename K>
+__device__ __forceinline__ void bwd_meta(const CoreParams& cp, int t, int cfirst, int j0, int ccount, int mb,
+                                         const K* __restrict__ uniq_keys, const int32_t* __restrict__ grp_start,
+                                         const int32_t* __restrict__ sorted_groups, BwdMeta<S>& M)
+{
+    const int tid = threadIdx.x;
+    const int cnt = min(S::MPB, ccount - j0);
+    if (tid < S::MPB) {
+        int u0 = 0, nu = 0, i1 = 0;
+        if (tid < cnt) {
+            const int g = sorted_groups[cfirst + j0 + tid];
+            u0 = grp_start[g];
+            nu = grp_start[g + 1] - u0;
+            i1 = (int)(key_row(uniq_keys[u0], cp.ibits) / cp.n[t][2] / cp.n[t][1]);
+        }
+        M.u0[mb][tid] = u0;
+        M.ucum[mb][tid] = nu;
+        M.i1[mb][tid] = i1;
+    }
+    if (tid == 0) M.cnt[mb] = cnt;
+    __syncthreads();
+    if (tid == 0) {
+        int run = 0;
+        for (int j = 0; j < S::MPB; ++j) {
+            const int v = M.ucum[mb][j];
+            M.ucum[mb][j] = run;
+            run += v;
+        }
+        M.ucum[mb][S::MPB] = run;
+    }
+    __syncthreads();
+}
+
+template <class S>
+__device__ __forceinline__ void bwd_issue_a(const CoreParams& cp, int t, int mb, const BwdMeta<S>& M, float* As)
+{
+    constexpr int R = S::R, MB = S::MB, D1 = S::D1;
+    const float* G1 = cp.cores[t][0];
+    const int cnt = M.cnt[mb];
+    for (int q = threadIdx.x; q < MB * (R / 4); q += kThreads) {
+        const int m = q / (R / 4), c4 = q % (R / 4);
+        const int j = m / D1, a1 = m % D1;
+        float* dst = &As[swz_a<R>(m, c4 * 4)];
+        if (j < cnt) cp_async16(dst, G1 + ((int64_t)M.i1[mb][j] * D1 + a1) * R + c4 * 4);
+        else *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    cp_async_commit();
+}
+
+// batch of distinct rows k0.. of chunk buffer mb into batch buffer bb: H rows and last slices (one group)
+template <class S, typename K>
+__device__ __forceinline__ void bwd_issue_batch(const CoreParams& cp, int t, int mb, int k0, int bb,
+                                                const K* __restrict__ uniq_keys, const float* __restrict__ rowbuf,
+                                                BwdMeta<S>& M, float* Hs, float* Ss)
+{
+    constexpr int R = S::R, D3 = S::D3, P = S::P, SR = S::SR;
+    const int tid = threadIdx.x;
+    const int total = M.ucum[mb][S::MPB];
+    const int nb = min(S::NUB, total - k0);
+    const uint32_t n3 = cp.n[t][2];
+    if (tid < nb) {
+        const int kq = k0 + tid;
+        int j = 0;
+        while (j + 1 < M.cnt[mb] && M.ucum[mb][j + 1] <= kq) ++j;
+        const int u = M.u0[mb][j] + (kq - M.ucum[mb][j]);
+        M.bu[bb][tid] = u;
+        M.bp[bb][tid] = j;
+        M.bi3[bb][tid] = (int)(key_row(uniq_keys[u], cp.ibits) % n3);
+    }
+    __syncthreads();
+    float* H = Hs + (size_t)bb * S::NUB * P * D3;
+    float* Sb = Ss + (size_t)bb * S::NUB * R * SR;
+    for (int q = tid; q < nb * (P * D3 / 4); q += kThreads) {
+        const int uu = q / (P * D3 / 4), c4 = q % (P * D3 / 4);
+        cp_async16(&H[uu * P * D3 + c4 * 4], rowbuf + (int64_t)M.bu[bb][uu] * S::D + c4 * 4);
+    }
+    const float* G3 = cp.cores[t][2];
+    for (int q = tid; q < nb * R * (D3 / 4); q += kThreads) {
+        const int uu = q / (R * (D3 / 4)), rem = q % (R * (D3 / 4));
+        const int rho = rem / (D3 / 4), c4 = rem % (D3 / 4);
+        cp_async16(&Sb[(uu * R + rho) * SR + c4 * 4], G3 + ((int64_t)rho * n3 + M.bi3[bb][uu]) * D3 + c4 * 4);
+    }
+    cp_async_commit();
+}
+
 template <class S, typename K>
 __global__ void __launch_bounds__(kThreads, 1)
 k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ uniq_keys,
@@ -425,29 +706,22 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
               PlanHeader* hdr, const float* __restrict__ rowbuf, int32_t* status)
 {
     constexpr int R = S::R, N = S::N, MB = S::MB, MPB = S::MPB, D1 = S::D1, D2 = S::D2, D3 = S::D3,
-                  P = S::P, NUB = S::NUB, DBR = S::DBR, DBC = S::DBC;
-    extern __shared__ __align__(16) float sm[];
-    float* Bs = sm;                       // [R][N] swizzled (key row/4)
-    float* As = Bs + R * N;               // [MB][R]
-    float* AsT = As + MB * R;             // [R][MB]
-    float* Cn = AsT + R * MB;             // [MB][N] swizzled (key row)
-    float* dCn = Cn + MB * N;             // [MB][N] swizzled (key row)
-    float* Hs = dCn + MB * N;             // [NUB][P][D3]
-    float* HsT = Hs + NUB * P * D3;       // [NUB][D3][P]
-    float* SsT = HsT + NUB * P * D3;      // [NUB][D3][R] (+4 pad per row block)
-    __shared__ int s_u0[MPB], s_ucum[MPB + 1], s_i1[MPB];
-    __shared__ int s_bu[NUB], s_bp[NUB], s_bi3[NUB];
-    __shared__ int s_task;
-    constexpr int SST = D3 * R + 4;
+                  P = S::P, NUB = S::NUB, DBR = S::DBR, DBC = S::DBC, SR = S::SR;
+    extern __shared__ __align__(16) float smem_f[];
+    __shared__ BwdMeta<S> M;
+    float* Bs = smem_f;                    // [R][N] swizzled (key row/4)
+    float* As = Bs + R * N;                // [2][MB][R] swizzled rows
+    float* Cn = As + 2 * MB * R;           // [MB][N] swizzled (key row)
+    float* dCn = Cn + MB * N;              // [MB][N] swizzled (key row)
+    float* Hs = dCn + MB * N;              // [2][NUB][P][D3]
+    float* Ss = Hs + 2 * NUB * P * D3;     // [2][NUB][R][SR]
     if (has_error(status)) return;
-    const int tid = threadIdx.x, lane = tid & 31;
-    const uint64_t rmask = (uint64_t(1) << cp.ibits) - 1;
-    (void)lane;
+    const int tid = threadIdx.x;
 
     for (int iter = 0;; ++iter) {
-        if (tid == 0) s_task = next_task(pp.sched, &hdr->col_head, iter);
+        if (tid == 0) M.task = next_task(pp.sched, &hdr->col_head, iter);
         __syncthreads();
-        const int c = s_task;
+        const int c = M.task;
         if (c >= pp.ncols) break;
         const int ccount = col_count[c];
         if (ccount == 0) {
@@ -459,22 +733,26 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
         const int i2 = c - pp.col_base[t];
         const int cfirst = col_start[c];
         const uint32_t n2 = cp.n[t][1], n3 = cp.n[t][2];
-        const float* __restrict__ G1 = cp.cores[t][0];
-        const float* __restrict__ G2 = cp.cores[t][1];
-        const float* __restrict__ G3 = cp.cores[t][2];
         float* __restrict__ dG1 = gp.g[t][0];
         float* __restrict__ dG2 = gp.g[t][1];
         float* __restrict__ dG3 = gp.g[t][2];
+        TT_PH_START();
 
-        for (int q = tid; q < R * N / 4; q += kThreads) {
-            const int rho = q / (N / 4), c4 = q % (N / 4);
-            const float4 v = __ldg(reinterpret_cast<const float4*>(G2 + ((int64_t)rho * n2 + i2) * N) + c4);
-            *reinterpret_cast<float4*>(&Bs[swz_b<N>(rho, c4 * 4)]) = v;
+        // B for the whole column group, and the first chunk's A
+        {
+            const float* G2 = cp.cores[t][1] + (int64_t)i2 * N;
+            const int64_t rs = (int64_t)n2 * N;
+            for (int q = tid; q < R * N / 4; q += kThreads) {
+                const int rho = q / (N / 4), c4 = q % (N / 4);
+                cp_async16(&Bs[swz_b<N>(rho, c4 * 4)], G2 + rho * rs + c4 * 4);
+            }
         }
-        // dB accumulators: rows {tr*(DBR/2)+i, R/2 + tr*(DBR/2)+i} (DBR >= 4) or {tr} (DBR == 1),
-        // cols: DBC/4 float4 chunks {tn*4, N/(DBC/4) + tn*4, ...}
+        bwd_meta<S, K>(cp, t, cfirst, 0, ccount, 0, uniq_keys, grp_start, sorted_groups, M);
+        bwd_issue_a<S>(cp, t, 0, M, As);
+        TT_PH(8);
+
         constexpr int NCH = DBC / 4;
-        constexpr int TNB = N / DBC;  // column tiles
+        constexpr int TNB = N / DBC;
         const int tnb = tid % TNB, trb = tid / TNB;
         float dB[DBR][DBC];
 #pragma unroll
@@ -482,41 +760,15 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
 #pragma unroll
             for (int j = 0; j < DBC; ++j) dB[i][j] = 0.f;
 
-        for (int j0 = 0; j0 < ccount; j0 += MPB) {
-            const int cnt = min(MPB, ccount - j0);
-            __syncthreads();   // previous chunk finished with As / dCn
-            if (tid < MPB) {
-                int u0 = 0, nu = 0, i1 = 0;
-                if (tid < cnt) {
-                    const int g = sorted_groups[cfirst + j0 + tid];
-                    u0 = grp_start[g];
-                    nu = grp_start[g + 1] - u0;
-                    i1 = (int)(key_row(uniq_keys[u0], cp.ibits) / n3 / n2);
-                }
-                s_u0[tid] = u0;
-                s_ucum[tid] = nu;
-                s_i1[tid] = i1;
-            }
-            __syncthreads();
-            if (tid == 0) {
-                int run = 0;
-                for (int j = 0; j < MPB; ++j) {
-                    const int v = s_ucum[j];
-                    s_ucum[j] = run;
-                    run += v;
-                }
-                s_ucum[MPB] = run;
-            }
-            for (int q = tid; q < MB * R; q += kThreads) {
-                const int m = q / R, rho = q % R;
-                const int j = m / D1, a1 = m % D1;
-                const float v = j < cnt ? __ldg(G1 + ((int64_t)s_i1[j] * D1 + a1) * R + rho) : 0.f;
-                As[m * R + rho] = v;
-                AsT[rho * MB + m] = v;
-            }
+        int mb = 0;
+        for (int j0 = 0; j0 < ccount; j0 += MPB, mb ^= 1) {
+            const int cnt = M.cnt[mb];
+            const float* Ab = As + mb * MB * R;
             for (int q = tid; q < MB * N / 4; q += kThreads)
                 reinterpret_cast<float4*>(dCn)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            cp_async_wait_all();
             __syncthreads();
+            TT_PH(9);
 
             // C_all = A . B  (MB x N): thread tile 4 rows x 8 cols
             {
@@ -527,17 +779,23 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                 for (int i = 0; i < 4; ++i)
 #pragma unroll
                     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-#pragma unroll 2
-                for (int rho = 0; rho < R; ++rho) {
-                    const float4 a0 = *reinterpret_cast<const float4*>(&AsT[rho * MB + tm * 4]);
-                    const float4 b0 = *reinterpret_cast<const float4*>(&Bs[swz_b<N>(rho, tn * 4)]);
-                    const float4 b1 = *reinterpret_cast<const float4*>(&Bs[swz_b<N>(rho, N / 2 + tn * 4)]);
-                    const float a[4] = {a0.x, a0.y, a0.z, a0.w};
-                    const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll 1
+                for (int rho = 0; rho < R; rho += 4) {
+                    float4 a[4];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
+                    for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(&Ab[swz_a<R>(tm * 4 + i, rho)]);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+                    for (int r = 0; r < 4; ++r) {
+                        const float4 b0 = *reinterpret_cast<const float4*>(&Bs[swz_b<N>(rho + r, tn * 4)]);
+                        const float4 b1 = *reinterpret_cast<const float4*>(&Bs[swz_b<N>(rho + r, N / 2 + tn * 4)]);
+                        const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float av = f4get(a[i], r);
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av, b[j], acc[i][j]);
+                        }
+                    }
                 }
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -549,42 +807,36 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                 }
             }
             __syncthreads();
+            TT_PH(10);
 
-            // distinct rows in batches: dS_u -> dG3 (vector reductions), dC_p accumulated in dCn
-            const int total = s_ucum[MPB];
-            for (int k0 = 0; k0 < total; k0 += NUB) {
+            // next chunk's metadata and A rows go in flight while this chunk's rows are processed
+            const bool more = j0 + MPB < ccount;
+            if (more) {
+                bwd_meta<S, K>(cp, t, cfirst, j0 + MPB, ccount, mb ^ 1, uniq_keys, grp_start, sorted_groups, M);
+                bwd_issue_a<S>(cp, t, mb ^ 1, M, As + (mb ^ 1) * MB * R);
+            }
+
+            // distinct rows in double-buffered batches: dS_u -> dG_3 (vector reductions), dC_p += H_u S_u^T
+            const int total = M.ucum[mb][MPB];
+            if (total > 0) bwd_issue_batch<S, K>(cp, t, mb, 0, 0, uniq_keys, rowbuf, M, Hs, Ss);
+            for (int k0 = 0, bb = 0; k0 < total; k0 += NUB, bb ^= 1) {
                 const int nb = min(NUB, total - k0);
-                if (tid < nb) {
-                    const int kq = k0 + tid;
-                    int j = 0;
-                    while (j + 1 < cnt && s_ucum[j + 1] <= kq) ++j;
-                    const int u = s_u0[j] + (kq - s_ucum[j]);
-                    s_bu[tid] = u;
-                    s_bp[tid] = j;
-                    s_bi3[tid] = (int)((uint32_t)((uint64_t)uniq_keys[u] & rmask) % n3);
+                if (k0 + NUB < total) {
+                    bwd_issue_batch<S, K>(cp, t, mb, k0 + NUB, bb ^ 1, uniq_keys, rowbuf, M, Hs, Ss);
+                    cp_async_wait<1>();
+                } else {
+                    cp_async_wait_all();
                 }
                 __syncthreads();
-                // stage H (both layouts) and S^T
-                for (int q = tid; q < nb * P * D3; q += kThreads) {
-                    const int uu = q / (P * D3), rem = q % (P * D3);
-                    const int row = rem / D3, a3 = rem % D3;
-                    const float v = __ldcg(rowbuf + (int64_t)s_bu[uu] * S::D + rem);
-                    Hs[uu * P * D3 + rem] = v;
-                    HsT[uu * P * D3 + a3 * P + row] = v;
-                }
-                for (int q = tid; q < nb * R * D3; q += kThreads) {
-                    const int uu = q / (R * D3), rem = q % (R * D3);
-                    const int rho = rem / D3, a3 = rem % D3;
-                    SsT[uu * SST + a3 * R + rho] = __ldg(G3 + ((int64_t)rho * n3 + s_bi3[uu]) * D3 + a3);
-                }
-                __syncthreads();
-                // dS_u[rho2][a3] = sum_row C_p[row][rho2] H_u[row][a3]; tile 4 rho2 x 4 a3
+                TT_PH(11);
+                const float* H = Hs + (size_t)bb * NUB * P * D3;
+                const float* Sb = Ss + (size_t)bb * NUB * R * SR;
+                // dS_u[rho2][a3]: tile 4 consecutive rho2 x 4 a3, one tile per thread
                 {
-                    constexpr int TPU = (R / 4) * (D3 / 4);
-                    for (int w = tid; w < nb * TPU; w += kThreads) {
-                        const int uu = w / TPU, rem = w % TPU;
-                        const int rc = rem / (D3 / 4), cg = rem % (D3 / 4);
-                        const int p = s_bp[uu];
+                    const int uu = tid / S::TPUB, rem = tid % S::TPUB;
+                    const int rc = rem / (D3 / 4), cg = rem % (D3 / 4);
+                    if (uu < nb) {
+                        const int p = M.bp[bb][uu];
                         float4 o[4];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -592,109 +844,134 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                         for (int row = 0; row < P; ++row) {
                             const int m = p * D1 + row / D2, a2 = row % D2;
                             const float4 cv = *reinterpret_cast<const float4*>(&Cn[swz_m<N>(m, a2 * R + rc * 4)]);
-                            const float4 h = *reinterpret_cast<const float4*>(&Hs[uu * P * D3 + row * D3 + cg * 4]);
-                            const float cr[4] = {cv.x, cv.y, cv.z, cv.w};
+                            const float4 h = *reinterpret_cast<const float4*>(&H[uu * P * D3 + row * D3 + cg * 4]);
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
-                                o[i].x = fmaf(cr[i], h.x, o[i].x);
-                                o[i].y = fmaf(cr[i], h.y, o[i].y);
-                                o[i].z = fmaf(cr[i], h.z, o[i].z);
-                                o[i].w = fmaf(cr[i], h.w, o[i].w);
+                                const float cr = f4get(cv, i);
+                                o[i].x = fmaf(cr, h.x, o[i].x);
+                                o[i].y = fmaf(cr, h.y, o[i].y);
+                                o[i].z = fmaf(cr, h.z, o[i].z);
+                                o[i].w = fmaf(cr, h.w, o[i].w);
                             }
                         }
-                        const int i3 = s_bi3[uu];
+                        const int i3 = M.bi3[bb][uu];
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
                             red_add_v4(dG3 + ((int64_t)(rc * 4 + i) * n3 + i3) * D3 + cg * 4, o[i]);
                     }
                 }
-                // dC_p[row][rho2] += sum_{u in p, a3} H_u[row][a3] S_u[rho2][a3]; tile rows (a1, a2=0..3) x 4 rho2
+                // dC_p[row][rho2] += sum_{u in p, a3} H_u[row][a3] S_u[rho2][a3]: each tile (prefix p,
+                // rows (a1, a2 = 0..3), rho2 in {rc, rc+R/4, rc+R/2, rc+3R/4}) is owned by one thread, which
+                // adds the batch's rows of its prefix in order (plain read-modify-write, deterministic)
                 {
-                    constexpr int TPP = D1 * (R / 4);
-                    for (int w = tid; w < cnt * TPP; w += kThreads) {
-                        const int p = w / TPP, rem = w % TPP;
+                    constexpr int TPD = D1 * (R / 4);
+                    for (int w = tid; w < cnt * TPD; w += kThreads) {
+                        const int p = w / TPD, rem = w % TPD;
                         const int a1 = rem / (R / 4), rc = rem % (R / 4);
-                        const int ulo = max(s_ucum[p], k0) - k0, uhi = min(s_ucum[p + 1], k0 + nb) - k0;
+                        const int ulo = max(M.ucum[mb][p], k0) - k0, uhi = min(M.ucum[mb][p + 1], k0 + nb) - k0;
                         if (ulo >= uhi) continue;
-                        float4 o[4];
+                        float o[4][4];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int i = 0; i < 4; ++i)
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) o[i][j] = 0.f;
                         for (int uu = ulo; uu < uhi; ++uu) {
 #pragma unroll
-                            for (int a3 = 0; a3 < D3; ++a3) {
-                                const float4 h = *reinterpret_cast<const float4*>(&HsT[uu * P * D3 + a3 * P + a1 * D2]);
-                                const float4 sv = *reinterpret_cast<const float4*>(&SsT[uu * SST + a3 * R + rc * 4]);
-                                const float hr[4] = {h.x, h.y, h.z, h.w};
+                            for (int ac = 0; ac < D3; ac += 4) {
+                                float4 h[4], sv[4];
 #pragma unroll
-                                for (int i = 0; i < 4; ++i) {
-                                    o[i].x = fmaf(hr[i], sv.x, o[i].x);
-                                    o[i].y = fmaf(hr[i], sv.y, o[i].y);
-                                    o[i].z = fmaf(hr[i], sv.z, o[i].z);
-                                    o[i].w = fmaf(hr[i], sv.w, o[i].w);
-                                }
+                                for (int i = 0; i < 4; ++i)
+                                    h[i] = *reinterpret_cast<const float4*>(&H[uu * P * D3 + (a1 * D2 + i) * D3 + ac]);
+#pragma unroll
+                                for (int j = 0; j < 4; ++j)
+                                    sv[j] = *reinterpret_cast<const float4*>(&Sb[(uu * R + rc + j * (R / 4)) * SR + ac]);
+#pragma unroll
+                                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j) {
+                                        o[i][j] = fmaf(h[i].x, sv[j].x, o[i][j]);
+                                        o[i][j] = fmaf(h[i].y, sv[j].y, o[i][j]);
+                                        o[i][j] = fmaf(h[i].z, sv[j].z, o[i][j]);
+                                        o[i][j] = fmaf(h[i].w, sv[j].w, o[i][j]);
+                                    }
                             }
                         }
                         const int m = p * D1 + a1;
 #pragma unroll
-                        for (int a2 = 0; a2 < 4; ++a2) {
-                            float4* d = reinterpret_cast<float4*>(&dCn[swz_m<N>(m, a2 * R + rc * 4)]);
-                            *d = f4add(*d, o[a2]);
-                        }
+                        for (int i = 0; i < 4; ++i)
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) dCn[swz_m<N>(m, i * R + rc + j * (R / 4))] += o[i][j];
                     }
                 }
                 __syncthreads();
+                TT_PH(12);
             }
 
-            // dA[m][rho1] = sum_n dC[m][n] B[rho1][n] -> dG_1 (vector reductions); tile 2 m x 4 rho1
+            // dA[m][rho1] = sum_n dC[m][n] B[rho1][n] -> dG_1; tiles 4 m x 4 rho1, the n range split
+            // between the two halves of the block and combined through shared memory
             {
                 constexpr int TRH = R / 4;
-                const int tr = tid % TRH, tm = tid / TRH;   // tm < MB / 2
-                float o[2][4];
+                const int kh = tid / 128, tl = tid % 128;
+                float* part = Hs;   // batch buffers are free here: 128 tiles x 16 partial sums
+                float o[4][4];
 #pragma unroll
-                for (int i = 0; i < 2; ++i)
+                for (int i = 0; i < 4; ++i)
 #pragma unroll
                     for (int j = 0; j < 4; ++j) o[i][j] = 0.f;
+                const bool act = tl < (MB / 4) * TRH;
+                const int tr = tl % TRH, tm = tl / TRH;
+                if (act) {
 #pragma unroll 2
-                for (int n = 0; n < N; n += 4) {
-                    float4 dc[2], b[4];
+                    for (int n = kh * (N / 2); n < (kh + 1) * (N / 2); n += 4) {
+                        float4 dc[4], b[4];
 #pragma unroll
-                    for (int i = 0; i < 2; ++i)
-                        dc[i] = *reinterpret_cast<const float4*>(&dCn[swz_m<N>(tm * 2 + i, n)]);
+                        for (int i = 0; i < 4; ++i)
+                            dc[i] = *reinterpret_cast<const float4*>(&dCn[swz_m<N>(tm * 4 + i, n)]);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        b[j] = *reinterpret_cast<const float4*>(&Bs[swz_b<N>(tr * 4 + j, n)]);
+                        for (int j = 0; j < 4; ++j)
+                            b[j] = *reinterpret_cast<const float4*>(&Bs[swz_b<N>(tr * 4 + j, n)]);
 #pragma unroll
-                    for (int i = 0; i < 2; ++i)
+                        for (int i = 0; i < 4; ++i)
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            o[i][j] = fmaf(dc[i].x, b[j].x, o[i][j]);
-                            o[i][j] = fmaf(dc[i].y, b[j].y, o[i][j]);
-                            o[i][j] = fmaf(dc[i].z, b[j].z, o[i][j]);
-                            o[i][j] = fmaf(dc[i].w, b[j].w, o[i][j]);
-                        }
+                            for (int j = 0; j < 4; ++j)
+                                o[i][j] += dc[i].x * b[j].x + dc[i].y * b[j].y + dc[i].z * b[j].z + dc[i].w * b[j].w;
+                    }
                 }
+                if (kh == 1 && act) {
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const int m = tm * 2 + i, p = m / D1, a1 = m % D1;
-                    if (p < cnt)
-                        red_add_v4(dG1 + ((int64_t)s_i1[p] * D1 + a1) * R + tr * 4,
-                                   make_float4(o[i][0], o[i][1], o[i][2], o[i][3]));
+                    for (int i = 0; i < 4; ++i)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) part[tl * 16 + i * 4 + j] = o[i][j];
+                }
+                __syncthreads();
+                if (kh == 0 && act) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int m = tm * 4 + i, p = m / D1, a1 = m % D1;
+                        if (p < cnt)
+                            red_add_v4(dG1 + ((int64_t)M.i1[mb][p] * D1 + a1) * R + tr * 4,
+                                       make_float4(o[i][0] + part[tl * 16 + i * 4 + 0],
+                                                   o[i][1] + part[tl * 16 + i * 4 + 1],
+                                                   o[i][2] + part[tl * 16 + i * 4 + 2],
+                                                   o[i][3] + part[tl * 16 + i * 4 + 3]));
+                    }
                 }
             }
+            TT_PH(13);
             // dB[rho1][n] += sum_m A[m][rho1] dC[m][n]
             {
 #pragma unroll 2
                 for (int m = 0; m < MB; ++m) {
                     float a[DBR];
                     if constexpr (DBR >= 4) {
-                        const float4 a0 = *reinterpret_cast<const float4*>(&As[m * R + trb * 4]);
+                        const float4 a0 = *reinterpret_cast<const float4*>(&Ab[swz_a<R>(m, trb * 4)]);
                         a[0] = a0.x; a[1] = a0.y; a[2] = a0.z; a[3] = a0.w;
                         if constexpr (DBR == 8) {
-                            const float4 a1v = *reinterpret_cast<const float4*>(&As[m * R + R / 2 + trb * 4]);
+                            const float4 a1v = *reinterpret_cast<const float4*>(&Ab[swz_a<R>(m, R / 2 + trb * 4)]);
                             a[4] = a1v.x; a[5] = a1v.y; a[6] = a1v.z; a[7] = a1v.w;
                         }
                     } else {
-                        a[0] = As[m * R + trb];
+                        a[0] = Ab[swz_a<R>(m, trb)];
                     }
                     float bv[DBC];
 #pragma unroll
@@ -708,6 +985,8 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                         for (int j = 0; j < DBC; ++j) dB[i][j] = fmaf(a[i], bv[j], dB[i][j]);
                 }
             }
+            __syncthreads();   // dCn, Ab and the partial buffer are reused by the next chunk
+            TT_PH(14);
         }
         // the column group is complete: dG_2[:, i_2] = dB (this block owns the slice)
 #pragma unroll
@@ -723,7 +1002,9 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                     make_float4(dB[i][ch * 4], dB[i][ch * 4 + 1], dB[i][ch * 4 + 2], dB[i][ch * 4 + 3]);
         }
         __syncthreads();
+        TT_PH(15);
     }
+    cp_async_wait_all();
 }
 
 // ---------------------------------------------------------------------------
@@ -732,7 +1013,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
 template <class S, typename K>
 cudaError_t fwd_launch(const K3Args& a, float* out, cudaStream_t s, int* nl)
 {
-    const size_t smem = sizeof(float) * S::fwd_smem_floats() + sizeof(int) * (S::MPF * 3 + 1 + S::NUF * 3 + 4);
+    const size_t smem = sizeof(float) * S::fwd_smem_floats();
     cudaError_t e = cudaFuncSetAttribute(k3_fwd_kernel<S, K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const PlanBuffers& pb = *a.pb;
@@ -777,7 +1058,7 @@ cudaError_t bwd_dispatch(const K3Args& a, const GradPtrs& gp, const float* g, cu
 template <class S>
 int occ_fwd()
 {
-    const size_t smem = sizeof(float) * S::fwd_smem_floats() + sizeof(int) * (S::MPF * 3 + 1 + S::NUF * 3 + 4);
+    const size_t smem = sizeof(float) * S::fwd_smem_floats();
     cudaFuncSetAttribute(k3_fwd_kernel<S, uint32_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k3_fwd_kernel<S, uint32_t>, kThreads, smem) != cudaSuccess) return 1;
@@ -841,3 +1122,15 @@ cudaError_t k3_backward(const K3Args& a, const GradPtrs& gp, const float* grad_o
 }
 
 }  // namespace tt
+
+#ifdef TT_PROFILE_PHASES
+extern "C" int tt_emb_debug_phase_cycles(unsigned long long* out, int n)
+{
+    if (!out || n < 1 || n > 32) return TT_ERR_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return TT_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(out, g_tt_phase_cycles, sizeof(unsigned long long) * n) != cudaSuccess) return TT_ERR_CUDA;
+    unsigned long long zero[32] = {};
+    if (cudaMemcpyToSymbol(g_tt_phase_cycles, zero, sizeof(zero)) != cudaSuccess) return TT_ERR_CUDA;
+    return TT_OK;
+}
+#endif
