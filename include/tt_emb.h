@@ -89,7 +89,8 @@ typedef struct {
     int32_t grouping;        /* tt_group_mode, default TT_GROUP_PREFIX */
     int32_t chunk;           /* rows per stealable chunk of a prefix group; 0 = library default */
     int32_t grid;            /* persistent blocks; 0 = one wave on the current device */
-    int32_t reserved[12];    /* must be zero */
+    int32_t force_generic;   /* 1: run the shape-generic kernels even where a specialised path exists */
+    int32_t reserved[11];    /* must be zero */
 } tt_emb_options;
 
 /* Fills *opt with the defaults. */

@@ -33,7 +33,7 @@ class TTEmbError(RuntimeError):
 class Options(ctypes.Structure):
     _fields_ = [("sched", ctypes.c_int32), ("grouping", ctypes.c_int32),
                 ("chunk", ctypes.c_int32), ("grid", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 12)]
+                ("force_generic", ctypes.c_int32), ("reserved", ctypes.c_int32 * 11)]
 
 
 class SegView(ctypes.Structure):

@@ -15,7 +15,7 @@ struct Layout {
         uniq_start, grp_start, bag_sorted;
     // specialised path only (zero when unused)
     size_t uid_at_pos, uid_sorted, rowbuf, pkeys[2], pvals[2], col_count, col_start, chunk_base,
-        hdr, chunks, tasks;
+        hdr, chunks, tasks, g12, dg12;
     int64_t chunk_cap, task_cap;
     size_t total;
 };
@@ -24,6 +24,7 @@ struct Layout {
 struct FastDims {
     bool on;
     int D, ncols, MP, T;
+    int64_t g12_floats;   // merged first cores of four-core tables (0 otherwise)
 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -69,6 +70,10 @@ Layout make_layout(int key_bytes, int64_t L, int64_t B, const FastDims& f)
         y.chunks = take((size_t)y.chunk_cap * sizeof(int4));
         y.task_cap = y.chunk_cap + (int64_t)f.T * ceil_div(B, kPoolBags);
         y.tasks = take((size_t)y.task_cap * 4);
+        if (f.g12_floats > 0) {
+            y.g12 = take((size_t)f.g12_floats * 4);
+            y.dg12 = take((size_t)f.g12_floats * 4);
+        }
     }
     y.total = p;
     return y;
@@ -106,10 +111,14 @@ struct tt_emb_handle {
     int64_t fwd_L = 0, fwd_B = 0;
     int fwd_which = 0;
     int device = 0, num_sms = 148;
-    // specialised three-core path
+    // specialised three-core path (four-core tables through the merged-core view)
     bool fast = false;
+    bool merged = false;
     int ncols = 0;
     int col_base[kMaxT + 1] = {};
+    int64_t vn[kMaxT][3] = {};      // three-core view: factors (n_1 n_2, n_3, n_4) when merged
+    int32_t vd[3] = {}, vr[4] = {};
+    int64_t g12_off[kMaxT + 1] = {};  // merged-core offsets (floats) in the workspace
     // timing and launch accounting
     bool timing = false;
     double phase_ms[TT_EMB_NUM_PHASES] = {};
@@ -168,25 +177,88 @@ struct tt_emb_handle {
         f.on = fast;
         f.D = D;
         f.ncols = ncols;
-        f.MP = fast ? k3_plan_mp(core_params()) : 1;
+        f.MP = fast ? k3_plan_mp(view_params()) : 1;
         f.T = T;
+        f.g12_floats = merged ? g12_off[T] : 0;
         return f;
+    }
+    // three-core view of the shapes (identity for three-core tables), without core pointers
+    CoreParams view_params() const
+    {
+        CoreParams cp;
+        memset(&cp, 0, sizeof(cp));
+        cp.T = T; cp.k = 3; cp.D = D;
+        for (int j = 0; j < 3; ++j) cp.d[j] = vd[j];
+        for (int j = 0; j < 4; ++j) cp.r[j] = vr[j];
+        cp.P = vd[0] * vd[1];
+        cp.ibits = ibits;
+        cp.unique_only = opt.grouping == TT_GROUP_UNIQUE_ONLY;
+        cp.B = fwd_B;
+        for (int t = 0; t < T; ++t)
+            for (int j = 0; j < 3; ++j) cp.n[t][j] = (uint32_t)vn[t][j];
+        return cp;
+    }
+    // view with cores (merged first core from the workspace) and the matching gradient pointers
+    CoreParams view_cores(int64_t batch, GradPtrs* gp) const
+    {
+        CoreParams cp = view_params();
+        cp.B = batch;
+        if (gp) memset(gp, 0, sizeof(*gp));
+        for (int t = 0; t < T; ++t) {
+            const int off = merged ? 1 : 0;   // real core j+off is view core j (j >= 1)
+            cp.cores[t][0] = merged ? (const float*)at(lay.g12) + g12_off[t] : cores[t * k];
+            cp.cores[t][1] = cores[t * k + 1 + off];
+            cp.cores[t][2] = cores[t * k + 2 + off];
+            if (gp) {
+                gp->g[t][0] = merged ? (float*)at(lay.dg12) + g12_off[t] : grads[t * k];
+                gp->g[t][1] = grads[t * k + 1 + off];
+                gp->g[t][2] = grads[t * k + 2 + off];
+            }
+        }
+        return cp;
+    }
+    MergeParams merge_params() const
+    {
+        MergeParams mp;
+        memset(&mp, 0, sizeof(mp));
+        mp.T = T;
+        mp.d1 = d[0];
+        mp.d2 = d[1];
+        mp.r1 = r[1];
+        mp.r2 = r[2];
+        int b = 0;
+        for (int t = 0; t < T; ++t) {
+            mp.blk_base[t] = b;
+            b += (int)n[t][1];
+            mp.n1[t] = (uint32_t)n[t][0];
+            mp.n2[t] = (uint32_t)n[t][1];
+            mp.g1[t] = cores[t * k];
+            mp.g2[t] = cores[t * k + 1];
+            if (ws) {
+                mp.g12[t] = (float*)at(lay.g12) + g12_off[t];
+                mp.dg12[t] = (const float*)at(lay.dg12) + g12_off[t];
+            }
+            mp.dg1[t] = grads[t * k];
+            mp.dg2[t] = grads[t * k + 1];
+        }
+        mp.blk_base[T] = b;
+        return mp;
     }
     PlanParams plan_params(int64_t batch) const
     {
         PlanParams pp;
         memset(&pp, 0, sizeof(pp));
         pp.T = T;
-        pp.k = k;
+        pp.k = 3;
         pp.ibits = ibits;
         pp.col_digit = 1;
         pp.B = batch;
-        pp.MP = k3_plan_mp(core_params());
+        pp.MP = k3_plan_mp(view_params());
         pp.NB = kPoolBags;
         pp.ncols = ncols;
         pp.sched = opt.sched;
         for (int t = 0; t < T; ++t)
-            for (int j = 0; j < k; ++j) pp.n[t][j] = (uint32_t)n[t][j];
+            for (int j = 0; j < 3; ++j) pp.n[t][j] = (uint32_t)vn[t][j];
         for (int t = 0; t <= T; ++t) pp.col_base[t] = col_base[t];
         return pp;
     }
@@ -320,8 +392,9 @@ int tt_emb_create(int32_t num_tables, int32_t num_cores, const int64_t* n_factor
     tt_emb_default_options(&o);
     if (opt) {
         o = *opt;
-        for (int i = 0; i < 12; ++i)
+        for (int i = 0; i < 11; ++i)
             if (o.reserved[i] != 0) return TT_ERR_ARG;
+        if (o.force_generic != 0 && o.force_generic != 1) return TT_ERR_ARG;
         if (o.sched < TT_SCHED_STATIC || o.sched > TT_SCHED_STEAL_L2) return TT_ERR_ARG;
         if (o.grouping < TT_GROUP_PREFIX || o.grouping > TT_GROUP_UNIQUE_ONLY) return TT_ERR_ARG;
         if (o.chunk < 0 || o.grid < 0) return TT_ERR_ARG;
@@ -366,15 +439,44 @@ int tt_emb_create(int32_t num_tables, int32_t num_cores, const int64_t* n_factor
     h->key64 = h->ibits + h->tbits > 32;
 
     const CoreParams cp = h->core_params();
-    h->fast = k3_supported(cp);
+    // three-core view: the shapes themselves, or (n_1 n_2, n_3, n_4) with the merged first core
+    if (k == 3 || k == 4) {
+        const bool m4 = k == 4;
+        h->vd[0] = m4 ? d_factors[0] * d_factors[1] : d_factors[0];
+        h->vd[1] = d_factors[m4 ? 2 : 1];
+        h->vd[2] = d_factors[m4 ? 3 : 2];
+        h->vr[0] = 1;
+        h->vr[1] = ranks[m4 ? 2 : 1];
+        h->vr[2] = ranks[m4 ? 3 : 2];
+        h->vr[3] = 1;
+        bool ok = true;
+        int64_t g12 = 0;
+        for (int t = 0; t < num_tables; ++t) {
+            const int64_t a = m4 ? h->n[t][0] * h->n[t][1] : h->n[t][0];
+            if (a > 0xffffffffLL) ok = false;
+            h->vn[t][0] = a;
+            h->vn[t][1] = h->n[t][m4 ? 2 : 1];
+            h->vn[t][2] = h->n[t][m4 ? 3 : 2];
+            h->g12_off[t] = g12;
+            if (m4) g12 += a * h->vd[0] * h->vr[1];
+        }
+        h->g12_off[num_tables] = g12;
+        h->merged = m4;
+        h->fast = ok && !o.force_generic && k3_supported(h->view_params());
+        if (h->fast && m4) {
+            MergeParams mp = h->merge_params();
+            if (!merge_fits(mp) || g12 * 4 > (int64_t)2 << 30) h->fast = false;
+        }
+        if (!h->fast) h->merged = false;
+    }
     if (h->fast) {
         int64_t nc = 0;
         for (int t = 0; t < num_tables; ++t) {
             h->col_base[t] = (int)nc;
-            nc += h->n[t][1];
+            nc += h->vn[t][1];
         }
         h->col_base[num_tables] = (int)nc;
-        if (nc >= (1LL << 24)) h->fast = false;
+        if (nc >= (1LL << 24)) h->fast = h->merged = false;
         h->ncols = (int)nc;
     }
     if (generic_backward_smem_floats(cp) * 4 > 200 * 1024 ||
@@ -508,7 +610,7 @@ int tt_emb_forward(tt_emb_t h, const int64_t* indices, const int64_t* offsets, i
                        h->fast ? (int32_t*)h->at(y.uid_sorted) : nullptr, h->d_status, s, &nl);
     PlanBuffers pb;
     PlanParams pp;
-    CoreParams cp = h->core_params();
+    CoreParams cp = h->fast ? h->view_cores(batch, nullptr) : h->core_params();
     cp.B = batch;
     if (e == cudaSuccess && h->fast) {
         pp = h->plan_params(batch);
@@ -521,8 +623,9 @@ int tt_emb_forward(tt_emb_t h, const int64_t* indices, const int64_t* offsets, i
     if (e != cudaSuccess) return TT_ERR_CUDA;
     h->begin(TT_PHASE_FWD_FUSED, s);
     if (h->fast) {
+        if (h->merged) e = launch_merge(h->merge_params(), h->d_status, s, &nl);
         K3Args a = h->k3_args(&cp, &pp, &pb, offsets, L, false);
-        e = k3_forward(a, out, s, &nl);
+        if (e == cudaSuccess) e = k3_forward(a, out, s, &nl);
     } else {
         const int grid = h->opt.grid > 0 ? h->opt.grid : h->num_sms * 8;
         e = launch_forward_generic(cp, h->key64, h->at(y.uniq_keys), (const int32_t*)h->at(y.uniq_start),
@@ -565,11 +668,16 @@ int tt_emb_backward(tt_emb_t h, const float* grad_out, tt_stream_t stream)
         memset(&sb, 0, sizeof(sb));
         PlanBuffers pb = h->plan_buffers(sb);
         pb.sorted_groups = h->plan_sorted_groups;
+        GradPtrs vgp;
+        const CoreParams vcp = h->view_cores(h->fwd_B, &vgp);
         e = cudaMemsetAsync(&pb.hdr->col_head, 0, sizeof(int32_t), s);
+        if (e == cudaSuccess && h->merged)
+            e = cudaMemsetAsync(h->at(y.dg12), 0, sizeof(float) * (size_t)h->g12_off[h->T], s);
         if (e == cudaSuccess) {
-            K3Args a = h->k3_args(&cp, &pp, &pb, nullptr, h->fwd_L, true);
-            e = k3_backward(a, gp, grad_out, s, &nl);
+            K3Args a = h->k3_args(&vcp, &pp, &pb, nullptr, h->fwd_L, true);
+            e = k3_backward(a, vgp, grad_out, s, &nl);
         }
+        if (e == cudaSuccess && h->merged) e = launch_unmerge(h->merge_params(), h->d_status, s, &nl);
     } else {
         const int grid = h->opt.grid > 0 ? h->opt.grid : h->num_sms * 8;
         e = launch_backward_generic(cp, gp, h->key64, h->at(y.uniq_keys),

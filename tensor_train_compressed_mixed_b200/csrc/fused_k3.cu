@@ -28,7 +28,8 @@
     X(4, 4, 8, 32)           \
     X(4, 4, 8, 16)           \
     X(4, 4, 4, 32)           \
-    X(4, 4, 4, 16)
+    X(4, 4, 4, 16)           \
+    X(8, 4, 4, 32)
 
 // Optional phase timing (build with -DTT_PROFILE_PHASES): thread 0 of every
 // block adds the clock64 cycles it spent in each phase to a device array that
@@ -84,8 +85,10 @@ struct S3 {
     static constexpr int DBR = (R * N) / (kThreads * 4) >= 16 ? 8 : ((R * N) / (kThreads * 4) >= 4 ? 4 : 1);
     static constexpr int DBC = (R * N) / (kThreads * DBR);   // dB columns per thread
     static_assert(D2 == 4, "specialised path needs d_2 = 4");
-    static_assert(D1 == 4, "specialised path needs d_1 = 4");
+    static_assert(D1 == 4 || D1 == 8, "specialised path needs d_1 in {4, 8}");
+    static_assert(MF % D1 == 0 && MB % D1 == 0, "chunk rows in whole prefixes");
     static_assert(D3 % 4 == 0, "d_3 must be a multiple of 4");
+    static_assert(D <= 128, "one warp (4 columns per lane) covers a pooled row");
     static_assert(N >= 32 && N % 32 == 0, "swizzle needs N >= 32");
     static_assert(MF % 8 == 0 && (MF / 8) * (N / 8) == kThreads, "forward GEMM tiling");
     static_assert(DBC % 4 == 0, "dB columns in float4 chunks");
@@ -389,7 +392,7 @@ __device__ void fwd_pool(const CoreParams& cp, int ptask, int nP, const int32_t*
     if (!s_flag[0]) return;
     const int64_t B = cp.B, TD = (int64_t)cp.T * D;
     const int sub = lane / LB, sl = lane % LB, col = sl * 4;
-    const unsigned smask = LB == 32 ? kFull : (((1u << LB) - 1u) << (sub * LB));
+    const unsigned smask = LB >= 32 ? kFull : (((1u << (LB & 31)) - 1u) << (sub * LB));
     const int b_lo = jb * kNB, b_hi = (int)min64((int64_t)b_lo + kNB, B);
     const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
     // one sub-warp of LB lanes per bag; every lane owns 4 columns
@@ -1079,7 +1082,7 @@ int occ_bwd()
 int k3_blocks_per_sm(const CoreParams& cp, bool backward)
 {
 #define TT_OCC_CASE(Q1, Q2, Q3, QR) \
-    if (cp.d[2] == Q3 && cp.r[1] == QR) return backward ? occ_bwd<S3<Q1, Q2, Q3, QR>>() : occ_fwd<S3<Q1, Q2, Q3, QR>>();
+    if (cp.d[0] == Q1 && cp.d[2] == Q3 && cp.r[1] == QR) return backward ? occ_bwd<S3<Q1, Q2, Q3, QR>>() : occ_fwd<S3<Q1, Q2, Q3, QR>>();
     TT_K3_CASES_INNER(TT_OCC_CASE)
 #undef TT_OCC_CASE
     return 1;
@@ -1087,10 +1090,12 @@ int k3_blocks_per_sm(const CoreParams& cp, bool backward)
 
 bool k3_supported(const CoreParams& cp)
 {
-    if (cp.k != 3 || cp.d[0] != 4 || cp.d[1] != 4 || cp.r[1] != cp.r[2]) return false;
-    const int R = cp.r[1], d3 = cp.d[2];
-    return (R == 64 && d3 == 8) || (R == 32 && d3 == 8) || (R == 16 && d3 == 4) || (R == 32 && d3 == 4) ||
-           (R == 16 && d3 == 8);
+    if (cp.k != 3 || cp.d[1] != 4 || cp.r[1] != cp.r[2] || cp.d[0] * cp.d[1] * cp.d[2] > 128) return false;
+#define TT_SUP_CASE(Q1, Q2, Q3, QR) \
+    if (cp.d[0] == Q1 && cp.d[2] == Q3 && cp.r[1] == QR) return true;
+    TT_K3_CASES_INNER(TT_SUP_CASE)
+#undef TT_SUP_CASE
+    return false;
 }
 
 int k3_plan_mp(const CoreParams& cp)
@@ -1105,7 +1110,7 @@ cudaError_t k3_forward(const K3Args& a, float* out, cudaStream_t s, int* nl)
 {
     const CoreParams& cp = *a.cp;
 #define TT_FWD_CASE(Q1, Q2, Q3, QR) \
-    if (cp.d[2] == Q3 && cp.r[1] == QR) return fwd_dispatch<S3<Q1, Q2, Q3, QR>>(a, out, s, nl);
+    if (cp.d[0] == Q1 && cp.d[2] == Q3 && cp.r[1] == QR) return fwd_dispatch<S3<Q1, Q2, Q3, QR>>(a, out, s, nl);
     TT_K3_CASES(TT_FWD_CASE)
 #undef TT_FWD_CASE
     return cudaErrorInvalidValue;
@@ -1115,7 +1120,7 @@ cudaError_t k3_backward(const K3Args& a, const GradPtrs& gp, const float* grad_o
 {
     const CoreParams& cp = *a.cp;
 #define TT_BWD_CASE(Q1, Q2, Q3, QR) \
-    if (cp.d[2] == Q3 && cp.r[1] == QR) return bwd_dispatch<S3<Q1, Q2, Q3, QR>>(a, gp, grad_out, s, nl);
+    if (cp.d[0] == Q1 && cp.d[2] == Q3 && cp.r[1] == QR) return bwd_dispatch<S3<Q1, Q2, Q3, QR>>(a, gp, grad_out, s, nl);
     TT_K3_CASES(TT_BWD_CASE)
 #undef TT_BWD_CASE
     return cudaErrorInvalidValue;

@@ -214,6 +214,23 @@ struct K3Args {
     int grid;
     int32_t* status;
 };
+// Four-core tables run the three-core kernels on the merged first core
+// G_12 = G_1 . G_2 (merge.cu).
+struct MergeParams {
+    int32_t T, d1, d2, r1, r2, pad;
+    int32_t blk_base[kMaxT + 1];   // first block of each table (prefix sums of n_2)
+    uint32_t n1[kMaxT], n2[kMaxT];
+    const float* g1[kMaxT];
+    const float* g2[kMaxT];
+    float* g12[kMaxT];
+    const float* dg12[kMaxT];
+    float* dg1[kMaxT];
+    float* dg2[kMaxT];
+};
+bool merge_fits(const MergeParams& mp);
+cudaError_t launch_merge(const MergeParams& mp, int32_t* status, cudaStream_t s, int* nl);
+cudaError_t launch_unmerge(const MergeParams& mp, int32_t* status, cudaStream_t s, int* nl);
+
 constexpr int kPoolBags = 64;     // bags per pooling task of the specialised forward
 bool k3_supported(const CoreParams& cp);
 int k3_plan_mp(const CoreParams& cp);

@@ -68,6 +68,11 @@ def test_create_rejects_bad_options_on_host():
         abi.tt_emb_create([[2, 3]], [6], [2, 2], [1, 4, 1], o)
     assert e.value.code == abi.TT_ERR_ARG
     o = abi.tt_emb_default_options()
+    o.force_generic = 2
+    with pytest.raises(abi.TTEmbError) as e:
+        abi.tt_emb_create([[2, 3]], [6], [2, 2], [1, 4, 1], o)
+    assert e.value.code == abi.TT_ERR_ARG
+    o = abi.tt_emb_default_options()
     o.reserved[3] = 1
     with pytest.raises(abi.TTEmbError) as e:
         abi.tt_emb_create([[2, 3]], [6], [2, 2], [1, 4, 1], o)
