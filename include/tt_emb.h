@@ -223,10 +223,11 @@ typedef enum {
     TT_PHASE_FWD_SORT = 1,   /* radix sort of the keys */
     TT_PHASE_FWD_SEGMENT = 2,/* unique + prefix run-length segmentation */
     TT_PHASE_FWD_FUSED = 3,  /* fused gather + pooling (includes zeroing out) */
-    TT_PHASE_BWD_FUSED = 4,  /* fused backward kernels */
-    TT_PHASE_BWD_REDUCE = 5, /* segmented reductions and gradient write-out */
+    TT_PHASE_BWD_FUSED = 4,  /* fused backward kernel (prefix/suffix partial products, dG per digit) */
+    TT_PHASE_BWD_REDUCE = 5, /* gradient zero fill and the merged-core split of four-core tables */
     TT_PHASE_SGD = 6,        /* SGD update */
-    TT_EMB_NUM_PHASES = 7
+    TT_PHASE_BWD_ROWSUM = 7, /* upstream gradient summed per distinct row (reverse of pooling) */
+    TT_EMB_NUM_PHASES = 8
 } tt_phase;
 
 int tt_emb_enable_timing(tt_emb_t h, int enable);

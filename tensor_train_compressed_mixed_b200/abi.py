@@ -76,7 +76,8 @@ _SIGS = {
 
 NOALLOC_MAX_LOOKUPS = 262144
 
-PHASES = ("fwd_keys", "fwd_sort", "fwd_segment", "fwd_fused", "bwd_fused", "bwd_reduce", "sgd")
+PHASES = ("fwd_keys", "fwd_sort", "fwd_segment", "fwd_fused", "bwd_fused", "bwd_reduce", "sgd",
+          "bwd_rowsum")
 
 
 def lib() -> ctypes.CDLL:

@@ -661,7 +661,6 @@ int tt_emb_backward(tt_emb_t h, const float* grad_out, tt_stream_t stream)
         for (int j = 0; j < h->k; ++j) gp.g[t][j] = h->grads[t * h->k + j];
     const CoreParams cp = h->core_params();
     nl = 0;
-    h->begin(TT_PHASE_BWD_FUSED, s);
     if (h->fast) {
         PlanParams pp = h->plan_params(h->fwd_B);
         SortBuffers sb;
@@ -670,15 +669,20 @@ int tt_emb_backward(tt_emb_t h, const float* grad_out, tt_stream_t stream)
         pb.sorted_groups = h->plan_sorted_groups;
         GradPtrs vgp;
         const CoreParams vcp = h->view_cores(h->fwd_B, &vgp);
-        e = cudaMemsetAsync(&pb.hdr->col_head, 0, sizeof(int32_t), s);
+        K3Args a = h->k3_args(&vcp, &pp, &pb, nullptr, h->fwd_L, true);
+        h->begin(TT_PHASE_BWD_ROWSUM, s);
+        e = k3_rowsum(a, grad_out, s, &nl);
+        h->end(s);
+        e = e == cudaSuccess ? cudaMemsetAsync(&pb.hdr->col_head, 0, sizeof(int32_t), s) : e;
         if (e == cudaSuccess && h->merged)
             e = cudaMemsetAsync(h->at(y.dg12), 0, sizeof(float) * (size_t)h->g12_off[h->T], s);
-        if (e == cudaSuccess) {
-            K3Args a = h->k3_args(&vcp, &pp, &pb, nullptr, h->fwd_L, true);
-            e = k3_backward(a, vgp, grad_out, s, &nl);
-        }
+        h->begin(TT_PHASE_BWD_FUSED, s);
+        if (e == cudaSuccess) e = k3_backward(a, vgp, grad_out, s, &nl);
+        h->end(s);
+        h->begin(TT_PHASE_BWD_REDUCE, s);
         if (e == cudaSuccess && h->merged) e = launch_unmerge(h->merge_params(), h->d_status, s, &nl);
     } else {
+        h->begin(TT_PHASE_BWD_FUSED, s);
         const int grid = h->opt.grid > 0 ? h->opt.grid : h->num_sms * 8;
         e = launch_backward_generic(cp, gp, h->key64, h->at(y.uniq_keys),
                                     (const int32_t*)h->at(y.uniq_start), (const int32_t*)h->at(y.grp_start),

@@ -1027,15 +1027,22 @@ cudaError_t fwd_launch(const K3Args& a, float* out, cudaStream_t s, int* nl)
     return cudaGetLastError();
 }
 
-template <class S, typename K>
-cudaError_t bwd_launch(const K3Args& a, const GradPtrs& gp, const float* grad_out, cudaStream_t s, int* nl)
+template <int D>
+cudaError_t rowsum_launch(const K3Args& a, const float* grad_out, cudaStream_t s, int* nl)
 {
     const int64_t L = a.L;
     const int64_t nwarps = ceil_div(L, kHChunk);
-    k3_hzero<S::D><<<148, 256, 0, s>>>(a.uid_sorted, L, a.rowbuf, a.status);
-    k3_hsum<S::D><<<(unsigned)ceil_div(nwarps * 32, 256), 256, 0, s>>>(
+    k3_hzero<D><<<148, 256, 0, s>>>(a.uid_sorted, L, a.rowbuf, a.status);
+    k3_hsum<D><<<(unsigned)ceil_div(nwarps * 32, 256), 256, 0, s>>>(
         a.uid_sorted, a.bag_sorted, a.uniq_start, grad_out, L, a.cp->B, a.cp->T, a.rowbuf, a.status);
     *nl += 2;
+    return cudaGetLastError();
+}
+
+template <class S, typename K>
+cudaError_t bwd_launch(const K3Args& a, const GradPtrs& gp, const float* grad_out, cudaStream_t s, int* nl)
+{
+    (void)grad_out;
     const size_t smem = sizeof(float) * S::bwd_smem_floats();
     cudaError_t e = cudaFuncSetAttribute(k3_bwd_kernel<S, K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -1113,6 +1120,14 @@ cudaError_t k3_forward(const K3Args& a, float* out, cudaStream_t s, int* nl)
     if (cp.d[0] == Q1 && cp.d[2] == Q3 && cp.r[1] == QR) return fwd_dispatch<S3<Q1, Q2, Q3, QR>>(a, out, s, nl);
     TT_K3_CASES(TT_FWD_CASE)
 #undef TT_FWD_CASE
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t k3_rowsum(const K3Args& a, const float* grad_out, cudaStream_t s, int* nl)
+{
+    const int D = a.cp->D;
+    if (D == 128) return rowsum_launch<128>(a, grad_out, s, nl);
+    if (D == 64) return rowsum_launch<64>(a, grad_out, s, nl);
     return cudaErrorInvalidValue;
 }
 

@@ -236,6 +236,8 @@ bool k3_supported(const CoreParams& cp);
 int k3_plan_mp(const CoreParams& cp);
 int k3_blocks_per_sm(const CoreParams& cp, bool backward);
 cudaError_t k3_forward(const K3Args& a, float* out, cudaStream_t s, int* nl);
+// upstream sums per distinct row (must run before k3_backward)
+cudaError_t k3_rowsum(const K3Args& a, const float* grad_out, cudaStream_t s, int* nl);
 cudaError_t k3_backward(const K3Args& a, const GradPtrs& gp, const float* grad_out, cudaStream_t s,
                         int* nl);
 
