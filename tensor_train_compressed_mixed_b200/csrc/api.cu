@@ -15,7 +15,7 @@ struct Layout {
         uniq_start, grp_start, bag_sorted;
     // specialised path only (zero when unused)
     size_t uid_at_pos, uid_sorted, rowbuf, pkeys[2], pvals[2], col_count, col_start, chunk_base,
-        hdr, chunks, tasks, g12, dg12;
+        hdr, chunks, tasks, g12, dg12, g3t;
     int64_t chunk_cap, task_cap;
     size_t total;
 };
@@ -25,6 +25,7 @@ struct FastDims {
     bool on;
     int D, ncols, MP, T;
     int64_t g12_floats;   // merged first cores of four-core tables (0 otherwise)
+    int64_t g3t_floats;   // transposed copies of the last cores
 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -74,6 +75,7 @@ Layout make_layout(int key_bytes, int64_t L, int64_t B, const FastDims& f)
             y.g12 = take((size_t)f.g12_floats * 4);
             y.dg12 = take((size_t)f.g12_floats * 4);
         }
+        y.g3t = take((size_t)f.g3t_floats * 4);
     }
     y.total = p;
     return y;
@@ -119,6 +121,7 @@ struct tt_emb_handle {
     int64_t vn[kMaxT][3] = {};      // three-core view: factors (n_1 n_2, n_3, n_4) when merged
     int32_t vd[3] = {}, vr[4] = {};
     int64_t g12_off[kMaxT + 1] = {};  // merged-core offsets (floats) in the workspace
+    int64_t g3t_off[kMaxT + 1] = {};  // transposed last-core offsets (floats) in the workspace
     // timing and launch accounting
     bool timing = false;
     double phase_ms[TT_EMB_NUM_PHASES] = {};
@@ -180,6 +183,7 @@ struct tt_emb_handle {
         f.MP = fast ? k3_plan_mp(view_params()) : 1;
         f.T = T;
         f.g12_floats = merged ? g12_off[T] : 0;
+        f.g3t_floats = g3t_off[T];
         return f;
     }
     // three-core view of the shapes (identity for three-core tables), without core pointers
@@ -209,6 +213,7 @@ struct tt_emb_handle {
             cp.cores[t][0] = merged ? (const float*)at(lay.g12) + g12_off[t] : cores[t * k];
             cp.cores[t][1] = cores[t * k + 1 + off];
             cp.cores[t][2] = cores[t * k + 2 + off];
+            cp.last_t[t] = (const float*)at(lay.g3t) + g3t_off[t];
             if (gp) {
                 gp->g[t][0] = merged ? (float*)at(lay.dg12) + g12_off[t] : grads[t * k];
                 gp->g[t][1] = grads[t * k + 1 + off];
@@ -461,6 +466,12 @@ int tt_emb_create(int32_t num_tables, int32_t num_cores, const int64_t* n_factor
             if (m4) g12 += a * h->vd[0] * h->vr[1];
         }
         h->g12_off[num_tables] = g12;
+        int64_t g3t = 0;
+        for (int t = 0; t < num_tables; ++t) {
+            h->g3t_off[t] = g3t;
+            g3t += h->vn[t][2] * h->vr[2] * h->vd[2];
+        }
+        h->g3t_off[num_tables] = g3t;
         h->merged = m4;
         h->fast = ok && !o.force_generic && k3_supported(h->view_params());
         if (h->fast && m4) {
@@ -624,6 +635,11 @@ int tt_emb_forward(tt_emb_t h, const int64_t* indices, const int64_t* offsets, i
     h->begin(TT_PHASE_FWD_FUSED, s);
     if (h->fast) {
         if (h->merged) e = launch_merge(h->merge_params(), h->d_status, s, &nl);
+        if (e == cudaSuccess) {
+            float* dst[kMaxT];
+            for (int t = 0; t < h->T; ++t) dst[t] = (float*)h->at(y.g3t) + h->g3t_off[t];
+            e = k3_transpose_last(cp, dst, s, &nl);
+        }
         K3Args a = h->k3_args(&cp, &pp, &pb, offsets, L, false);
         if (e == cudaSuccess) e = k3_forward(a, out, s, &nl);
     } else {

@@ -21,6 +21,8 @@
 //     and dB += A^T dC.  dB is reduced on chip over the whole column group and
 //     written once; dA and the last-slice gradients are reduced into the
 //     small, L2-resident gradient arrays with 16-byte vector reductions.
+#include <string.h>
+
 #include "tt_common.cuh"
 
 #define TT_K3_CASES_INNER(X) \
@@ -315,12 +317,11 @@ __device__ __forceinline__ void fwd_issue_batch(const CoreParams& cp, int mb, in
         M.bi3[bb][tid] = (int)(key_row(uniq_keys[u], cp.ibits) % n3);
     }
     __syncthreads();
-    const float* G3 = cp.cores[t][2];
+    const float* G3t = cp.last_t[t];   // [n3][R][D3]: one row's slice is contiguous
     float* Ss = sm.Ss + (size_t)bb * S::NUF * S::SU;
     for (int q = tid; q < nb * R * (D3 / 4); q += kThreads) {
         const int uu = q / (R * (D3 / 4)), rem = q % (R * (D3 / 4));
-        const int rho = rem / (D3 / 4), c4 = rem % (D3 / 4);
-        cp_async16(&Ss[uu * S::SU + rho * D3 + c4 * 4], G3 + ((int64_t)rho * n3 + M.bi3[bb][uu]) * D3 + c4 * 4);
+        cp_async16(&Ss[uu * S::SU + rem * 4], G3t + (int64_t)M.bi3[bb][uu] * (R * D3) + rem * 4);
     }
     cp_async_commit();
 }
@@ -692,11 +693,11 @@ __device__ __forceinline__ void bwd_issue_batch(const CoreParams& cp, int t, int
         const int uu = q / (P * D3 / 4), c4 = q % (P * D3 / 4);
         cp_async16(&H[uu * P * D3 + c4 * 4], rowbuf + (int64_t)M.bu[bb][uu] * S::D + c4 * 4);
     }
-    const float* G3 = cp.cores[t][2];
+    const float* G3t = cp.last_t[t];   // [n3][R][D3]
     for (int q = tid; q < nb * R * (D3 / 4); q += kThreads) {
         const int uu = q / (R * (D3 / 4)), rem = q % (R * (D3 / 4));
         const int rho = rem / (D3 / 4), c4 = rem % (D3 / 4);
-        cp_async16(&Sb[(uu * R + rho) * SR + c4 * 4], G3 + ((int64_t)rho * n3 + M.bi3[bb][uu]) * D3 + c4 * 4);
+        cp_async16(&Sb[(uu * R + rho) * SR + c4 * 4], G3t + (int64_t)M.bi3[bb][uu] * (R * D3) + rem * 4);
     }
     cp_async_commit();
 }
@@ -1011,6 +1012,33 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
 }
 
 // ---------------------------------------------------------------------------
+// last core [R][n3][D3] -> [n3][R][D3]; one thread per (table, i3, rho) row of D3 floats
+// ---------------------------------------------------------------------------
+struct TransposeJob {
+    int32_t T, R, D3, pad;
+    int64_t row_base[kMaxT + 1];   // prefix sums of n3 * R
+    uint32_t n3[kMaxT];
+    const float* src[kMaxT];
+    float* dst[kMaxT];
+};
+
+__global__ void __launch_bounds__(256) k3_transpose_last_kernel(TransposeJob tj, const int32_t* status)
+{
+    if (status && has_error(status)) return;
+    const int64_t total = tj.row_base[tj.T];
+    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < total;
+         q += (int64_t)gridDim.x * blockDim.x) {
+        int t = 0;
+        while (t + 1 < tj.T && tj.row_base[t + 1] <= q) ++t;
+        const int64_t rq = q - tj.row_base[t];
+        const int64_t i3 = rq / tj.R, rho = rq % tj.R;
+        const float4* src = reinterpret_cast<const float4*>(tj.src[t] + (rho * tj.n3[t] + i3) * tj.D3);
+        float4* dst = reinterpret_cast<float4*>(tj.dst[t] + (i3 * tj.R + rho) * tj.D3);
+        for (int c = 0; c < tj.D3 / 4; ++c) dst[c] = __ldg(src + c);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // host launchers
 // ---------------------------------------------------------------------------
 template <class S, typename K>
@@ -1121,6 +1149,29 @@ cudaError_t k3_forward(const K3Args& a, float* out, cudaStream_t s, int* nl)
     TT_K3_CASES(TT_FWD_CASE)
 #undef TT_FWD_CASE
     return cudaErrorInvalidValue;
+}
+
+cudaError_t k3_transpose_last(const CoreParams& cp, float* const* dst, cudaStream_t s, int* nl)
+{
+    TransposeJob tj;
+    memset(&tj, 0, sizeof(tj));
+    tj.T = cp.T;
+    tj.R = cp.r[2];
+    tj.D3 = cp.d[2];
+    int64_t b = 0;
+    for (int t = 0; t < cp.T; ++t) {
+        tj.row_base[t] = b;
+        b += (int64_t)cp.n[t][2] * tj.R;
+        tj.n3[t] = cp.n[t][2];
+        tj.src[t] = cp.cores[t][2];
+        tj.dst[t] = dst[t];
+    }
+    tj.row_base[cp.T] = b;
+    if (b == 0) return cudaSuccess;
+    const int grid = (int)min64(ceil_div(b, 256), 148 * 16);
+    k3_transpose_last_kernel<<<grid, 256, 0, s>>>(tj, nullptr);
+    *nl += 1;
+    return cudaGetLastError();
 }
 
 cudaError_t k3_rowsum(const K3Args& a, const float* grad_out, cudaStream_t s, int* nl)

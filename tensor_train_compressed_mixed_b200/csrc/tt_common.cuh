@@ -60,6 +60,9 @@ struct CoreParams {
     int64_t B;
     uint32_t n[kMaxT][kMaxK];
     const float* cores[kMaxT][kMaxK];
+    // specialised path: the last core re-laid out as [n_k][r_{k-1}][d_k], so that one
+    // row's last slice is a contiguous block (built by k3_transpose_last each forward)
+    const float* last_t[kMaxT];
 };
 
 struct GradPtrs {
@@ -236,6 +239,8 @@ bool k3_supported(const CoreParams& cp);
 int k3_plan_mp(const CoreParams& cp);
 int k3_blocks_per_sm(const CoreParams& cp, bool backward);
 cudaError_t k3_forward(const K3Args& a, float* out, cudaStream_t s, int* nl);
+// last core [r][n_k][d_k] -> [n_k][r][d_k] into cp.last_t (before k3_forward / k3_backward)
+cudaError_t k3_transpose_last(const CoreParams& cp, float* const* dst, cudaStream_t s, int* nl);
 // upstream sums per distinct row (must run before k3_backward)
 cudaError_t k3_rowsum(const K3Args& a, const float* grad_out, cudaStream_t s, int* nl);
 cudaError_t k3_backward(const K3Args& a, const GradPtrs& gp, const float* grad_out, cudaStream_t s,
