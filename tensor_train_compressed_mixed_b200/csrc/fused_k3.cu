@@ -59,7 +59,8 @@ __device__ unsigned long long g_tt_phase_cycles[32];
 namespace tt {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kFwdThreads = 512;  // forward: 16 warps, at most 128 registers per thread
+constexpr int kBwdThreads = 256;  // backward: 8 warps, up to 255 registers per thread
 constexpr int kNB = kPoolBags;    // bags per pooling task
 constexpr int kHChunk = 256;      // sorted lookups per upstream-sum warp
 constexpr int kSpinLimit = 1 << 22;
@@ -70,11 +71,11 @@ struct S3 {
     static constexpr int N = D2 * R;          // columns of B and of C_all
     static constexpr int P = D1 * D2;         // rows of C_p
     static constexpr int D = P * D3;          // embedding width
-    // forward: GEMM of MF x N per chunk, 8x8 outputs per thread
+    // forward: GEMM of MF x N per chunk, 4 x 8 outputs per thread
     static constexpr int MF = 16384 / N;
     static constexpr int MPF = MF / D1;       // prefixes per forward chunk
-    static constexpr int TPU = D1 * (D3 / 4); // threads per distinct row in the suffix step
-    static constexpr int NUF = kThreads / TPU;
+    static constexpr int TPU = D1 * 2 * (D3 / 4); // threads per distinct row in the suffix step
+    static constexpr int NUF = kFwdThreads / TPU;
     static constexpr int SU = R * D3 + 8;     // padded stride of one staged last slice
     static constexpr size_t FWD_FIXED = (size_t)R * N + (size_t)MF * R + (size_t)MF * N;
     static constexpr int FBUF = (FWD_FIXED + 2 * (size_t)NUF * SU) * 4 <= 220 * 1024 ? 2 : 1;
@@ -82,19 +83,20 @@ struct S3 {
     static constexpr int MB = 2048 / R;
     static constexpr int MPB = MB / D1;
     static constexpr int TPUB = (R / 4) * (D3 / 4);   // dS tiles per distinct row
-    static constexpr int NUB = kThreads / TPUB;      // distinct rows per backward batch
+    static constexpr int NUB = kBwdThreads / TPUB;      // distinct rows per backward batch
     static constexpr int SR = D3 + 4;                // padded row of a staged last slice (backward)
-    static constexpr int DBR = (R * N) / (kThreads * 4) >= 16 ? 8 : ((R * N) / (kThreads * 4) >= 4 ? 4 : 1);
-    static constexpr int DBC = (R * N) / (kThreads * DBR);   // dB columns per thread
+    static constexpr int DBR = (R * N) / (kBwdThreads * 4) >= 16 ? 8 : ((R * N) / (kBwdThreads * 4) >= 4 ? 4 : 1);
+    static constexpr int DBC = (R * N) / (kBwdThreads * DBR);   // dB columns per thread
     static_assert(D2 == 4, "specialised path needs d_2 = 4");
     static_assert(D1 == 4 || D1 == 8, "specialised path needs d_1 in {4, 8}");
     static_assert(MF % D1 == 0 && MB % D1 == 0, "chunk rows in whole prefixes");
     static_assert(D3 % 4 == 0, "d_3 must be a multiple of 4");
     static_assert(D <= 128, "one warp (4 columns per lane) covers a pooled row");
     static_assert(N >= 32 && N % 32 == 0, "swizzle needs N >= 32");
-    static_assert(MF % 8 == 0 && (MF / 8) * (N / 8) == kThreads, "forward GEMM tiling");
+    static_assert(MF % 4 == 0 && (MF / 4) * (N / 8) == kFwdThreads, "forward GEMM tiling (4 x 8 per thread)");
+    static_assert((2048 / R / 4) * (N / 8) == kBwdThreads, "backward GEMM tiling (4 x 8 per thread)");
     static_assert(DBC % 4 == 0, "dB columns in float4 chunks");
-    static_assert(NUB >= 1 && NUB * TPUB == kThreads, "backward batch tiling");
+    static_assert(NUB >= 1 && NUB * TPUB == kBwdThreads, "backward batch tiling");
 
     static constexpr size_t fwd_smem_floats() { return FWD_FIXED + (size_t)FBUF * NUF * SU; }
     static constexpr size_t bwd_smem_floats()
@@ -235,7 +237,7 @@ __device__ __forceinline__ void fwd_issue_ab(const CoreParams& cp, int mb, const
     if (t != cur_t || i2 != cur_i2) {
         const float* G2 = cp.cores[t][1] + (int64_t)i2 * N;
         const int64_t rs = (int64_t)cp.n[t][1] * N;
-        for (int q = tid; q < R * N / 4; q += kThreads) {
+        for (int q = tid; q < R * N / 4; q += kFwdThreads) {
             const int rho = q / (N / 4), c4 = q % (N / 4);
             cp_async16(&sm.Bs[swz_b<N>(rho, c4 * 4)], G2 + rho * rs + c4 * 4);
         }
@@ -243,7 +245,7 @@ __device__ __forceinline__ void fwd_issue_ab(const CoreParams& cp, int mb, const
         cur_i2 = i2;
     }
     const float* G1 = cp.cores[t][0];
-    for (int q = tid; q < MF * (R / 4); q += kThreads) {
+    for (int q = tid; q < MF * (R / 4); q += kFwdThreads) {
         const int m = q / (R / 4), c4 = q % (R / 4);
         const int j = m / D1, a1 = m % D1;
         float* dst = &sm.As[swz_a<R>(m, c4 * 4)];
@@ -253,33 +255,33 @@ __device__ __forceinline__ void fwd_issue_ab(const CoreParams& cp, int mb, const
     cp_async_commit();
 }
 
-// C_all = A . B into Cn; thread tile rows {4tm+i, MF/2+4tm+i} x cols {4tn+j, N/2+4tn+j}
+// C_all = A . B into Cn; thread tile rows {4tm+i} x cols {4tn+j, N/2+4tn+j}
 template <class S>
 __device__ __forceinline__ void fwd_gemm(const FwdSmem<S>& sm)
 {
-    constexpr int R = S::R, N = S::N, MF = S::MF;
+    constexpr int R = S::R, N = S::N;
     constexpr int TN = N / 8;
     const int tn = threadIdx.x % TN, tm = threadIdx.x / TN;
-    int rows[8];
+    int rows[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) rows[i] = (i < 4) ? tm * 4 + i : MF / 2 + tm * 4 + (i - 4);
-    float acc[8][8];
+    for (int i = 0; i < 4; ++i) rows[i] = tm * 4 + i;
+    float acc[4][8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
 #pragma unroll 1
     for (int rho = 0; rho < R; rho += 4) {
-        float4 a[8];
+        float4 a[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) a[i] = *reinterpret_cast<const float4*>(&sm.As[swz_a<R>(rows[i], rho)]);
+        for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(&sm.As[swz_a<R>(rows[i], rho)]);
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const float4 b0 = *reinterpret_cast<const float4*>(&sm.Bs[swz_b<N>(rho + r, tn * 4)]);
             const float4 b1 = *reinterpret_cast<const float4*>(&sm.Bs[swz_b<N>(rho + r, N / 2 + tn * 4)]);
             const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < 4; ++i) {
                 const float av = f4get(a[i], r);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av, b[j], acc[i][j]);
@@ -287,7 +289,7 @@ __device__ __forceinline__ void fwd_gemm(const FwdSmem<S>& sm)
         }
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 4; ++i) {
         *reinterpret_cast<float4*>(&sm.Cn[swz_m<N>(rows[i], tn * 4)]) =
             make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
         *reinterpret_cast<float4*>(&sm.Cn[swz_m<N>(rows[i], N / 2 + tn * 4)]) =
@@ -319,14 +321,14 @@ __device__ __forceinline__ void fwd_issue_batch(const CoreParams& cp, int mb, in
     __syncthreads();
     const float* G3t = cp.last_t[t];   // [n3][R][D3]: one row's slice is contiguous
     float* Ss = sm.Ss + (size_t)bb * S::NUF * S::SU;
-    for (int q = tid; q < nb * R * (D3 / 4); q += kThreads) {
+    for (int q = tid; q < nb * R * (D3 / 4); q += kFwdThreads) {
         const int uu = q / (R * (D3 / 4)), rem = q % (R * (D3 / 4));
         cp_async16(&Ss[uu * S::SU + rem * 4], G3t + (int64_t)M.bi3[bb][uu] * (R * D3) + rem * 4);
     }
     cp_async_commit();
 }
 
-// E_u = C_p . S_u for the batch in buffer bb; tile: rows (a1, a2 = 0..3) x 4 columns of a3
+// E_u = C_p . S_u for the batch in buffer bb; tile: rows (a1, a2 = 2h, 2h+1) x 4 columns of a3
 template <class S>
 __device__ __forceinline__ void fwd_batch_compute(int nb, int bb, const FwdMeta<S>& M, const FwdSmem<S>& sm,
                                                   float* __restrict__ rowbuf)
@@ -335,33 +337,34 @@ __device__ __forceinline__ void fwd_batch_compute(int nb, int bb, const FwdMeta<
     const int tid = threadIdx.x;
     const int uu = tid / S::TPU;
     if (uu >= nb) return;
-    const int a1 = (tid % S::TPU) / (D3 / 4), cg = tid % (D3 / 4);
+    const int rem = tid % S::TPU;
+    const int a1 = rem / (2 * (D3 / 4)), h = (rem / (D3 / 4)) % 2, cg = rem % (D3 / 4);
     const int m = M.bp[bb][uu] * D1 + a1;
     const float* srow = sm.Ss + (size_t)bb * S::NUF * S::SU + uu * S::SU + cg * 4;
-    float4 e[4];
+    float4 e[2];
 #pragma unroll
-    for (int a2 = 0; a2 < 4; ++a2) e[a2] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < 2; ++q) e[q] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 2
     for (int rho = 0; rho < R; rho += 4) {
-        float4 c[4], s4[4];
+        float4 c[2], s4[4];
 #pragma unroll
-        for (int a2 = 0; a2 < 4; ++a2) c[a2] = *reinterpret_cast<const float4*>(&sm.Cn[swz_m<N>(m, a2 * R + rho)]);
+        for (int q = 0; q < 2; ++q) c[q] = *reinterpret_cast<const float4*>(&sm.Cn[swz_m<N>(m, (2 * h + q) * R + rho)]);
 #pragma unroll
         for (int r = 0; r < 4; ++r) s4[r] = *reinterpret_cast<const float4*>(srow + (rho + r) * D3);
 #pragma unroll
-        for (int a2 = 0; a2 < 4; ++a2)
+        for (int q = 0; q < 2; ++q)
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
-                const float cv = f4get(c[a2], r);
-                e[a2].x = fmaf(cv, s4[r].x, e[a2].x);
-                e[a2].y = fmaf(cv, s4[r].y, e[a2].y);
-                e[a2].z = fmaf(cv, s4[r].z, e[a2].z);
-                e[a2].w = fmaf(cv, s4[r].w, e[a2].w);
+                const float cv = f4get(c[q], r);
+                e[q].x = fmaf(cv, s4[r].x, e[q].x);
+                e[q].y = fmaf(cv, s4[r].y, e[q].y);
+                e[q].z = fmaf(cv, s4[r].z, e[q].z);
+                e[q].w = fmaf(cv, s4[r].w, e[q].w);
             }
     }
     float* dst = rowbuf + (int64_t)M.bu[bb][uu] * S::D + cg * 4;
 #pragma unroll
-    for (int a2 = 0; a2 < 4; ++a2) *reinterpret_cast<float4*>(dst + (a1 * D2 + a2) * D3) = e[a2];
+    for (int q = 0; q < 2; ++q) *reinterpret_cast<float4*>(dst + (a1 * D2 + 2 * h + q) * D3) = e[q];
 }
 
 template <class S>
@@ -397,23 +400,23 @@ __device__ void fwd_pool(const CoreParams& cp, int ptask, int nP, const int32_t*
     const int b_lo = jb * kNB, b_hi = (int)min64((int64_t)b_lo + kNB, B);
     const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
     // one sub-warp of LB lanes per bag; every lane owns 4 columns
-    for (int b = b_lo + wid * BPW + sub; b < b_hi; b += (kThreads / 32) * BPW) {
+    for (int b = b_lo + wid * BPW + sub; b < b_hi; b += (kFwdThreads / 32) * BPW) {
         const int64_t g = (int64_t)t * B + b;
         const int64_t l0 = offsets[g], l1 = offsets[g + 1];
         float4 acc = zero;
         for (int64_t base = l0; base < l1; base += LB) {
             const int n = (int)min64(LB, l1 - base);
             const int myu = sl < n ? uid_at_pos[base + sl] : 0;   // row ids of up to LB lookups
-            for (int k = 0; k < n; k += 16) {
-                float4 v[16];
+            for (int k = 0; k < n; k += 8) {
+                float4 v[8];
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
+                for (int q = 0; q < 8; ++q) {
                     const int u = __shfl_sync(smask, myu, (k + q) & (LB - 1), LB);
                     v[q] = (k + q < n) ? __ldcg(reinterpret_cast<const float4*>(rowbuf + (int64_t)u * D + col))
                                        : zero;
                 }
 #pragma unroll
-                for (int q = 0; q < 16; ++q)   // lookup order: the sum is the same for every schedule
+                for (int q = 0; q < 8; ++q)   // lookup order: the sum is the same for every schedule
                     if (k + q < n) acc = f4add(acc, v[q]);
             }
         }
@@ -429,7 +432,7 @@ __device__ void fwd_pool(const CoreParams& cp, int ptask, int nP, const int32_t*
 // chunk's distinct rows are contracted batch by batch (double-buffered last
 // slices when shared memory allows).
 template <class S, typename K>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
 k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
               const int32_t* __restrict__ grp_start, const int32_t* __restrict__ uid_at_pos,
               const int64_t* __restrict__ offsets, const int32_t* __restrict__ sorted_groups,
@@ -471,9 +474,13 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
             fwd_meta<S, K>(cp, tv, mb, uniq_keys, grp_start, sorted_groups, chunks, M);
             fwd_issue_ab<S>(cp, mb, M, sm, cur_t, cur_i2);
         }
+        // the first batch of last slices is in flight during the GEMM
+        const int total = M.ucum[mb][S::MPF];
+        if (total > 0) fwd_issue_batch<S, K>(cp, mb, 0, 0, uniq_keys, M, sm);
         if (tid == 0) M.task[1] = next_task(sched, &hdr->queue_head, iter);   // result used after the GEMM
         ++iter;
-        cp_async_wait_all();
+        if (total > 0) cp_async_wait<1>();   // A/B landed; the batch may still be in flight
+        else cp_async_wait_all();
         __syncthreads();
         TT_PH(0);
         fwd_gemm<S>(sm);
@@ -485,14 +492,15 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
             fwd_meta<S, K>(cp, tasks[qn], mb ^ 1, uniq_keys, grp_start, sorted_groups, chunks, M);
             fwd_issue_ab<S>(cp, mb ^ 1, M, sm, cur_t, cur_i2);
         }
-        // distinct rows of this chunk, in batches of NUF
-        const int total = M.ucum[mb][S::MPF];
+        // distinct rows of this chunk, in batches of NUF (commit groups in flight: the batch,
+        // then possibly the next chunk's A/B, then possibly the next batch)
         if (S::FBUF == 2) {
-            if (total > 0) fwd_issue_batch<S, K>(cp, mb, 0, 0, uniq_keys, M, sm);
             for (int k0 = 0, b = 0; k0 < total; k0 += S::NUF, b ^= 1) {
                 const bool more = k0 + S::NUF < total;
                 if (more) {
                     fwd_issue_batch<S, K>(cp, mb, k0 + S::NUF, b ^ 1, uniq_keys, M, sm);
+                    cp_async_wait<1>();
+                } else if (k0 == 0 && next_chunk) {
                     cp_async_wait<1>();
                 } else {
                     cp_async_wait_all();
@@ -505,8 +513,9 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
             }
         } else {
             for (int k0 = 0; k0 < total; k0 += S::NUF) {
-                fwd_issue_batch<S, K>(cp, mb, k0, 0, uniq_keys, M, sm);
-                cp_async_wait_all();
+                if (k0 > 0) fwd_issue_batch<S, K>(cp, mb, k0, 0, uniq_keys, M, sm);
+                if (k0 == 0 && next_chunk) cp_async_wait<1>();
+                else cp_async_wait_all();
                 __syncthreads();
                 TT_PH(2);
                 fwd_batch_compute<S>(min(S::NUF, total - k0), 0, M, sm, rowbuf);
@@ -656,7 +665,7 @@ __device__ __forceinline__ void bwd_issue_a(const CoreParams& cp, int t, int mb,
     constexpr int R = S::R, MB = S::MB, D1 = S::D1;
     const float* G1 = cp.cores[t][0];
     const int cnt = M.cnt[mb];
-    for (int q = threadIdx.x; q < MB * (R / 4); q += kThreads) {
+    for (int q = threadIdx.x; q < MB * (R / 4); q += kBwdThreads) {
         const int m = q / (R / 4), c4 = q % (R / 4);
         const int j = m / D1, a1 = m % D1;
         float* dst = &As[swz_a<R>(m, c4 * 4)];
@@ -689,12 +698,12 @@ __device__ __forceinline__ void bwd_issue_batch(const CoreParams& cp, int t, int
     __syncthreads();
     float* H = Hs + (size_t)bb * S::NUB * P * D3;
     float* Sb = Ss + (size_t)bb * S::NUB * R * SR;
-    for (int q = tid; q < nb * (P * D3 / 4); q += kThreads) {
+    for (int q = tid; q < nb * (P * D3 / 4); q += kBwdThreads) {
         const int uu = q / (P * D3 / 4), c4 = q % (P * D3 / 4);
         cp_async16(&H[uu * P * D3 + c4 * 4], rowbuf + (int64_t)M.bu[bb][uu] * S::D + c4 * 4);
     }
     const float* G3t = cp.last_t[t];   // [n3][R][D3]
-    for (int q = tid; q < nb * R * (D3 / 4); q += kThreads) {
+    for (int q = tid; q < nb * R * (D3 / 4); q += kBwdThreads) {
         const int uu = q / (R * (D3 / 4)), rem = q % (R * (D3 / 4));
         const int rho = rem / (D3 / 4), c4 = rem % (D3 / 4);
         cp_async16(&Sb[(uu * R + rho) * SR + c4 * 4], G3t + (int64_t)M.bi3[bb][uu] * (R * D3) + rem * 4);
@@ -703,7 +712,7 @@ __device__ __forceinline__ void bwd_issue_batch(const CoreParams& cp, int t, int
 }
 
 template <class S, typename K>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
 k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ uniq_keys,
               const int32_t* __restrict__ grp_start, const int32_t* __restrict__ sorted_groups,
               const int32_t* __restrict__ col_count, const int32_t* __restrict__ col_start,
@@ -746,7 +755,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
         {
             const float* G2 = cp.cores[t][1] + (int64_t)i2 * N;
             const int64_t rs = (int64_t)n2 * N;
-            for (int q = tid; q < R * N / 4; q += kThreads) {
+            for (int q = tid; q < R * N / 4; q += kBwdThreads) {
                 const int rho = q / (N / 4), c4 = q % (N / 4);
                 cp_async16(&Bs[swz_b<N>(rho, c4 * 4)], G2 + rho * rs + c4 * 4);
             }
@@ -768,9 +777,13 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
         for (int j0 = 0; j0 < ccount; j0 += MPB, mb ^= 1) {
             const int cnt = M.cnt[mb];
             const float* Ab = As + mb * MB * R;
-            for (int q = tid; q < MB * N / 4; q += kThreads)
+            // the first batch of distinct rows is in flight during the C GEMM
+            const int total = M.ucum[mb][MPB];
+            if (total > 0) bwd_issue_batch<S, K>(cp, t, mb, 0, 0, uniq_keys, rowbuf, M, Hs, Ss);
+            for (int q = tid; q < MB * N / 4; q += kBwdThreads)
                 reinterpret_cast<float4*>(dCn)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-            cp_async_wait_all();
+            if (total > 0) cp_async_wait<1>();   // B and A landed; the batch may still be in flight
+            else cp_async_wait_all();
             __syncthreads();
             TT_PH(9);
 
@@ -821,12 +834,13 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             }
 
             // distinct rows in double-buffered batches: dS_u -> dG_3 (vector reductions), dC_p += H_u S_u^T
-            const int total = M.ucum[mb][MPB];
-            if (total > 0) bwd_issue_batch<S, K>(cp, t, mb, 0, 0, uniq_keys, rowbuf, M, Hs, Ss);
+            // (commit groups in flight: the batch, then possibly the next chunk's A, then possibly the next batch)
             for (int k0 = 0, bb = 0; k0 < total; k0 += NUB, bb ^= 1) {
                 const int nb = min(NUB, total - k0);
                 if (k0 + NUB < total) {
                     bwd_issue_batch<S, K>(cp, t, mb, k0 + NUB, bb ^ 1, uniq_keys, rowbuf, M, Hs, Ss);
+                    cp_async_wait<1>();
+                } else if (k0 == 0 && more) {
                     cp_async_wait<1>();
                 } else {
                     cp_async_wait_all();
@@ -869,7 +883,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                 // adds the batch's rows of its prefix in order (plain read-modify-write, deterministic)
                 {
                     constexpr int TPD = D1 * (R / 4);
-                    for (int w = tid; w < cnt * TPD; w += kThreads) {
+                    for (int w = tid; w < cnt * TPD; w += kBwdThreads) {
                         const int p = w / TPD, rem = w % TPD;
                         const int a1 = rem / (R / 4), rc = rem % (R / 4);
                         const int ulo = max(M.ucum[mb][p], k0) - k0, uhi = min(M.ucum[mb][p + 1], k0 + nb) - k0;
@@ -1048,7 +1062,7 @@ cudaError_t fwd_launch(const K3Args& a, float* out, cudaStream_t s, int* nl)
     cudaError_t e = cudaFuncSetAttribute(k3_fwd_kernel<S, K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const PlanBuffers& pb = *a.pb;
-    k3_fwd_kernel<S, K><<<a.grid, kThreads, smem, s>>>(
+    k3_fwd_kernel<S, K><<<a.grid, kFwdThreads, smem, s>>>(
         *a.cp, a.pp->sched, (const K*)a.uniq_keys, a.grp_start, a.uid_at_pos, a.offsets,
         pb.sorted_groups, pb.chunks, pb.tasks, pb.hdr, a.rowbuf, out, a.status);
     *nl += 1;
@@ -1075,7 +1089,7 @@ cudaError_t bwd_launch(const K3Args& a, const GradPtrs& gp, const float* grad_ou
     cudaError_t e = cudaFuncSetAttribute(k3_bwd_kernel<S, K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const PlanBuffers& pb = *a.pb;
-    k3_bwd_kernel<S, K><<<a.grid, kThreads, smem, s>>>(
+    k3_bwd_kernel<S, K><<<a.grid, kBwdThreads, smem, s>>>(
         *a.cp, gp, *a.pp, (const K*)a.uniq_keys, a.grp_start, pb.sorted_groups, pb.col_count,
         pb.col_start, pb.hdr, a.rowbuf, a.status);
     *nl += 1;
@@ -1099,7 +1113,7 @@ int occ_fwd()
     const size_t smem = sizeof(float) * S::fwd_smem_floats();
     cudaFuncSetAttribute(k3_fwd_kernel<S, uint32_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k3_fwd_kernel<S, uint32_t>, kThreads, smem) != cudaSuccess) return 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k3_fwd_kernel<S, uint32_t>, kFwdThreads, smem) != cudaSuccess) return 1;
     return n > 0 ? n : 1;
 }
 template <class S>
@@ -1108,7 +1122,7 @@ int occ_bwd()
     const size_t smem = sizeof(float) * S::bwd_smem_floats();
     cudaFuncSetAttribute(k3_bwd_kernel<S, uint32_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k3_bwd_kernel<S, uint32_t>, kThreads, smem) != cudaSuccess) return 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k3_bwd_kernel<S, uint32_t>, kBwdThreads, smem) != cudaSuccess) return 1;
     return n > 0 ? n : 1;
 }
 
