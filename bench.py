@@ -32,6 +32,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "pooled TT lookups/sec fwd and fwd+bwd at batch 32768; % of roofline"
 FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # FFMA lanes x 2 flops x max SM clock
+BF16_PEAK_TFLOPS = 1644.9   # cuBLAS bf16 GEMM, burst, measured on this B200 pool (MEASURED_PEAKS.json)
 
 
 def parse_args():
@@ -43,9 +44,15 @@ def parse_args():
     p.add_argument("--config", type=int, default=4)
     p.add_argument("--batch", type=int, default=None, help="smaller batch (profiling runs)")
     p.add_argument("--tables", type=int, default=None, help="fewer tables (profiling runs)")
+    p.add_argument("--sched", choices=["static", "steal", "steal_l2"], default="steal_l2",
+                   help="work distribution of the fused kernels (ablation)")
+    p.add_argument("--grouping", choices=["prefix", "unique"], default="prefix",
+                   help="prefix reuse, or one unit per unique row (ablation)")
+    p.add_argument("--precision", choices=["fp32", "bf16"], default="fp32",
+                   help="forward prefix contraction: fp32 FFMA, or bf16 on the tcgen05 tensor cores")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--cpu-seconds", type=float, default=12.0,
+    p.add_argument("--cpu-seconds", type=float, default=15.0,
                    help="target CPU time of the oracle sample")
     return p.parse_args()
 
@@ -95,6 +102,7 @@ def algorithmic(w, U, G):
     b_fwd = io + out_bytes + core_bytes
     b_train = b_fwd + out_bytes + core_bytes + 3 * core_bytes
     return {"f_fwd": f_fwd, "f_bwd": f_bwd, "f_bwd_kernel": f_bwd_kernel, "f_sgd": 2.0 * core_bytes / 4,
+            "f_fwd_prefix": 2.0 * shared,
             "b_fwd": b_fwd, "b_train": b_train, "b_rowsum": out_bytes + 4.0 * U * D, "Mp": Mp, "Ms": Ms}
 
 
@@ -215,13 +223,18 @@ def oracle_step(w_sample, threads):
 
 
 def cpu_sample(w, target_s, threads):
-    """Pick the number of samples whose oracle step takes about target_s seconds."""
+    """Pick the number of samples whose oracle step takes about target_s seconds.
+
+    Small probes underuse the thread pool, so the probe grows geometrically until
+    it takes a quarter of the target, and the last probe's rate is extrapolated."""
     from workloads import sub_batch
-    probe = sub_batch(w, np.arange(1))
-    t1 = oracle_step(probe, threads)
-    per_lookup = t1 / max(probe.num_lookups, 1)
-    avg = w.num_lookups / w.batch
-    S = int(max(1, min(w.batch, target_s / max(per_lookup * avg, 1e-9))))
+    S = 1
+    while True:
+        t = oracle_step(sub_batch(w, np.arange(S)), threads)
+        if t >= 0.25 * target_s or S >= w.batch:
+            break
+        S = min(w.batch, int(S * min(16.0, max(2.0, 0.3 * target_s / max(t, 1e-3)))))
+    S = int(max(1, min(w.batch, S * target_s / max(t, 1e-6))))
     return sub_batch(w, np.arange(S)), S
 
 
@@ -271,7 +284,12 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     w = config_workload(args.config, batch=args.batch, tables=args.tables, with_grad=True)
     train = w.grad_out is not None and args.config in (4, 5)
-    emb, cores, idx, off = from_workload(w, device=dev, with_grads=True)
+    opts = abi.tt_emb_default_options()
+    opts.sched = {"static": abi.TT_SCHED_STATIC, "steal": abi.TT_SCHED_STEAL,
+                  "steal_l2": abi.TT_SCHED_STEAL_L2}[args.sched]
+    opts.grouping = abi.TT_GROUP_PREFIX if args.grouping == "prefix" else abi.TT_GROUP_UNIQUE_ONLY
+    opts.precision = abi.TT_PREC_FP32 if args.precision == "fp32" else abi.TT_PREC_BF16_TC
+    emb, cores, idx, off = from_workload(w, device=dev, options=opts, with_grads=True)
     g = torch.from_numpy(w.grad_out).to(dev)
     L, B, T, D = w.num_lookups, w.batch, w.num_tables, w.dim
     out = torch.empty(B, T * D, dtype=torch.float32, device=dev)
@@ -322,7 +340,20 @@ def run_ours(args):
     per_step = {k: v / args.steps for k, v in ph.items()}
     dom = max(per_step, key=per_step.get)
     flops = {"fwd_fused": alg["f_fwd"], "bwd_fused": alg["f_bwd_kernel"]}
-    if dom in flops:
+    if dom == "fwd_fused" and args.precision == "bf16":
+        # prefix step on the tensor cores, the rest on the FP32 pipes: the peak is the
+        # work-weighted combination of the two (time = F_tc / P_tc + F_fp32 / P_fp32)
+        f_tc = alg["f_fwd_prefix"]
+        f_rest = alg["f_fwd"] - f_tc
+        t_ideal = f_tc / (BF16_PEAK_TFLOPS * 1e12) + f_rest / (FP32_PEAK_TFLOPS * 1e12)
+        peak = alg["f_fwd"] / t_ideal / 1e12
+        achieved = alg["f_fwd"] / (per_step[dom] / 1e3) / 1e12
+        roof = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "peak_source": f"work-weighted: prefix step {f_tc / 1e9:.1f} GFLOP at the measured bf16 "
+                               f"tensor peak {BF16_PEAK_TFLOPS:.0f} TF/s, the rest {f_rest / 1e9:.1f} GFLOP at "
+                               f"the derived FP32 peak {FP32_PEAK_TFLOPS:.1f} TF/s"}
+    elif dom in flops:
         achieved = flops[dom] / (per_step[dom] / 1e3) / 1e12
         roof = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": FP32_PEAK_TFLOPS,
                 "unit": "TFLOP/s", "frac": achieved / FP32_PEAK_TFLOPS,
@@ -338,31 +369,76 @@ def run_ours(args):
     t_roof_fwd = max(alg["f_fwd"] / (FP32_PEAK_TFLOPS * 1e12), alg["b_fwd"] / 6550.4e9)
 
     # --- end to end through the public API with host buffers ---
+    # Every step copies its inputs from pinned host memory and reads its pooled output
+    # back.  The copies run on two copy streams, double-buffered, so step i+1's inputs
+    # and step i's output cross the host link while the compute stream works.
     e2e = None
     if not args.no_e2e:
         h_idx = torch.from_numpy(w.indices).pin_memory()
         h_off = torch.from_numpy(w.offsets).pin_memory()
         h_g = torch.from_numpy(w.grad_out).pin_memory()
-        h_out = torch.empty(B, T * D, dtype=torch.float32).pin_memory()
-        d_idx, d_off, d_g = torch.empty_like(idx), torch.empty_like(off), torch.empty_like(g)
+        h_out = [torch.empty(B, T * D, dtype=torch.float32).pin_memory() for _ in range(2)]
+        d_idx = [torch.empty_like(idx) for _ in range(2)]
+        d_off = [torch.empty_like(off) for _ in range(2)]
+        d_g = [torch.empty_like(g) for _ in range(2)] if train else None
+        d_out = [torch.empty_like(out) for _ in range(2)]
+        comp = torch.cuda.current_stream(dev)
+        up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]     # a slot's inputs are on the device
+        ev_used = [torch.cuda.Event() for _ in range(2)]   # the step using a slot is done
+        ev_fwd = [torch.cuda.Event() for _ in range(2)]    # a slot's pooled output is written
+        ev_read = [torch.cuda.Event() for _ in range(2)]   # a slot's output is back on the host
 
-        def e2e_step():
-            d_idx.copy_(h_idx, non_blocking=True)
-            d_off.copy_(h_off, non_blocking=True)
-            if train:
-                d_g.copy_(h_g, non_blocking=True)
-            emb.forward(d_idx, d_off, B, out)
-            if train:
-                emb.backward(d_g)
-                if args.config == 4:
-                    emb.sgd_update(w.lr)
-            h_out.copy_(out, non_blocking=True)
+        def upload(s):
+            up.wait_event(ev_used[s])
+            with torch.cuda.stream(up):
+                d_idx[s].copy_(h_idx, non_blocking=True)
+                d_off[s].copy_(h_off, non_blocking=True)
+                if train:
+                    d_g[s].copy_(h_g, non_blocking=True)
+            ev_in[s].record(up)
 
-        e2e_step()
-        ms_e2e = timed(e2e_step, max(2, args.steps // 2)) / max(2, args.steps // 2)
+        def run_steps(K):
+            upload(0)
+            for i in range(K):
+                s = i % 2
+                if i + 1 < K:
+                    upload((i + 1) % 2)
+                comp.wait_event(ev_in[s])
+                comp.wait_event(ev_read[s])
+                emb.forward(d_idx[s], d_off[s], B, d_out[s])
+                ev_fwd[s].record(comp)
+                down.wait_event(ev_fwd[s])
+                with torch.cuda.stream(down):
+                    h_out[s].copy_(d_out[s], non_blocking=True)
+                ev_read[s].record(down)
+                if train:
+                    emb.backward(d_g[s])
+                    if args.config == 4:
+                        emb.sgd_update(w.lr)
+                ev_used[s].record(comp)
+            for s in range(2):
+                comp.wait_event(ev_read[s])
+
+        run_steps(2)
+        torch.cuda.synchronize()
+        K = max(4, args.steps // 2)
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(comp)
+        up.wait_event(e0)
+        down.wait_event(e0)
+        run_steps(K)
+        e1.record(comp)
+        torch.cuda.synchronize()
+        emb.sync()
+        barrier(world)
+        ms_e2e = max_over_ranks(world, e0.elapsed_time(e1)) / K
         h2d = 8 * L + 8 * (T * B + 1) + (4 * B * T * D if train else 0)
         e2e = {"value": world * L / (ms_e2e / 1e3), "unit": "lookups/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": 4 * B * T * D, "ms_per_step": ms_e2e}
+               "d2h_bytes_per_step": 4 * B * T * D, "ms_per_step": ms_e2e,
+               "copies": "pinned host buffers, double-buffered on two copy streams, overlapped with compute"}
 
     # --- CPU oracle on a bounded sample (rank 0, one GPU only) ---
     cpu = None
@@ -379,13 +455,17 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": value, "unit": "lookups/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32" if args.precision == "fp32" else "bf16 prefix GEMM, f32 elsewhere",
             "data": "synthetic",
             "config": {"workload": w.name, "batch": B, "tables": T, "lookups": L,
                        "unique_rows": U, "prefix_groups": G,
                        "step": "fwd+bwd+sgd" if train else "fwd",
                        "l2": "inputs larger than L2 (indices+grad+cores ~800 MB), no flush",
-                       "parallelism": f"replicas{world}" if world > 1 else "single"},
+                       "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "sched": args.sched, "grouping": args.grouping,
+                       "prefix_step": "fp32 FFMA" if args.precision == "fp32" else
+                                      "bf16 operands, fp32 accumulation, tcgen05"},
             "fwd": {"value": world * L / (ms_fwd / 1e3), "unit": "lookups/s", "ms": ms_fwd,
                     "roofline_frac": t_roof_fwd / (ms_fwd / 1e3)},
             "step_roofline_frac": t_roof_step / (ms_step / 1e3),

@@ -84,13 +84,29 @@ typedef enum {
     TT_GROUP_UNIQUE_ONLY = 1 /* deduplicate rows only: every distinct row is contracted on its own */
 } tt_group_mode;
 
+/*
+ * Arithmetic of the prefix contraction C_p = G_1[0, i_1] . G_2[:, i_2] in the forward
+ * (FlowTT section 3.3 computes it once per prefix group; the pages compute in fp32).
+ * TT_PREC_BF16_TC rounds both operands to bf16 (round to nearest even) and runs the
+ * contraction on the fifth-generation tensor cores, accumulating in fp32 in tensor
+ * memory; the suffix contraction, the pooling and the whole backward stay fp32.  Its
+ * results agree with the exact (fp64) definition to within 2e-2, measured normwise per
+ * pooled row.  It needs three cores with d = (4, 4, 8) and r_1 = r_2 in {32, 64};
+ * tt_emb_create returns TT_ERR_SHAPE for other shapes.
+ */
+typedef enum {
+    TT_PREC_FP32 = 0,        /* fp32 operands and accumulation on the FP32 pipes (default) */
+    TT_PREC_BF16_TC = 1      /* bf16 operands, fp32 accumulation, tcgen05 tensor cores */
+} tt_precision;
+
 typedef struct {
     int32_t sched;           /* tt_sched_mode, default TT_SCHED_STEAL_L2 */
     int32_t grouping;        /* tt_group_mode, default TT_GROUP_PREFIX */
     int32_t chunk;           /* rows per stealable chunk of a prefix group; 0 = library default */
     int32_t grid;            /* persistent blocks; 0 = one wave on the current device */
     int32_t force_generic;   /* 1: run the shape-generic kernels even where a specialised path exists */
-    int32_t reserved[11];    /* must be zero */
+    int32_t precision;       /* tt_precision, default TT_PREC_FP32 */
+    int32_t reserved[10];    /* must be zero */
 } tt_emb_options;
 
 /* Fills *opt with the defaults. */

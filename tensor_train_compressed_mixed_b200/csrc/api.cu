@@ -15,7 +15,7 @@ struct Layout {
         uniq_start, grp_start, bag_sorted;
     // specialised path only (zero when unused)
     size_t uid_at_pos, uid_sorted, rowbuf, pkeys[2], pvals[2], col_count, col_start, chunk_base,
-        hdr, chunks, tasks, g12, dg12, g3t;
+        hdr, chunks, tasks, g12, dg12, g3t, bf1, bf2;
     int64_t chunk_cap, task_cap;
     size_t total;
 };
@@ -26,6 +26,7 @@ struct FastDims {
     int D, ncols, MP, T;
     int64_t g12_floats;   // merged first cores of four-core tables (0 otherwise)
     int64_t g3t_floats;   // transposed copies of the last cores
+    int64_t bf1_elems, bf2_elems;   // bf16 operand copies of G_1 and G_2 (tensor-core forward)
 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -76,6 +77,10 @@ Layout make_layout(int key_bytes, int64_t L, int64_t B, const FastDims& f)
             y.dg12 = take((size_t)f.g12_floats * 4);
         }
         y.g3t = take((size_t)f.g3t_floats * 4);
+        if (f.bf1_elems > 0) {
+            y.bf1 = take((size_t)f.bf1_elems * 2);
+            y.bf2 = take((size_t)f.bf2_elems * 2);
+        }
     }
     y.total = p;
     return y;
@@ -122,6 +127,9 @@ struct tt_emb_handle {
     int32_t vd[3] = {}, vr[4] = {};
     int64_t g12_off[kMaxT + 1] = {};  // merged-core offsets (floats) in the workspace
     int64_t g3t_off[kMaxT + 1] = {};  // transposed last-core offsets (floats) in the workspace
+    bool tc = false;                  // forward prefix GEMM on the tensor cores (bf16 operands)
+    int64_t bf1_off[kMaxT + 1] = {};  // bf16 copies of G_1 and G_2 (elements) in the workspace
+    int64_t bf2_off[kMaxT + 1] = {};
     // timing and launch accounting
     bool timing = false;
     double phase_ms[TT_EMB_NUM_PHASES] = {};
@@ -184,6 +192,8 @@ struct tt_emb_handle {
         f.T = T;
         f.g12_floats = merged ? g12_off[T] : 0;
         f.g3t_floats = g3t_off[T];
+        f.bf1_elems = tc ? bf1_off[T] : 0;
+        f.bf2_elems = tc ? bf2_off[T] : 0;
         return f;
     }
     // three-core view of the shapes (identity for three-core tables), without core pointers
@@ -214,6 +224,10 @@ struct tt_emb_handle {
             cp.cores[t][1] = cores[t * k + 1 + off];
             cp.cores[t][2] = cores[t * k + 2 + off];
             cp.last_t[t] = (const float*)at(lay.g3t) + g3t_off[t];
+            if (tc) {
+                cp.bf1[t] = (const uint16_t*)at(lay.bf1) + bf1_off[t];
+                cp.bf2[t] = (const uint16_t*)at(lay.bf2) + bf2_off[t];
+            }
             if (gp) {
                 gp->g[t][0] = merged ? (float*)at(lay.dg12) + g12_off[t] : grads[t * k];
                 gp->g[t][1] = grads[t * k + 1 + off];
@@ -347,7 +361,8 @@ struct tt_emb_handle {
         a.offsets = offsets;
         a.rowbuf = (float*)at(lay.rowbuf);
         a.L = L;
-        a.grid = opt.grid > 0 ? opt.grid : num_sms * k3_blocks_per_sm(*cp, backward);
+        a.tc = (tc && !backward) ? 1 : 0;
+        a.grid = opt.grid > 0 ? opt.grid : num_sms * k3_blocks_per_sm(*cp, backward, a.tc != 0);
         a.status = d_status;
         return a;
     }
@@ -397,9 +412,10 @@ int tt_emb_create(int32_t num_tables, int32_t num_cores, const int64_t* n_factor
     tt_emb_default_options(&o);
     if (opt) {
         o = *opt;
-        for (int i = 0; i < 11; ++i)
+        for (int i = 0; i < 10; ++i)
             if (o.reserved[i] != 0) return TT_ERR_ARG;
         if (o.force_generic != 0 && o.force_generic != 1) return TT_ERR_ARG;
+        if (o.precision != TT_PREC_FP32 && o.precision != TT_PREC_BF16_TC) return TT_ERR_ARG;
         if (o.sched < TT_SCHED_STATIC || o.sched > TT_SCHED_STEAL_L2) return TT_ERR_ARG;
         if (o.grouping < TT_GROUP_PREFIX || o.grouping > TT_GROUP_UNIQUE_ONLY) return TT_ERR_ARG;
         if (o.chunk < 0 || o.grid < 0) return TT_ERR_ARG;
@@ -489,6 +505,23 @@ int tt_emb_create(int32_t num_tables, int32_t num_cores, const int64_t* n_factor
         h->col_base[num_tables] = (int)nc;
         if (nc >= (1LL << 24)) h->fast = h->merged = false;
         h->ncols = (int)nc;
+    }
+    if (o.precision == TT_PREC_BF16_TC) {
+        // the tensor-core prefix GEMM exists for three-core tables of the listed shapes only
+        if (!h->fast || h->merged || !k3_tc_supported(h->view_params())) {
+            delete h;
+            return TT_ERR_SHAPE;
+        }
+        h->tc = true;
+        int64_t b1 = 0, b2 = 0;
+        for (int t = 0; t < num_tables; ++t) {
+            h->bf1_off[t] = b1;
+            h->bf2_off[t] = b2;
+            b1 += h->vn[t][0] * h->vd[0] * h->vr[1];
+            b2 += h->vn[t][1] * h->vr[1] * h->vd[1] * h->vr[2];
+        }
+        h->bf1_off[num_tables] = b1;
+        h->bf2_off[num_tables] = b2;
     }
     if (generic_backward_smem_floats(cp) * 4 > 200 * 1024 ||
         generic_forward_smem_floats(cp) * 4 > 200 * 1024) {
@@ -639,6 +672,15 @@ int tt_emb_forward(tt_emb_t h, const int64_t* indices, const int64_t* offsets, i
             float* dst[kMaxT];
             for (int t = 0; t < h->T; ++t) dst[t] = (float*)h->at(y.g3t) + h->g3t_off[t];
             e = k3_transpose_last(cp, dst, s, &nl);
+        }
+        if (e == cudaSuccess && h->tc) {
+            uint16_t* d1[kMaxT];
+            uint16_t* d2[kMaxT];
+            for (int t = 0; t < h->T; ++t) {
+                d1[t] = (uint16_t*)h->at(y.bf1) + h->bf1_off[t];
+                d2[t] = (uint16_t*)h->at(y.bf2) + h->bf2_off[t];
+            }
+            e = k3_to_bf16(cp, d1, d2, s, &nl);
         }
         K3Args a = h->k3_args(&cp, &pp, &pb, offsets, L, false);
         if (e == cudaSuccess) e = k3_forward(a, out, s, &nl);

@@ -21,6 +21,7 @@
 //     and dB += A^T dC.  dB is reduced on chip over the whole column group and
 //     written once; dA and the last-slice gradients are reduced into the
 //     small, L2-resident gradient arrays with 16-byte vector reductions.
+#include <cuda_bf16.h>
 #include <string.h>
 
 #include "tt_common.cuh"
@@ -99,6 +100,11 @@ struct S3 {
     static_assert(NUB >= 1 && NUB * TPUB == kBwdThreads, "backward batch tiling");
 
     static constexpr size_t fwd_smem_floats() { return FWD_FIXED + (size_t)FBUF * NUF * SU; }
+    // tensor-core variant: A and B in bf16
+    static constexpr size_t fwd_smem_floats_tc()
+    {
+        return ((size_t)R * N + (size_t)MF * R) / 2 + (size_t)MF * N + (size_t)FBUF * NUF * SU;
+    }
     static constexpr size_t bwd_smem_floats()
     {
         return (size_t)R * N + 2 * (size_t)MB * R + 2 * (size_t)MB * N + 2 * (size_t)NUB * P * D3 +
@@ -165,12 +171,111 @@ __device__ __forceinline__ int next_task(int sched, int* head, int iter)
 }
 
 // ---------------------------------------------------------------------------
+// fifth-generation tensor cores: tensor memory, mbarrier, tcgen05.mma (bf16 x bf16 -> f32)
+// ---------------------------------------------------------------------------
+constexpr int kMbarSpin = 1 << 20;   // bounded wait for an MMA completion (tens of ms at most)
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// Shared-memory matrix descriptor for a K-major operand without swizzle.  The operand is
+// stored as 8-row x 16-byte core matrices (8 rows of 8 bf16 along K, 128 contiguous bytes);
+// lbo = bytes between the two K-adjacent core matrices one MMA (K = 16) reads, sbo = bytes
+// between consecutive 8-row groups.  Bits: start >> 4 [0,14), lbo >> 4 [16,30),
+// sbo >> 4 [32,46), descriptor version 1 [46,48), base offset 0, layout 0 (no swizzle).
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
+}
+
+// Instruction descriptor of kind::f16: f32 accumulator [4,6) = 1, A = bf16 [7,10) = 1,
+// B = bf16 [10,13) = 1, both K-major (bits 15, 16 clear), N >> 3 at [17,23), M >> 4 at [24,29).
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols)   // one warp
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)   // the same warp
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// makes this thread's generic-proxy shared-memory writes visible to the tensor cores
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
+        : "memory");
+}
+// arrives once on the mbarrier when every MMA this thread issued so far has completed
+__device__ __forceinline__ void tc_commit(uint64_t* bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// bounded wait for the completion of phase `parity`; false when the bound ran out
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
+{
+    const uint32_t a = smem_u32(bar);
+    for (int it = 0; it < kMbarSpin; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.b32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(a), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if (it >= 8) __nanosleep(64);
+    }
+    return false;
+}
+// 32 lanes x 32 consecutive 32-bit columns of tensor memory: lane i of the warp gets row
+// (taddr lane + i), columns taddr column .. +31
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ---------------------------------------------------------------------------
 // forward
 // ---------------------------------------------------------------------------
 template <class S>
 struct FwdSmem {
     float* Bs;   // [R][N]        B = G_2[:, i_2], swizzled
     float* As;   // [MF][R]       A_j = G_1[0, i1_j] rows, swizzled
+    uint16_t* Bb;   // tensor-core variant: B as N x R bf16 core matrices (K-major)
+    uint16_t* Ab;   // tensor-core variant: A as MF x R bf16 core matrices (K-major)
     float* Cn;   // [MF][N]       C_all, swizzled
     float* Ss;   // [FBUF][NUF][SU] last slices of a batch of distinct rows
 };
@@ -295,6 +400,85 @@ __device__ __forceinline__ void fwd_gemm(const FwdSmem<S>& sm)
         *reinterpret_cast<float4*>(&sm.Cn[swz_m<N>(rows[i], N / 2 + tn * 4)]) =
             make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
     }
+}
+
+// Tensor-core variant of fwd_issue_ab: bf16 B tile (already in operand order, one flat
+// copy) and the chunk's A rows placed into 8 x 16-byte core matrices; one commit group.
+template <class S>
+__device__ __forceinline__ void fwd_issue_ab_tc(const CoreParams& cp, int mb, const FwdMeta<S>& M,
+                                                const FwdSmem<S>& sm, int& cur_t, int& cur_i2)
+{
+    constexpr int R = S::R, N = S::N, MF = S::MF, D1 = S::D1;
+    constexpr int KC = R / 8;   // 16-byte K chunks per operand row
+    const int tid = threadIdx.x;
+    const int t = M.t[mb], i2 = M.i2[mb], cnt = M.cnt[mb];
+    if (t != cur_t || i2 != cur_i2) {
+        const uint16_t* src = cp.bf2[t] + (int64_t)i2 * (R * N);
+        for (int q = tid; q < R * N / 8; q += kFwdThreads) cp_async16(sm.Bb + q * 8, src + q * 8);
+        cur_t = t;
+        cur_i2 = i2;
+    }
+    const uint16_t* G1 = cp.bf1[t];
+    for (int q = tid; q < MF * KC; q += kFwdThreads) {
+        const int m = q / KC, kc = q % KC;
+        const int j = m / D1, a1 = m % D1;
+        uint16_t* dst = sm.Ab + ((m >> 3) * KC + kc) * 64 + (m & 7) * 8;
+        if (j < cnt) cp_async16(dst, G1 + ((int64_t)M.i1[mb][j] * D1 + a1) * R + kc * 8);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    cp_async_commit();
+}
+
+// C_all = A . B on the tensor cores: one thread issues R / 16 MMAs (M = MF, N, K = 16)
+// into tensor memory and commits them to the mbarrier; after the bounded wait every warp
+// moves its share of the fp32 accumulator (sub-partition warp % 4, a quarter of the
+// columns) into Cn.  The caller has waited for the A/B copies; returns false (all
+// threads) when the completion wait ran out.
+template <class S>
+__device__ __forceinline__ bool fwd_gemm_tc(const FwdSmem<S>& sm, uint32_t tmem, uint64_t* bar, uint32_t& parity,
+                                            int* s_ok)
+{
+    constexpr int R = S::R, N = S::N, MF = S::MF;
+    static_assert(MF == 64 || MF == 128, "tensor-core M is 64 or 128");
+    static_assert(kFwdThreads == 512, "16 warps: 4 sub-partitions x 4 column blocks");
+    const int tid = threadIdx.x;
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t SBO = (R / 8) * 128;
+        constexpr uint32_t idesc = umma_idesc_bf16(MF, N);
+        const uint32_t a0 = smem_u32(sm.Ab), b0 = smem_u32(sm.Bb);
+#pragma unroll
+        for (int k = 0; k < R / 16; ++k)
+            tc_mma_bf16(tmem, umma_desc(a0 + k * 256, 128, SBO), umma_desc(b0 + k * 256, 128, SBO), idesc, k > 0);
+        tc_commit(bar);
+        *s_ok = mbar_wait(bar, parity) ? 1 : 0;
+    }
+    __syncthreads();
+    parity ^= 1u;
+    if (!*s_ok) return false;
+    tc_fence_after();
+    const int warp = tid >> 5, lane = tid & 31;
+    const int sub = warp & 3, cb = warp >> 2;
+    constexpr int CPB = N / 4;   // accumulator columns per warp
+    // M = 128: row m in lane m; M = 64: rows 16 s .. 16 s + 15 in lanes 32 s .. 32 s + 15
+    const int m = MF == 128 ? 32 * sub + lane : 16 * sub + lane;
+    const bool valid = MF == 128 || lane < 16;
+#pragma unroll 1
+    for (int g = 0; g < CPB / 32; ++g) {
+        const int c0 = cb * CPB + g * 32;
+        float v[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)c0, v);
+        if (valid) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<float4*>(&sm.Cn[swz_m<N>(m, c0 + 4 * j)]) =
+                    make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        }
+    }
+    tc_fence_before();
+    return true;
 }
 
 // distinct rows k0..k0+nb of the chunk into batch buffer bb; issues their last slices (one commit group)
@@ -431,7 +615,7 @@ __device__ void fwd_pool(const CoreParams& cp, int ptask, int nP, const int32_t*
 // metadata and A/B rows (As and Bs are free once the GEMM is done) while this
 // chunk's distinct rows are contracted batch by batch (double-buffered last
 // slices when shared memory allows).
-template <class S, typename K>
+template <class S, typename K, bool TC>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
               const int32_t* __restrict__ grp_start, const int32_t* __restrict__ uid_at_pos,
@@ -441,13 +625,32 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
 {
     extern __shared__ __align__(16) float smem_f[];
     __shared__ FwdMeta<S> M;
+    __shared__ __align__(8) uint64_t s_mbar;
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_ok;
     if (has_error(status)) return;
     FwdSmem<S> sm;
-    sm.Bs = smem_f;
-    sm.As = sm.Bs + S::R * S::N;
-    sm.Cn = sm.As + S::MF * S::R;
-    sm.Ss = sm.Cn + S::MF * S::N;
     const int tid = threadIdx.x;
+    uint32_t tmem = 0, parity = 0;
+    if constexpr (TC) {
+        // bf16 operands take half the room of fp32 ones
+        sm.Bs = sm.As = nullptr;
+        sm.Bb = reinterpret_cast<uint16_t*>(smem_f);
+        sm.Ab = sm.Bb + S::R * S::N;
+        sm.Cn = smem_f + (S::R * S::N + S::MF * S::R) / 2;
+        if (tid < 32) tmem_alloc(&s_tmem, (uint32_t)S::N);
+        if (tid == 0) mbar_init(&s_mbar, 1);
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        tmem = s_tmem;
+    } else {
+        sm.Bs = smem_f;
+        sm.As = sm.Bs + S::R * S::N;
+        sm.Bb = sm.Ab = nullptr;
+        sm.Cn = sm.As + S::MF * S::R;
+    }
+    sm.Ss = sm.Cn + S::MF * S::N;
     const int ntasks = hdr->ntasks, nP = hdr->nP;
     int iter = 0;
     int cur_t = -1, cur_i2 = -1;   // column of the B now in (or on its way to) Bs
@@ -472,7 +675,8 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
         TT_PH_START();
         if (!staged) {
             fwd_meta<S, K>(cp, tv, mb, uniq_keys, grp_start, sorted_groups, chunks, M);
-            fwd_issue_ab<S>(cp, mb, M, sm, cur_t, cur_i2);
+            if constexpr (TC) fwd_issue_ab_tc<S>(cp, mb, M, sm, cur_t, cur_i2);
+            else fwd_issue_ab<S>(cp, mb, M, sm, cur_t, cur_i2);
         }
         // the first batch of last slices is in flight during the GEMM
         const int total = M.ucum[mb][S::MPF];
@@ -483,14 +687,22 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
         else cp_async_wait_all();
         __syncthreads();
         TT_PH(0);
-        fwd_gemm<S>(sm);
+        if constexpr (TC) {
+            if (!fwd_gemm_tc<S>(sm, tmem, &s_mbar, parity, &s_ok)) {
+                if (tid == 0) raise_error(status, TT_ERR_TIMEOUT, 100);
+                break;
+            }
+        } else {
+            fwd_gemm<S>(sm);
+        }
         __syncthreads();
         TT_PH(1);
         const int qn = M.task[1];
         const bool next_chunk = qn < ntasks && tasks[qn] >= 0;
         if (next_chunk) {
             fwd_meta<S, K>(cp, tasks[qn], mb ^ 1, uniq_keys, grp_start, sorted_groups, chunks, M);
-            fwd_issue_ab<S>(cp, mb ^ 1, M, sm, cur_t, cur_i2);
+            if constexpr (TC) fwd_issue_ab_tc<S>(cp, mb ^ 1, M, sm, cur_t, cur_i2);
+            else fwd_issue_ab<S>(cp, mb ^ 1, M, sm, cur_t, cur_i2);
         }
         // distinct rows of this chunk, in batches of NUF (commit groups in flight: the batch,
         // then possibly the next chunk's A/B, then possibly the next batch)
@@ -531,6 +743,14 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
         if (next_chunk) mb ^= 1;
     }
     cp_async_wait_all();
+    if constexpr (TC) {
+        tc_fence_before();
+        __syncthreads();
+        if (tid < 32) {
+            tc_fence_after();
+            tmem_dealloc(tmem, (uint32_t)S::N);
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -1028,6 +1248,73 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
 // ---------------------------------------------------------------------------
 // last core [R][n3][D3] -> [n3][R][D3]; one thread per (table, i3, rho) row of D3 floats
 // ---------------------------------------------------------------------------
+// bf16 operand copies for the tensor-core forward.  Items are 16-byte output chunks:
+// first every table's G_1 (a plain [n_1][d_1][r_1] copy), then every table's G_2 tiles,
+// one per i_2, in the operand order of fwd_issue_ab_tc: element (n, k) of the tile
+// (n = a_2 r_2 + rho_2, k = rho_1) at ((n / 8) (R / 8) + k / 8) 64 + (n % 8) 8 + k % 8.
+struct Bf16Job {
+    int32_t T, R, N, pad;
+    int64_t base1[kMaxT + 1], base2[kMaxT + 1];   // prefix sums of chunk counts
+    uint32_t n2[kMaxT];
+    const float* src1[kMaxT];
+    const float* src2[kMaxT];
+    uint16_t* dst1[kMaxT];
+    uint16_t* dst2[kMaxT];
+};
+
+__device__ __forceinline__ int table_of(const int64_t* base, int T, int64_t q)
+{
+    int lo = 0, hi = T - 1;   // last t with base[t] <= q
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (base[mid] <= q) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ uint4 pack_bf16x8(const float (&v)[8])
+{
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        w[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i])) |
+               ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i + 1])) << 16);
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__global__ void __launch_bounds__(256) k3_bf16_kernel(Bf16Job j)
+{
+    const int64_t tot1 = j.base1[j.T], tot2 = j.base2[j.T];
+    const int KC = j.R / 8;
+    const int64_t per_tile = (int64_t)j.R * j.N / 8;
+    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < tot1 + tot2;
+         q += (int64_t)gridDim.x * blockDim.x) {
+        float v[8];
+        if (q < tot1) {
+            const int t = table_of(j.base1, j.T, q);
+            const int64_t off = (q - j.base1[t]) * 8;
+            const float4 x0 = __ldg(reinterpret_cast<const float4*>(j.src1[t] + off));
+            const float4 x1 = __ldg(reinterpret_cast<const float4*>(j.src1[t] + off + 4));
+            v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
+            v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+            *reinterpret_cast<uint4*>(j.dst1[t] + off) = pack_bf16x8(v);
+        } else {
+            const int64_t q2 = q - tot1;
+            const int t = table_of(j.base2, j.T, q2);
+            const int64_t r = q2 - j.base2[t];
+            const int64_t i2 = r / per_tile;
+            const int c = (int)(r % per_tile);          // chunk ((n / 8) KC + kc) 8 + n % 8
+            const int n = (c / (8 * KC)) * 8 + (c % 8), kc = (c / 8) % KC;
+            const int64_t rs = (int64_t)j.n2[t] * j.N;  // stride between rho_1 rows of G_2
+            const float* src = j.src2[t] + i2 * j.N + n + (int64_t)kc * 8 * rs;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = __ldg(src + e * rs);
+            *reinterpret_cast<uint4*>(j.dst2[t] + i2 * (j.R * j.N) + (int64_t)c * 8) = pack_bf16x8(v);
+        }
+    }
+}
+
 struct TransposeJob {
     int32_t T, R, D3, pad;
     int64_t row_base[kMaxT + 1];   // prefix sums of n3 * R
@@ -1055,14 +1342,14 @@ __global__ void __launch_bounds__(256) k3_transpose_last_kernel(TransposeJob tj,
 // ---------------------------------------------------------------------------
 // host launchers
 // ---------------------------------------------------------------------------
-template <class S, typename K>
+template <class S, typename K, bool TC>
 cudaError_t fwd_launch(const K3Args& a, float* out, cudaStream_t s, int* nl)
 {
-    const size_t smem = sizeof(float) * S::fwd_smem_floats();
-    cudaError_t e = cudaFuncSetAttribute(k3_fwd_kernel<S, K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = sizeof(float) * (TC ? S::fwd_smem_floats_tc() : S::fwd_smem_floats());
+    cudaError_t e = cudaFuncSetAttribute(k3_fwd_kernel<S, K, TC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const PlanBuffers& pb = *a.pb;
-    k3_fwd_kernel<S, K><<<a.grid, kFwdThreads, smem, s>>>(
+    k3_fwd_kernel<S, K, TC><<<a.grid, kFwdThreads, smem, s>>>(
         *a.cp, a.pp->sched, (const K*)a.uniq_keys, a.grp_start, a.uid_at_pos, a.offsets,
         pb.sorted_groups, pb.chunks, pb.tasks, pb.hdr, a.rowbuf, out, a.status);
     *nl += 1;
@@ -1099,7 +1386,12 @@ cudaError_t bwd_launch(const K3Args& a, const GradPtrs& gp, const float* grad_ou
 template <class S>
 cudaError_t fwd_dispatch(const K3Args& a, float* out, cudaStream_t s, int* nl)
 {
-    return a.key64 ? fwd_launch<S, uint64_t>(a, out, s, nl) : fwd_launch<S, uint32_t>(a, out, s, nl);
+    return a.key64 ? fwd_launch<S, uint64_t, false>(a, out, s, nl) : fwd_launch<S, uint32_t, false>(a, out, s, nl);
+}
+template <class S>
+cudaError_t fwd_dispatch_tc(const K3Args& a, float* out, cudaStream_t s, int* nl)
+{
+    return a.key64 ? fwd_launch<S, uint64_t, true>(a, out, s, nl) : fwd_launch<S, uint32_t, true>(a, out, s, nl);
 }
 template <class S>
 cudaError_t bwd_dispatch(const K3Args& a, const GradPtrs& gp, const float* g, cudaStream_t s, int* nl)
@@ -1107,14 +1399,16 @@ cudaError_t bwd_dispatch(const K3Args& a, const GradPtrs& gp, const float* g, cu
     return a.key64 ? bwd_launch<S, uint64_t>(a, gp, g, s, nl) : bwd_launch<S, uint32_t>(a, gp, g, s, nl);
 }
 
-template <class S>
+template <class S, bool TC>
 int occ_fwd()
 {
-    const size_t smem = sizeof(float) * S::fwd_smem_floats();
-    cudaFuncSetAttribute(k3_fwd_kernel<S, uint32_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = sizeof(float) * (TC ? S::fwd_smem_floats_tc() : S::fwd_smem_floats());
+    cudaFuncSetAttribute(k3_fwd_kernel<S, uint32_t, TC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k3_fwd_kernel<S, uint32_t>, kFwdThreads, smem) != cudaSuccess) return 1;
-    return n > 0 ? n : 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k3_fwd_kernel<S, uint32_t, TC>, kFwdThreads, smem) != cudaSuccess)
+        return 1;
+    // one block per SM holds tensor memory: the kernel allocates N columns and keeps them
+    return n > 0 ? (TC ? 1 : n) : 1;
 }
 template <class S>
 int occ_bwd()
@@ -1128,13 +1422,23 @@ int occ_bwd()
 
 }  // namespace
 
-int k3_blocks_per_sm(const CoreParams& cp, bool backward)
+int k3_blocks_per_sm(const CoreParams& cp, bool backward, bool tc)
 {
+    if (tc && !backward) {
+        if (cp.d[0] == 4 && cp.d[2] == 8 && cp.r[1] == 64) return occ_fwd<S3<4, 4, 8, 64>, true>();
+        if (cp.d[0] == 4 && cp.d[2] == 8 && cp.r[1] == 32) return occ_fwd<S3<4, 4, 8, 32>, true>();
+        return 1;
+    }
 #define TT_OCC_CASE(Q1, Q2, Q3, QR) \
-    if (cp.d[0] == Q1 && cp.d[2] == Q3 && cp.r[1] == QR) return backward ? occ_bwd<S3<Q1, Q2, Q3, QR>>() : occ_fwd<S3<Q1, Q2, Q3, QR>>();
+    if (cp.d[0] == Q1 && cp.d[2] == Q3 && cp.r[1] == QR) return backward ? occ_bwd<S3<Q1, Q2, Q3, QR>>() : occ_fwd<S3<Q1, Q2, Q3, QR>, false>();
     TT_K3_CASES_INNER(TT_OCC_CASE)
 #undef TT_OCC_CASE
     return 1;
+}
+
+bool k3_tc_supported(const CoreParams& cp)
+{
+    return k3_supported(cp) && cp.d[0] == 4 && cp.d[1] == 4 && cp.d[2] == 8 && (cp.r[1] == 64 || cp.r[1] == 32);
 }
 
 bool k3_supported(const CoreParams& cp)
@@ -1158,6 +1462,11 @@ int k3_plan_mp(const CoreParams& cp)
 cudaError_t k3_forward(const K3Args& a, float* out, cudaStream_t s, int* nl)
 {
     const CoreParams& cp = *a.cp;
+    if (a.tc) {
+        if (cp.d[0] == 4 && cp.d[2] == 8 && cp.r[1] == 64) return fwd_dispatch_tc<S3<4, 4, 8, 64>>(a, out, s, nl);
+        if (cp.d[0] == 4 && cp.d[2] == 8 && cp.r[1] == 32) return fwd_dispatch_tc<S3<4, 4, 8, 32>>(a, out, s, nl);
+        return cudaErrorInvalidValue;
+    }
 #define TT_FWD_CASE(Q1, Q2, Q3, QR) \
     if (cp.d[0] == Q1 && cp.d[2] == Q3 && cp.r[1] == QR) return fwd_dispatch<S3<Q1, Q2, Q3, QR>>(a, out, s, nl);
     TT_K3_CASES(TT_FWD_CASE)
@@ -1184,6 +1493,34 @@ cudaError_t k3_transpose_last(const CoreParams& cp, float* const* dst, cudaStrea
     if (b == 0) return cudaSuccess;
     const int grid = (int)min64(ceil_div(b, 256), 148 * 16);
     k3_transpose_last_kernel<<<grid, 256, 0, s>>>(tj, nullptr);
+    *nl += 1;
+    return cudaGetLastError();
+}
+
+cudaError_t k3_to_bf16(const CoreParams& cp, uint16_t* const* dst1, uint16_t* const* dst2, cudaStream_t s, int* nl)
+{
+    Bf16Job j;
+    memset(&j, 0, sizeof(j));
+    j.T = cp.T;
+    j.R = cp.r[1];
+    j.N = cp.d[1] * cp.r[2];
+    int64_t b1 = 0, b2 = 0;
+    for (int t = 0; t < cp.T; ++t) {
+        j.base1[t] = b1;
+        j.base2[t] = b2;
+        b1 += (int64_t)cp.n[t][0] * cp.d[0] * cp.r[1] / 8;
+        b2 += (int64_t)cp.n[t][1] * j.R * j.N / 8;
+        j.n2[t] = cp.n[t][1];
+        j.src1[t] = cp.cores[t][0];
+        j.src2[t] = cp.cores[t][1];
+        j.dst1[t] = dst1[t];
+        j.dst2[t] = dst2[t];
+    }
+    j.base1[cp.T] = b1;
+    j.base2[cp.T] = b2;
+    if (b1 + b2 == 0) return cudaSuccess;
+    const int grid = (int)min64(ceil_div(b1 + b2, 256), 148 * 16);
+    k3_bf16_kernel<<<grid, 256, 0, s>>>(j);
     *nl += 1;
     return cudaGetLastError();
 }

@@ -63,6 +63,10 @@ struct CoreParams {
     // specialised path: the last core re-laid out as [n_k][r_{k-1}][d_k], so that one
     // row's last slice is a contiguous block (built by k3_transpose_last each forward)
     const float* last_t[kMaxT];
+    // bf16 tensor-core prefix step: G_1 as [n_1][d_1][r_1] and G_2 as one operand tile per
+    // i_2 (n = (a_2, rho_2) rows x K = rho_1, 8 x 8 core matrices), built by k3_to_bf16
+    const uint16_t* bf1[kMaxT];
+    const uint16_t* bf2[kMaxT];
 };
 
 struct GradPtrs {
@@ -215,6 +219,7 @@ struct K3Args {
     float* rowbuf;                 // [U][D]: pooled-row checkpoint (forward), upstream sums (backward)
     int64_t L;
     int grid;
+    int tc;                        // 1: prefix GEMM on the tensor cores (bf16 operands)
     int32_t* status;
 };
 // Four-core tables run the three-core kernels on the merged first core
@@ -237,7 +242,11 @@ cudaError_t launch_unmerge(const MergeParams& mp, int32_t* status, cudaStream_t 
 constexpr int kPoolBags = 64;     // bags per pooling task of the specialised forward
 bool k3_supported(const CoreParams& cp);
 int k3_plan_mp(const CoreParams& cp);
-int k3_blocks_per_sm(const CoreParams& cp, bool backward);
+int k3_blocks_per_sm(const CoreParams& cp, bool backward, bool tc = false);
+// shapes with a tensor-core (bf16) variant of the forward prefix GEMM
+bool k3_tc_supported(const CoreParams& cp);
+// bf16 operand copies of G_1 and G_2 for the tensor-core forward (cp.cores -> dst1/dst2)
+cudaError_t k3_to_bf16(const CoreParams& cp, uint16_t* const* dst1, uint16_t* const* dst2, cudaStream_t s, int* nl);
 cudaError_t k3_forward(const K3Args& a, float* out, cudaStream_t s, int* nl);
 // last core [r][n_k][d_k] -> [n_k][r][d_k] into cp.last_t (before k3_forward / k3_backward)
 cudaError_t k3_transpose_last(const CoreParams& cp, float* const* dst, cudaStream_t s, int* nl);

@@ -73,6 +73,11 @@ def test_create_rejects_bad_options_on_host():
         abi.tt_emb_create([[2, 3]], [6], [2, 2], [1, 4, 1], o)
     assert e.value.code == abi.TT_ERR_ARG
     o = abi.tt_emb_default_options()
+    o.precision = 2
+    with pytest.raises(abi.TTEmbError) as e:
+        abi.tt_emb_create([[2, 3]], [6], [2, 2], [1, 4, 1], o)
+    assert e.value.code == abi.TT_ERR_ARG
+    o = abi.tt_emb_default_options()
     o.reserved[3] = 1
     with pytest.raises(abi.TTEmbError) as e:
         abi.tt_emb_create([[2, 3]], [6], [2, 2], [1, 4, 1], o)
@@ -86,3 +91,19 @@ def test_null_handle_calls_fail_cleanly():
     assert lib.tt_emb_sgd_update(None, 0.1, None) == abi.TT_ERR_ARG
     assert lib.tt_emb_sync(None) == abi.TT_ERR_ARG
     lib.tt_emb_destroy(None)
+
+
+@pytest.mark.parametrize("n,d,r", [
+    ([[5, 6, 7]], [4, 4, 4], [1, 32, 32, 1]),      # d_3 = 4
+    ([[5, 6, 7]], [4, 4, 8], [1, 16, 16, 1]),      # rank 16
+    ([[5, 6, 7]], [4, 4, 8], [1, 32, 64, 1]),      # r_1 != r_2
+    ([[2, 3]], [2, 2], [1, 4, 1]),                 # two cores
+    ([[2, 5, 6, 7]], [2, 4, 4, 4], [1, 32, 32, 32, 1]),  # four cores
+])
+def test_bf16_tensor_core_precision_rejects_other_shapes(n, d, r):
+    o = abi.tt_emb_default_options()
+    o.precision = abi.TT_PREC_BF16_TC
+    rows = [int(__import__("numpy").prod(x)) for x in n]
+    with pytest.raises(abi.TTEmbError) as e:
+        abi.tt_emb_create(n, rows, d, r, o)
+    assert e.value.code == abi.TT_ERR_SHAPE

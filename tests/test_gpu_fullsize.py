@@ -1,0 +1,135 @@
+"""Parity at the benchmark sizes, in the launch configuration bench.py times.
+
+The oracle cannot run a whole step at these sizes, so the tests check
+  * sampled bags: the GPU rows of a seeded sample of bags (plus the largest bags)
+    against the oracle run on exactly those bags;
+  * a property of the backward that holds at any size: every pooled output is linear
+    in each core, so for each table t and core j
+        <dG_{t,j}, G_{t,j}> = <grad_out[:, t], out[:, t]>
+    (Euler's identity for a function homogeneous of degree one in G_{t,j}).  The
+    difference is measured against ||dG|| ||G|| + ||grad_out[:, t]|| ||out[:, t]||, the
+    Cauchy-Schwarz bounds of the two inner products, so cancellation inside them does
+    not inflate it.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from tests.parity import FP32_TOL, output_err
+from workloads import config_workload, sub_batch
+
+pytestmark = pytest.mark.gpu
+
+BF16_TOL = 2e-2
+
+
+def _sample_bags(w, n=48, seed=5):
+    rng = np.random.default_rng(seed)
+    sizes = np.diff(w.offsets).reshape(w.num_tables, w.batch).sum(axis=0)
+    heavy = np.argsort(sizes)[-8:]
+    return np.unique(np.concatenate([rng.choice(w.batch, size=n, replace=False), heavy]))
+
+
+def _forward_full(w, options=None):
+    import torch
+    from tensor_train_compressed_mixed_b200 import from_workload
+    emb, cores, idx, off = from_workload(w, options=options, with_grads=w.grad_out is not None)
+    emb.reserve(w.num_lookups, w.batch)
+    out = torch.empty(w.batch, w.num_tables * w.dim, dtype=torch.float32, device="cuda")
+    emb.forward(idx, off, w.batch, out)
+    emb.sync()
+    return emb, cores, out
+
+
+@pytest.mark.parametrize("cfg", [4, 5])
+def test_full_size_forward_sampled_bags(cfg):
+    w = config_workload(cfg, with_grad=False)
+    emb, cores, out = _forward_full(w)
+    bags = _sample_bags(w)
+    got = out.cpu().numpy()[bags]
+    want = oracle.workload_forward(sub_batch(w, bags))
+    assert output_err(got, want, w.dim) <= FP32_TOL
+    emb.close()
+
+
+@pytest.mark.parametrize("cfg", [3, 4])
+def test_full_size_bf16_forward_sampled_bags(cfg):
+    from tensor_train_compressed_mixed_b200 import abi
+    w = config_workload(cfg, with_grad=False)
+    o = abi.tt_emb_default_options()
+    o.precision = abi.TT_PREC_BF16_TC
+    emb, cores, out = _forward_full(w, o)
+    bags = _sample_bags(w)
+    got = out.cpu().numpy()[bags]
+    want = oracle.workload_forward(sub_batch(w, bags))
+    assert output_err(got, want, w.dim) <= BF16_TOL
+    emb.close()
+
+
+@pytest.mark.parametrize("cfg", [4, 5])
+def test_full_size_backward_euler_identity(cfg):
+    import torch
+    w = config_workload(cfg, with_grad=True)
+    emb, cores, out = _forward_full(w)
+    g = torch.from_numpy(w.grad_out).cuda()
+    emb.backward(g)
+    emb.sync()
+    o64 = out.double().reshape(w.batch, w.num_tables, w.dim)
+    g64 = g.double().reshape(w.batch, w.num_tables, w.dim)
+    lhs_all = (o64 * g64).sum(dim=(0, 2)).cpu().numpy()
+    lhs_scale = (o64.pow(2).sum(dim=(0, 2)).sqrt() * g64.pow(2).sum(dim=(0, 2)).sqrt()).cpu().numpy()
+    worst = 0.0
+    for t in range(w.num_tables):
+        for j in range(w.num_cores):
+            G = cores[t][j].double()
+            dG = emb.grads[t * w.num_cores + j].double()
+            val = float((G * dG).sum())
+            scale = float(G.norm() * dG.norm()) + float(lhs_scale[t])
+            assert scale > 0, (t, j)
+            worst = max(worst, abs(val - lhs_all[t]) / scale)
+    assert worst <= FP32_TOL, worst
+    emb.close()
+
+
+def _digit_of(idx, n, j):
+    stride = int(np.prod(n[j + 1:])) if j + 1 < len(n) else 1
+    return (idx // stride) % n[j]
+
+
+def _restrict(w, t, j, digit):
+    """The lookups of table t whose core-j digit is `digit`, with the same bags and grad_out."""
+    from workloads.gen import Workload
+    T, B = w.num_tables, w.batch
+    parts, sizes = [], np.zeros(T * B, dtype=np.int64)
+    lo_t, hi_t = w.offsets[t * B], w.offsets[(t + 1) * B]
+    seg = w.indices[lo_t:hi_t]
+    keep = _digit_of(seg, w.n[t], j) == digit
+    bag = np.repeat(np.arange(B), np.diff(w.offsets[t * B:(t + 1) * B + 1]))
+    sizes[t * B:(t + 1) * B] = np.bincount(bag[keep], minlength=B)
+    offsets = np.zeros(T * B + 1, dtype=np.int64)
+    np.cumsum(sizes, out=offsets[1:])
+    return Workload(name=w.name + "_slice", d=w.d, r=w.r, n=w.n, n_rows=w.n_rows, batch=B,
+                    indices=seg[keep].astype(np.int64), offsets=offsets, cores=w.cores,
+                    grad_out=w.grad_out, lr=w.lr, train=w.train, meta=dict(w.meta))
+
+
+def test_full_size_backward_sampled_slices():
+    """Whole digit slices dG_{t,j}[:, i] of the rank-64 training step: only the lookups
+    with digit i touch the slice, so the oracle run on those lookups alone gives it."""
+    import torch
+    from tests.parity import core_grad_err
+    w = config_workload(4, with_grad=True)
+    emb, cores, out = _forward_full(w)
+    g = torch.from_numpy(w.grad_out).cuda()
+    emb.backward(g)
+    emb.sync()
+    t = int(np.argmin([np.prod(x) for x in w.n]))   # the smallest table: fewest lookups per slice
+    rng = np.random.default_rng(11)
+    for j in range(w.num_cores):
+        digit = int(rng.integers(0, w.n[t][j]))
+        sub = _restrict(w, t, j, digit)
+        assert sub.num_lookups > 0
+        want = oracle.workload_backward(sub)[t][j][:, digit:digit + 1]
+        got = emb.grads[t * w.num_cores + j][:, digit:digit + 1].cpu().numpy()
+        assert core_grad_err(got, want) <= FP32_TOL, (j, digit)
+    emb.close()

@@ -1,0 +1,95 @@
+"""Parity of the bf16 tensor-core forward (TT_PREC_BF16_TC) with the fp64 oracle.
+
+The prefix contraction C_p = G_1[0, i_1] . G_2[:, i_2] runs on tcgen05 with bf16
+operands and fp32 accumulation in tensor memory; the bound is the pages' 2e-2 for a
+bf16 tensor-core step, read normwise per bag row like the fp32 bound (tests/parity.py).
+The backward stays fp32 and does not read the forward's rows, so its gradients must
+agree with the fp32 handle's up to the order of the floating-point reductions (the
+first and last core gradients are accumulated with vector atomics).  Shapes: the two supported ones, with factors
+that give several chunks per column group, ragged and empty bags.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from tests.parity import FP32_TOL, core_grad_err, gpu_forward, gpu_train_step, output_err
+from workloads import config_workload, random_workload
+
+pytestmark = pytest.mark.gpu
+
+BF16_TOL = 2e-2
+
+TC_SHAPES = [
+    # d, r, n per table, rows per table, batch
+    ((4, 4, 8), (1, 64, 64, 1), [(40, 3, 17), (9, 5, 11)], None, 300),
+    ((4, 4, 8), (1, 32, 32, 1), [(70, 2, 13), (25, 7, 9), (3, 3, 3)], [1800, 1500, 20], 200),
+]
+
+
+def _opts(precision):
+    from tensor_train_compressed_mixed_b200 import abi
+    o = abi.tt_emb_default_options()
+    o.precision = precision
+    return o
+
+
+@pytest.mark.parametrize("case", range(len(TC_SHAPES)))
+def test_bf16_forward_matches_oracle(case):
+    from tensor_train_compressed_mixed_b200 import abi
+    d, r, n, rows, batch = TC_SHAPES[case]
+    w = random_workload(900 + case, d, r, n, rows, batch=batch,
+                        pooling={"kind": "uniform", "lo": 0, "hi": 40}, with_grad=False)
+    emb, cores, out = gpu_forward(w, options=_opts(abi.TT_PREC_BF16_TC))
+    got = out.cpu().numpy()
+    want = oracle.workload_forward(w)
+    err = output_err(got, want, w.dim)
+    assert err <= BF16_TOL, err
+    # bf16 rounding is visible: the result is not the fp32 one
+    emb32, _, out32 = gpu_forward(w)
+    assert output_err(out32.cpu().numpy(), want, w.dim) <= FP32_TOL
+    assert not np.array_equal(got, out32.cpu().numpy())
+
+
+@pytest.mark.parametrize("cfg,batch,tables", [(3, 64, 4), (4, 40, 3)])
+def test_bf16_forward_benchmark_shapes(cfg, batch, tables):
+    from tensor_train_compressed_mixed_b200 import abi
+    w = config_workload(cfg, batch=batch, tables=tables, with_grad=False)
+    emb, cores, out = gpu_forward(w, options=_opts(abi.TT_PREC_BF16_TC))
+    err = output_err(out.cpu().numpy(), oracle.workload_forward(w), w.dim)
+    assert err <= BF16_TOL, err
+
+
+def test_bf16_training_step_keeps_fp32_backward():
+    from tensor_train_compressed_mixed_b200 import abi
+    w = config_workload(4, batch=24, tables=3, with_grad=True)
+    _, out_tc, g_tc, new_tc = gpu_train_step(w, options=_opts(abi.TT_PREC_BF16_TC), lr=0.01)
+    _, out_32, g_32, new_32 = gpu_train_step(w, lr=0.01)
+    for t in range(w.num_tables):
+        for j in range(w.num_cores):
+            assert core_grad_err(g_tc[t][j], g_32[t][j]) <= 1e-5, (t, j)
+            assert core_grad_err(new_tc[t][j], new_32[t][j]) <= 1e-5, (t, j)
+    want = oracle.workload_backward(w)
+    for t in range(w.num_tables):
+        for j in range(w.num_cores):
+            assert core_grad_err(g_tc[t][j], want[t][j]) <= FP32_TOL, (t, j)
+    assert output_err(out_tc, oracle.workload_forward(w), w.dim) <= BF16_TOL
+
+
+def test_bf16_all_bags_empty():
+    from tensor_train_compressed_mixed_b200 import abi
+    w = random_workload(950, (4, 4, 8), (1, 64, 64, 1), [(5, 6, 7)], batch=16,
+                        pooling={"kind": "uniform", "lo": 0, "hi": 0}, with_grad=False)
+    assert w.num_lookups == 0
+    emb, cores, out = gpu_forward(w, options=_opts(abi.TT_PREC_BF16_TC))
+    assert not out.cpu().numpy().any()
+
+
+def test_bf16_scheduler_modes_agree_bitwise():
+    from tensor_train_compressed_mixed_b200 import abi
+    w = config_workload(3, batch=48, tables=4, with_grad=False)
+    outs = []
+    for sched in (abi.TT_SCHED_STATIC, abi.TT_SCHED_STEAL, abi.TT_SCHED_STEAL_L2):
+        o = _opts(abi.TT_PREC_BF16_TC)
+        o.sched = sched
+        outs.append(gpu_forward(w, options=o)[2].cpu().numpy())
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2])
