@@ -15,7 +15,7 @@ struct Layout {
         uniq_start, grp_start, bag_sorted;
     // specialised path only (zero when unused)
     size_t uid_at_pos, uid_sorted, rowbuf, pkeys[2], pvals[2], col_count, col_start, chunk_base,
-        hdr, chunks, tasks, g12, dg12, g3t, bf1, bf2;
+        hdr, chunks, tasks, grec, g12, dg12, g3t, bf1, bf2;
     int64_t chunk_cap, task_cap;
     size_t total;
 };
@@ -72,6 +72,7 @@ Layout make_layout(int key_bytes, int64_t L, int64_t B, const FastDims& f)
         y.chunks = take((size_t)y.chunk_cap * sizeof(int4));
         y.task_cap = y.chunk_cap + (int64_t)f.T * ceil_div(B, kPoolBags);
         y.tasks = take((size_t)y.task_cap * 4);
+        y.grec = take(Lz * sizeof(int4));
         if (f.g12_floats > 0) {
             y.g12 = take((size_t)f.g12_floats * 4);
             y.dg12 = take((size_t)f.g12_floats * 4);
@@ -339,6 +340,7 @@ struct tt_emb_handle {
         pb.hdr = (PlanHeader*)at(lay.hdr);
         pb.chunks = (int4*)at(lay.chunks);
         pb.tasks = (int32_t*)at(lay.tasks);
+        pb.grec = (int4*)at(lay.grec);
         return pb;
     }
 
@@ -358,6 +360,7 @@ struct tt_emb_handle {
         a.uid_sorted = (const int32_t*)at(lay.uid_sorted);
         a.counters = (const WsCounters*)at(lay.counters);
         a.pb = pb;
+        a.grec = pb ? pb->grec : nullptr;
         a.offsets = offsets;
         a.rowbuf = (float*)at(lay.rowbuf);
         a.L = L;

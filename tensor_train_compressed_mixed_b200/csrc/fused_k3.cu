@@ -65,6 +65,7 @@ constexpr int kBwdThreads = 256;  // backward: 8 warps, up to 255 registers per 
 constexpr int kNB = kPoolBags;    // bags per pooling task
 constexpr int kHChunk = 256;      // sorted lookups per upstream-sum warp
 constexpr int kSpinLimit = 1 << 22;
+constexpr int kKeyCap = 256;      // distinct rows per chunk whose keys are staged with the chunk
 
 template <int D1_, int D2_, int D3_, int R_>
 struct S3 {
@@ -96,6 +97,7 @@ struct S3 {
     static_assert(N >= 32 && N % 32 == 0, "swizzle needs N >= 32");
     static_assert(MF % 4 == 0 && (MF / 4) * (N / 8) == kFwdThreads, "forward GEMM tiling (4 x 8 per thread)");
     static_assert((2048 / R / 4) * (N / 8) == kBwdThreads, "backward GEMM tiling (4 x 8 per thread)");
+    static_assert((MF / 4) % 4 == 0 && (MB / 4) % 4 == 0 && (N / 8) % 8 == 0, "warps of 4 x 8 thread tiles");
     static_assert(DBC % 4 == 0, "dB columns in float4 chunks");
     static_assert(NUB >= 1 && NUB * TPUB == kBwdThreads, "backward batch tiling");
 
@@ -147,11 +149,29 @@ __device__ __forceinline__ float f4get(const float4& v, int i)
     return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
 }
 
+// Thread tile coordinates of a register-tiled GEMM with TN tiles across N: each warp
+// covers 4 tile rows x 8 tile columns, so one fragment load of A touches 4 rows and one
+// of B 8 consecutive 16-byte chunks (one shared-memory wavefront each) instead of 32.
+template <int TN>
+__device__ __forceinline__ void warp_tile_2d(int tid, int& tm, int& tn)
+{
+    static_assert(TN % 8 == 0, "tile columns in groups of 8");
+    const int warp = tid >> 5, lane = tid & 31;
+    tm = (warp / (TN / 8)) * 4 + (lane >> 3);
+    tn = (warp % (TN / 8)) * 8 + (lane & 7);
+}
+
 // 16-byte asynchronous global -> shared copies (L2 only), grouped and awaited
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
 {
     const unsigned a = (unsigned)__cvta_generic_to_shared(smem);
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(a), "l"(gmem) : "memory");
+}
+template <typename K>
+__device__ __forceinline__ void cp_async_key(K* smem, const K* gmem)   // 4- or 8-byte copy (L1 path)
+{
+    const unsigned a = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(a), "l"(gmem), "n"(sizeof(K)) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
@@ -291,31 +311,33 @@ struct FwdMeta {   // shared-memory metadata of a chunk (double buffered)
     int flag;
 };
 
-// metadata of chunk `cid` into buffer mb (all threads call; ends with a barrier)
+// Index of the prefix (0..cnt-1) holding the chunk's distinct row number kq.
+__device__ __forceinline__ int prefix_of(const int* ucum, int cnt, int kq)
+{
+    int j = 0;
+    while (j + 1 < cnt && ucum[j + 1] <= kq) ++j;
+    return j;
+}
+
+// Metadata of chunk `cid` into buffer mb (all threads call; ends with a barrier), and
+// asynchronous copies of the keys of its first kKeyCap distinct rows into keys[mb]; those
+// join the caller's next commit group (the chunk's A/B copies).
 template <class S, typename K>
 __device__ __forceinline__ void fwd_meta(const CoreParams& cp, int cid, int mb, const K* __restrict__ uniq_keys,
-                                         const int32_t* __restrict__ grp_start,
-                                         const int32_t* __restrict__ sorted_groups,
-                                         const int4* __restrict__ chunks, FwdMeta<S>& M)
+                                         const int4* __restrict__ grec, const int4* __restrict__ chunks,
+                                         FwdMeta<S>& M, K* keys)
 {
     const int tid = threadIdx.x;
     const int4 ch = chunks[cid];
-    const int t = ch.z;
     if (tid < S::MPF) {
-        int u0 = 0, nu = 0, i1 = 0;
-        if (tid < ch.y) {
-            const int g = sorted_groups[ch.x + tid];
-            u0 = grp_start[g];
-            nu = grp_start[g + 1] - u0;
-            i1 = (int)(key_row(uniq_keys[u0], cp.ibits) / cp.n[t][2] / cp.n[t][1]);
-        }
-        M.u0[mb][tid] = u0;
-        M.ucum[mb][tid] = nu;
-        M.i1[mb][tid] = i1;
+        const int4 g = tid < ch.y ? grec[ch.x + tid] : make_int4(0, 0, 0, 0);
+        M.u0[mb][tid] = g.x;
+        M.ucum[mb][tid] = g.y;
+        M.i1[mb][tid] = g.z;
     }
     if (tid == 0) {
         M.cnt[mb] = ch.y;
-        M.t[mb] = t;
+        M.t[mb] = ch.z;
         M.i2[mb] = ch.w;
     }
     __syncthreads();
@@ -329,6 +351,11 @@ __device__ __forceinline__ void fwd_meta(const CoreParams& cp, int cid, int mb, 
         M.ucum[mb][S::MPF] = run;
     }
     __syncthreads();
+    const int nk = min(M.ucum[mb][S::MPF], kKeyCap);
+    for (int kq = tid; kq < nk; kq += kFwdThreads) {
+        const int j = prefix_of(M.ucum[mb], M.cnt[mb], kq);
+        cp_async_key(keys + mb * kKeyCap + kq, uniq_keys + M.u0[mb][j] + (kq - M.ucum[mb][j]));
+    }
 }
 
 // asynchronous copies of the chunk's A rows (and B when its column changes); one commit group
@@ -366,7 +393,8 @@ __device__ __forceinline__ void fwd_gemm(const FwdSmem<S>& sm)
 {
     constexpr int R = S::R, N = S::N;
     constexpr int TN = N / 8;
-    const int tn = threadIdx.x % TN, tm = threadIdx.x / TN;
+    int tm, tn;
+    warp_tile_2d<TN>(threadIdx.x, tm, tn);
     int rows[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) rows[i] = tm * 4 + i;
@@ -481,11 +509,13 @@ __device__ __forceinline__ bool fwd_gemm_tc(const FwdSmem<S>& sm, uint32_t tmem,
     return true;
 }
 
-// distinct rows k0..k0+nb of the chunk into batch buffer bb; issues their last slices (one commit group)
+// distinct rows k0..k0+nb of the chunk into batch buffer bb; issues their last slices (one
+// commit group).  Row keys come from the chunk's staged keys (landed and made visible by the
+// caller) for the first kKeyCap rows, from global memory beyond.
 template <class S, typename K>
 __device__ __forceinline__ void fwd_issue_batch(const CoreParams& cp, int mb, int k0, int bb,
                                                 const K* __restrict__ uniq_keys, FwdMeta<S>& M,
-                                                const FwdSmem<S>& sm)
+                                                const FwdSmem<S>& sm, const K* keys)
 {
     constexpr int R = S::R, D3 = S::D3;
     const int tid = threadIdx.x;
@@ -495,12 +525,12 @@ __device__ __forceinline__ void fwd_issue_batch(const CoreParams& cp, int mb, in
     const uint32_t n3 = cp.n[t][2];
     if (tid < nb) {
         const int kq = k0 + tid;
-        int j = 0;
-        while (j + 1 < M.cnt[mb] && M.ucum[mb][j + 1] <= kq) ++j;
+        const int j = prefix_of(M.ucum[mb], M.cnt[mb], kq);
         const int u = M.u0[mb][j] + (kq - M.ucum[mb][j]);
+        const K key = kq < kKeyCap ? keys[mb * kKeyCap + kq] : uniq_keys[u];
         M.bu[bb][tid] = u;
         M.bp[bb][tid] = j;
-        M.bi3[bb][tid] = (int)(key_row(uniq_keys[u], cp.ibits) % n3);
+        M.bi3[bb][tid] = (int)(key_row(key, cp.ibits) % n3);
     }
     __syncthreads();
     const float* G3t = cp.last_t[t];   // [n3][R][D3]: one row's slice is contiguous
@@ -618,13 +648,14 @@ __device__ void fwd_pool(const CoreParams& cp, int ptask, int nP, const int32_t*
 template <class S, typename K, bool TC>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
-              const int32_t* __restrict__ grp_start, const int32_t* __restrict__ uid_at_pos,
-              const int64_t* __restrict__ offsets, const int32_t* __restrict__ sorted_groups,
-              const int4* __restrict__ chunks, const int32_t* __restrict__ tasks, PlanHeader* hdr,
+              const int4* __restrict__ grec, const int32_t* __restrict__ uid_at_pos,
+              const int64_t* __restrict__ offsets, const int4* __restrict__ chunks,
+              const int32_t* __restrict__ tasks, PlanHeader* hdr,
               float* __restrict__ rowbuf, float* __restrict__ out, int32_t* status)
 {
     extern __shared__ __align__(16) float smem_f[];
     __shared__ FwdMeta<S> M;
+    __shared__ __align__(16) K s_keys[2 * kKeyCap];   // keys of each chunk buffer's first rows
     __shared__ __align__(8) uint64_t s_mbar;
     __shared__ uint32_t s_tmem;
     __shared__ int s_ok;
@@ -674,18 +705,17 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
         }
         TT_PH_START();
         if (!staged) {
-            fwd_meta<S, K>(cp, tv, mb, uniq_keys, grp_start, sorted_groups, chunks, M);
+            fwd_meta<S, K>(cp, tv, mb, uniq_keys, grec, chunks, M, s_keys);
             if constexpr (TC) fwd_issue_ab_tc<S>(cp, mb, M, sm, cur_t, cur_i2);
             else fwd_issue_ab<S>(cp, mb, M, sm, cur_t, cur_i2);
         }
-        // the first batch of last slices is in flight during the GEMM
-        const int total = M.ucum[mb][S::MPF];
-        if (total > 0) fwd_issue_batch<S, K>(cp, mb, 0, 0, uniq_keys, M, sm);
         if (tid == 0) M.task[1] = next_task(sched, &hdr->queue_head, iter);   // result used after the GEMM
         ++iter;
-        if (total > 0) cp_async_wait<1>();   // A/B landed; the batch may still be in flight
-        else cp_async_wait_all();
+        cp_async_wait_all();   // the chunk's A/B rows and row keys (usually prefetched long ago)
         __syncthreads();
+        // the first batch of last slices is in flight during the GEMM
+        const int total = M.ucum[mb][S::MPF];
+        if (total > 0) fwd_issue_batch<S, K>(cp, mb, 0, 0, uniq_keys, M, sm, s_keys);
         TT_PH(0);
         if constexpr (TC) {
             if (!fwd_gemm_tc<S>(sm, tmem, &s_mbar, parity, &s_ok)) {
@@ -700,7 +730,7 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
         const int qn = M.task[1];
         const bool next_chunk = qn < ntasks && tasks[qn] >= 0;
         if (next_chunk) {
-            fwd_meta<S, K>(cp, tasks[qn], mb ^ 1, uniq_keys, grp_start, sorted_groups, chunks, M);
+            fwd_meta<S, K>(cp, tasks[qn], mb ^ 1, uniq_keys, grec, chunks, M, s_keys);
             if constexpr (TC) fwd_issue_ab_tc<S>(cp, mb ^ 1, M, sm, cur_t, cur_i2);
             else fwd_issue_ab<S>(cp, mb ^ 1, M, sm, cur_t, cur_i2);
         }
@@ -710,7 +740,7 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
             for (int k0 = 0, b = 0; k0 < total; k0 += S::NUF, b ^= 1) {
                 const bool more = k0 + S::NUF < total;
                 if (more) {
-                    fwd_issue_batch<S, K>(cp, mb, k0 + S::NUF, b ^ 1, uniq_keys, M, sm);
+                    fwd_issue_batch<S, K>(cp, mb, k0 + S::NUF, b ^ 1, uniq_keys, M, sm, s_keys);
                     cp_async_wait<1>();
                 } else if (k0 == 0 && next_chunk) {
                     cp_async_wait<1>();
@@ -725,7 +755,7 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
             }
         } else {
             for (int k0 = 0; k0 < total; k0 += S::NUF) {
-                if (k0 > 0) fwd_issue_batch<S, K>(cp, mb, k0, 0, uniq_keys, M, sm);
+                if (k0 > 0) fwd_issue_batch<S, K>(cp, mb, k0, 0, uniq_keys, M, sm, s_keys);
                 if (k0 == 0 && next_chunk) cp_async_wait<1>();
                 else cp_async_wait_all();
                 __syncthreads();
@@ -845,25 +875,20 @@ struct BwdMeta {
     int task;
 };
 
-// chunk metadata (groups cfirst+j0 .. +MPB of the column) into buffer mb; ends with a barrier
+// chunk metadata (groups cfirst+j0 .. +MPB of the column, from the plan's per-group records)
+// into buffer mb, ending with a barrier; then asynchronous copies of the keys of its first
+// kKeyCap distinct rows into keys[mb], which join the caller's next commit group
 template <class S, typename K>
-__device__ __forceinline__ void bwd_meta(const CoreParams& cp, int t, int cfirst, int j0, int ccount, int mb,
-                                         const K* __restrict__ uniq_keys, const int32_t* __restrict__ grp_start,
-                                         const int32_t* __restrict__ sorted_groups, BwdMeta<S>& M)
+__device__ __forceinline__ void bwd_meta(int cfirst, int j0, int ccount, int mb, const K* __restrict__ uniq_keys,
+                                         const int4* __restrict__ grec, BwdMeta<S>& M, K* keys)
 {
     const int tid = threadIdx.x;
     const int cnt = min(S::MPB, ccount - j0);
     if (tid < S::MPB) {
-        int u0 = 0, nu = 0, i1 = 0;
-        if (tid < cnt) {
-            const int g = sorted_groups[cfirst + j0 + tid];
-            u0 = grp_start[g];
-            nu = grp_start[g + 1] - u0;
-            i1 = (int)(key_row(uniq_keys[u0], cp.ibits) / cp.n[t][2] / cp.n[t][1]);
-        }
-        M.u0[mb][tid] = u0;
-        M.ucum[mb][tid] = nu;
-        M.i1[mb][tid] = i1;
+        const int4 g = tid < cnt ? grec[cfirst + j0 + tid] : make_int4(0, 0, 0, 0);
+        M.u0[mb][tid] = g.x;
+        M.ucum[mb][tid] = g.y;
+        M.i1[mb][tid] = g.z;
     }
     if (tid == 0) M.cnt[mb] = cnt;
     __syncthreads();
@@ -877,6 +902,11 @@ __device__ __forceinline__ void bwd_meta(const CoreParams& cp, int t, int cfirst
         M.ucum[mb][S::MPB] = run;
     }
     __syncthreads();
+    const int nk = min(M.ucum[mb][S::MPB], kKeyCap);
+    for (int kq = tid; kq < nk; kq += kBwdThreads) {
+        const int j = prefix_of(M.ucum[mb], cnt, kq);
+        cp_async_key(keys + mb * kKeyCap + kq, uniq_keys + M.u0[mb][j] + (kq - M.ucum[mb][j]));
+    }
 }
 
 template <class S>
@@ -899,7 +929,7 @@ __device__ __forceinline__ void bwd_issue_a(const CoreParams& cp, int t, int mb,
 template <class S, typename K>
 __device__ __forceinline__ void bwd_issue_batch(const CoreParams& cp, int t, int mb, int k0, int bb,
                                                 const K* __restrict__ uniq_keys, const float* __restrict__ rowbuf,
-                                                BwdMeta<S>& M, float* Hs, float* Ss)
+                                                BwdMeta<S>& M, float* Hs, float* Ss, const K* keys)
 {
     constexpr int R = S::R, D3 = S::D3, P = S::P, SR = S::SR;
     const int tid = threadIdx.x;
@@ -908,12 +938,12 @@ __device__ __forceinline__ void bwd_issue_batch(const CoreParams& cp, int t, int
     const uint32_t n3 = cp.n[t][2];
     if (tid < nb) {
         const int kq = k0 + tid;
-        int j = 0;
-        while (j + 1 < M.cnt[mb] && M.ucum[mb][j + 1] <= kq) ++j;
+        const int j = prefix_of(M.ucum[mb], M.cnt[mb], kq);
         const int u = M.u0[mb][j] + (kq - M.ucum[mb][j]);
+        const K key = kq < kKeyCap ? keys[mb * kKeyCap + kq] : uniq_keys[u];
         M.bu[bb][tid] = u;
         M.bp[bb][tid] = j;
-        M.bi3[bb][tid] = (int)(key_row(uniq_keys[u], cp.ibits) % n3);
+        M.bi3[bb][tid] = (int)(key_row(key, cp.ibits) % n3);
     }
     __syncthreads();
     float* H = Hs + (size_t)bb * S::NUB * P * D3;
@@ -934,14 +964,15 @@ __device__ __forceinline__ void bwd_issue_batch(const CoreParams& cp, int t, int
 template <class S, typename K>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ uniq_keys,
-              const int32_t* __restrict__ grp_start, const int32_t* __restrict__ sorted_groups,
-              const int32_t* __restrict__ col_count, const int32_t* __restrict__ col_start,
-              PlanHeader* hdr, const float* __restrict__ rowbuf, int32_t* status)
+              const int4* __restrict__ grec, const int32_t* __restrict__ col_count,
+              const int32_t* __restrict__ col_start, PlanHeader* hdr, const float* __restrict__ rowbuf,
+              int32_t* status)
 {
     constexpr int R = S::R, N = S::N, MB = S::MB, MPB = S::MPB, D1 = S::D1, D2 = S::D2, D3 = S::D3,
                   P = S::P, NUB = S::NUB, DBR = S::DBR, DBC = S::DBC, SR = S::SR;
     extern __shared__ __align__(16) float smem_f[];
     __shared__ BwdMeta<S> M;
+    __shared__ __align__(16) K s_keys[2 * kKeyCap];   // keys of each chunk buffer's first rows
     float* Bs = smem_f;                    // [R][N] swizzled (key row/4)
     float* As = Bs + R * N;                // [2][MB][R] swizzled rows
     float* Cn = As + 2 * MB * R;           // [MB][N] swizzled (key row)
@@ -980,7 +1011,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                 cp_async16(&Bs[swz_b<N>(rho, c4 * 4)], G2 + rho * rs + c4 * 4);
             }
         }
-        bwd_meta<S, K>(cp, t, cfirst, 0, ccount, 0, uniq_keys, grp_start, sorted_groups, M);
+        bwd_meta<S, K>(cfirst, 0, ccount, 0, uniq_keys, grec, M, s_keys);
         bwd_issue_a<S>(cp, t, 0, M, As);
         TT_PH(8);
 
@@ -997,20 +1028,21 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
         for (int j0 = 0; j0 < ccount; j0 += MPB, mb ^= 1) {
             const int cnt = M.cnt[mb];
             const float* Ab = As + mb * MB * R;
+            cp_async_wait_all();   // B, this chunk's A rows and row keys (usually prefetched long ago)
+            __syncthreads();
             // the first batch of distinct rows is in flight during the C GEMM
             const int total = M.ucum[mb][MPB];
-            if (total > 0) bwd_issue_batch<S, K>(cp, t, mb, 0, 0, uniq_keys, rowbuf, M, Hs, Ss);
+            if (total > 0) bwd_issue_batch<S, K>(cp, t, mb, 0, 0, uniq_keys, rowbuf, M, Hs, Ss, s_keys);
             for (int q = tid; q < MB * N / 4; q += kBwdThreads)
                 reinterpret_cast<float4*>(dCn)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (total > 0) cp_async_wait<1>();   // B and A landed; the batch may still be in flight
-            else cp_async_wait_all();
             __syncthreads();
             TT_PH(9);
 
             // C_all = A . B  (MB x N): thread tile 4 rows x 8 cols
             {
                 constexpr int TN = N / 8;
-                const int tn = tid % TN, tm = tid / TN;   // tm < MB / 4
+                int tm, tn;   // tm < MB / 4
+                warp_tile_2d<TN>(tid, tm, tn);
                 float acc[4][8];
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
@@ -1049,7 +1081,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             // next chunk's metadata and A rows go in flight while this chunk's rows are processed
             const bool more = j0 + MPB < ccount;
             if (more) {
-                bwd_meta<S, K>(cp, t, cfirst, j0 + MPB, ccount, mb ^ 1, uniq_keys, grp_start, sorted_groups, M);
+                bwd_meta<S, K>(cfirst, j0 + MPB, ccount, mb ^ 1, uniq_keys, grec, M, s_keys);
                 bwd_issue_a<S>(cp, t, mb ^ 1, M, As + (mb ^ 1) * MB * R);
             }
 
@@ -1058,7 +1090,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             for (int k0 = 0, bb = 0; k0 < total; k0 += NUB, bb ^= 1) {
                 const int nb = min(NUB, total - k0);
                 if (k0 + NUB < total) {
-                    bwd_issue_batch<S, K>(cp, t, mb, k0 + NUB, bb ^ 1, uniq_keys, rowbuf, M, Hs, Ss);
+                    bwd_issue_batch<S, K>(cp, t, mb, k0 + NUB, bb ^ 1, uniq_keys, rowbuf, M, Hs, Ss, s_keys);
                     cp_async_wait<1>();
                 } else if (k0 == 0 && more) {
                     cp_async_wait<1>();
@@ -1350,8 +1382,8 @@ cudaError_t fwd_launch(const K3Args& a, float* out, cudaStream_t s, int* nl)
     if (e != cudaSuccess) return e;
     const PlanBuffers& pb = *a.pb;
     k3_fwd_kernel<S, K, TC><<<a.grid, kFwdThreads, smem, s>>>(
-        *a.cp, a.pp->sched, (const K*)a.uniq_keys, a.grp_start, a.uid_at_pos, a.offsets,
-        pb.sorted_groups, pb.chunks, pb.tasks, pb.hdr, a.rowbuf, out, a.status);
+        *a.cp, a.pp->sched, (const K*)a.uniq_keys, a.grec, a.uid_at_pos, a.offsets,
+        pb.chunks, pb.tasks, pb.hdr, a.rowbuf, out, a.status);
     *nl += 1;
     return cudaGetLastError();
 }
@@ -1377,8 +1409,8 @@ cudaError_t bwd_launch(const K3Args& a, const GradPtrs& gp, const float* grad_ou
     if (e != cudaSuccess) return e;
     const PlanBuffers& pb = *a.pb;
     k3_bwd_kernel<S, K><<<a.grid, kBwdThreads, smem, s>>>(
-        *a.cp, gp, *a.pp, (const K*)a.uniq_keys, a.grp_start, pb.sorted_groups, pb.col_count,
-        pb.col_start, pb.hdr, a.rowbuf, a.status);
+        *a.cp, gp, *a.pp, (const K*)a.uniq_keys, a.grec, pb.col_count, pb.col_start, pb.hdr, a.rowbuf,
+        a.status);
     *nl += 1;
     return cudaGetLastError();
 }

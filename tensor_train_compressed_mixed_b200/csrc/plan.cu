@@ -179,6 +179,29 @@ __global__ void __launch_bounds__(256) k_plan_chunks(PlanParams pp, const WsCoun
     }
 }
 
+// Per sorted group position: first distinct row, row count and the first digit of the
+// three-core view (i_1 = row / (n_2 n_3)), so that the fused kernels read a chunk's
+// metadata with one load per group instead of a chain of three dependent loads.
+template <typename K>
+__global__ void __launch_bounds__(256) k_plan_grec(PlanParams pp, const WsCounters* __restrict__ counters,
+                                                   const int32_t* __restrict__ sorted_groups,
+                                                   const int32_t* __restrict__ grp_start,
+                                                   const K* __restrict__ uniq_keys, int4* __restrict__ grec,
+                                                   const int32_t* status)
+{
+    if (has_error(status)) return;
+    const int64_t G = counters->num_groups;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < G; i += (int64_t)gridDim.x * blockDim.x) {
+        const int g = sorted_groups[i];
+        const int u0 = grp_start[g];
+        const uint64_t key = (uint64_t)uniq_keys[u0];
+        const int t = (int)(key >> pp.ibits);
+        const uint32_t row = (uint32_t)(key & ((uint64_t(1) << pp.ibits) - 1));
+        const uint32_t i1 = row / pp.n[t][pp.k - 1] / pp.n[t][pp.k - 2];
+        grec[i] = make_int4(u0, grp_start[g + 1] - u0, (int)i1, 0);
+    }
+}
+
 cudaError_t launch_plan(const PlanParams& pp, bool key64, const void* uniq_keys,
                         const int32_t* grp_start, const WsCounters* counters, int64_t max_groups,
                         PlanBuffers& pb, int32_t* status, cudaStream_t s, int* nl)
@@ -205,7 +228,13 @@ cudaError_t launch_plan(const PlanParams& pp, bool key64, const void* uniq_keys,
     k_plan_cols<<<1, 1024, 0, s>>>(pp, pb.col_count, pb.col_start, pb.chunk_base, pb.hdr, status);
     k_plan_chunks<<<grid, 256, 0, s>>>(pp, counters, (const uint32_t*)pb.sort.keys[which], pb.col_count,
                                        pb.col_start, pb.chunk_base, pb.hdr, pb.chunks, pb.tasks, status);
-    *nl += 2;
+    if (key64)
+        k_plan_grec<uint64_t><<<grid, 256, 0, s>>>(pp, counters, pb.sorted_groups, grp_start,
+                                                   (const uint64_t*)uniq_keys, pb.grec, status);
+    else
+        k_plan_grec<uint32_t><<<grid, 256, 0, s>>>(pp, counters, pb.sorted_groups, grp_start,
+                                                   (const uint32_t*)uniq_keys, pb.grec, status);
+    *nl += 3;
     return cudaGetLastError();
 }
 

@@ -124,6 +124,8 @@ struct PlanBuffers {
     PlanHeader* hdr;
     int4* chunks;                  // (first sorted position, groups, table, column digit)
     int32_t* tasks;                // >= 0: chunk id; < 0: pooling task -1 - (t * nP + j)
+    int4* grec;                    // [G] per sorted group position: (first distinct row, rows,
+                                   //     first digit i_1, 0), so chunk metadata is one load
 };
 
 // ---------------------------------------------------------------------------
@@ -215,6 +217,7 @@ struct K3Args {
     const int32_t* uid_sorted;
     const WsCounters* counters;
     const PlanBuffers* pb;
+    const int4* grec;              // plan's per-group records in sorted (column) order
     const int64_t* offsets;
     float* rowbuf;                 // [U][D]: pooled-row checkpoint (forward), upstream sums (backward)
     int64_t L;
