@@ -85,14 +85,17 @@ typedef enum {
 } tt_group_mode;
 
 /*
- * Arithmetic of the prefix contraction C_p = G_1[0, i_1] . G_2[:, i_2] in the forward
- * (FlowTT section 3.3 computes it once per prefix group; the pages compute in fp32).
- * TT_PREC_BF16_TC rounds both operands to bf16 (round to nearest even) and runs the
- * contraction on the fifth-generation tensor cores, accumulating in fp32 in tensor
- * memory; the suffix contraction, the pooling and the whole backward stay fp32.  Its
- * results agree with the exact (fp64) definition to within 2e-2, measured normwise per
- * pooled row.  It needs three cores with d = (4, 4, 8) and r_1 = r_2 in {32, 64};
- * tt_emb_create returns TT_ERR_SHAPE for other shapes.
+ * Arithmetic of the prefix-level products (FlowTT section 3.3 computes the prefix
+ * contraction C_p = G_1[0, i_1] . G_2[:, i_2] once per prefix group; the pages compute in
+ * fp32).  TT_PREC_BF16_TC rounds the operands to bf16 (round to nearest even) and runs
+ * the products on the fifth-generation tensor cores, accumulating in fp32 in tensor
+ * memory: in the forward the prefix contraction; in the backward, for r_1 = r_2 = 64,
+ * also the recomputed C_p and the two gradient products dG_1 += dC_p . G_2[:, i_2]^T and
+ * dG_2[:, i_2] += G_1[0, i_1]^T . dC_p (dC_p itself is rounded to bf16 for them).  The
+ * suffix contraction, the pooling and the per-row backward (dG_3, dC_p) stay fp32.
+ * Results agree with the exact (fp64) definition to within 2e-2, measured normwise per
+ * pooled row and per digit slice of a core gradient.  It needs three cores with
+ * d = (4, 4, 8) and r_1 = r_2 in {32, 64}; tt_emb_create returns TT_ERR_SHAPE otherwise.
  */
 typedef enum {
     TT_PREC_FP32 = 0,        /* fp32 operands and accumulation on the FP32 pipes (default) */

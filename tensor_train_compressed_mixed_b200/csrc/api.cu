@@ -364,7 +364,7 @@ struct tt_emb_handle {
         a.offsets = offsets;
         a.rowbuf = (float*)at(lay.rowbuf);
         a.L = L;
-        a.tc = (tc && !backward) ? 1 : 0;
+        a.tc = (tc && (!backward || k3_tc_bwd_supported(*cp))) ? 1 : 0;
         a.grid = opt.grid > 0 ? opt.grid : num_sms * k3_blocks_per_sm(*cp, backward, a.tc != 0);
         a.status = d_status;
         return a;

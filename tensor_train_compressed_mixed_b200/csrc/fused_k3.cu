@@ -107,6 +107,12 @@ struct S3 {
     {
         return ((size_t)R * N + (size_t)MF * R) / 2 + (size_t)MF * N + (size_t)FBUF * NUF * SU;
     }
+    // tensor-core backward (rank 64): bf16 B, two bf16 A buffers and a bf16 dC tile, M = 64
+    static constexpr size_t bwd_smem_floats_tc()
+    {
+        return (size_t)R * N / 2 + 64 * (size_t)R + 2 * (size_t)MB * N + 64 * (size_t)N / 2 +
+               2 * (size_t)NUB * P * D3 + 2 * (size_t)NUB * R * SR;
+    }
     static constexpr size_t bwd_smem_floats()
     {
         return (size_t)R * N + 2 * (size_t)MB * R + 2 * (size_t)MB * N + 2 * (size_t)NUB * P * D3 +
@@ -209,10 +215,19 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint
 }
 
 // Instruction descriptor of kind::f16: f32 accumulator [4,6) = 1, A = bf16 [7,10) = 1,
-// B = bf16 [10,13) = 1, both K-major (bits 15, 16 clear), N >> 3 at [17,23), M >> 4 at [24,29).
-__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N)
+// B = bf16 [10,13) = 1, A / B major at bits 15 / 16 (0 = K-major, 1 = MN-major),
+// N >> 3 at [17,23), M >> 4 at [24,29).
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool a_mn = false, bool b_mn = false)
 {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// Descriptor of an MN-major operand without swizzle over the same 8 x 16-byte core matrices:
+// each core matrix holds 8 K-rows of 8 contiguous MN-elements; sbo = bytes between
+// MN-adjacent core matrices, lbo = bytes between K-adjacent ones.
+__device__ __forceinline__ uint64_t umma_desc_mn(uint32_t saddr, uint32_t sbo, uint32_t lbo)
+{
+    return umma_desc(saddr, lbo, sbo);
 }
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols)   // one warp
@@ -268,6 +283,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
     }
     return false;
 }
+// eight fp32 values rounded to bf16 (nearest even), packed in order into 16 bytes
+__device__ __forceinline__ uint4 pack_bf16x8(const float (&v)[8])
+{
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        w[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i])) |
+               ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i + 1])) << 16);
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // 32 lanes x 32 consecutive 32-bit columns of tensor memory: lane i of the warp gets row
 // (taddr lane + i), columns taddr column .. +31
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
@@ -961,7 +987,37 @@ __device__ __forceinline__ void bwd_issue_batch(const CoreParams& cp, int t, int
     cp_async_commit();
 }
 
-template <class S, typename K>
+// Tensor-core variant of bwd_issue_a: the chunk's G_1 rows (bf16) into 8 x 16-byte core
+// matrices of an M = 64 operand (rows MB..63 stay zero); one commit group.
+template <class S>
+__device__ __forceinline__ void bwd_issue_a_tc(const CoreParams& cp, int t, int mb, const BwdMeta<S>& M, uint16_t* Ab)
+{
+    constexpr int R = S::R, MB = S::MB, D1 = S::D1, KC = R / 8;
+    const uint16_t* G1 = cp.bf1[t];
+    const int cnt = M.cnt[mb];
+    for (int q = threadIdx.x; q < MB * KC; q += kBwdThreads) {
+        const int m = q / KC, kc = q % KC;
+        const int j = m / D1, a1 = m % D1;
+        uint16_t* dst = Ab + ((m >> 3) * KC + kc) * 64 + (m & 7) * 8;
+        if (j < cnt) cp_async16(dst, G1 + ((int64_t)M.i1[mb][j] * D1 + a1) * R + kc * 8);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    cp_async_commit();
+}
+
+// one thread issues, the others wait at the barrier; false (all threads) when the wait ran out
+__device__ __forceinline__ bool tc_commit_wait(uint64_t* bar, uint32_t& parity, int* s_ok)
+{
+    if (threadIdx.x == 0) {
+        tc_commit(bar);
+        *s_ok = mbar_wait(bar, parity) ? 1 : 0;
+    }
+    __syncthreads();
+    parity ^= 1u;
+    return *s_ok != 0;
+}
+
+template <class S, typename K, bool TC>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ uniq_keys,
               const int4* __restrict__ grec, const int32_t* __restrict__ col_count,
@@ -973,14 +1029,45 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
     extern __shared__ __align__(16) float smem_f[];
     __shared__ BwdMeta<S> M;
     __shared__ __align__(16) K s_keys[2 * kKeyCap];   // keys of each chunk buffer's first rows
-    float* Bs = smem_f;                    // [R][N] swizzled (key row/4)
-    float* As = Bs + R * N;                // [2][MB][R] swizzled rows
-    float* Cn = As + 2 * MB * R;           // [MB][N] swizzled (key row)
+    __shared__ __align__(8) uint64_t s_mbar;
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_ok;
+    // tensor-core variant: MMA row count (MB rows padded to 64) and bf16 operand tiles
+    constexpr int MT = TC ? 64 : MB;
+    static_assert(!TC || (R == 64 && MB == 32 && N == 256), "tensor-core backward: rank 64, d_2 = 4");
+    float* Bs = smem_f;                    // [R][N] swizzled (key row/4)            (fp32 variant)
+    uint16_t* Bb = reinterpret_cast<uint16_t*>(smem_f);   // N x R bf16 core matrices  (tensor-core variant)
+    float* As = smem_f + (TC ? R * N / 2 : R * N);        // [2][MT][R] fp32 swizzled or bf16 core matrices
+    uint16_t* Abt = reinterpret_cast<uint16_t*>(As);
+    float* Cn = As + (TC ? MT * R : 2 * MB * R);          // [MB][N] swizzled (key row)
     float* dCn = Cn + MB * N;              // [MB][N] swizzled (key row)
-    float* Hs = dCn + MB * N;              // [2][NUB][P][D3]
+    uint16_t* dCb = reinterpret_cast<uint16_t*>(dCn + MB * N);   // MT x N bf16 core matrices (tensor cores)
+    float* Hs = dCn + MB * N + (TC ? MT * N / 2 : 0);   // [2][NUB][P][D3]
     float* Ss = Hs + 2 * NUB * P * D3;     // [2][NUB][R][SR]
     if (has_error(status)) return;
     const int tid = threadIdx.x;
+    uint32_t tmem = 0, parity = 0;
+    bool failed = false;
+    if constexpr (TC) {
+        // rows MB..63 of both A buffers and of the dC tile stay zero for the whole kernel
+        for (int q = tid; q < 2 * (MT - MB) * R / 8; q += kBwdThreads) {
+            const int buf = q / ((MT - MB) * R / 8), r = q % ((MT - MB) * R / 8);
+            const int m = MB + r / (R / 8), kc = r % (R / 8);
+            *reinterpret_cast<uint4*>(Abt + buf * MT * R + ((m >> 3) * (R / 8) + kc) * 64 + (m & 7) * 8) =
+                make_uint4(0u, 0u, 0u, 0u);
+        }
+        for (int q = tid; q < (MT - MB) * N / 8; q += kBwdThreads) {
+            const int m = MB + q / (N / 8), nc = q % (N / 8);
+            *reinterpret_cast<uint4*>(dCb + ((m >> 3) * (N / 8) + nc) * 64 + (m & 7) * 8) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        // tensor memory: columns [0, N) hold dB of the current column group, [N, 2N) C and then dA
+        if (tid < 32) tmem_alloc(&s_tmem, 2 * N);
+        if (tid == 0) mbar_init(&s_mbar, 1);
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        tmem = s_tmem;
+    }
 
     for (int iter = 0;; ++iter) {
         if (tid == 0) M.task = next_task(pp.sched, &hdr->col_head, iter);
@@ -1003,7 +1090,10 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
         TT_PH_START();
 
         // B for the whole column group, and the first chunk's A
-        {
+        if constexpr (TC) {
+            const uint16_t* src = cp.bf2[t] + (int64_t)i2 * (R * N);
+            for (int q = tid; q < R * N / 8; q += kBwdThreads) cp_async16(Bb + q * 8, src + q * 8);
+        } else {
             const float* G2 = cp.cores[t][1] + (int64_t)i2 * N;
             const int64_t rs = (int64_t)n2 * N;
             for (int q = tid; q < R * N / 4; q += kBwdThreads) {
@@ -1012,22 +1102,25 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             }
         }
         bwd_meta<S, K>(cfirst, 0, ccount, 0, uniq_keys, grec, M, s_keys);
-        bwd_issue_a<S>(cp, t, 0, M, As);
+        if constexpr (TC) bwd_issue_a_tc<S>(cp, t, 0, M, Abt);
+        else bwd_issue_a<S>(cp, t, 0, M, As);
         TT_PH(8);
 
-        constexpr int NCH = DBC / 4;
-        constexpr int TNB = N / DBC;
+        constexpr int XR = TC ? 1 : DBR, XC = TC ? 4 : DBC;   // register dB (FP32 variant only)
+        constexpr int NCH = XC / 4;
+        constexpr int TNB = N / XC;
         const int tnb = tid % TNB, trb = tid / TNB;
-        float dB[DBR][DBC];
+        float dB[XR][XC];
 #pragma unroll
-        for (int i = 0; i < DBR; ++i)
+        for (int i = 0; i < XR; ++i)
 #pragma unroll
-            for (int j = 0; j < DBC; ++j) dB[i][j] = 0.f;
+            for (int j = 0; j < XC; ++j) dB[i][j] = 0.f;
 
         int mb = 0;
         for (int j0 = 0; j0 < ccount; j0 += MPB, mb ^= 1) {
             const int cnt = M.cnt[mb];
             const float* Ab = As + mb * MB * R;
+            const uint16_t* Ab16 = Abt + mb * MT * R;
             cp_async_wait_all();   // B, this chunk's A rows and row keys (usually prefetched long ago)
             __syncthreads();
             // the first batch of distinct rows is in flight during the C GEMM
@@ -1038,8 +1131,44 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             __syncthreads();
             TT_PH(9);
 
-            // C_all = A . B  (MB x N): thread tile 4 rows x 8 cols
-            {
+            if constexpr (TC) {
+                // C_all = A . B on the tensor cores (M = 64 with rows MB.. zero, N, K = R) into
+                // tensor-memory columns [N, 2N), then rows < MB into Cn (sub-partitions 0 and 1)
+                fence_async_smem();
+                __syncthreads();
+                if (tid == 0) {
+                    tc_fence_after();
+                    constexpr uint32_t SBO = (R / 8) * 128;
+                    const uint32_t a0 = smem_u32(Ab16), b0 = smem_u32(Bb);
+#pragma unroll
+                    for (int k = 0; k < R / 16; ++k)
+                        tc_mma_bf16(tmem + N, umma_desc(a0 + k * 256, 128, SBO), umma_desc(b0 + k * 256, 128, SBO),
+                                    umma_idesc_bf16(MT, N), k > 0);
+                }
+                if (!tc_commit_wait(&s_mbar, parity, &s_ok)) {
+                    failed = true;
+                    break;
+                }
+                tc_fence_after();
+                const int warp = tid >> 5, lane = tid & 31, sub = warp & 3, half = warp >> 2;
+                if (sub < 2) {   // rows 16 sub + lane (lane < 16)
+                    const int m = 16 * sub + lane;
+#pragma unroll 1
+                    for (int g = 0; g < N / 64; ++g) {
+                        const int c0 = half * (N / 2) + g * 32;
+                        float v[32];
+                        tmem_ld32(tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)(N + c0), v);
+                        if (lane < 16) {
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                *reinterpret_cast<float4*>(&Cn[swz_m<N>(m, c0 + 4 * j)]) =
+                                    make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                        }
+                    }
+                }
+                tc_fence_before();
+            } else {
+                // C_all = A . B  (MB x N): thread tile 4 rows x 8 cols
                 constexpr int TN = N / 8;
                 int tm, tn;   // tm < MB / 4
                 warp_tile_2d<TN>(tid, tm, tn);
@@ -1082,7 +1211,8 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             const bool more = j0 + MPB < ccount;
             if (more) {
                 bwd_meta<S, K>(cfirst, j0 + MPB, ccount, mb ^ 1, uniq_keys, grec, M, s_keys);
-                bwd_issue_a<S>(cp, t, mb ^ 1, M, As + (mb ^ 1) * MB * R);
+                if constexpr (TC) bwd_issue_a_tc<S>(cp, t, mb ^ 1, M, Abt + (mb ^ 1) * MT * R);
+                else bwd_issue_a<S>(cp, t, mb ^ 1, M, As + (mb ^ 1) * MB * R);
             }
 
             // distinct rows in double-buffered batches: dS_u -> dG_3 (vector reductions), dC_p += H_u S_u^T
@@ -1130,6 +1260,10 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                             red_add_v4(dG3 + ((int64_t)(rc * 4 + i) * n3 + i3) * D3 + cg * 4, o[i]);
                     }
                 }
+#ifdef TT_PROFILE_PHASES
+                __syncthreads();   // profiling builds only: separates the dS and dC times
+#endif
+                TT_PH(6);
                 // dC_p[row][rho2] += sum_{u in p, a3} H_u[row][a3] S_u[rho2][a3]: each tile (prefix p,
                 // rows (a1, a2 = 0..3), rho2 in {rc, rc+R/4, rc+R/2, rc+3R/4}) is owned by one thread, which
                 // adds the batch's rows of its prefix in order (plain read-modify-write, deterministic)
@@ -1177,6 +1311,58 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                 TT_PH(12);
             }
 
+            if constexpr (TC) {
+                // dC -> bf16 core matrices (M = 64, K = N); then on the tensor cores
+                //   dA = dC . B^T   (M = 64, N = R, K = N) into columns [N, N + R)
+                //   dB += A^T . dC  (M = R, N, K = MB)     into columns [0, N), over the column group
+                for (int q = tid; q < MB * N / 8; q += kBwdThreads) {
+                    const int m = q / (N / 8), nc = q % (N / 8);
+                    const float4 x0 = *reinterpret_cast<const float4*>(&dCn[swz_m<N>(m, nc * 8)]);
+                    const float4 x1 = *reinterpret_cast<const float4*>(&dCn[swz_m<N>(m, nc * 8 + 4)]);
+                    const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                    *reinterpret_cast<uint4*>(dCb + ((m >> 3) * (N / 8) + nc) * 64 + (m & 7) * 8) = pack_bf16x8(v);
+                }
+                fence_async_smem();
+                __syncthreads();
+                if (tid == 0) {
+                    tc_fence_after();
+                    const uint32_t c0 = smem_u32(dCb), b0 = smem_u32(Bb), a0 = smem_u32(Ab16);
+                    // dA: A = dC (K-major: 8-row groups 16 N bytes apart), B = B viewed MN-major
+#pragma unroll 1
+                    for (int k = 0; k < N / 16; ++k)
+                        tc_mma_bf16(tmem + N, umma_desc(c0 + k * 256, 128, (N / 8) * 128),
+                                    umma_desc_mn(b0 + k * 2 * (R / 8) * 128, 128, (R / 8) * 128),
+                                    umma_idesc_bf16(MT, R, false, true), k > 0);
+                    // dB: A = A^T (MN-major over the A tile), B = dC viewed MN-major
+#pragma unroll
+                    for (int k = 0; k < MB / 16; ++k)
+                        tc_mma_bf16(tmem, umma_desc_mn(a0 + k * 2 * (R / 8) * 128, 128, (R / 8) * 128),
+                                    umma_desc_mn(c0 + k * 2 * (N / 8) * 128, 128, (N / 8) * 128),
+                                    umma_idesc_bf16(R, N, true, true), (j0 > 0 || k > 0) ? 1u : 0u);
+                }
+                if (!tc_commit_wait(&s_mbar, parity, &s_ok)) {
+                    failed = true;
+                    break;
+                }
+                tc_fence_after();
+                TT_PH(13);
+                const int warp = tid >> 5, lane = tid & 31, sub = warp & 3, half = warp >> 2;
+                if (sub < 2) {   // dA rows 16 sub + lane, columns half * R / 2 ..
+                    const int m = 16 * sub + lane, p = m / D1, a1 = m % D1;
+                    float v[32];
+                    tmem_ld32(tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)(N + half * 32), v);
+                    if (lane < 16 && p < cnt) {
+                        float* dst = dG1 + ((int64_t)M.i1[mb][p] * D1 + a1) * R + half * 32;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            red_add_v4(dst + 4 * j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+                    }
+                }
+                tc_fence_before();
+                __syncthreads();   // dCn, the dC tile and the A buffer are reused by the next chunks
+                TT_PH(14);
+                // (the FP32 variant follows)
+            } else {
             // dA[m][rho1] = sum_n dC[m][n] B[rho1][n] -> dG_1; tiles 4 m x 4 rho1, the n range split
             // between the two halves of the block and combined through shared memory
             {
@@ -1257,7 +1443,28 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             }
             __syncthreads();   // dCn, Ab and the partial buffer are reused by the next chunk
             TT_PH(14);
+            }
         }
+        if (failed) break;
+        if constexpr (TC) {
+            // dG_2[:, i_2] = dB from tensor memory: rows rho_1 = 16 sub + lane (lane < 16), half the columns
+            tc_fence_after();
+            const int warp = tid >> 5, lane = tid & 31, sub = warp & 3, half = warp >> 2;
+            const int rho1 = 16 * sub + lane;
+#pragma unroll 1
+            for (int g = 0; g < N / 64; ++g) {
+                const int c0 = half * (N / 2) + g * 32;
+                float v[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)c0, v);
+                if (lane < 16) {
+                    float* dst = dG2 + ((int64_t)rho1 * n2 + i2) * N + c0;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<float4*>(dst + 4 * j) = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                }
+            }
+            tc_fence_before();
+        } else {
         // the column group is complete: dG_2[:, i_2] = dB (this block owns the slice)
 #pragma unroll
         for (int i = 0; i < DBR; ++i) {
@@ -1271,10 +1478,20 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                 *reinterpret_cast<float4*>(dst + ch * (N / NCH) + tnb * 4) =
                     make_float4(dB[i][ch * 4], dB[i][ch * 4 + 1], dB[i][ch * 4 + 2], dB[i][ch * 4 + 3]);
         }
+        }
         __syncthreads();
         TT_PH(15);
     }
     cp_async_wait_all();
+    if constexpr (TC) {
+        if (failed && tid == 0) raise_error(status, TT_ERR_TIMEOUT, 101);
+        tc_fence_before();
+        __syncthreads();
+        if (tid < 32) {
+            tc_fence_after();
+            tmem_dealloc(tmem, 2 * N);
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -1303,16 +1520,6 @@ __device__ __forceinline__ int table_of(const int64_t* base, int T, int64_t q)
         else hi = mid - 1;
     }
     return lo;
-}
-
-__device__ __forceinline__ uint4 pack_bf16x8(const float (&v)[8])
-{
-    uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        w[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i])) |
-               ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i + 1])) << 16);
-    return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 __global__ void __launch_bounds__(256) k3_bf16_kernel(Bf16Job j)
@@ -1400,15 +1607,15 @@ cudaError_t rowsum_launch(const K3Args& a, const float* grad_out, cudaStream_t s
     return cudaGetLastError();
 }
 
-template <class S, typename K>
+template <class S, typename K, bool TC>
 cudaError_t bwd_launch(const K3Args& a, const GradPtrs& gp, const float* grad_out, cudaStream_t s, int* nl)
 {
     (void)grad_out;
-    const size_t smem = sizeof(float) * S::bwd_smem_floats();
-    cudaError_t e = cudaFuncSetAttribute(k3_bwd_kernel<S, K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = sizeof(float) * (TC ? S::bwd_smem_floats_tc() : S::bwd_smem_floats());
+    cudaError_t e = cudaFuncSetAttribute(k3_bwd_kernel<S, K, TC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const PlanBuffers& pb = *a.pb;
-    k3_bwd_kernel<S, K><<<a.grid, kBwdThreads, smem, s>>>(
+    k3_bwd_kernel<S, K, TC><<<a.grid, kBwdThreads, smem, s>>>(
         *a.cp, gp, *a.pp, (const K*)a.uniq_keys, a.grec, pb.col_count, pb.col_start, pb.hdr, a.rowbuf,
         a.status);
     *nl += 1;
@@ -1428,7 +1635,12 @@ cudaError_t fwd_dispatch_tc(const K3Args& a, float* out, cudaStream_t s, int* nl
 template <class S>
 cudaError_t bwd_dispatch(const K3Args& a, const GradPtrs& gp, const float* g, cudaStream_t s, int* nl)
 {
-    return a.key64 ? bwd_launch<S, uint64_t>(a, gp, g, s, nl) : bwd_launch<S, uint32_t>(a, gp, g, s, nl);
+    return a.key64 ? bwd_launch<S, uint64_t, false>(a, gp, g, s, nl) : bwd_launch<S, uint32_t, false>(a, gp, g, s, nl);
+}
+template <class S>
+cudaError_t bwd_dispatch_tc(const K3Args& a, const GradPtrs& gp, const float* g, cudaStream_t s, int* nl)
+{
+    return a.key64 ? bwd_launch<S, uint64_t, true>(a, gp, g, s, nl) : bwd_launch<S, uint32_t, true>(a, gp, g, s, nl);
 }
 
 template <class S, bool TC>
@@ -1446,9 +1658,11 @@ template <class S>
 int occ_bwd()
 {
     const size_t smem = sizeof(float) * S::bwd_smem_floats();
-    cudaFuncSetAttribute(k3_bwd_kernel<S, uint32_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(k3_bwd_kernel<S, uint32_t, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k3_bwd_kernel<S, uint32_t>, kBwdThreads, smem) != cudaSuccess) return 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k3_bwd_kernel<S, uint32_t, false>, kBwdThreads, smem) !=
+        cudaSuccess)
+        return 1;
     return n > 0 ? n : 1;
 }
 
@@ -1456,11 +1670,7 @@ int occ_bwd()
 
 int k3_blocks_per_sm(const CoreParams& cp, bool backward, bool tc)
 {
-    if (tc && !backward) {
-        if (cp.d[0] == 4 && cp.d[2] == 8 && cp.r[1] == 64) return occ_fwd<S3<4, 4, 8, 64>, true>();
-        if (cp.d[0] == 4 && cp.d[2] == 8 && cp.r[1] == 32) return occ_fwd<S3<4, 4, 8, 32>, true>();
-        return 1;
-    }
+    if (tc) return 1;   // tensor-core variants hold tensor memory: one block per SM
 #define TT_OCC_CASE(Q1, Q2, Q3, QR) \
     if (cp.d[0] == Q1 && cp.d[2] == Q3 && cp.r[1] == QR) return backward ? occ_bwd<S3<Q1, Q2, Q3, QR>>() : occ_fwd<S3<Q1, Q2, Q3, QR>, false>();
     TT_K3_CASES_INNER(TT_OCC_CASE)
@@ -1471,6 +1681,11 @@ int k3_blocks_per_sm(const CoreParams& cp, bool backward, bool tc)
 bool k3_tc_supported(const CoreParams& cp)
 {
     return k3_supported(cp) && cp.d[0] == 4 && cp.d[1] == 4 && cp.d[2] == 8 && (cp.r[1] == 64 || cp.r[1] == 32);
+}
+
+bool k3_tc_bwd_supported(const CoreParams& cp)
+{
+    return k3_tc_supported(cp) && cp.r[1] == 64;
 }
 
 bool k3_supported(const CoreParams& cp)
@@ -1568,6 +1783,10 @@ cudaError_t k3_rowsum(const K3Args& a, const float* grad_out, cudaStream_t s, in
 cudaError_t k3_backward(const K3Args& a, const GradPtrs& gp, const float* grad_out, cudaStream_t s, int* nl)
 {
     const CoreParams& cp = *a.cp;
+    if (a.tc) {
+        if (k3_tc_bwd_supported(cp)) return bwd_dispatch_tc<S3<4, 4, 8, 64>>(a, gp, grad_out, s, nl);
+        return cudaErrorInvalidValue;
+    }
 #define TT_BWD_CASE(Q1, Q2, Q3, QR) \
     if (cp.d[0] == Q1 && cp.d[2] == Q3 && cp.r[1] == QR) return bwd_dispatch<S3<Q1, Q2, Q3, QR>>(a, gp, grad_out, s, nl);
     TT_K3_CASES(TT_BWD_CASE)

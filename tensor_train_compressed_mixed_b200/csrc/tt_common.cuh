@@ -248,6 +248,8 @@ int k3_plan_mp(const CoreParams& cp);
 int k3_blocks_per_sm(const CoreParams& cp, bool backward, bool tc = false);
 // shapes with a tensor-core (bf16) variant of the forward prefix GEMM
 bool k3_tc_supported(const CoreParams& cp);
+// shapes whose backward also runs its prefix-level products on the tensor cores (rank 64)
+bool k3_tc_bwd_supported(const CoreParams& cp);
 // bf16 operand copies of G_1 and G_2 for the tensor-core forward (cp.cores -> dst1/dst2)
 cudaError_t k3_to_bf16(const CoreParams& cp, uint16_t* const* dst1, uint16_t* const* dst2, cudaStream_t s, int* nl);
 cudaError_t k3_forward(const K3Args& a, float* out, cudaStream_t s, int* nl);
