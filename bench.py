@@ -48,8 +48,10 @@ def parse_args():
                    help="work distribution of the fused kernels (ablation)")
     p.add_argument("--grouping", choices=["prefix", "unique"], default="prefix",
                    help="prefix reuse, or one unit per unique row (ablation)")
-    p.add_argument("--precision", choices=["fp32", "bf16"], default="fp32",
-                   help="forward prefix contraction: fp32 FFMA, or bf16 on the tcgen05 tensor cores")
+    p.add_argument("--precision", choices=["auto", "fp32", "split", "bf16"], default="auto",
+                   help="prefix-level products: fp32 on the FP32 pipes; split = fp32-accurate on the "
+                        "tcgen05 tensor cores (two bf16 terms per value, three products); bf16 on the "
+                        "tensor cores; auto = split where the shape has tensor-core kernels, else fp32")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -283,12 +285,17 @@ def run_ours(args):
     world, rank, local = dist_init(args.gpus)
     dev = torch.device("cuda", local)
     w = config_workload(args.config, batch=args.batch, tables=args.tables, with_grad=True)
+    if args.precision == "auto":
+        # the tensor-core kernels cover three cores with d = (4, 4, 8) and r = 32 or 64
+        tc_shape = len(w.d) == 3 and tuple(w.d) == (4, 4, 8) and w.r[1] == w.r[2] and w.r[1] in (32, 64)
+        args.precision = "split" if tc_shape else "fp32"
     train = w.grad_out is not None and args.config in (4, 5)
     opts = abi.tt_emb_default_options()
     opts.sched = {"static": abi.TT_SCHED_STATIC, "steal": abi.TT_SCHED_STEAL,
                   "steal_l2": abi.TT_SCHED_STEAL_L2}[args.sched]
     opts.grouping = abi.TT_GROUP_PREFIX if args.grouping == "prefix" else abi.TT_GROUP_UNIQUE_ONLY
-    opts.precision = abi.TT_PREC_FP32 if args.precision == "fp32" else abi.TT_PREC_BF16_TC
+    opts.precision = {"fp32": abi.TT_PREC_FP32, "split": abi.TT_PREC_FP32_SPLIT_TC,
+                      "bf16": abi.TT_PREC_BF16_TC}[args.precision]
     emb, cores, idx, off = from_workload(w, device=dev, options=opts, with_grads=True)
     g = torch.from_numpy(w.grad_out).to(dev)
     L, B, T, D = w.num_lookups, w.batch, w.num_tables, w.dim
@@ -340,19 +347,29 @@ def run_ours(args):
     per_step = {k: v / args.steps for k, v in ph.items()}
     dom = max(per_step, key=per_step.get)
     flops = {"fwd_fused": alg["f_fwd"], "bwd_fused": alg["f_bwd_kernel"]}
-    if dom == "fwd_fused" and args.precision == "bf16":
-        # prefix step on the tensor cores, the rest on the FP32 pipes: the peak is the
-        # work-weighted combination of the two (time = F_tc / P_tc + F_fp32 / P_fp32)
-        f_tc = alg["f_fwd_prefix"]
-        f_rest = alg["f_fwd"] - f_tc
-        t_ideal = f_tc / (BF16_PEAK_TFLOPS * 1e12) + f_rest / (FP32_PEAK_TFLOPS * 1e12)
-        peak = alg["f_fwd"] / t_ideal / 1e12
-        achieved = alg["f_fwd"] / (per_step[dom] / 1e3) / 1e12
+    # tensor-core share of each fused kernel's algorithmic work in bf16 mode: the forward's
+    # prefix step; at rank 64 also the backward's two prefix-level gradient products
+    tc_work = {}
+    if args.precision in ("bf16", "split"):
+        tc_work["fwd_fused"] = alg["f_fwd_prefix"]
+        if len(w.d) == 3 and w.r[1] == 64:
+            tc_work["bwd_fused"] = 2.0 * alg["f_fwd_prefix"]
+    if dom in tc_work:
+        # tensor-core work and FP32 work: the peak is their work-weighted combination
+        # (ideal time = F_tc / P_tc + F_fp32 / P_fp32)
+        f_all = flops[dom]
+        f_tc = tc_work[dom]
+        f_rest = f_all - f_tc
+        products = 3 if args.precision == "split" else 1   # tensor-core products per algorithmic one
+        t_ideal = products * f_tc / (BF16_PEAK_TFLOPS * 1e12) + f_rest / (FP32_PEAK_TFLOPS * 1e12)
+        peak = f_all / t_ideal / 1e12
+        achieved = f_all / (per_step[dom] / 1e3) / 1e12
         roof = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": None,
-                "peak_source": f"work-weighted: prefix step {f_tc / 1e9:.1f} GFLOP at the measured bf16 "
-                               f"tensor peak {BF16_PEAK_TFLOPS:.0f} TF/s, the rest {f_rest / 1e9:.1f} GFLOP at "
-                               f"the derived FP32 peak {FP32_PEAK_TFLOPS:.1f} TF/s"}
+                "peak_source": f"work-weighted: {f_tc / 1e9:.1f} GFLOP of prefix-level products as {products} "
+                               f"bf16 tensor-core product(s) each at the measured bf16 peak "
+                               f"{BF16_PEAK_TFLOPS:.0f} TF/s, {f_rest / 1e9:.1f} GFLOP at the derived FP32 peak "
+                               f"{FP32_PEAK_TFLOPS:.1f} TF/s"}
     elif dom in flops:
         achieved = flops[dom] / (per_step[dom] / 1e3) / 1e12
         roof = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": FP32_PEAK_TFLOPS,
@@ -456,7 +473,8 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "lookups/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32" if args.precision == "fp32" else "bf16 prefix GEMM, f32 elsewhere",
+            "dtype": {"fp32": "f32", "split": "f32 (prefix-level products as split bf16 on tensor cores)",
+                      "bf16": "bf16 prefix-level products, f32 elsewhere"}[args.precision],
             "data": "synthetic",
             "config": {"workload": w.name, "batch": B, "tables": T, "lookups": L,
                        "unique_rows": U, "prefix_groups": G,
@@ -464,8 +482,10 @@ def run_ours(args):
                        "l2": "inputs larger than L2 (indices+grad+cores ~800 MB), no flush",
                        "parallelism": f"replicas{world}" if world > 1 else "single",
                        "sched": args.sched, "grouping": args.grouping,
-                       "prefix_step": "fp32 FFMA" if args.precision == "fp32" else
-                                      "bf16 operands, fp32 accumulation, tcgen05"},
+                       "prefix_step": {"fp32": "fp32 FFMA",
+                                       "split": "fp32-accurate: two bf16 terms per value, three tcgen05 "
+                                                "products, fp32 accumulation",
+                                       "bf16": "bf16 operands, fp32 accumulation, tcgen05"}[args.precision]},
             "fwd": {"value": world * L / (ms_fwd / 1e3), "unit": "lookups/s", "ms": ms_fwd,
                     "roofline_frac": t_roof_fwd / (ms_fwd / 1e3)},
             "step_roofline_frac": t_roof_step / (ms_step / 1e3),

@@ -99,7 +99,11 @@ typedef enum {
  */
 typedef enum {
     TT_PREC_FP32 = 0,        /* fp32 operands and accumulation on the FP32 pipes (default) */
-    TT_PREC_BF16_TC = 1      /* bf16 operands, fp32 accumulation, tcgen05 tensor cores */
+    TT_PREC_BF16_TC = 1,     /* bf16 operands, fp32 accumulation, tcgen05 tensor cores (bound 2e-2) */
+    TT_PREC_FP32_SPLIT_TC = 2 /* fp32-accurate on the tensor cores: every operand value x is held as
+                                 two bf16 terms hi = bf16(x), lo = bf16(x - hi) (|x - hi - lo| <=
+                                 2^-18 |x|) and each product is hi.hi + hi.lo + lo.hi with fp32
+                                 accumulation; same coverage as TT_PREC_BF16_TC, bound 1e-4 */
 } tt_precision;
 
 typedef struct {

@@ -21,7 +21,7 @@ TT_OK, TT_ERR_ARG, TT_ERR_SHAPE, TT_ERR_INDEX_RANGE, TT_ERR_OFFSETS = 0, 1, 2, 3
 TT_ERR_WORKSPACE, TT_ERR_STATE, TT_ERR_CUDA, TT_ERR_TIMEOUT, TT_ERR_UNSUPPORTED = 5, 6, 7, 8, 9
 TT_SCHED_STATIC, TT_SCHED_STEAL, TT_SCHED_STEAL_L2 = 0, 1, 2
 TT_GROUP_PREFIX, TT_GROUP_UNIQUE_ONLY = 0, 1
-TT_PREC_FP32, TT_PREC_BF16_TC = 0, 1
+TT_PREC_FP32, TT_PREC_BF16_TC, TT_PREC_FP32_SPLIT_TC = 0, 1, 2
 MAX_TABLES, MAX_CORES = 64, 4
 
 

@@ -128,7 +128,7 @@ struct tt_emb_handle {
     int32_t vd[3] = {}, vr[4] = {};
     int64_t g12_off[kMaxT + 1] = {};  // merged-core offsets (floats) in the workspace
     int64_t g3t_off[kMaxT + 1] = {};  // transposed last-core offsets (floats) in the workspace
-    bool tc = false;                  // forward prefix GEMM on the tensor cores (bf16 operands)
+    int tc = 0;                       // tensor-core prefix products: 0 none, 1 bf16, 3 split bf16 (two terms)
     int64_t bf1_off[kMaxT + 1] = {};  // bf16 copies of G_1 and G_2 (elements) in the workspace
     int64_t bf2_off[kMaxT + 1] = {};
     // timing and launch accounting
@@ -364,7 +364,7 @@ struct tt_emb_handle {
         a.offsets = offsets;
         a.rowbuf = (float*)at(lay.rowbuf);
         a.L = L;
-        a.tc = (tc && (!backward || k3_tc_bwd_supported(*cp))) ? 1 : 0;
+        a.tc = (tc && (!backward || k3_tc_bwd_supported(*cp))) ? tc : 0;
         a.grid = opt.grid > 0 ? opt.grid : num_sms * k3_blocks_per_sm(*cp, backward, a.tc != 0);
         a.status = d_status;
         return a;
@@ -418,7 +418,8 @@ int tt_emb_create(int32_t num_tables, int32_t num_cores, const int64_t* n_factor
         for (int i = 0; i < 10; ++i)
             if (o.reserved[i] != 0) return TT_ERR_ARG;
         if (o.force_generic != 0 && o.force_generic != 1) return TT_ERR_ARG;
-        if (o.precision != TT_PREC_FP32 && o.precision != TT_PREC_BF16_TC) return TT_ERR_ARG;
+        if (o.precision != TT_PREC_FP32 && o.precision != TT_PREC_BF16_TC && o.precision != TT_PREC_FP32_SPLIT_TC)
+            return TT_ERR_ARG;
         if (o.sched < TT_SCHED_STATIC || o.sched > TT_SCHED_STEAL_L2) return TT_ERR_ARG;
         if (o.grouping < TT_GROUP_PREFIX || o.grouping > TT_GROUP_UNIQUE_ONLY) return TT_ERR_ARG;
         if (o.chunk < 0 || o.grid < 0) return TT_ERR_ARG;
@@ -509,19 +510,20 @@ int tt_emb_create(int32_t num_tables, int32_t num_cores, const int64_t* n_factor
         if (nc >= (1LL << 24)) h->fast = h->merged = false;
         h->ncols = (int)nc;
     }
-    if (o.precision == TT_PREC_BF16_TC) {
+    if (o.precision == TT_PREC_BF16_TC || o.precision == TT_PREC_FP32_SPLIT_TC) {
         // the tensor-core prefix GEMM exists for three-core tables of the listed shapes only
         if (!h->fast || h->merged || !k3_tc_supported(h->view_params())) {
             delete h;
             return TT_ERR_SHAPE;
         }
-        h->tc = true;
+        h->tc = o.precision == TT_PREC_FP32_SPLIT_TC ? 3 : 1;
+        const int terms = h->tc == 3 ? 2 : 1;
         int64_t b1 = 0, b2 = 0;
         for (int t = 0; t < num_tables; ++t) {
             h->bf1_off[t] = b1;
             h->bf2_off[t] = b2;
-            b1 += h->vn[t][0] * h->vd[0] * h->vr[1];
-            b2 += h->vn[t][1] * h->vr[1] * h->vd[1] * h->vr[2];
+            b1 += terms * h->vn[t][0] * h->vd[0] * h->vr[1];
+            b2 += terms * h->vn[t][1] * h->vr[1] * h->vd[1] * h->vr[2];
         }
         h->bf1_off[num_tables] = b1;
         h->bf2_off[num_tables] = b2;
@@ -683,7 +685,7 @@ int tt_emb_forward(tt_emb_t h, const int64_t* indices, const int64_t* offsets, i
                 d1[t] = (uint16_t*)h->at(y.bf1) + h->bf1_off[t];
                 d2[t] = (uint16_t*)h->at(y.bf2) + h->bf2_off[t];
             }
-            e = k3_to_bf16(cp, d1, d2, s, &nl);
+            e = k3_to_bf16(cp, h->tc == 3 ? 2 : 1, d1, d2, s, &nl);
         }
         K3Args a = h->k3_args(&cp, &pp, &pb, offsets, L, false);
         if (e == cudaSuccess) e = k3_forward(a, out, s, &nl);

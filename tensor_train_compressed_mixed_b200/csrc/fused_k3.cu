@@ -102,16 +102,17 @@ struct S3 {
     static_assert(NUB >= 1 && NUB * TPUB == kBwdThreads, "backward batch tiling");
 
     static constexpr size_t fwd_smem_floats() { return FWD_FIXED + (size_t)FBUF * NUF * SU; }
-    // tensor-core variant: A and B in bf16
-    static constexpr size_t fwd_smem_floats_tc()
+    // tensor-core variants: A and B as NS bf16 terms
+    static constexpr size_t fwd_smem_floats_tc(int NS)
     {
-        return ((size_t)R * N + (size_t)MF * R) / 2 + (size_t)MF * N + (size_t)FBUF * NUF * SU;
+        return (size_t)NS * ((size_t)R * N + (size_t)MF * R) / 2 + (size_t)MF * N + (size_t)FBUF * NUF * SU;
     }
-    // tensor-core backward (rank 64): bf16 B, two bf16 A buffers and a bf16 dC tile, M = 64
-    static constexpr size_t bwd_smem_floats_tc()
+    // tensor-core backward (rank 64): B and two A buffers as NS bf16 terms; dC's bf16 terms
+    // overwrite dCn
+    static constexpr size_t bwd_smem_floats_tc(int NS)
     {
-        return (size_t)R * N / 2 + 64 * (size_t)R + 2 * (size_t)MB * N + 64 * (size_t)N / 2 +
-               2 * (size_t)NUB * P * D3 + 2 * (size_t)NUB * R * SR;
+        return (size_t)NS * R * N / 2 + (size_t)NS * MB * R + 2 * (size_t)MB * N + 2 * (size_t)NUB * P * D3 +
+               2 * (size_t)NUB * R * SR;
     }
     static constexpr size_t bwd_smem_floats()
     {
@@ -283,15 +284,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
     }
     return false;
 }
-// eight fp32 values rounded to bf16 (nearest even), packed in order into 16 bytes
-__device__ __forceinline__ uint4 pack_bf16x8(const float (&v)[8])
+// eight fp32 values as two bf16 terms: hi = bf16(x), lo = bf16(x - hi); |x - hi - lo| <= 2^-18 |x|
+__device__ __forceinline__ void split_bf16x8(const float (&v)[8], uint4& hi, uint4& lo)
 {
-    uint32_t w[4];
+    uint32_t h[4], l[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-        w[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i])) |
-               ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i + 1])) << 16);
-    return make_uint4(w[0], w[1], w[2], w[3]);
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * i]), h1 = __float2bfloat16_rn(v[2 * i + 1]);
+        const __nv_bfloat16 l0 = __float2bfloat16_rn(v[2 * i] - __bfloat162float(h0));
+        const __nv_bfloat16 l1 = __float2bfloat16_rn(v[2 * i + 1] - __bfloat162float(h1));
+        h[i] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+        l[i] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
 // 32 lanes x 32 consecutive 32-bit columns of tensor memory: lane i of the warp gets row
@@ -456,9 +462,10 @@ __device__ __forceinline__ void fwd_gemm(const FwdSmem<S>& sm)
     }
 }
 
-// Tensor-core variant of fwd_issue_ab: bf16 B tile (already in operand order, one flat
+// Tensor-core variant of fwd_issue_ab: the bf16 B tile (already in operand order, one flat
 // copy) and the chunk's A rows placed into 8 x 16-byte core matrices; one commit group.
-template <class S>
+// NS = 2 stores each operand as two bf16 terms (hi tile, then lo tile).
+template <class S, int NS>
 __device__ __forceinline__ void fwd_issue_ab_tc(const CoreParams& cp, int mb, const FwdMeta<S>& M,
                                                 const FwdSmem<S>& sm, int& cur_t, int& cur_i2)
 {
@@ -467,20 +474,35 @@ __device__ __forceinline__ void fwd_issue_ab_tc(const CoreParams& cp, int mb, co
     const int tid = threadIdx.x;
     const int t = M.t[mb], i2 = M.i2[mb], cnt = M.cnt[mb];
     if (t != cur_t || i2 != cur_i2) {
-        const uint16_t* src = cp.bf2[t] + (int64_t)i2 * (R * N);
-        for (int q = tid; q < R * N / 8; q += kFwdThreads) cp_async16(sm.Bb + q * 8, src + q * 8);
+        const uint16_t* src = cp.bf2[t] + (int64_t)i2 * (NS * R * N);
+        for (int q = tid; q < NS * R * N / 8; q += kFwdThreads) cp_async16(sm.Bb + q * 8, src + q * 8);
         cur_t = t;
         cur_i2 = i2;
     }
     const uint16_t* G1 = cp.bf1[t];
-    for (int q = tid; q < MF * KC; q += kFwdThreads) {
-        const int m = q / KC, kc = q % KC;
+    for (int q = tid; q < NS * MF * KC; q += kFwdThreads) {
+        const int term = q / (MF * KC), r = q % (MF * KC);
+        const int m = r / KC, kc = r % KC;
         const int j = m / D1, a1 = m % D1;
-        uint16_t* dst = sm.Ab + ((m >> 3) * KC + kc) * 64 + (m & 7) * 8;
-        if (j < cnt) cp_async16(dst, G1 + ((int64_t)M.i1[mb][j] * D1 + a1) * R + kc * 8);
+        uint16_t* dst = sm.Ab + term * (MF * R) + ((m >> 3) * KC + kc) * 64 + (m & 7) * 8;
+        if (j < cnt) cp_async16(dst, G1 + ((int64_t)M.i1[mb][j] * D1 + a1) * (NS * R) + term * R + kc * 8);
         else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
     }
     cp_async_commit();
+}
+
+// The MMAs of one K = 16 step of a product whose operands are stored as NT = 1 term
+// (bf16) or as two terms hi + lo (NT = 3 products: hi.hi + hi.lo + lo.hi).  a_lo / b_lo
+// are the byte distances from the hi tiles to the lo tiles.
+template <int NT>
+__device__ __forceinline__ void tc_mma_terms(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t a_lo,
+                                             uint32_t b_lo, uint32_t idesc, bool accumulate)
+{
+    tc_mma_bf16(tmem_d, adesc, bdesc, idesc, accumulate ? 1u : 0u);
+    if constexpr (NT == 3) {
+        tc_mma_bf16(tmem_d, adesc, bdesc + (b_lo >> 4), idesc, 1u);
+        tc_mma_bf16(tmem_d, adesc + (a_lo >> 4), bdesc, idesc, 1u);
+    }
 }
 
 // C_all = A . B on the tensor cores: one thread issues R / 16 MMAs (M = MF, N, K = 16)
@@ -488,7 +510,7 @@ __device__ __forceinline__ void fwd_issue_ab_tc(const CoreParams& cp, int mb, co
 // moves its share of the fp32 accumulator (sub-partition warp % 4, a quarter of the
 // columns) into Cn.  The caller has waited for the A/B copies; returns false (all
 // threads) when the completion wait ran out.
-template <class S>
+template <class S, int NT>
 __device__ __forceinline__ bool fwd_gemm_tc(const FwdSmem<S>& sm, uint32_t tmem, uint64_t* bar, uint32_t& parity,
                                             int* s_ok)
 {
@@ -505,7 +527,8 @@ __device__ __forceinline__ bool fwd_gemm_tc(const FwdSmem<S>& sm, uint32_t tmem,
         const uint32_t a0 = smem_u32(sm.Ab), b0 = smem_u32(sm.Bb);
 #pragma unroll
         for (int k = 0; k < R / 16; ++k)
-            tc_mma_bf16(tmem, umma_desc(a0 + k * 256, 128, SBO), umma_desc(b0 + k * 256, 128, SBO), idesc, k > 0);
+            tc_mma_terms<NT>(tmem, umma_desc(a0 + k * 256, 128, SBO), umma_desc(b0 + k * 256, 128, SBO),
+                             MF * R * 2, R * N * 2, idesc, k > 0);
         tc_commit(bar);
         *s_ok = mbar_wait(bar, parity) ? 1 : 0;
     }
@@ -671,7 +694,7 @@ __device__ void fwd_pool(const CoreParams& cp, int ptask, int nP, const int32_t*
 // metadata and A/B rows (As and Bs are free once the GEMM is done) while this
 // chunk's distinct rows are contracted batch by batch (double-buffered last
 // slices when shared memory allows).
-template <class S, typename K, bool TC>
+template <class S, typename K, int NT>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
               const int4* __restrict__ grec, const int32_t* __restrict__ uid_at_pos,
@@ -686,15 +709,17 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
     __shared__ uint32_t s_tmem;
     __shared__ int s_ok;
     if (has_error(status)) return;
+    constexpr bool TC = NT > 0;
+    constexpr int NS = NT == 3 ? 2 : 1;   // bf16 terms stored per operand element
     FwdSmem<S> sm;
     const int tid = threadIdx.x;
     uint32_t tmem = 0, parity = 0;
     if constexpr (TC) {
-        // bf16 operands take half the room of fp32 ones
+        // one bf16 term takes half the room of an fp32 operand, two terms the same room
         sm.Bs = sm.As = nullptr;
         sm.Bb = reinterpret_cast<uint16_t*>(smem_f);
-        sm.Ab = sm.Bb + S::R * S::N;
-        sm.Cn = smem_f + (S::R * S::N + S::MF * S::R) / 2;
+        sm.Ab = sm.Bb + NS * S::R * S::N;
+        sm.Cn = smem_f + NS * (S::R * S::N + S::MF * S::R) / 2;
         if (tid < 32) tmem_alloc(&s_tmem, (uint32_t)S::N);
         if (tid == 0) mbar_init(&s_mbar, 1);
         tc_fence_before();
@@ -732,7 +757,7 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
         TT_PH_START();
         if (!staged) {
             fwd_meta<S, K>(cp, tv, mb, uniq_keys, grec, chunks, M, s_keys);
-            if constexpr (TC) fwd_issue_ab_tc<S>(cp, mb, M, sm, cur_t, cur_i2);
+            if constexpr (TC) fwd_issue_ab_tc<S, NS>(cp, mb, M, sm, cur_t, cur_i2);
             else fwd_issue_ab<S>(cp, mb, M, sm, cur_t, cur_i2);
         }
         if (tid == 0) M.task[1] = next_task(sched, &hdr->queue_head, iter);   // result used after the GEMM
@@ -744,7 +769,7 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
         if (total > 0) fwd_issue_batch<S, K>(cp, mb, 0, 0, uniq_keys, M, sm, s_keys);
         TT_PH(0);
         if constexpr (TC) {
-            if (!fwd_gemm_tc<S>(sm, tmem, &s_mbar, parity, &s_ok)) {
+            if (!fwd_gemm_tc<S, NT>(sm, tmem, &s_mbar, parity, &s_ok)) {
                 if (tid == 0) raise_error(status, TT_ERR_TIMEOUT, 100);
                 break;
             }
@@ -757,7 +782,7 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
         const bool next_chunk = qn < ntasks && tasks[qn] >= 0;
         if (next_chunk) {
             fwd_meta<S, K>(cp, tasks[qn], mb ^ 1, uniq_keys, grec, chunks, M, s_keys);
-            if constexpr (TC) fwd_issue_ab_tc<S>(cp, mb ^ 1, M, sm, cur_t, cur_i2);
+            if constexpr (TC) fwd_issue_ab_tc<S, NS>(cp, mb ^ 1, M, sm, cur_t, cur_i2);
             else fwd_issue_ab<S>(cp, mb ^ 1, M, sm, cur_t, cur_i2);
         }
         // distinct rows of this chunk, in batches of NUF (commit groups in flight: the batch,
@@ -987,19 +1012,22 @@ __device__ __forceinline__ void bwd_issue_batch(const CoreParams& cp, int t, int
     cp_async_commit();
 }
 
-// Tensor-core variant of bwd_issue_a: the chunk's G_1 rows (bf16) into 8 x 16-byte core
-// matrices of an M = 64 operand (rows MB..63 stay zero); one commit group.
-template <class S>
+// Tensor-core variant of bwd_issue_a: the chunk's G_1 rows (NS bf16 terms: hi tile, then
+// lo tile) into 8 x 16-byte core matrices of MB rows; one commit group.  The M = 64 MMAs
+// read 64 rows: rows MB..63 fall on the following tile, and the output rows they feed are
+// never read.
+template <class S, int NS>
 __device__ __forceinline__ void bwd_issue_a_tc(const CoreParams& cp, int t, int mb, const BwdMeta<S>& M, uint16_t* Ab)
 {
     constexpr int R = S::R, MB = S::MB, D1 = S::D1, KC = R / 8;
     const uint16_t* G1 = cp.bf1[t];
     const int cnt = M.cnt[mb];
-    for (int q = threadIdx.x; q < MB * KC; q += kBwdThreads) {
-        const int m = q / KC, kc = q % KC;
+    for (int q = threadIdx.x; q < NS * MB * KC; q += kBwdThreads) {
+        const int term = q / (MB * KC), r = q % (MB * KC);
+        const int m = r / KC, kc = r % KC;
         const int j = m / D1, a1 = m % D1;
-        uint16_t* dst = Ab + ((m >> 3) * KC + kc) * 64 + (m & 7) * 8;
-        if (j < cnt) cp_async16(dst, G1 + ((int64_t)M.i1[mb][j] * D1 + a1) * R + kc * 8);
+        uint16_t* dst = Ab + term * (MB * R) + ((m >> 3) * KC + kc) * 64 + (m & 7) * 8;
+        if (j < cnt) cp_async16(dst, G1 + ((int64_t)M.i1[mb][j] * D1 + a1) * (NS * R) + term * R + kc * 8);
         else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
     }
     cp_async_commit();
@@ -1017,7 +1045,7 @@ __device__ __forceinline__ bool tc_commit_wait(uint64_t* bar, uint32_t& parity, 
     return *s_ok != 0;
 }
 
-template <class S, typename K, bool TC>
+template <class S, typename K, int NT>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ uniq_keys,
               const int4* __restrict__ grec, const int32_t* __restrict__ col_count,
@@ -1032,34 +1060,27 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
     __shared__ __align__(8) uint64_t s_mbar;
     __shared__ uint32_t s_tmem;
     __shared__ int s_ok;
-    // tensor-core variant: MMA row count (MB rows padded to 64) and bf16 operand tiles
+    // tensor-core variants: MMA row count 64 (the MB chunk rows, then rows nobody reads) and
+    // bf16 operand tiles of NS terms each (NT = 3 products for two terms)
+    constexpr bool TC = NT > 0;
+    constexpr int NS = NT == 3 ? 2 : 1;
     constexpr int MT = TC ? 64 : MB;
-    static_assert(!TC || (R == 64 && MB == 32 && N == 256), "tensor-core backward: rank 64, d_2 = 4");
+    constexpr int DAQ = 4;   // dA accumulators in tensor-memory columns [N, N + DAQ R)
+    static_assert(!TC || (R == 64 && MB == 32 && N == 256 && DAQ * R <= N), "tensor-core backward: rank 64, d_2 = 4");
     float* Bs = smem_f;                    // [R][N] swizzled (key row/4)            (fp32 variant)
-    uint16_t* Bb = reinterpret_cast<uint16_t*>(smem_f);   // N x R bf16 core matrices  (tensor-core variant)
-    float* As = smem_f + (TC ? R * N / 2 : R * N);        // [2][MT][R] fp32 swizzled or bf16 core matrices
+    uint16_t* Bb = reinterpret_cast<uint16_t*>(smem_f);   // NS x (N x R) bf16 core matrices (tensor cores)
+    float* As = smem_f + (TC ? NS * R * N / 2 : R * N);   // [2][MB][R] fp32 swizzled, or [2][NS][MB x R] bf16
     uint16_t* Abt = reinterpret_cast<uint16_t*>(As);
-    float* Cn = As + (TC ? MT * R : 2 * MB * R);          // [MB][N] swizzled (key row)
-    float* dCn = Cn + MB * N;              // [MB][N] swizzled (key row)
-    uint16_t* dCb = reinterpret_cast<uint16_t*>(dCn + MB * N);   // MT x N bf16 core matrices (tensor cores)
-    float* Hs = dCn + MB * N + (TC ? MT * N / 2 : 0);   // [2][NUB][P][D3]
+    float* Cn = As + (TC ? NS * MB * R : 2 * MB * R);     // [MB][N] swizzled (key row)
+    float* dCn = Cn + MB * N;              // [MB][N] swizzled (key row); tensor cores: then NS x (MB x N) bf16
+    uint16_t* dCb = reinterpret_cast<uint16_t*>(dCn);
+    float* Hs = dCn + MB * N;              // [2][NUB][P][D3]
     float* Ss = Hs + 2 * NUB * P * D3;     // [2][NUB][R][SR]
     if (has_error(status)) return;
     const int tid = threadIdx.x;
     uint32_t tmem = 0, parity = 0;
     bool failed = false;
     if constexpr (TC) {
-        // rows MB..63 of both A buffers and of the dC tile stay zero for the whole kernel
-        for (int q = tid; q < 2 * (MT - MB) * R / 8; q += kBwdThreads) {
-            const int buf = q / ((MT - MB) * R / 8), r = q % ((MT - MB) * R / 8);
-            const int m = MB + r / (R / 8), kc = r % (R / 8);
-            *reinterpret_cast<uint4*>(Abt + buf * MT * R + ((m >> 3) * (R / 8) + kc) * 64 + (m & 7) * 8) =
-                make_uint4(0u, 0u, 0u, 0u);
-        }
-        for (int q = tid; q < (MT - MB) * N / 8; q += kBwdThreads) {
-            const int m = MB + q / (N / 8), nc = q % (N / 8);
-            *reinterpret_cast<uint4*>(dCb + ((m >> 3) * (N / 8) + nc) * 64 + (m & 7) * 8) = make_uint4(0u, 0u, 0u, 0u);
-        }
         // tensor memory: columns [0, N) hold dB of the current column group, [N, 2N) C and then dA
         if (tid < 32) tmem_alloc(&s_tmem, 2 * N);
         if (tid == 0) mbar_init(&s_mbar, 1);
@@ -1091,8 +1112,8 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
 
         // B for the whole column group, and the first chunk's A
         if constexpr (TC) {
-            const uint16_t* src = cp.bf2[t] + (int64_t)i2 * (R * N);
-            for (int q = tid; q < R * N / 8; q += kBwdThreads) cp_async16(Bb + q * 8, src + q * 8);
+            const uint16_t* src = cp.bf2[t] + (int64_t)i2 * (NS * R * N);
+            for (int q = tid; q < NS * R * N / 8; q += kBwdThreads) cp_async16(Bb + q * 8, src + q * 8);
         } else {
             const float* G2 = cp.cores[t][1] + (int64_t)i2 * N;
             const int64_t rs = (int64_t)n2 * N;
@@ -1102,7 +1123,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             }
         }
         bwd_meta<S, K>(cfirst, 0, ccount, 0, uniq_keys, grec, M, s_keys);
-        if constexpr (TC) bwd_issue_a_tc<S>(cp, t, 0, M, Abt);
+        if constexpr (TC) bwd_issue_a_tc<S, NS>(cp, t, 0, M, Abt);
         else bwd_issue_a<S>(cp, t, 0, M, As);
         TT_PH(8);
 
@@ -1120,7 +1141,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
         for (int j0 = 0; j0 < ccount; j0 += MPB, mb ^= 1) {
             const int cnt = M.cnt[mb];
             const float* Ab = As + mb * MB * R;
-            const uint16_t* Ab16 = Abt + mb * MT * R;
+            const uint16_t* Ab16 = Abt + mb * NS * MB * R;
             cp_async_wait_all();   // B, this chunk's A rows and row keys (usually prefetched long ago)
             __syncthreads();
             // the first batch of distinct rows is in flight during the C GEMM
@@ -1132,8 +1153,8 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             TT_PH(9);
 
             if constexpr (TC) {
-                // C_all = A . B on the tensor cores (M = 64 with rows MB.. zero, N, K = R) into
-                // tensor-memory columns [N, 2N), then rows < MB into Cn (sub-partitions 0 and 1)
+                // C_all = A . B on the tensor cores (M = 64, N, K = R) into tensor-memory columns
+                // [N, 2N), then rows < MB into Cn (sub-partitions 0 and 1)
                 fence_async_smem();
                 __syncthreads();
                 if (tid == 0) {
@@ -1142,8 +1163,8 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                     const uint32_t a0 = smem_u32(Ab16), b0 = smem_u32(Bb);
 #pragma unroll
                     for (int k = 0; k < R / 16; ++k)
-                        tc_mma_bf16(tmem + N, umma_desc(a0 + k * 256, 128, SBO), umma_desc(b0 + k * 256, 128, SBO),
-                                    umma_idesc_bf16(MT, N), k > 0);
+                        tc_mma_terms<NT>(tmem + N, umma_desc(a0 + k * 256, 128, SBO), umma_desc(b0 + k * 256, 128, SBO),
+                                         MB * R * 2, R * N * 2, umma_idesc_bf16(MT, N), k > 0);
                 }
                 if (!tc_commit_wait(&s_mbar, parity, &s_ok)) {
                     failed = true;
@@ -1211,7 +1232,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             const bool more = j0 + MPB < ccount;
             if (more) {
                 bwd_meta<S, K>(cfirst, j0 + MPB, ccount, mb ^ 1, uniq_keys, grec, M, s_keys);
-                if constexpr (TC) bwd_issue_a_tc<S>(cp, t, mb ^ 1, M, Abt + (mb ^ 1) * MT * R);
+                if constexpr (TC) bwd_issue_a_tc<S, NS>(cp, t, mb ^ 1, M, Abt + (mb ^ 1) * NS * MB * R);
                 else bwd_issue_a<S>(cp, t, mb ^ 1, M, As + (mb ^ 1) * MB * R);
             }
 
@@ -1312,33 +1333,56 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             }
 
             if constexpr (TC) {
-                // dC -> bf16 core matrices (M = 64, K = N); then on the tensor cores
+                // dC -> NS bf16 terms in core matrices (MB rows, K = N), written over dCn once
+                // every thread holds its share in registers; then on the tensor cores
                 //   dA = dC . B^T   (M = 64, N = R, K = N) into columns [N, N + R)
                 //   dB += A^T . dC  (M = R, N, K = MB)     into columns [0, N), over the column group
-                for (int q = tid; q < MB * N / 8; q += kBwdThreads) {
-                    const int m = q / (N / 8), nc = q % (N / 8);
-                    const float4 x0 = *reinterpret_cast<const float4*>(&dCn[swz_m<N>(m, nc * 8)]);
-                    const float4 x1 = *reinterpret_cast<const float4*>(&dCn[swz_m<N>(m, nc * 8 + 4)]);
-                    const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-                    *reinterpret_cast<uint4*>(dCb + ((m >> 3) * (N / 8) + nc) * 64 + (m & 7) * 8) = pack_bf16x8(v);
+                {
+                    constexpr int CPT = MB * N / 8 / kBwdThreads;   // 16-byte chunks per thread
+                    static_assert(CPT * kBwdThreads * 8 == MB * N, "dC conversion tiling");
+                    float v[CPT][8];
+#pragma unroll
+                    for (int i = 0; i < CPT; ++i) {
+                        const int q = tid + i * kBwdThreads, m = q / (N / 8), nc = q % (N / 8);
+                        const float4 x0 = *reinterpret_cast<const float4*>(&dCn[swz_m<N>(m, nc * 8)]);
+                        const float4 x1 = *reinterpret_cast<const float4*>(&dCn[swz_m<N>(m, nc * 8 + 4)]);
+                        v[i][0] = x0.x; v[i][1] = x0.y; v[i][2] = x0.z; v[i][3] = x0.w;
+                        v[i][4] = x1.x; v[i][5] = x1.y; v[i][6] = x1.z; v[i][7] = x1.w;
+                    }
+                    __syncthreads();
+#pragma unroll
+                    for (int i = 0; i < CPT; ++i) {
+                        const int q = tid + i * kBwdThreads, m = q / (N / 8), nc = q % (N / 8);
+                        uint16_t* dst = dCb + ((m >> 3) * (N / 8) + nc) * 64 + (m & 7) * 8;
+                        uint4 hi, lo;
+                        split_bf16x8(v[i], hi, lo);
+                        *reinterpret_cast<uint4*>(dst) = hi;
+                        if constexpr (NS == 2) *reinterpret_cast<uint4*>(dst + MB * N) = lo;
+                    }
                 }
                 fence_async_smem();
                 __syncthreads();
                 if (tid == 0) {
                     tc_fence_after();
                     const uint32_t c0 = smem_u32(dCb), b0 = smem_u32(Bb), a0 = smem_u32(Ab16);
-                    // dA: A = dC (K-major: 8-row groups 16 N bytes apart), B = B viewed MN-major
+                    // dA: A = dC (K-major: 8-row groups 16 N bytes apart), B = B viewed MN-major.
+                    // The K range is split over DAQ accumulators (columns N + q R) issued in turn,
+                    // so the small M = 64 x N = R products do not form one serial chain.
 #pragma unroll 1
-                    for (int k = 0; k < N / 16; ++k)
-                        tc_mma_bf16(tmem + N, umma_desc(c0 + k * 256, 128, (N / 8) * 128),
-                                    umma_desc_mn(b0 + k * 2 * (R / 8) * 128, 128, (R / 8) * 128),
-                                    umma_idesc_bf16(MT, R, false, true), k > 0);
+                    for (int kk = 0; kk < N / 16 / DAQ; ++kk)
+#pragma unroll
+                        for (int q = 0; q < DAQ; ++q) {
+                            const int k = q * (N / 16 / DAQ) + kk;
+                            tc_mma_terms<NT>(tmem + N + q * R, umma_desc(c0 + k * 256, 128, (N / 8) * 128),
+                                             umma_desc_mn(b0 + k * 2 * (R / 8) * 128, 128, (R / 8) * 128),
+                                             MB * N * 2, R * N * 2, umma_idesc_bf16(MT, R, false, true), kk > 0);
+                        }
                     // dB: A = A^T (MN-major over the A tile), B = dC viewed MN-major
 #pragma unroll
                     for (int k = 0; k < MB / 16; ++k)
-                        tc_mma_bf16(tmem, umma_desc_mn(a0 + k * 2 * (R / 8) * 128, 128, (R / 8) * 128),
-                                    umma_desc_mn(c0 + k * 2 * (N / 8) * 128, 128, (N / 8) * 128),
-                                    umma_idesc_bf16(R, N, true, true), (j0 > 0 || k > 0) ? 1u : 0u);
+                        tc_mma_terms<NT>(tmem, umma_desc_mn(a0 + k * 2 * (R / 8) * 128, 128, (R / 8) * 128),
+                                         umma_desc_mn(c0 + k * 2 * (N / 8) * 128, 128, (N / 8) * 128),
+                                         MB * R * 2, MB * N * 2, umma_idesc_bf16(R, N, true, true), j0 > 0 || k > 0);
                 }
                 if (!tc_commit_wait(&s_mbar, parity, &s_ok)) {
                     failed = true;
@@ -1347,10 +1391,17 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                 tc_fence_after();
                 TT_PH(13);
                 const int warp = tid >> 5, lane = tid & 31, sub = warp & 3, half = warp >> 2;
-                if (sub < 2) {   // dA rows 16 sub + lane, columns half * R / 2 ..
+                if (sub < 2) {   // dA rows 16 sub + lane, columns half * R / 2 .., summed over the accumulators
                     const int m = 16 * sub + lane, p = m / D1, a1 = m % D1;
                     float v[32];
                     tmem_ld32(tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)(N + half * 32), v);
+#pragma unroll 1
+                    for (int q = 1; q < DAQ; ++q) {
+                        float x[32];
+                        tmem_ld32(tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)(N + q * R + half * 32), x);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] += x[i];
+                    }
                     if (lane < 16 && p < cnt) {
                         float* dst = dG1 + ((int64_t)M.i1[mb][p] * D1 + a1) * R + half * 32;
 #pragma unroll
@@ -1502,7 +1553,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
 // one per i_2, in the operand order of fwd_issue_ab_tc: element (n, k) of the tile
 // (n = a_2 r_2 + rho_2, k = rho_1) at ((n / 8) (R / 8) + k / 8) 64 + (n % 8) 8 + k % 8.
 struct Bf16Job {
-    int32_t T, R, N, pad;
+    int32_t T, R, N, NS;   // NS = 2: every value as two bf16 terms (hi, lo), stored as two tiles / row halves
     int64_t base1[kMaxT + 1], base2[kMaxT + 1];   // prefix sums of chunk counts
     uint32_t n2[kMaxT];
     const float* src1[kMaxT];
@@ -1530,6 +1581,7 @@ __global__ void __launch_bounds__(256) k3_bf16_kernel(Bf16Job j)
     for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < tot1 + tot2;
          q += (int64_t)gridDim.x * blockDim.x) {
         float v[8];
+        uint4 hi, lo;
         if (q < tot1) {
             const int t = table_of(j.base1, j.T, q);
             const int64_t off = (q - j.base1[t]) * 8;
@@ -1537,7 +1589,12 @@ __global__ void __launch_bounds__(256) k3_bf16_kernel(Bf16Job j)
             const float4 x1 = __ldg(reinterpret_cast<const float4*>(j.src1[t] + off + 4));
             v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
             v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
-            *reinterpret_cast<uint4*>(j.dst1[t] + off) = pack_bf16x8(v);
+            // row (i_1, a_1) of R values -> NS halves of R bf16 values
+            const int64_t row = off / j.R, e = off % j.R;
+            uint16_t* dst = j.dst1[t] + row * (j.NS * j.R) + e;
+            split_bf16x8(v, hi, lo);
+            *reinterpret_cast<uint4*>(dst) = hi;
+            if (j.NS == 2) *reinterpret_cast<uint4*>(dst + j.R) = lo;
         } else {
             const int64_t q2 = q - tot1;
             const int t = table_of(j.base2, j.T, q2);
@@ -1549,7 +1606,10 @@ __global__ void __launch_bounds__(256) k3_bf16_kernel(Bf16Job j)
             const float* src = j.src2[t] + i2 * j.N + n + (int64_t)kc * 8 * rs;
 #pragma unroll
             for (int e = 0; e < 8; ++e) v[e] = __ldg(src + e * rs);
-            *reinterpret_cast<uint4*>(j.dst2[t] + i2 * (j.R * j.N) + (int64_t)c * 8) = pack_bf16x8(v);
+            uint16_t* dst = j.dst2[t] + i2 * ((int64_t)j.NS * j.R * j.N) + (int64_t)c * 8;
+            split_bf16x8(v, hi, lo);
+            *reinterpret_cast<uint4*>(dst) = hi;
+            if (j.NS == 2) *reinterpret_cast<uint4*>(dst + (int64_t)j.R * j.N) = lo;
         }
     }
 }
@@ -1581,14 +1641,26 @@ __global__ void __launch_bounds__(256) k3_transpose_last_kernel(TransposeJob tj,
 // ---------------------------------------------------------------------------
 // host launchers
 // ---------------------------------------------------------------------------
-template <class S, typename K, bool TC>
+// NT: 0 = FP32 pipes, 1 = bf16 tensor-core products, 3 = fp32-accurate split-bf16 products
+template <class S, int NT>
+constexpr size_t fwd_smem_bytes()
+{
+    return sizeof(float) * (NT == 0 ? S::fwd_smem_floats() : S::fwd_smem_floats_tc(NT == 3 ? 2 : 1));
+}
+template <class S, int NT>
+constexpr size_t bwd_smem_bytes()
+{
+    return sizeof(float) * (NT == 0 ? S::bwd_smem_floats() : S::bwd_smem_floats_tc(NT == 3 ? 2 : 1));
+}
+
+template <class S, typename K, int NT>
 cudaError_t fwd_launch(const K3Args& a, float* out, cudaStream_t s, int* nl)
 {
-    const size_t smem = sizeof(float) * (TC ? S::fwd_smem_floats_tc() : S::fwd_smem_floats());
-    cudaError_t e = cudaFuncSetAttribute(k3_fwd_kernel<S, K, TC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = fwd_smem_bytes<S, NT>();
+    cudaError_t e = cudaFuncSetAttribute(k3_fwd_kernel<S, K, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const PlanBuffers& pb = *a.pb;
-    k3_fwd_kernel<S, K, TC><<<a.grid, kFwdThreads, smem, s>>>(
+    k3_fwd_kernel<S, K, NT><<<a.grid, kFwdThreads, smem, s>>>(
         *a.cp, a.pp->sched, (const K*)a.uniq_keys, a.grec, a.uid_at_pos, a.offsets,
         pb.chunks, pb.tasks, pb.hdr, a.rowbuf, out, a.status);
     *nl += 1;
@@ -1607,15 +1679,15 @@ cudaError_t rowsum_launch(const K3Args& a, const float* grad_out, cudaStream_t s
     return cudaGetLastError();
 }
 
-template <class S, typename K, bool TC>
+template <class S, typename K, int NT>
 cudaError_t bwd_launch(const K3Args& a, const GradPtrs& gp, const float* grad_out, cudaStream_t s, int* nl)
 {
     (void)grad_out;
-    const size_t smem = sizeof(float) * (TC ? S::bwd_smem_floats_tc() : S::bwd_smem_floats());
-    cudaError_t e = cudaFuncSetAttribute(k3_bwd_kernel<S, K, TC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = bwd_smem_bytes<S, NT>();
+    cudaError_t e = cudaFuncSetAttribute(k3_bwd_kernel<S, K, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const PlanBuffers& pb = *a.pb;
-    k3_bwd_kernel<S, K, TC><<<a.grid, kBwdThreads, smem, s>>>(
+    k3_bwd_kernel<S, K, NT><<<a.grid, kBwdThreads, smem, s>>>(
         *a.cp, gp, *a.pp, (const K*)a.uniq_keys, a.grec, pb.col_count, pb.col_start, pb.hdr, a.rowbuf,
         a.status);
     *nl += 1;
@@ -1625,42 +1697,45 @@ cudaError_t bwd_launch(const K3Args& a, const GradPtrs& gp, const float* grad_ou
 template <class S>
 cudaError_t fwd_dispatch(const K3Args& a, float* out, cudaStream_t s, int* nl)
 {
-    return a.key64 ? fwd_launch<S, uint64_t, false>(a, out, s, nl) : fwd_launch<S, uint32_t, false>(a, out, s, nl);
+    return a.key64 ? fwd_launch<S, uint64_t, 0>(a, out, s, nl) : fwd_launch<S, uint32_t, 0>(a, out, s, nl);
 }
 template <class S>
 cudaError_t fwd_dispatch_tc(const K3Args& a, float* out, cudaStream_t s, int* nl)
 {
-    return a.key64 ? fwd_launch<S, uint64_t, true>(a, out, s, nl) : fwd_launch<S, uint32_t, true>(a, out, s, nl);
+    if (a.tc == 3)
+        return a.key64 ? fwd_launch<S, uint64_t, 3>(a, out, s, nl) : fwd_launch<S, uint32_t, 3>(a, out, s, nl);
+    return a.key64 ? fwd_launch<S, uint64_t, 1>(a, out, s, nl) : fwd_launch<S, uint32_t, 1>(a, out, s, nl);
 }
 template <class S>
 cudaError_t bwd_dispatch(const K3Args& a, const GradPtrs& gp, const float* g, cudaStream_t s, int* nl)
 {
-    return a.key64 ? bwd_launch<S, uint64_t, false>(a, gp, g, s, nl) : bwd_launch<S, uint32_t, false>(a, gp, g, s, nl);
+    return a.key64 ? bwd_launch<S, uint64_t, 0>(a, gp, g, s, nl) : bwd_launch<S, uint32_t, 0>(a, gp, g, s, nl);
 }
 template <class S>
 cudaError_t bwd_dispatch_tc(const K3Args& a, const GradPtrs& gp, const float* g, cudaStream_t s, int* nl)
 {
-    return a.key64 ? bwd_launch<S, uint64_t, true>(a, gp, g, s, nl) : bwd_launch<S, uint32_t, true>(a, gp, g, s, nl);
+    if (a.tc == 3)
+        return a.key64 ? bwd_launch<S, uint64_t, 3>(a, gp, g, s, nl) : bwd_launch<S, uint32_t, 3>(a, gp, g, s, nl);
+    return a.key64 ? bwd_launch<S, uint64_t, 1>(a, gp, g, s, nl) : bwd_launch<S, uint32_t, 1>(a, gp, g, s, nl);
 }
 
-template <class S, bool TC>
+template <class S, int NT>
 int occ_fwd()
 {
-    const size_t smem = sizeof(float) * (TC ? S::fwd_smem_floats_tc() : S::fwd_smem_floats());
-    cudaFuncSetAttribute(k3_fwd_kernel<S, uint32_t, TC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = fwd_smem_bytes<S, NT>();
+    cudaFuncSetAttribute(k3_fwd_kernel<S, uint32_t, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k3_fwd_kernel<S, uint32_t, TC>, kFwdThreads, smem) != cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k3_fwd_kernel<S, uint32_t, NT>, kFwdThreads, smem) != cudaSuccess)
         return 1;
-    // one block per SM holds tensor memory: the kernel allocates N columns and keeps them
-    return n > 0 ? (TC ? 1 : n) : 1;
+    return n > 0 ? n : 1;
 }
 template <class S>
 int occ_bwd()
 {
     const size_t smem = sizeof(float) * S::bwd_smem_floats();
-    cudaFuncSetAttribute(k3_bwd_kernel<S, uint32_t, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(k3_bwd_kernel<S, uint32_t, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k3_bwd_kernel<S, uint32_t, false>, kBwdThreads, smem) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k3_bwd_kernel<S, uint32_t, 0>, kBwdThreads, smem) !=
         cudaSuccess)
         return 1;
     return n > 0 ? n : 1;
@@ -1672,7 +1747,7 @@ int k3_blocks_per_sm(const CoreParams& cp, bool backward, bool tc)
 {
     if (tc) return 1;   // tensor-core variants hold tensor memory: one block per SM
 #define TT_OCC_CASE(Q1, Q2, Q3, QR) \
-    if (cp.d[0] == Q1 && cp.d[2] == Q3 && cp.r[1] == QR) return backward ? occ_bwd<S3<Q1, Q2, Q3, QR>>() : occ_fwd<S3<Q1, Q2, Q3, QR>, false>();
+    if (cp.d[0] == Q1 && cp.d[2] == Q3 && cp.r[1] == QR) return backward ? occ_bwd<S3<Q1, Q2, Q3, QR>>() : occ_fwd<S3<Q1, Q2, Q3, QR>, 0>();
     TT_K3_CASES_INNER(TT_OCC_CASE)
 #undef TT_OCC_CASE
     return 1;
@@ -1744,11 +1819,13 @@ cudaError_t k3_transpose_last(const CoreParams& cp, float* const* dst, cudaStrea
     return cudaGetLastError();
 }
 
-cudaError_t k3_to_bf16(const CoreParams& cp, uint16_t* const* dst1, uint16_t* const* dst2, cudaStream_t s, int* nl)
+cudaError_t k3_to_bf16(const CoreParams& cp, int terms, uint16_t* const* dst1, uint16_t* const* dst2,
+                      cudaStream_t s, int* nl)
 {
     Bf16Job j;
     memset(&j, 0, sizeof(j));
     j.T = cp.T;
+    j.NS = terms;
     j.R = cp.r[1];
     j.N = cp.d[1] * cp.r[2];
     int64_t b1 = 0, b2 = 0;

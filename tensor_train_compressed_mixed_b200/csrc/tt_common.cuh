@@ -63,8 +63,8 @@ struct CoreParams {
     // specialised path: the last core re-laid out as [n_k][r_{k-1}][d_k], so that one
     // row's last slice is a contiguous block (built by k3_transpose_last each forward)
     const float* last_t[kMaxT];
-    // bf16 tensor-core prefix step: G_1 as [n_1][d_1][r_1] and G_2 as one operand tile per
-    // i_2 (n = (a_2, rho_2) rows x K = rho_1, 8 x 8 core matrices), built by k3_to_bf16
+    // tensor-core prefix step: G_1 as [n_1][d_1][terms][r_1] and G_2 as [n_2][terms] operand
+    // tiles (n = (a_2, rho_2) rows x K = rho_1, 8 x 8 core matrices) in bf16, built by k3_to_bf16
     const uint16_t* bf1[kMaxT];
     const uint16_t* bf2[kMaxT];
 };
@@ -222,7 +222,8 @@ struct K3Args {
     float* rowbuf;                 // [U][D]: pooled-row checkpoint (forward), upstream sums (backward)
     int64_t L;
     int grid;
-    int tc;                        // 1: prefix GEMM on the tensor cores (bf16 operands)
+    int tc;                        // prefix-level products on the tensor cores: 0 = no (FP32 pipes),
+                                   // 1 = bf16 operands, 3 = two bf16 terms per operand (three products)
     int32_t* status;
 };
 // Four-core tables run the three-core kernels on the merged first core
@@ -251,7 +252,9 @@ bool k3_tc_supported(const CoreParams& cp);
 // shapes whose backward also runs its prefix-level products on the tensor cores (rank 64)
 bool k3_tc_bwd_supported(const CoreParams& cp);
 // bf16 operand copies of G_1 and G_2 for the tensor-core forward (cp.cores -> dst1/dst2)
-cudaError_t k3_to_bf16(const CoreParams& cp, uint16_t* const* dst1, uint16_t* const* dst2, cudaStream_t s, int* nl);
+// terms = 2 stores every value as hi = bf16(x) and lo = bf16(x - hi)
+cudaError_t k3_to_bf16(const CoreParams& cp, int terms, uint16_t* const* dst1, uint16_t* const* dst2,
+                      cudaStream_t s, int* nl);
 cudaError_t k3_forward(const K3Args& a, float* out, cudaStream_t s, int* nl);
 // last core [r][n_k][d_k] -> [n_k][r][d_k] into cp.last_t (before k3_forward / k3_backward)
 cudaError_t k3_transpose_last(const CoreParams& cp, float* const* dst, cudaStream_t s, int* nl);

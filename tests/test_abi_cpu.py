@@ -73,7 +73,7 @@ def test_create_rejects_bad_options_on_host():
         abi.tt_emb_create([[2, 3]], [6], [2, 2], [1, 4, 1], o)
     assert e.value.code == abi.TT_ERR_ARG
     o = abi.tt_emb_default_options()
-    o.precision = 2
+    o.precision = 3
     with pytest.raises(abi.TTEmbError) as e:
         abi.tt_emb_create([[2, 3]], [6], [2, 2], [1, 4, 1], o)
     assert e.value.code == abi.TT_ERR_ARG
@@ -100,10 +100,11 @@ def test_null_handle_calls_fail_cleanly():
     ([[2, 3]], [2, 2], [1, 4, 1]),                 # two cores
     ([[2, 5, 6, 7]], [2, 4, 4, 4], [1, 32, 32, 32, 1]),  # four cores
 ])
-def test_bf16_tensor_core_precision_rejects_other_shapes(n, d, r):
-    o = abi.tt_emb_default_options()
-    o.precision = abi.TT_PREC_BF16_TC
+def test_tensor_core_precisions_reject_other_shapes(n, d, r):
     rows = [int(__import__("numpy").prod(x)) for x in n]
-    with pytest.raises(abi.TTEmbError) as e:
-        abi.tt_emb_create(n, rows, d, r, o)
-    assert e.value.code == abi.TT_ERR_SHAPE
+    for prec in (abi.TT_PREC_BF16_TC, abi.TT_PREC_FP32_SPLIT_TC):
+        o = abi.tt_emb_default_options()
+        o.precision = prec
+        with pytest.raises(abi.TTEmbError) as e:
+            abi.tt_emb_create(n, rows, d, r, o)
+        assert e.value.code == abi.TT_ERR_SHAPE

@@ -52,17 +52,17 @@ def test_full_size_forward_sampled_bags(cfg):
     emb.close()
 
 
-@pytest.mark.parametrize("cfg", [3, 4])
-def test_full_size_bf16_forward_sampled_bags(cfg):
+@pytest.mark.parametrize("cfg,prec", [(3, "bf16"), (4, "bf16"), (4, "split")])
+def test_full_size_tensor_core_forward_sampled_bags(cfg, prec):
     from tensor_train_compressed_mixed_b200 import abi
     w = config_workload(cfg, with_grad=False)
     o = abi.tt_emb_default_options()
-    o.precision = abi.TT_PREC_BF16_TC
+    o.precision = abi.TT_PREC_BF16_TC if prec == "bf16" else abi.TT_PREC_FP32_SPLIT_TC
     emb, cores, out = _forward_full(w, o)
     bags = _sample_bags(w)
     got = out.cpu().numpy()[bags]
     want = oracle.workload_forward(sub_batch(w, bags))
-    assert output_err(got, want, w.dim) <= BF16_TOL
+    assert output_err(got, want, w.dim) <= (BF16_TOL if prec == "bf16" else FP32_TOL)
     emb.close()
 
 
@@ -113,13 +113,17 @@ def _restrict(w, t, j, digit):
                     grad_out=w.grad_out, lr=w.lr, train=w.train, meta=dict(w.meta))
 
 
-def test_full_size_backward_sampled_slices():
+@pytest.mark.parametrize("prec", ["fp32", "split"])
+def test_full_size_backward_sampled_slices(prec):
     """Whole digit slices dG_{t,j}[:, i] of the rank-64 training step: only the lookups
     with digit i touch the slice, so the oracle run on those lookups alone gives it."""
     import torch
+    from tensor_train_compressed_mixed_b200 import abi
     from tests.parity import core_grad_err
     w = config_workload(4, with_grad=True)
-    emb, cores, out = _forward_full(w)
+    o = abi.tt_emb_default_options()
+    o.precision = abi.TT_PREC_FP32 if prec == "fp32" else abi.TT_PREC_FP32_SPLIT_TC
+    emb, cores, out = _forward_full(w, o)
     g = torch.from_numpy(w.grad_out).cuda()
     emb.backward(g)
     emb.sync()

@@ -120,3 +120,53 @@ def test_bf16_scheduler_modes_agree_bitwise():
         o.sched = sched
         outs.append(gpu_forward(w, options=o)[2].cpu().numpy())
     assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2])
+
+
+# ---------------------------------------------------------------------------
+# TT_PREC_FP32_SPLIT_TC: two bf16 terms per operand value, three products; the fp32 bound
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("case", range(len(TC_SHAPES)))
+def test_split_forward_meets_fp32_bound(case):
+    from tensor_train_compressed_mixed_b200 import abi
+    d, r, n, rows, batch = TC_SHAPES[case]
+    w = random_workload(900 + case, d, r, n, rows, batch=batch,
+                        pooling={"kind": "uniform", "lo": 0, "hi": 40}, with_grad=False)
+    emb, cores, out = gpu_forward(w, options=_opts(abi.TT_PREC_FP32_SPLIT_TC))
+    err = output_err(out.cpu().numpy(), oracle.workload_forward(w), w.dim)
+    assert err <= FP32_TOL, err
+
+
+@pytest.mark.parametrize("cfg,batch,tables", [(3, 64, 4), (4, 40, 3)])
+def test_split_forward_benchmark_shapes(cfg, batch, tables):
+    from tensor_train_compressed_mixed_b200 import abi
+    w = config_workload(cfg, batch=batch, tables=tables, with_grad=False)
+    emb, cores, out = gpu_forward(w, options=_opts(abi.TT_PREC_FP32_SPLIT_TC))
+    err = output_err(out.cpu().numpy(), oracle.workload_forward(w), w.dim)
+    assert err <= FP32_TOL, err
+
+
+def test_split_training_step_rank64_meets_fp32_bound():
+    from tensor_train_compressed_mixed_b200 import abi
+    w = config_workload(4, batch=24, tables=3, with_grad=True)
+    _, out, grads, new = gpu_train_step(w, options=_opts(abi.TT_PREC_FP32_SPLIT_TC), lr=0.01)
+    assert output_err(out, oracle.workload_forward(w), w.dim) <= FP32_TOL
+    want = oracle.workload_backward(w)
+    for t in range(w.num_tables):
+        for j in range(w.num_cores):
+            assert core_grad_err(grads[t][j], want[t][j]) <= FP32_TOL, (t, j)
+    upd = oracle.sgd(w.cores, want, 0.01)
+    for t in range(w.num_tables):
+        for j in range(w.num_cores):
+            assert core_grad_err(new[t][j], upd[t][j]) <= FP32_TOL, (t, j)
+
+
+def test_split_training_many_chunks_per_column():
+    from tensor_train_compressed_mixed_b200 import abi
+    w = random_workload(960, (4, 4, 8), (1, 64, 64, 1), [(60, 2, 9), (33, 3, 5)], batch=120,
+                        pooling={"kind": "uniform", "lo": 0, "hi": 30}, with_grad=True)
+    _, out, grads, _ = gpu_train_step(w, options=_opts(abi.TT_PREC_FP32_SPLIT_TC))
+    assert output_err(out, oracle.workload_forward(w), w.dim) <= FP32_TOL
+    want = oracle.workload_backward(w)
+    for t in range(w.num_tables):
+        for j in range(w.num_cores):
+            assert core_grad_err(grads[t][j], want[t][j]) <= FP32_TOL, (t, j)
