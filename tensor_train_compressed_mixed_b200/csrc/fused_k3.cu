@@ -481,8 +481,10 @@ __device__ __forceinline__ void fwd_issue_ab_tc(const CoreParams& cp, int mb, co
     }
     const uint16_t* G1 = cp.bf1[t];
     for (int q = tid; q < NS * MF * KC; q += kFwdThreads) {
+        // 8 consecutive threads fill one 128-byte core matrix (rows m % 8), so shared-memory
+        // writes of a warp are contiguous
         const int term = q / (MF * KC), r = q % (MF * KC);
-        const int m = r / KC, kc = r % KC;
+        const int m = (r / (8 * KC)) * 8 + (r & 7), kc = (r >> 3) % KC;
         const int j = m / D1, a1 = m % D1;
         uint16_t* dst = sm.Ab + term * (MF * R) + ((m >> 3) * KC + kc) * 64 + (m & 7) * 8;
         if (j < cnt) cp_async16(dst, G1 + ((int64_t)M.i1[mb][j] * D1 + a1) * (NS * R) + term * R + kc * 8);
@@ -1024,7 +1026,7 @@ __device__ __forceinline__ void bwd_issue_a_tc(const CoreParams& cp, int t, int 
     const int cnt = M.cnt[mb];
     for (int q = threadIdx.x; q < NS * MB * KC; q += kBwdThreads) {
         const int term = q / (MB * KC), r = q % (MB * KC);
-        const int m = r / KC, kc = r % KC;
+        const int m = (r / (8 * KC)) * 8 + (r & 7), kc = (r >> 3) % KC;   // 8 threads per core matrix
         const int j = m / D1, a1 = m % D1;
         uint16_t* dst = Ab + term * (MB * R) + ((m >> 3) * KC + kc) * 64 + (m & 7) * 8;
         if (j < cnt) cp_async16(dst, G1 + ((int64_t)M.i1[mb][j] * D1 + a1) * (NS * R) + term * R + kc * 8);
@@ -1340,10 +1342,13 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                 {
                     constexpr int CPT = MB * N / 8 / kBwdThreads;   // 16-byte chunks per thread
                     static_assert(CPT * kBwdThreads * 8 == MB * N, "dC conversion tiling");
+                    // chunk q: core matrix (m / 8, nc), row m % 8 = q % 8: 8 consecutive threads
+                    // write one contiguous 128-byte core matrix
                     float v[CPT][8];
 #pragma unroll
                     for (int i = 0; i < CPT; ++i) {
-                        const int q = tid + i * kBwdThreads, m = q / (N / 8), nc = q % (N / 8);
+                        const int q = tid + i * kBwdThreads;
+                        const int m = (q / (8 * (N / 8))) * 8 + (q & 7), nc = (q >> 3) % (N / 8);
                         const float4 x0 = *reinterpret_cast<const float4*>(&dCn[swz_m<N>(m, nc * 8)]);
                         const float4 x1 = *reinterpret_cast<const float4*>(&dCn[swz_m<N>(m, nc * 8 + 4)]);
                         v[i][0] = x0.x; v[i][1] = x0.y; v[i][2] = x0.z; v[i][3] = x0.w;
@@ -1352,7 +1357,8 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                     __syncthreads();
 #pragma unroll
                     for (int i = 0; i < CPT; ++i) {
-                        const int q = tid + i * kBwdThreads, m = q / (N / 8), nc = q % (N / 8);
+                        const int q = tid + i * kBwdThreads;
+                        const int m = (q / (8 * (N / 8))) * 8 + (q & 7), nc = (q >> 3) % (N / 8);
                         uint16_t* dst = dCb + ((m >> 3) * (N / 8) + nc) * 64 + (m & 7) * 8;
                         uint4 hi, lo;
                         split_bf16x8(v[i], hi, lo);
