@@ -332,6 +332,11 @@ struct FwdSmem {
     float* Ss;   // [FBUF][NUF][SU] last slices of a batch of distinct rows
 };
 
+// Per chunk buffer, for the chunk's first kKeyCap distinct rows: row id, prefix slot, last digit.
+struct RowTable {
+    int u[2][kKeyCap], p[2][kKeyCap], i3[2][kKeyCap];
+};
+
 template <class S>
 struct FwdMeta {   // shared-memory metadata of a chunk (double buffered)
     int u0[2][S::MPF];
@@ -341,6 +346,7 @@ struct FwdMeta {   // shared-memory metadata of a chunk (double buffered)
     int bu[2][S::NUF], bp[2][S::NUF], bi3[2][S::NUF];
     int task[2];
     int flag;
+    RowTable rows;
 };
 
 // Index of the prefix (0..cnt-1) holding the chunk's distinct row number kq.
@@ -349,6 +355,35 @@ __device__ __forceinline__ int prefix_of(const int* ucum, int cnt, int kq)
     int j = 0;
     while (j + 1 < cnt && ucum[j + 1] <= kq) ++j;
     return j;
+}
+
+// The chunk's row table: for its first kKeyCap distinct rows, the row id, the prefix slot and
+// the last digit, computed once per chunk by all threads from the staged keys (which must have
+// landed and be visible).  Batches inside the table then need no per-batch metadata pass.
+template <typename K>
+__device__ __forceinline__ void build_rows(RowTable& rt, int mb, const int* ucum, const int* u0, int cnt, int total,
+                                           const K* keys, int ibits, uint32_t n3, int nthreads)
+{
+    const int n = min(total, kKeyCap);
+    for (int kq = threadIdx.x; kq < n; kq += nthreads) {
+        const int j = prefix_of(ucum, cnt, kq);
+        rt.u[mb][kq] = u0[j] + (kq - ucum[j]);
+        rt.p[mb][kq] = j;
+        rt.i3[mb][kq] = (int)(key_row(keys[mb * kKeyCap + kq], ibits) % n3);
+    }
+}
+// Rows k0 .. k0 + nb of chunk buffer mb: the row table when it covers them, else the batch's own
+// metadata (filled by the batch issue)
+struct RowRef {
+    const int* u;
+    const int* p;
+    const int* i3;
+};
+__device__ __forceinline__ RowRef batch_rows(const RowTable& rt, int mb, int k0, int nb, const int* bu,
+                                             const int* bp, const int* bi3)
+{
+    if (k0 + nb <= kKeyCap) return RowRef{rt.u[mb] + k0, rt.p[mb] + k0, rt.i3[mb] + k0};
+    return RowRef{bu, bp, bi3};
 }
 
 // Metadata of chunk `cid` into buffer mb (all threads call; ends with a barrier), and
@@ -574,37 +609,41 @@ __device__ __forceinline__ void fwd_issue_batch(const CoreParams& cp, int mb, in
     const int nb = min(S::NUF, total - k0);
     const int t = M.t[mb];
     const uint32_t n3 = cp.n[t][2];
-    if (tid < nb) {
-        const int kq = k0 + tid;
-        const int j = prefix_of(M.ucum[mb], M.cnt[mb], kq);
-        const int u = M.u0[mb][j] + (kq - M.ucum[mb][j]);
-        const K key = kq < kKeyCap ? keys[mb * kKeyCap + kq] : uniq_keys[u];
-        M.bu[bb][tid] = u;
-        M.bp[bb][tid] = j;
-        M.bi3[bb][tid] = (int)(key_row(key, cp.ibits) % n3);
+    if (k0 + nb > kKeyCap) {   // beyond the row table: this batch's metadata
+        if (tid < nb) {
+            const int kq = k0 + tid;
+            const int j = prefix_of(M.ucum[mb], M.cnt[mb], kq);
+            const int u = M.u0[mb][j] + (kq - M.ucum[mb][j]);
+            const K key = kq < kKeyCap ? keys[mb * kKeyCap + kq] : uniq_keys[u];
+            M.bu[bb][tid] = u;
+            M.bp[bb][tid] = j;
+            M.bi3[bb][tid] = (int)(key_row(key, cp.ibits) % n3);
+        }
+        __syncthreads();
     }
-    __syncthreads();
+    const RowRef rr = batch_rows(M.rows, mb, k0, nb, M.bu[bb], M.bp[bb], M.bi3[bb]);
     const float* G3t = cp.last_t[t];   // [n3][R][D3]: one row's slice is contiguous
     float* Ss = sm.Ss + (size_t)bb * S::NUF * S::SU;
     for (int q = tid; q < nb * R * (D3 / 4); q += kFwdThreads) {
         const int uu = q / (R * (D3 / 4)), rem = q % (R * (D3 / 4));
-        cp_async16(&Ss[uu * S::SU + rem * 4], G3t + (int64_t)M.bi3[bb][uu] * (R * D3) + rem * 4);
+        cp_async16(&Ss[uu * S::SU + rem * 4], G3t + (int64_t)rr.i3[uu] * (R * D3) + rem * 4);
     }
     cp_async_commit();
 }
 
 // E_u = C_p . S_u for the batch in buffer bb; tile: rows (a1, a2 = 2h, 2h+1) x 4 columns of a3
 template <class S>
-__device__ __forceinline__ void fwd_batch_compute(int nb, int bb, const FwdMeta<S>& M, const FwdSmem<S>& sm,
-                                                  float* __restrict__ rowbuf)
+__device__ __forceinline__ void fwd_batch_compute(int mb, int k0, int nb, int bb, const FwdMeta<S>& M,
+                                                  const FwdSmem<S>& sm, float* __restrict__ rowbuf)
 {
     constexpr int R = S::R, N = S::N, D1 = S::D1, D2 = S::D2, D3 = S::D3;
     const int tid = threadIdx.x;
     const int uu = tid / S::TPU;
     if (uu >= nb) return;
+    const RowRef rr = batch_rows(M.rows, mb, k0, nb, M.bu[bb], M.bp[bb], M.bi3[bb]);
     const int rem = tid % S::TPU;
     const int a1 = rem / (2 * (D3 / 4)), h = (rem / (D3 / 4)) % 2, cg = rem % (D3 / 4);
-    const int m = M.bp[bb][uu] * D1 + a1;
+    const int m = rr.p[uu] * D1 + a1;
     const float* srow = sm.Ss + (size_t)bb * S::NUF * S::SU + uu * S::SU + cg * 4;
     float4 e[2];
 #pragma unroll
@@ -627,7 +666,7 @@ __device__ __forceinline__ void fwd_batch_compute(int nb, int bb, const FwdMeta<
                 e[q].w = fmaf(cv, s4[r].w, e[q].w);
             }
     }
-    float* dst = rowbuf + (int64_t)M.bu[bb][uu] * S::D + cg * 4;
+    float* dst = rowbuf + (int64_t)rr.u[uu] * S::D + cg * 4;
 #pragma unroll
     for (int q = 0; q < 2; ++q) *reinterpret_cast<float4*>(dst + (a1 * D2 + 2 * h + q) * D3) = e[q];
 }
@@ -766,8 +805,11 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
         ++iter;
         cp_async_wait_all();   // the chunk's A/B rows and row keys (usually prefetched long ago)
         __syncthreads();
-        // the first batch of last slices is in flight during the GEMM
         const int total = M.ucum[mb][S::MPF];
+        build_rows(M.rows, mb, M.ucum[mb], M.u0[mb], M.cnt[mb], total, s_keys, cp.ibits, cp.n[M.t[mb]][2],
+                   kFwdThreads);
+        __syncthreads();
+        // the first batch of last slices is in flight during the GEMM
         if (total > 0) fwd_issue_batch<S, K>(cp, mb, 0, 0, uniq_keys, M, sm, s_keys);
         TT_PH(0);
         if constexpr (TC) {
@@ -802,7 +844,7 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
                 }
                 __syncthreads();
                 TT_PH(2);
-                fwd_batch_compute<S>(min(S::NUF, total - k0), b, M, sm, rowbuf);
+                fwd_batch_compute<S>(mb, k0, min(S::NUF, total - k0), b, M, sm, rowbuf);
                 __syncthreads();
                 TT_PH(3);
             }
@@ -813,7 +855,7 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
                 else cp_async_wait_all();
                 __syncthreads();
                 TT_PH(2);
-                fwd_batch_compute<S>(min(S::NUF, total - k0), 0, M, sm, rowbuf);
+                fwd_batch_compute<S>(mb, k0, min(S::NUF, total - k0), 0, M, sm, rowbuf);
                 __syncthreads();
                 TT_PH(3);
             }
@@ -926,19 +968,22 @@ struct BwdMeta {
     int cnt[2];
     int bu[2][S::NUB], bp[2][S::NUB], bi3[2][S::NUB];
     int task;
+    RowTable rows;
+    int4 rec[2][S::MPB];   // the next chunk's per-group records, prefetched
 };
 
 // chunk metadata (groups cfirst+j0 .. +MPB of the column, from the plan's per-group records)
 // into buffer mb, ending with a barrier; then asynchronous copies of the keys of its first
 // kKeyCap distinct rows into keys[mb], which join the caller's next commit group
 template <class S, typename K>
-__device__ __forceinline__ void bwd_meta(int cfirst, int j0, int ccount, int mb, const K* __restrict__ uniq_keys,
-                                         const int4* __restrict__ grec, BwdMeta<S>& M, K* keys)
+__device__ __forceinline__ void bwd_meta(const int4* recs, int j0, int ccount, int mb, const K* __restrict__ uniq_keys,
+                                         BwdMeta<S>& M, K* keys)
 {
+    // recs: the chunk's per-group records (global memory, or the prefetched shared copy)
     const int tid = threadIdx.x;
     const int cnt = min(S::MPB, ccount - j0);
     if (tid < S::MPB) {
-        const int4 g = tid < cnt ? grec[cfirst + j0 + tid] : make_int4(0, 0, 0, 0);
+        const int4 g = tid < cnt ? recs[tid] : make_int4(0, 0, 0, 0);
         M.u0[mb][tid] = g.x;
         M.ucum[mb][tid] = g.y;
         M.i1[mb][tid] = g.z;
@@ -989,27 +1034,30 @@ __device__ __forceinline__ void bwd_issue_batch(const CoreParams& cp, int t, int
     const int total = M.ucum[mb][S::MPB];
     const int nb = min(S::NUB, total - k0);
     const uint32_t n3 = cp.n[t][2];
-    if (tid < nb) {
-        const int kq = k0 + tid;
-        const int j = prefix_of(M.ucum[mb], M.cnt[mb], kq);
-        const int u = M.u0[mb][j] + (kq - M.ucum[mb][j]);
-        const K key = kq < kKeyCap ? keys[mb * kKeyCap + kq] : uniq_keys[u];
-        M.bu[bb][tid] = u;
-        M.bp[bb][tid] = j;
-        M.bi3[bb][tid] = (int)(key_row(key, cp.ibits) % n3);
+    if (k0 + nb > kKeyCap) {   // beyond the row table: this batch's metadata
+        if (tid < nb) {
+            const int kq = k0 + tid;
+            const int j = prefix_of(M.ucum[mb], M.cnt[mb], kq);
+            const int u = M.u0[mb][j] + (kq - M.ucum[mb][j]);
+            const K key = kq < kKeyCap ? keys[mb * kKeyCap + kq] : uniq_keys[u];
+            M.bu[bb][tid] = u;
+            M.bp[bb][tid] = j;
+            M.bi3[bb][tid] = (int)(key_row(key, cp.ibits) % n3);
+        }
+        __syncthreads();
     }
-    __syncthreads();
+    const RowRef rr = batch_rows(M.rows, mb, k0, nb, M.bu[bb], M.bp[bb], M.bi3[bb]);
     float* H = Hs + (size_t)bb * S::NUB * P * D3;
     float* Sb = Ss + (size_t)bb * S::NUB * R * SR;
     for (int q = tid; q < nb * (P * D3 / 4); q += kBwdThreads) {
         const int uu = q / (P * D3 / 4), c4 = q % (P * D3 / 4);
-        cp_async16(&H[uu * P * D3 + c4 * 4], rowbuf + (int64_t)M.bu[bb][uu] * S::D + c4 * 4);
+        cp_async16(&H[uu * P * D3 + c4 * 4], rowbuf + (int64_t)rr.u[uu] * S::D + c4 * 4);
     }
     const float* G3t = cp.last_t[t];   // [n3][R][D3]
     for (int q = tid; q < nb * R * (D3 / 4); q += kBwdThreads) {
         const int uu = q / (R * (D3 / 4)), rem = q % (R * (D3 / 4));
         const int rho = rem / (D3 / 4), c4 = rem % (D3 / 4);
-        cp_async16(&Sb[(uu * R + rho) * SR + c4 * 4], G3t + (int64_t)M.bi3[bb][uu] * (R * D3) + rem * 4);
+        cp_async16(&Sb[(uu * R + rho) * SR + c4 * 4], G3t + (int64_t)rr.i3[uu] * (R * D3) + rem * 4);
     }
     cp_async_commit();
 }
@@ -1124,7 +1172,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                 cp_async16(&Bs[swz_b<N>(rho, c4 * 4)], G2 + rho * rs + c4 * 4);
             }
         }
-        bwd_meta<S, K>(cfirst, 0, ccount, 0, uniq_keys, grec, M, s_keys);
+        bwd_meta<S, K>(grec + cfirst, 0, ccount, 0, uniq_keys, M, s_keys);
         if constexpr (TC) bwd_issue_a_tc<S, NS>(cp, t, 0, M, Abt);
         else bwd_issue_a<S>(cp, t, 0, M, As);
         TT_PH(8);
@@ -1146,9 +1194,15 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             const uint16_t* Ab16 = Abt + mb * NS * MB * R;
             cp_async_wait_all();   // B, this chunk's A rows and row keys (usually prefetched long ago)
             __syncthreads();
-            // the first batch of distinct rows is in flight during the C GEMM
             const int total = M.ucum[mb][MPB];
+            const bool more = j0 + MPB < ccount;
+            build_rows(M.rows, mb, M.ucum[mb], M.u0[mb], cnt, total, s_keys, cp.ibits, n3, kBwdThreads);
+            // the next chunk's group records travel with this chunk's first batch
+            if (more && tid < min(MPB, ccount - j0 - MPB)) cp_async16(&M.rec[mb ^ 1][tid], grec + cfirst + j0 + MPB + tid);
+            __syncthreads();
+            // the first batch of distinct rows is in flight during the C GEMM
             if (total > 0) bwd_issue_batch<S, K>(cp, t, mb, 0, 0, uniq_keys, rowbuf, M, Hs, Ss, s_keys);
+            else cp_async_commit();
             for (int q = tid; q < MB * N / 4; q += kBwdThreads)
                 reinterpret_cast<float4*>(dCn)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
             __syncthreads();
@@ -1231,12 +1285,14 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             TT_PH(10);
 
             // next chunk's metadata and A rows go in flight while this chunk's rows are processed
-            const bool more = j0 + MPB < ccount;
             if (more) {
-                bwd_meta<S, K>(cfirst, j0 + MPB, ccount, mb ^ 1, uniq_keys, grec, M, s_keys);
+                cp_async_wait_all();   // its group records (and this chunk's first batch)
+                __syncthreads();
+                bwd_meta<S, K>(M.rec[mb ^ 1], j0 + MPB, ccount, mb ^ 1, uniq_keys, M, s_keys);
                 if constexpr (TC) bwd_issue_a_tc<S, NS>(cp, t, mb ^ 1, M, Abt + (mb ^ 1) * NS * MB * R);
                 else bwd_issue_a<S>(cp, t, mb ^ 1, M, As + (mb ^ 1) * MB * R);
             }
+            TT_PH(16);
 
             // distinct rows in double-buffered batches: dS_u -> dG_3 (vector reductions), dC_p += H_u S_u^T
             // (commit groups in flight: the batch, then possibly the next chunk's A, then possibly the next batch)
@@ -1244,6 +1300,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                 const int nb = min(NUB, total - k0);
                 if (k0 + NUB < total) {
                     bwd_issue_batch<S, K>(cp, t, mb, k0 + NUB, bb ^ 1, uniq_keys, rowbuf, M, Hs, Ss, s_keys);
+                    TT_PH(7);
                     cp_async_wait<1>();
                 } else if (k0 == 0 && more) {
                     cp_async_wait<1>();
@@ -1259,7 +1316,8 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                     const int uu = tid / S::TPUB, rem = tid % S::TPUB;
                     const int rc = rem / (D3 / 4), cg = rem % (D3 / 4);
                     if (uu < nb) {
-                        const int p = M.bp[bb][uu];
+                        const RowRef rr = batch_rows(M.rows, mb, k0, nb, M.bu[bb], M.bp[bb], M.bi3[bb]);
+                        const int p = rr.p[uu];
                         float4 o[4];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1277,7 +1335,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                                 o[i].w = fmaf(cr, h.w, o[i].w);
                             }
                         }
-                        const int i3 = M.bi3[bb][uu];
+                        const int i3 = rr.i3[uu];
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
                             red_add_v4(dG3 + ((int64_t)(rc * 4 + i) * n3 + i3) * D3 + cg * 4, o[i]);
