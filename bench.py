@@ -279,12 +279,13 @@ def run_reference(args):
 
 def run_ours(args):
     import torch
-    from tensor_train_compressed_mixed_b200 import abi, from_workload
+    from tensor_train_compressed_mixed_b200 import abi, dp, from_workload
     from workloads import config_workload
 
     world, rank, local = dist_init(args.gpus)
     dev = torch.device("cuda", local)
-    w = config_workload(args.config, batch=args.batch, tables=args.tables, with_grad=True)
+    # every rank draws its own batch of the same workload (rank 0's is the single-GPU one)
+    w = config_workload(args.config, batch=args.batch, tables=args.tables, with_grad=True, shard=rank)
     if args.precision == "auto":
         # the tensor-core kernels cover three cores with d = (4, 4, 8) and r = 32 or 64
         tc_shape = len(w.d) == 3 and tuple(w.d) == (4, 4, 8) and w.r[1] == w.r[2] and w.r[1] in (32, 64)
@@ -296,7 +297,10 @@ def run_ours(args):
     opts.grouping = abi.TT_GROUP_PREFIX if args.grouping == "prefix" else abi.TT_GROUP_UNIQUE_ONLY
     opts.precision = {"fp32": abi.TT_PREC_FP32, "split": abi.TT_PREC_FP32_SPLIT_TC,
                       "bf16": abi.TT_PREC_BF16_TC}[args.precision]
-    emb, cores, idx, off = from_workload(w, device=dev, options=opts, with_grads=True)
+    # data-parallel training: the core gradients of all ranks are summed (one NCCL
+    # all-reduce over a flat buffer) before the SGD step
+    dp_train = world > 1 and train
+    emb, cores, idx, off = from_workload(w, device=dev, options=opts, with_grads=True, flat_grads=dp_train)
     g = torch.from_numpy(w.grad_out).to(dev)
     L, B, T, D = w.num_lookups, w.batch, w.num_tables, w.dim
     out = torch.empty(B, T * D, dtype=torch.float32, device=dev)
@@ -306,6 +310,8 @@ def run_ours(args):
         emb.forward(idx, off, B, out)
         if train:
             emb.backward(g)
+            if dp_train:
+                dp.allreduce_grads(emb)
             if args.config == 4:
                 emb.sgd_update(w.lr)
 
@@ -431,6 +437,8 @@ def run_ours(args):
                 ev_read[s].record(down)
                 if train:
                     emb.backward(d_g[s])
+                    if dp_train:
+                        dp.allreduce_grads(emb)
                     if args.config == 4:
                         emb.sgd_update(w.lr)
                 ev_used[s].record(comp)
@@ -480,7 +488,9 @@ def run_ours(args):
                        "unique_rows": U, "prefix_groups": G,
                        "step": "fwd+bwd+sgd" if train else "fwd",
                        "l2": "inputs larger than L2 (indices+grad+cores ~800 MB), no flush",
-                       "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "parallelism": (f"dp{world}: own batch per GPU, NCCL all-reduce of the core gradients"
+                                       if dp_train else (f"shards{world}: own batch per GPU, no exchange"
+                                                         if world > 1 else "single")),
                        "sched": args.sched, "grouping": args.grouping,
                        "prefix_step": {"fp32": "fp32 FFMA",
                                        "split": "fp32-accurate: two bf16 terms per value, three tcgen05 "
@@ -498,6 +508,10 @@ def run_ours(args):
         }
         print(json.dumps(line), flush=True)
     emb.close()
+    if world > 1:
+        import torch.distributed as dist
+        barrier(world)
+        dist.destroy_process_group()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

@@ -30,20 +30,31 @@ class TTEmbeddingBag:
         self.D = int(np.prod(self.d))
         self.cores = None
         self.grads = None
+        self.grad_flat = None
         self._ws = None
         self._ws_dims = (0, 0)
 
     def core_shape(self, t: int, j: int) -> tuple:
         return (self.r[j], self.n[t][j], self.d[j], self.r[j + 1])
 
-    def set_cores(self, cores, with_grads: bool = True):
-        """cores: [T][k] float32 CUDA tensors (borrowed); allocates gradient buffers."""
+    def set_cores(self, cores, with_grads: bool = True, flat_grads: bool = False):
+        """cores: [T][k] float32 CUDA tensors (borrowed); allocates gradient buffers.
+
+        flat_grads: the gradients are views of one buffer (``self.grad_flat``), so that a
+        data-parallel exchange is a single collective (dp.allreduce_grads)."""
         flat = [cores[t][j] for t in range(self.T) for j in range(self.k)]
         for q, c in enumerate(flat):
             if tuple(c.shape) != self.core_shape(q // self.k, q % self.k):
                 raise ValueError(f"core {q} has shape {tuple(c.shape)}")
         self.cores = flat
-        self.grads = [torch.empty_like(c) for c in flat] if with_grads else None
+        self.grad_flat = None
+        if with_grads and flat_grads:
+            from .dp import grad_layout
+            offs, total = grad_layout([tuple(c.shape) for c in flat])
+            self.grad_flat = torch.zeros(total, dtype=torch.float32, device=self.device)
+            self.grads = [self.grad_flat[o:o + c.numel()].view(c.shape) for o, c in zip(offs, flat)]
+        else:
+            self.grads = [torch.empty_like(c) for c in flat] if with_grads else None
         abi.tt_emb_set_cores(self.handle, flat, self.grads)
 
     def reserve(self, max_lookups: int, batch: int):
@@ -90,11 +101,11 @@ class TTEmbeddingBag:
             pass
 
 
-def from_workload(w, device="cuda", options=None, with_grads=None):
+def from_workload(w, device="cuda", options=None, with_grads=None, flat_grads=False):
     """A TTEmbeddingBag holding a seeded workload's cores, plus its inputs on the device."""
     emb = TTEmbeddingBag(w.n, w.n_rows, w.d, w.r, options=options, device=device)
     cores = [[torch.from_numpy(c).to(device) for c in tab] for tab in w.cores]
-    emb.set_cores(cores, with_grads=w.train if with_grads is None else with_grads)
+    emb.set_cores(cores, with_grads=w.train if with_grads is None else with_grads, flat_grads=flat_grads)
     idx = torch.from_numpy(w.indices).to(device)
     off = torch.from_numpy(w.offsets).to(device)
     return emb, cores, idx, off

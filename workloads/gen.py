@@ -227,18 +227,34 @@ CONFIG_NAMES = {
 }
 
 
+SHARD_SEED_STRIDE = 1_000_003
+
+
 def config_workload(cfg: int, batch: int | None = None, with_grad: bool | None = None,
-                    tables: int | None = None) -> Workload:
-    """One of the five benchmark workloads; ``batch``/``tables`` shrink it."""
+                    tables: int | None = None, shard: int = 0) -> Workload:
+    """One of the five benchmark workloads; ``batch``/``tables`` shrink it.
+
+    ``shard`` > 0 draws another batch of the same workload (data-parallel ranks): the cores,
+    the tables and the popularity of their rows (the rank-to-row bijection) are shared; the
+    bag sizes, the drawn indices and the upstream gradient come from shifted seeds.  Shard 0
+    is the workload itself."""
     s = BASE_SEED
+    build = build_workload
+    if shard:
+        def build(name, d, r, n_list, n_rows_list, B, pooling, law, index_seeds, core_seeds,
+                  grad_seed=None, **kw):
+            return build_workload(name, d, r, n_list, n_rows_list, B, pooling, law,
+                                  [x + shard * SHARD_SEED_STRIDE for x in index_seeds], core_seeds,
+                                  grad_seed=None if grad_seed is None else grad_seed + shard * SHARD_SEED_STRIDE,
+                                  perm_seeds=list(index_seeds), **kw)
     if cfg == 1:
         B = batch or 1024
-        w = build_workload(CONFIG_NAMES[1], (2, 2, 4), (1, 8, 8, 1), [(100, 100, 100)], [1_000_000],
+        w = build(CONFIG_NAMES[1], (2, 2, 4), (1, 8, 8, 1), [(100, 100, 100)], [1_000_000],
                            B, {"kind": "fixed", "size": 1}, {"kind": "uniform"},
                            [s + 1000], [s + 1500], grad_seed=(s + 1777) if with_grad else None)
     elif cfg == 2:
         B = batch or 32768
-        w = build_workload(CONFIG_NAMES[2], (4, 4, 4), (1, 16, 16, 1), [(200, 200, 250)],
+        w = build(CONFIG_NAMES[2], (4, 4, 4), (1, 16, 16, 1), [(200, 200, 250)],
                            [10_000_000], B, {"kind": "poisson_plus1", "mean": 8},
                            {"kind": "zipf", "alpha": 1.05}, [s + 2000], [s + 2500],
                            grad_seed=(s + 2777) if with_grad else None)
@@ -251,7 +267,7 @@ def config_workload(cfg: int, batch: int | None = None, with_grad: bool | None =
         train = cfg == 4
         if with_grad is None:
             with_grad = train
-        w = build_workload(CONFIG_NAMES[cfg], (4, 4, 8), r, n_list, rows, B,
+        w = build(CONFIG_NAMES[cfg], (4, 4, 8), r, n_list, rows, B,
                            {"kind": "poisson_plus1", "mean": 20}, {"kind": "zipf", "alpha": 1.1},
                            [s + 3000 + t for t in range(T)],
                            [s + 1000 * cfg + 500 + t for t in range(T)],
@@ -262,7 +278,7 @@ def config_workload(cfg: int, batch: int | None = None, with_grad: bool | None =
         T = tables or 8
         if with_grad is None:
             with_grad = True
-        w = build_workload(CONFIG_NAMES[5], (2, 4, 4, 4), (1, 32, 32, 32, 1),
+        w = build(CONFIG_NAMES[5], (2, 4, 4, 4), (1, 32, 32, 32, 1),
                            [(178, 178, 178, 178)] * T, [1_000_000_000] * T, B,
                            {"kind": "uniform", "lo": 1, "hi": 64},
                            {"kind": "mix", "alpha": 1.4, "p_zipf": 0.9},
@@ -272,9 +288,10 @@ def config_workload(cfg: int, batch: int | None = None, with_grad: bool | None =
         raise ValueError(f"no workload {cfg}")
     if with_grad and w.grad_out is None:
         D = w.dim
-        w.grad_out = np.random.default_rng(s + 1000 * cfg + 777).normal(
+        w.grad_out = np.random.default_rng(s + 1000 * cfg + 777 + shard * SHARD_SEED_STRIDE).normal(
             0.0, 1.0, size=(w.batch, w.num_tables * D)).astype(np.float32)
     w.meta["config"] = cfg
+    w.meta["shard"] = shard
     return w
 
 
