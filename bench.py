@@ -306,13 +306,18 @@ def run_ours(args):
     out = torch.empty(B, T * D, dtype=torch.float32, device=dev)
     emb.reserve(L, B)
 
+    sgd = args.config == 4
+    fused_sgd = sgd and not dp_train   # data parallel: the gradients are exchanged before SGD
+
     def step():
         emb.forward(idx, off, B, out)
-        if train:
+        if fused_sgd:
+            emb.backward_sgd(g, w.lr)
+        elif train:
             emb.backward(g)
             if dp_train:
                 dp.allreduce_grads(emb)
-            if args.config == 4:
+            if sgd:
                 emb.sgd_update(w.lr)
 
     def timed(fn, K):
@@ -435,11 +440,13 @@ def run_ours(args):
                 with torch.cuda.stream(down):
                     h_out[s].copy_(d_out[s], non_blocking=True)
                 ev_read[s].record(down)
-                if train:
+                if fused_sgd:
+                    emb.backward_sgd(d_g[s], w.lr)
+                elif train:
                     emb.backward(d_g[s])
                     if dp_train:
                         dp.allreduce_grads(emb)
-                    if args.config == 4:
+                    if sgd:
                         emb.sgd_update(w.lr)
                 ev_used[s].record(comp)
             for s in range(2):
@@ -486,7 +493,8 @@ def run_ours(args):
             "data": "synthetic",
             "config": {"workload": w.name, "batch": B, "tables": T, "lookups": L,
                        "unique_rows": U, "prefix_groups": G,
-                       "step": "fwd+bwd+sgd" if train else "fwd",
+                       "step": ("fwd+bwd+sgd (fused sparse update of the middle cores)" if fused_sgd else
+                                "fwd+bwd+sgd" if sgd else "fwd+bwd" if train else "fwd"),
                        "l2": "inputs larger than L2 (indices+grad+cores ~800 MB), no flush",
                        "parallelism": (f"dp{world}: own batch per GPU, NCCL all-reduce of the core gradients"
                                        if dp_train else (f"shards{world}: own batch per GPU, no exchange"

@@ -191,6 +191,21 @@ int tt_emb_backward(tt_emb_t h, const float* grad_out, tt_stream_t stream);
 int tt_emb_sgd_update(tt_emb_t h, float lr, tt_stream_t stream);
 
 /*
+ * Backward pass and SGD step fused, with a sparse update of the middle core (the
+ * "sparse fused optimizer" follow-on to FlowTT section 3.2's backward).  The result for the
+ * cores is that of tt_emb_backward followed by tt_emb_sgd_update(lr).  On three-core
+ * tables served by the shape-specialised kernels, the block that reduces a column group's
+ * dG_2[:, i_2] on chip applies G_2[:, i_2] -= lr * dG_2[:, i_2] itself, so dG_2 is neither
+ * zero-filled, written nor read back; G_2 slices no lookup touched are not visited.  In that
+ * case the registered core_grads of the middle cores are left unchanged (not gradients);
+ * those of the other cores hold their gradients.  Other tables take the unfused
+ * path (every registered gradient is written).  Same arguments and errors as
+ * tt_emb_backward; registered core_grads are required (the first and last cores' gradients
+ * are reduced there).
+ */
+int tt_emb_backward_sgd(tt_emb_t h, const float* grad_out, float lr, tt_stream_t stream);
+
+/*
  * Test and inspection hook: device views of the last forward's segmentation,
  * valid until the next forward on the handle.  Synchronises the stream of the
  * last call to read the counts.

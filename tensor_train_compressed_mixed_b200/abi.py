@@ -65,6 +65,7 @@ _SIGS = {
                         ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
     "tt_emb_backward": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
     "tt_emb_sgd_update": ([ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p], ctypes.c_int),
+    "tt_emb_backward_sgd": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p], ctypes.c_int),
     "tt_emb_get_segmentation": ([ctypes.c_void_p, ctypes.POINTER(SegView)], ctypes.c_int),
     "tt_emb_copy_segmentation": ([ctypes.c_void_p] + [ctypes.c_void_p] * 6, ctypes.c_int),
     "tt_emb_sync": ([ctypes.c_void_p], ctypes.c_int),
@@ -196,6 +197,12 @@ def tt_emb_backward(h, grad_out, stream=None):
 
 def tt_emb_sgd_update(h, lr: float, stream=None):
     _check(lib().tt_emb_sgd_update(h, float(lr), _stream(stream)), "tt_emb_sgd_update")
+
+
+def tt_emb_backward_sgd(h, grad_out, lr: float, stream=None):
+    import torch
+    _check(lib().tt_emb_backward_sgd(h, _dev_ptr(grad_out, torch.float32, "grad_out"), float(lr),
+                                     _stream(stream)), "tt_emb_backward_sgd")
 
 
 def tt_emb_sync(h):

@@ -302,14 +302,15 @@ struct tt_emb_handle {
         return cp;
     }
 
-    BufferList buffers(bool with_grads_as_b, bool grads_as_a) const
+    // every core (or its gradient); skip_middle leaves out core 1 of every table (size 0)
+    BufferList buffers(bool with_grads_as_b, bool grads_as_a, bool skip_middle = false) const
     {
         BufferList bl;
         memset(&bl, 0, sizeof(bl));
         bl.count = T * k;
         int64_t c = 0;
         for (int q = 0; q < T * k; ++q) {
-            const int64_t sz = core_floats(q / k, q % k);
+            const int64_t sz = (skip_middle && q % k == 1) ? 0 : core_floats(q / k, q % k);
             bl.chunk_start[q] = c;
             bl.size[q] = sz;
             bl.a[q] = grads_as_a ? grads[q] : cores[q];
@@ -703,16 +704,18 @@ int tt_emb_forward(tt_emb_t h, const int64_t* indices, const int64_t* offsets, i
     return TT_OK;
 }
 
-int tt_emb_backward(tt_emb_t h, const float* grad_out, tt_stream_t stream)
+// Backward of the last forward; fused: the middle cores take their SGD step inside the
+// column-group kernel (the caller checked that the handle qualifies) and their gradient
+// buffers are skipped by the zero fill.
+static int backward_impl(tt_emb_t h, const float* grad_out, tt_stream_t stream, bool fused, float lr)
 {
-    if (!h || !grad_out) return TT_ERR_ARG;
-    if (!h->have_fwd || !h->have_grads || !h->have_cores) return TT_ERR_STATE;
     cudaStream_t s = (cudaStream_t)stream;
     h->last_stream = s;
     h->used_stream = true;
     int nl = 0;
     h->begin(TT_PHASE_BWD_REDUCE, s);
-    cudaError_t e = launch_fill_zero(h->buffers(false, true), h->d_status, s, &nl);
+    // fused: dG_2 is never materialised, so it is not zero-filled either
+    cudaError_t e = launch_fill_zero(h->buffers(false, true, fused), h->d_status, s, &nl);
     h->end(s);
     h->launches += nl;
     if (e != cudaSuccess) return TT_ERR_CUDA;
@@ -732,6 +735,11 @@ int tt_emb_backward(tt_emb_t h, const float* grad_out, tt_stream_t stream)
         pb.sorted_groups = h->plan_sorted_groups;
         GradPtrs vgp;
         const CoreParams vcp = h->view_cores(h->fwd_B, &vgp);
+        if (fused) {
+            vgp.fused = 1;
+            vgp.lr = lr;
+            for (int t = 0; t < h->T; ++t) vgp.upd1[t] = h->cores[t * h->k + 1];
+        }
         K3Args a = h->k3_args(&vcp, &pp, &pb, nullptr, h->fwd_L, true);
         h->begin(TT_PHASE_BWD_ROWSUM, s);
         e = k3_rowsum(a, grad_out, s, &nl);
@@ -752,6 +760,31 @@ int tt_emb_backward(tt_emb_t h, const float* grad_out, tt_stream_t stream)
                                     (const int32_t*)h->at(y.bag_sorted), (const WsCounters*)h->at(y.counters),
                                     h->fwd_L, grad_out, h->d_status, s, grid, &nl);
     }
+    h->end(s);
+    h->launches += nl;
+    return cuda_status(e);
+}
+
+int tt_emb_backward(tt_emb_t h, const float* grad_out, tt_stream_t stream)
+{
+    if (!h || !grad_out) return TT_ERR_ARG;
+    if (!h->have_fwd || !h->have_grads || !h->have_cores) return TT_ERR_STATE;
+    return backward_impl(h, grad_out, stream, false, 0.f);
+}
+
+int tt_emb_backward_sgd(tt_emb_t h, const float* grad_out, float lr, tt_stream_t stream)
+{
+    if (!h || !grad_out) return TT_ERR_ARG;
+    if (!h->have_fwd || !h->have_grads || !h->have_cores) return TT_ERR_STATE;
+    // the middle core's column groups are reduced on chip only by the three-core specialised kernel
+    const bool fused = h->fast && !h->merged && h->k == 3;
+    int rc = backward_impl(h, grad_out, stream, fused, lr);
+    if (rc != TT_OK) return rc;
+    if (!fused) return tt_emb_sgd_update(h, lr, stream);
+    cudaStream_t s = (cudaStream_t)stream;
+    int nl = 0;
+    h->begin(TT_PHASE_SGD, s);
+    const cudaError_t e = launch_sgd(h->buffers(true, false, true), lr, h->d_status, s, &nl);
     h->end(s);
     h->launches += nl;
     return cuda_status(e);

@@ -1572,10 +1572,22 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                 float v[32];
                 tmem_ld32(tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)c0, v);
                 if (lane < 16) {
-                    float* dst = dG2 + ((int64_t)rho1 * n2 + i2) * N + c0;
+                    if (gp.fused) {   // sparse fused SGD: G_2[:, i_2] -= lr dB
+                        float* g2 = gp.upd1[t] + ((int64_t)rho1 * n2 + i2) * N + c0;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        *reinterpret_cast<float4*>(dst + 4 * j) = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                        for (int j = 0; j < 8; ++j) {
+                            const float4 x = *reinterpret_cast<const float4*>(g2 + 4 * j);
+                            *reinterpret_cast<float4*>(g2 + 4 * j) =
+                                make_float4(x.x - gp.lr * v[4 * j], x.y - gp.lr * v[4 * j + 1],
+                                            x.z - gp.lr * v[4 * j + 2], x.w - gp.lr * v[4 * j + 3]);
+                        }
+                    } else {
+                        float* dst = dG2 + ((int64_t)rho1 * n2 + i2) * N + c0;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            *reinterpret_cast<float4*>(dst + 4 * j) =
+                                make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                    }
                 }
             }
             tc_fence_before();
@@ -1587,11 +1599,22 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             if constexpr (DBR == 8) rho1 = (i < 4) ? trb * 4 + i : R / 2 + trb * 4 + (i - 4);
             else if constexpr (DBR == 4) rho1 = trb * 4 + i;
             else rho1 = trb;
-            float* dst = dG2 + ((int64_t)rho1 * n2 + i2) * N;
+            if (gp.fused) {   // sparse fused SGD: G_2[:, i_2] -= lr dB
+                float* g2 = gp.upd1[t] + ((int64_t)rho1 * n2 + i2) * N;
 #pragma unroll
-            for (int ch = 0; ch < NCH; ++ch)
-                *reinterpret_cast<float4*>(dst + ch * (N / NCH) + tnb * 4) =
-                    make_float4(dB[i][ch * 4], dB[i][ch * 4 + 1], dB[i][ch * 4 + 2], dB[i][ch * 4 + 3]);
+                for (int ch = 0; ch < NCH; ++ch) {
+                    float4* q = reinterpret_cast<float4*>(g2 + ch * (N / NCH) + tnb * 4);
+                    const float4 x = *q;
+                    *q = make_float4(x.x - gp.lr * dB[i][ch * 4], x.y - gp.lr * dB[i][ch * 4 + 1],
+                                     x.z - gp.lr * dB[i][ch * 4 + 2], x.w - gp.lr * dB[i][ch * 4 + 3]);
+                }
+            } else {
+                float* dst = dG2 + ((int64_t)rho1 * n2 + i2) * N;
+#pragma unroll
+                for (int ch = 0; ch < NCH; ++ch)
+                    *reinterpret_cast<float4*>(dst + ch * (N / NCH) + tnb * 4) =
+                        make_float4(dB[i][ch * 4], dB[i][ch * 4 + 1], dB[i][ch * 4 + 2], dB[i][ch * 4 + 3]);
+            }
         }
         }
         __syncthreads();

@@ -71,6 +71,11 @@ struct CoreParams {
 
 struct GradPtrs {
     float* g[kMaxT][kMaxK];
+    // fused SGD (tt_emb_backward_sgd): the middle core is updated in place by the block that
+    // reduces its column group, G_2[:, i_2] -= lr * dB, instead of writing dG_2
+    float* upd1[kMaxT];
+    float lr;
+    int32_t fused;
 };
 
 // Up to T*k float buffers handled by one elementwise launch (zero fill, SGD).

@@ -83,6 +83,10 @@ class TTEmbeddingBag:
     def sgd_update(self, lr: float, stream=None):
         abi.tt_emb_sgd_update(self.handle, lr, stream)
 
+    def backward_sgd(self, grad_out: torch.Tensor, lr: float, stream=None):
+        """Backward and SGD step fused (the middle cores are updated sparsely in place)."""
+        abi.tt_emb_backward_sgd(self.handle, grad_out, lr, stream)
+
     def sync(self):
         abi.tt_emb_sync(self.handle)
 

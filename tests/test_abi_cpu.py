@@ -89,6 +89,7 @@ def test_null_handle_calls_fail_cleanly():
     assert lib.tt_emb_forward(None, None, None, 0, 1, None, None) == abi.TT_ERR_ARG
     assert lib.tt_emb_backward(None, None, None) == abi.TT_ERR_ARG
     assert lib.tt_emb_sgd_update(None, 0.1, None) == abi.TT_ERR_ARG
+    assert lib.tt_emb_backward_sgd(None, None, 0.1, None) == abi.TT_ERR_ARG
     assert lib.tt_emb_sync(None) == abi.TT_ERR_ARG
     lib.tt_emb_destroy(None)
 
