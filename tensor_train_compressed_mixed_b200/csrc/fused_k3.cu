@@ -905,7 +905,8 @@ __global__ void __launch_bounds__(256) k3_hsum(const int32_t* __restrict__ uid_s
                                                const int32_t* __restrict__ bag_sorted,
                                                const int32_t* __restrict__ uniq_start,
                                                const float* __restrict__ grad_out, int64_t L, int64_t B,
-                                               int T, float* __restrict__ rowbuf, const int32_t* status)
+                                               float inv_b, int T, float* __restrict__ rowbuf,
+                                               const int32_t* status)
 {
     if (has_error(status)) return;
     constexpr int LB = D / 4;
@@ -936,7 +937,10 @@ __global__ void __launch_bounds__(256) k3_hsum(const int32_t* __restrict__ uid_s
             for (int q = 0; q < 8; ++q) {
                 uq[q] = __shfl_sync(kFull, myu, k + q);
                 const int bag = __shfl_sync(kFull, myb, k + q);
-                const int t = (int)(bag / B);
+                // table t = bag / B (t < 64): a float estimate, corrected to the exact quotient
+                int t = __float2int_rz(__int2float_rz(bag) * inv_b);
+                if ((int64_t)t * B > bag) --t;
+                else if ((int64_t)(t + 1) * B <= bag) ++t;
                 const int64_t b = bag - (int64_t)t * B;
                 v[q] = (active && k + q < n)
                            ? __ldg(reinterpret_cast<const float4*>(grad_out + b * TD + (int64_t)t * D) + lane)
@@ -1761,7 +1765,8 @@ cudaError_t rowsum_launch(const K3Args& a, const float* grad_out, cudaStream_t s
     const int64_t nwarps = ceil_div(L, kHChunk);
     k3_hzero<D><<<148, 256, 0, s>>>(a.uid_sorted, L, a.rowbuf, a.status);
     k3_hsum<D><<<(unsigned)ceil_div(nwarps * 32, 256), 256, 0, s>>>(
-        a.uid_sorted, a.bag_sorted, a.uniq_start, grad_out, L, a.cp->B, a.cp->T, a.rowbuf, a.status);
+        a.uid_sorted, a.bag_sorted, a.uniq_start, grad_out, L, a.cp->B, (float)(1.0 / (double)a.cp->B), a.cp->T,
+        a.rowbuf, a.status);
     *nl += 2;
     return cudaGetLastError();
 }
