@@ -1087,6 +1087,128 @@ __device__ __forceinline__ void bwd_issue_a_tc(const CoreParams& cp, int t, int 
     cp_async_commit();
 }
 
+// Per-row backward of a chunk with one warp per contiguous range of its distinct rows (rank 64,
+// d = (4, 4, 8)); lane l owns rho_2 in {2l, 2l + 1}.  For each row u of prefix p:
+//   dS_u[rho][a3] = sum_r C_p[r][rho] H_u[r][a3]    -> dG_3[rho, i3(u), a3] (vector reductions)
+//   dC_p[r][rho] += sum_a3 H_u[r][a3] S_u[rho][a3]   (registers; into dCn when the prefix ends:
+//                                                      a plain store when the prefix lies inside
+//                                                      this warp's range, shared atomics if not)
+// C_p for the lane's columns sits in registers, H_u is broadcast through a per-warp slot, and the
+// lane's two rows of S_u with its quarter-row of H_u are loaded two rows ahead.  No block
+// barrier is taken between rows.
+struct WarpRow {
+    float4 s[4];   // S_u rows 2l, 2l + 1 (8 values each)
+    float4 h;      // H_u[4 l .. 4 l + 3]
+    int u, j, i3;
+};
+
+template <class S, typename K>
+__device__ __forceinline__ void warp_row_load(const CoreParams& cp, int t, int mb, int kq, int cnt, const BwdMeta<S>& M,
+                                              const K* __restrict__ uniq_keys, const float* __restrict__ rowbuf,
+                                              uint32_t n3, WarpRow& w)
+{
+    constexpr int R = S::R, D3 = S::D3, D = S::D;
+    const int lane = threadIdx.x & 31;
+    if (kq < kKeyCap) {
+        w.u = M.rows.u[mb][kq];
+        w.j = M.rows.p[mb][kq];
+        w.i3 = M.rows.i3[mb][kq];
+    } else {
+        w.j = prefix_of(M.ucum[mb], cnt, kq);
+        w.u = M.u0[mb][w.j] + (kq - M.ucum[mb][w.j]);
+        w.i3 = (int)(key_row(uniq_keys[w.u], cp.ibits) % n3);
+    }
+    const float4* sp = reinterpret_cast<const float4*>(cp.last_t[t] + (int64_t)w.i3 * (R * D3) + lane * 2 * D3);
+    w.s[0] = __ldg(sp);
+    w.s[1] = __ldg(sp + 1);
+    w.s[2] = __ldg(sp + 2);
+    w.s[3] = __ldg(sp + 3);
+    w.h = __ldcg(reinterpret_cast<const float4*>(rowbuf + (int64_t)w.u * D) + lane);
+}
+
+template <class S, typename K>
+__device__ __forceinline__ void bwd_rows_warp(const CoreParams& cp, int t, int mb, int total, int cnt,
+                                              const BwdMeta<S>& M, const K* __restrict__ uniq_keys,
+                                              const float* __restrict__ rowbuf, const float* Cn, float* dCn,
+                                              float* __restrict__ dG3, uint32_t n3, float* hslots)
+{
+    constexpr int R = S::R, N = S::N, D1 = S::D1, D2 = S::D2, D3 = S::D3, P = S::P;
+    static_assert(R == 64 && D3 == 8 && P == 16 && S::D == 128, "warp row path: rank 64, d = (4, 4, 8)");
+    constexpr int NW = kBwdThreads / 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int lo = (int)((int64_t)total * warp / NW), hi = (int)((int64_t)total * (warp + 1) / NW);
+    if (lo >= hi) return;
+    float* hs = hslots + warp * 2 * P * D3;   // two slots of one row's H (P x D3 floats each)
+    float c[P][2], o[P][2];
+    int cur = -1;
+    auto flush = [&]() {
+        const bool whole = M.ucum[mb][cur] >= lo && M.ucum[mb][cur + 1] <= hi;
+#pragma unroll
+        for (int r = 0; r < P; ++r) {
+            float* d = &dCn[swz_m<N>(cur * D1 + r / D2, (r % D2) * R + 2 * lane)];
+            if (whole) {
+                *reinterpret_cast<float2*>(d) = make_float2(o[r][0], o[r][1]);
+            } else {
+                atomicAdd(d, o[r][0]);
+                atomicAdd(d + 1, o[r][1]);
+            }
+        }
+    };
+    WarpRow a, b;
+    warp_row_load<S, K>(cp, t, mb, lo, cnt, M, uniq_keys, rowbuf, n3, a);
+    if (lo + 1 < hi) warp_row_load<S, K>(cp, t, mb, lo + 1, cnt, M, uniq_keys, rowbuf, n3, b);
+#pragma unroll 1
+    for (int kq = lo; kq < hi; ++kq) {
+        const WarpRow w = a;
+        a = b;
+        if (kq + 2 < hi) warp_row_load<S, K>(cp, t, mb, kq + 2, cnt, M, uniq_keys, rowbuf, n3, b);
+        if (w.j != cur) {
+            if (cur >= 0) flush();
+            cur = w.j;
+#pragma unroll
+            for (int r = 0; r < P; ++r) {
+                const float2 cv = *reinterpret_cast<const float2*>(&Cn[swz_m<N>(cur * D1 + r / D2, (r % D2) * R + 2 * lane)]);
+                c[r][0] = cv.x;
+                c[r][1] = cv.y;
+                o[r][0] = o[r][1] = 0.f;
+            }
+        }
+        float* hb = hs + (kq & 1) * (P * D3);
+        reinterpret_cast<float4*>(hb)[lane] = w.h;
+        __syncwarp();
+        const float sv[2][8] = {{w.s[0].x, w.s[0].y, w.s[0].z, w.s[0].w, w.s[1].x, w.s[1].y, w.s[1].z, w.s[1].w},
+                                {w.s[2].x, w.s[2].y, w.s[2].z, w.s[2].w, w.s[3].x, w.s[3].y, w.s[3].z, w.s[3].w}};
+        float ds[2][8];
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+            for (int a3 = 0; a3 < 8; ++a3) ds[q][a3] = 0.f;
+#pragma unroll
+        for (int r = 0; r < P; ++r) {
+            const float4 h0 = *reinterpret_cast<const float4*>(hb + r * D3);
+            const float4 h1 = *reinterpret_cast<const float4*>(hb + r * D3 + 4);
+            const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                float acc = o[r][q];
+#pragma unroll
+                for (int a3 = 0; a3 < 8; ++a3) {
+                    ds[q][a3] = fmaf(c[r][q], hv[a3], ds[q][a3]);
+                    acc = fmaf(hv[a3], sv[q][a3], acc);
+                }
+                o[r][q] = acc;
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            float* dst = dG3 + ((int64_t)(2 * lane + q) * n3 + w.i3) * D3;
+            red_add_v4(dst, make_float4(ds[q][0], ds[q][1], ds[q][2], ds[q][3]));
+            red_add_v4(dst + 4, make_float4(ds[q][4], ds[q][5], ds[q][6], ds[q][7]));
+        }
+    }
+    flush();
+}
+
 // one thread issues, the others wait at the barrier; false (all threads) when the wait ran out
 __device__ __forceinline__ bool tc_commit_wait(uint64_t* bar, uint32_t& parity, int* s_ok)
 {
@@ -1120,6 +1242,9 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
     constexpr int NS = NT == 3 ? 2 : 1;
     constexpr int MT = TC ? 64 : MB;
     constexpr int DAQ = 4;   // dA accumulators in tensor-memory columns [N, N + DAQ R)
+    // per-row backward by warps over contiguous row ranges (rank 64, d = (4, 4, 8)); other
+    // shapes use barrier-synchronised batches of NUB rows
+    constexpr bool WARP_ROWS = R == 64 && D1 == 4 && D2 == 4 && D3 == 8;
     static_assert(!TC || (R == 64 && MB == 32 && N == 256 && DAQ * R <= N), "tensor-core backward: rank 64, d_2 = 4");
     float* Bs = smem_f;                    // [R][N] swizzled (key row/4)            (fp32 variant)
     uint16_t* Bb = reinterpret_cast<uint16_t*>(smem_f);   // NS x (N x R) bf16 core matrices (tensor cores)
@@ -1205,7 +1330,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             if (more && tid < min(MPB, ccount - j0 - MPB)) cp_async16(&M.rec[mb ^ 1][tid], grec + cfirst + j0 + MPB + tid);
             __syncthreads();
             // the first batch of distinct rows is in flight during the C GEMM
-            if (total > 0) bwd_issue_batch<S, K>(cp, t, mb, 0, 0, uniq_keys, rowbuf, M, Hs, Ss, s_keys);
+            if (!WARP_ROWS && total > 0) bwd_issue_batch<S, K>(cp, t, mb, 0, 0, uniq_keys, rowbuf, M, Hs, Ss, s_keys);
             else cp_async_commit();
             for (int q = tid; q < MB * N / 4; q += kBwdThreads)
                 reinterpret_cast<float4*>(dCn)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1298,9 +1423,14 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             }
             TT_PH(16);
 
+            if constexpr (WARP_ROWS) {
+                bwd_rows_warp<S, K>(cp, t, mb, total, cnt, M, uniq_keys, rowbuf, Cn, dCn, dG3, n3, Hs);
+                __syncthreads();
+                TT_PH(12);
+            }
             // distinct rows in double-buffered batches: dS_u -> dG_3 (vector reductions), dC_p += H_u S_u^T
             // (commit groups in flight: the batch, then possibly the next chunk's A, then possibly the next batch)
-            for (int k0 = 0, bb = 0; k0 < total; k0 += NUB, bb ^= 1) {
+            for (int k0 = 0, bb = 0; !WARP_ROWS && k0 < total; k0 += NUB, bb ^= 1) {
                 const int nb = min(NUB, total - k0);
                 if (k0 + NUB < total) {
                     bwd_issue_batch<S, K>(cp, t, mb, k0 + NUB, bb ^ 1, uniq_keys, rowbuf, M, Hs, Ss, s_keys);
