@@ -61,7 +61,8 @@ namespace tt {
 namespace {
 
 constexpr int kFwdThreads = 512;  // forward: 16 warps, at most 128 registers per thread
-constexpr int kBwdThreads = 256;  // backward: 8 warps, up to 255 registers per thread
+constexpr int kBwdThreads = 256;  // backward, FP32 variant: 8 warps, up to 255 registers per thread
+constexpr int kBwdThreadsTC = 512; // backward, tensor-core variants: 16 warps, at most 128 registers
 constexpr int kNB = kPoolBags;    // bags per pooling task
 constexpr int kHChunk = 256;      // sorted lookups per upstream-sum warp
 constexpr int kSpinLimit = 1 << 22;
@@ -1005,7 +1006,7 @@ __device__ __forceinline__ void bwd_meta(const int4* recs, int j0, int ccount, i
     }
     __syncthreads();
     const int nk = min(M.ucum[mb][S::MPB], kKeyCap);
-    for (int kq = tid; kq < nk; kq += kBwdThreads) {
+    for (int kq = tid; kq < nk; kq += (int)blockDim.x) {
         const int j = prefix_of(M.ucum[mb], cnt, kq);
         cp_async_key(keys + mb * kKeyCap + kq, uniq_keys + M.u0[mb][j] + (kq - M.ucum[mb][j]));
     }
@@ -1017,7 +1018,7 @@ __device__ __forceinline__ void bwd_issue_a(const CoreParams& cp, int t, int mb,
     constexpr int R = S::R, MB = S::MB, D1 = S::D1;
     const float* G1 = cp.cores[t][0];
     const int cnt = M.cnt[mb];
-    for (int q = threadIdx.x; q < MB * (R / 4); q += kBwdThreads) {
+    for (int q = threadIdx.x; q < MB * (R / 4); q += (int)blockDim.x) {
         const int m = q / (R / 4), c4 = q % (R / 4);
         const int j = m / D1, a1 = m % D1;
         float* dst = &As[swz_a<R>(m, c4 * 4)];
@@ -1053,12 +1054,12 @@ __device__ __forceinline__ void bwd_issue_batch(const CoreParams& cp, int t, int
     const RowRef rr = batch_rows(M.rows, mb, k0, nb, M.bu[bb], M.bp[bb], M.bi3[bb]);
     float* H = Hs + (size_t)bb * S::NUB * P * D3;
     float* Sb = Ss + (size_t)bb * S::NUB * R * SR;
-    for (int q = tid; q < nb * (P * D3 / 4); q += kBwdThreads) {
+    for (int q = tid; q < nb * (P * D3 / 4); q += (int)blockDim.x) {
         const int uu = q / (P * D3 / 4), c4 = q % (P * D3 / 4);
         cp_async16(&H[uu * P * D3 + c4 * 4], rowbuf + (int64_t)rr.u[uu] * S::D + c4 * 4);
     }
     const float* G3t = cp.last_t[t];   // [n3][R][D3]
-    for (int q = tid; q < nb * R * (D3 / 4); q += kBwdThreads) {
+    for (int q = tid; q < nb * R * (D3 / 4); q += (int)blockDim.x) {
         const int uu = q / (R * (D3 / 4)), rem = q % (R * (D3 / 4));
         const int rho = rem / (D3 / 4), c4 = rem % (D3 / 4);
         cp_async16(&Sb[(uu * R + rho) * SR + c4 * 4], G3t + (int64_t)rr.i3[uu] * (R * D3) + rem * 4);
@@ -1076,7 +1077,7 @@ __device__ __forceinline__ void bwd_issue_a_tc(const CoreParams& cp, int t, int 
     constexpr int R = S::R, MB = S::MB, D1 = S::D1, KC = R / 8;
     const uint16_t* G1 = cp.bf1[t];
     const int cnt = M.cnt[mb];
-    for (int q = threadIdx.x; q < NS * MB * KC; q += kBwdThreads) {
+    for (int q = threadIdx.x; q < NS * MB * KC; q += (int)blockDim.x) {
         const int term = q / (MB * KC), r = q % (MB * KC);
         const int m = (r / (8 * KC)) * 8 + (r & 7), kc = (r >> 3) % KC;   // 8 threads per core matrix
         const int j = m / D1, a1 = m % D1;
@@ -1209,6 +1210,106 @@ __device__ __forceinline__ void bwd_rows_warp(const CoreParams& cp, int t, int m
     flush();
 }
 
+// The same per-row backward with 16 warps: a pair of warps shares each row range, warp 2p + h
+// taking rho_2 = 32 h + lane (one column per lane), so that C_p, dC_p, dS and the streamed rows fit
+// in 128 registers.  Both warps of a pair load the row's H (the second load hits L2).
+struct WarpRow1 {
+    float4 s[2];   // S_u row rho (8 values)
+    float4 h;      // H_u[4 lane .. 4 lane + 3]
+    int u, j, i3;
+};
+
+template <class S, typename K>
+__device__ __forceinline__ void warp_row_load1(const CoreParams& cp, int t, int mb, int kq, int cnt, int rho,
+                                               const BwdMeta<S>& M, const K* __restrict__ uniq_keys,
+                                               const float* __restrict__ rowbuf, uint32_t n3, WarpRow1& w)
+{
+    constexpr int R = S::R, D3 = S::D3, D = S::D;
+    const int lane = threadIdx.x & 31;
+    if (kq < kKeyCap) {
+        w.u = M.rows.u[mb][kq];
+        w.j = M.rows.p[mb][kq];
+        w.i3 = M.rows.i3[mb][kq];
+    } else {
+        w.j = prefix_of(M.ucum[mb], cnt, kq);
+        w.u = M.u0[mb][w.j] + (kq - M.ucum[mb][w.j]);
+        w.i3 = (int)(key_row(uniq_keys[w.u], cp.ibits) % n3);
+    }
+    const float4* sp = reinterpret_cast<const float4*>(cp.last_t[t] + (int64_t)w.i3 * (R * D3) + rho * D3);
+    w.s[0] = __ldg(sp);
+    w.s[1] = __ldg(sp + 1);
+    w.h = __ldcg(reinterpret_cast<const float4*>(rowbuf + (int64_t)w.u * D) + lane);
+}
+
+template <class S, typename K>
+__device__ __forceinline__ void bwd_rows_warp2(const CoreParams& cp, int t, int mb, int total, int cnt,
+                                               const BwdMeta<S>& M, const K* __restrict__ uniq_keys,
+                                               const float* __restrict__ rowbuf, const float* Cn, float* dCn,
+                                               float* __restrict__ dG3, uint32_t n3, float* hslots)
+{
+    constexpr int R = S::R, N = S::N, D1 = S::D1, D2 = S::D2, D3 = S::D3, P = S::P;
+    static_assert(R == 64 && D3 == 8 && P == 16 && S::D == 128, "warp row path: rank 64, d = (4, 4, 8)");
+    constexpr int NPAIR = kBwdThreadsTC / 64;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, pair = warp >> 1;
+    const int rho = (warp & 1) * 32 + lane;
+    const int lo = (int)((int64_t)total * pair / NPAIR), hi = (int)((int64_t)total * (pair + 1) / NPAIR);
+    if (lo >= hi) return;
+    float* hs = hslots + warp * 2 * P * D3;
+    float c[P], o[P];
+    int cur = -1;
+    auto flush = [&]() {
+        const bool whole = M.ucum[mb][cur] >= lo && M.ucum[mb][cur + 1] <= hi;
+#pragma unroll
+        for (int r = 0; r < P; ++r) {
+            float* d = &dCn[swz_m<N>(cur * D1 + r / D2, (r % D2) * R + rho)];
+            if (whole) *d = o[r];
+            else atomicAdd(d, o[r]);
+        }
+    };
+    WarpRow1 a, b;
+    warp_row_load1<S, K>(cp, t, mb, lo, cnt, rho, M, uniq_keys, rowbuf, n3, a);
+    if (lo + 1 < hi) warp_row_load1<S, K>(cp, t, mb, lo + 1, cnt, rho, M, uniq_keys, rowbuf, n3, b);
+#pragma unroll 1
+    for (int kq = lo; kq < hi; ++kq) {
+        const WarpRow1 w = a;
+        a = b;
+        if (kq + 2 < hi) warp_row_load1<S, K>(cp, t, mb, kq + 2, cnt, rho, M, uniq_keys, rowbuf, n3, b);
+        if (w.j != cur) {
+            if (cur >= 0) flush();
+            cur = w.j;
+#pragma unroll
+            for (int r = 0; r < P; ++r) {
+                c[r] = Cn[swz_m<N>(cur * D1 + r / D2, (r % D2) * R + rho)];
+                o[r] = 0.f;
+            }
+        }
+        float* hb = hs + (kq & 1) * (P * D3);
+        reinterpret_cast<float4*>(hb)[lane] = w.h;
+        __syncwarp();
+        const float sv[8] = {w.s[0].x, w.s[0].y, w.s[0].z, w.s[0].w, w.s[1].x, w.s[1].y, w.s[1].z, w.s[1].w};
+        float ds[8];
+#pragma unroll
+        for (int a3 = 0; a3 < 8; ++a3) ds[a3] = 0.f;
+#pragma unroll
+        for (int r = 0; r < P; ++r) {
+            const float4 h0 = *reinterpret_cast<const float4*>(hb + r * D3);
+            const float4 h1 = *reinterpret_cast<const float4*>(hb + r * D3 + 4);
+            const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+            float acc = o[r];
+#pragma unroll
+            for (int a3 = 0; a3 < 8; ++a3) {
+                ds[a3] = fmaf(c[r], hv[a3], ds[a3]);
+                acc = fmaf(hv[a3], sv[a3], acc);
+            }
+            o[r] = acc;
+        }
+        float* dst = dG3 + ((int64_t)rho * n3 + w.i3) * D3;
+        red_add_v4(dst, make_float4(ds[0], ds[1], ds[2], ds[3]));
+        red_add_v4(dst + 4, make_float4(ds[4], ds[5], ds[6], ds[7]));
+    }
+    flush();
+}
+
 // one thread issues, the others wait at the barrier; false (all threads) when the wait ran out
 __device__ __forceinline__ bool tc_commit_wait(uint64_t* bar, uint32_t& parity, int* s_ok)
 {
@@ -1222,7 +1323,7 @@ __device__ __forceinline__ bool tc_commit_wait(uint64_t* bar, uint32_t& parity, 
 }
 
 template <class S, typename K, int NT>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(NT > 0 ? kBwdThreadsTC : kBwdThreads, 1)
 k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ uniq_keys,
               const int4* __restrict__ grec, const int32_t* __restrict__ col_count,
               const int32_t* __restrict__ col_start, PlanHeader* hdr, const float* __restrict__ rowbuf,
@@ -1241,6 +1342,8 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
     constexpr bool TC = NT > 0;
     constexpr int NS = NT == 3 ? 2 : 1;
     constexpr int MT = TC ? 64 : MB;
+    constexpr int BT = TC ? kBwdThreadsTC : kBwdThreads;   // threads of this variant
+    constexpr int CB = BT / 128;                           // column blocks per tensor-memory sub-partition
     constexpr int DAQ = 4;   // dA accumulators in tensor-memory columns [N, N + DAQ R)
     // per-row backward by warps over contiguous row ranges (rank 64, d = (4, 4, 8)); other
     // shapes use barrier-synchronised batches of NUB rows
@@ -1292,11 +1395,11 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
         // B for the whole column group, and the first chunk's A
         if constexpr (TC) {
             const uint16_t* src = cp.bf2[t] + (int64_t)i2 * (NS * R * N);
-            for (int q = tid; q < NS * R * N / 8; q += kBwdThreads) cp_async16(Bb + q * 8, src + q * 8);
+            for (int q = tid; q < NS * R * N / 8; q += BT) cp_async16(Bb + q * 8, src + q * 8);
         } else {
             const float* G2 = cp.cores[t][1] + (int64_t)i2 * N;
             const int64_t rs = (int64_t)n2 * N;
-            for (int q = tid; q < R * N / 4; q += kBwdThreads) {
+            for (int q = tid; q < R * N / 4; q += BT) {
                 const int rho = q / (N / 4), c4 = q % (N / 4);
                 cp_async16(&Bs[swz_b<N>(rho, c4 * 4)], G2 + rho * rs + c4 * 4);
             }
@@ -1325,14 +1428,14 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             __syncthreads();
             const int total = M.ucum[mb][MPB];
             const bool more = j0 + MPB < ccount;
-            build_rows(M.rows, mb, M.ucum[mb], M.u0[mb], cnt, total, s_keys, cp.ibits, n3, kBwdThreads);
+            build_rows(M.rows, mb, M.ucum[mb], M.u0[mb], cnt, total, s_keys, cp.ibits, n3, BT);
             // the next chunk's group records travel with this chunk's first batch
             if (more && tid < min(MPB, ccount - j0 - MPB)) cp_async16(&M.rec[mb ^ 1][tid], grec + cfirst + j0 + MPB + tid);
             __syncthreads();
             // the first batch of distinct rows is in flight during the C GEMM
             if (!WARP_ROWS && total > 0) bwd_issue_batch<S, K>(cp, t, mb, 0, 0, uniq_keys, rowbuf, M, Hs, Ss, s_keys);
             else cp_async_commit();
-            for (int q = tid; q < MB * N / 4; q += kBwdThreads)
+            for (int q = tid; q < MB * N / 4; q += BT)
                 reinterpret_cast<float4*>(dCn)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
             __syncthreads();
             TT_PH(9);
@@ -1356,12 +1459,12 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                     break;
                 }
                 tc_fence_after();
-                const int warp = tid >> 5, lane = tid & 31, sub = warp & 3, half = warp >> 2;
-                if (sub < 2) {   // rows 16 sub + lane (lane < 16)
+                const int warp = tid >> 5, lane = tid & 31, sub = warp & 3, cblk = warp >> 2;
+                if (sub < 2) {   // rows 16 sub + lane (lane < 16), column block cblk of CB
                     const int m = 16 * sub + lane;
 #pragma unroll 1
-                    for (int g = 0; g < N / 64; ++g) {
-                        const int c0 = half * (N / 2) + g * 32;
+                    for (int g = 0; g < N / CB / 32; ++g) {
+                        const int c0 = cblk * (N / CB) + g * 32;
                         float v[32];
                         tmem_ld32(tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)(N + c0), v);
                         if (lane < 16) {
@@ -1423,7 +1526,11 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             }
             TT_PH(16);
 
-            if constexpr (WARP_ROWS) {
+            if constexpr (WARP_ROWS && BT == 512) {
+                bwd_rows_warp2<S, K>(cp, t, mb, total, cnt, M, uniq_keys, rowbuf, Cn, dCn, dG3, n3, Ss);
+                __syncthreads();
+                TT_PH(12);
+            } else if constexpr (WARP_ROWS) {
                 bwd_rows_warp<S, K>(cp, t, mb, total, cnt, M, uniq_keys, rowbuf, Cn, dCn, dG3, n3, Hs);
                 __syncthreads();
                 TT_PH(12);
@@ -1532,14 +1639,14 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                 //   dA = dC . B^T   (M = 64, N = R, K = N) into columns [N, N + R)
                 //   dB += A^T . dC  (M = R, N, K = MB)     into columns [0, N), over the column group
                 {
-                    constexpr int CPT = MB * N / 8 / kBwdThreads;   // 16-byte chunks per thread
-                    static_assert(CPT * kBwdThreads * 8 == MB * N, "dC conversion tiling");
+                    constexpr int CPT = MB * N / 8 / BT;   // 16-byte chunks per thread
+                    static_assert(CPT * BT * 8 == MB * N, "dC conversion tiling");
                     // chunk q: core matrix (m / 8, nc), row m % 8 = q % 8: 8 consecutive threads
                     // write one contiguous 128-byte core matrix
                     float v[CPT][8];
 #pragma unroll
                     for (int i = 0; i < CPT; ++i) {
-                        const int q = tid + i * kBwdThreads;
+                        const int q = tid + i * BT;
                         const int m = (q / (8 * (N / 8))) * 8 + (q & 7), nc = (q >> 3) % (N / 8);
                         const float4 x0 = *reinterpret_cast<const float4*>(&dCn[swz_m<N>(m, nc * 8)]);
                         const float4 x1 = *reinterpret_cast<const float4*>(&dCn[swz_m<N>(m, nc * 8 + 4)]);
@@ -1549,7 +1656,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                     __syncthreads();
 #pragma unroll
                     for (int i = 0; i < CPT; ++i) {
-                        const int q = tid + i * kBwdThreads;
+                        const int q = tid + i * BT;
                         const int m = (q / (8 * (N / 8))) * 8 + (q & 7), nc = (q >> 3) % (N / 8);
                         uint16_t* dst = dCb + ((m >> 3) * (N / 8) + nc) * 64 + (m & 7) * 8;
                         uint4 hi, lo;
@@ -1589,7 +1696,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                 tc_fence_after();
                 TT_PH(13);
                 const int warp = tid >> 5, lane = tid & 31, sub = warp & 3, half = warp >> 2;
-                if (sub < 2) {   // dA rows 16 sub + lane, columns half * R / 2 .., summed over the accumulators
+                if (sub < 2 && half < 2) {   // dA rows 16 sub + lane, columns half * R / 2 .., summed over the accumulators
                     const int m = 16 * sub + lane, p = m / D1, a1 = m % D1;
                     float v[32];
                     tmem_ld32(tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)(N + half * 32), v);
@@ -1698,11 +1805,11 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
         if constexpr (TC) {
             // dG_2[:, i_2] = dB from tensor memory: rows rho_1 = 16 sub + lane (lane < 16), half the columns
             tc_fence_after();
-            const int warp = tid >> 5, lane = tid & 31, sub = warp & 3, half = warp >> 2;
+            const int warp = tid >> 5, lane = tid & 31, sub = warp & 3, cblk = warp >> 2;
             const int rho1 = 16 * sub + lane;
 #pragma unroll 1
-            for (int g = 0; g < N / 64; ++g) {
-                const int c0 = half * (N / 2) + g * 32;
+            for (int g = 0; g < N / CB / 32; ++g) {
+                const int c0 = cblk * (N / CB) + g * 32;
                 float v[32];
                 tmem_ld32(tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)c0, v);
                 if (lane < 16) {
@@ -1909,7 +2016,7 @@ cudaError_t bwd_launch(const K3Args& a, const GradPtrs& gp, const float* grad_ou
     cudaError_t e = cudaFuncSetAttribute(k3_bwd_kernel<S, K, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const PlanBuffers& pb = *a.pb;
-    k3_bwd_kernel<S, K, NT><<<a.grid, kBwdThreads, smem, s>>>(
+    k3_bwd_kernel<S, K, NT><<<a.grid, NT > 0 ? kBwdThreadsTC : kBwdThreads, smem, s>>>(
         *a.cp, gp, *a.pp, (const K*)a.uniq_keys, a.grec, pb.col_count, pb.col_start, pb.hdr, a.rowbuf,
         a.status);
     *nl += 1;
