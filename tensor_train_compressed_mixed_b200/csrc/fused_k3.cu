@@ -65,7 +65,6 @@ constexpr int kBwdThreads = 256;  // backward, FP32 variant: 8 warps, up to 255 
 constexpr int kBwdThreadsTC = 512; // backward, tensor-core variants: 16 warps, at most 128 registers
 constexpr int kNB = kPoolBags;    // bags per pooling task
 constexpr int kHChunk = 256;      // sorted lookups per upstream-sum warp
-constexpr int kHLoads = 8;        // upstream-gradient rows in flight per warp
 constexpr int kSpinLimit = 1 << 22;
 constexpr int kKeyCap = 256;      // distinct rows per chunk whose keys are staged with the chunk
 
@@ -932,11 +931,11 @@ __global__ void __launch_bounds__(256) k3_hsum(const int32_t* __restrict__ uid_s
         const int n = (int)min64(32, c1 - base);
         const int myu = lane < n ? uid_sorted[base + lane] : -1;
         const int myb = lane < n ? bag_sorted[base + lane] : 0;
-        for (int k = 0; k < n; k += kHLoads) {
-            float4 v[kHLoads];
-            int uq[kHLoads];
+        for (int k = 0; k < n; k += 8) {
+            float4 v[8];
+            int uq[8];
 #pragma unroll
-            for (int q = 0; q < kHLoads; ++q) {
+            for (int q = 0; q < 8; ++q) {
                 uq[q] = __shfl_sync(kFull, myu, k + q);
                 const int bag = __shfl_sync(kFull, myb, k + q);
                 // table t = bag / B (t < 64): a float estimate, corrected to the exact quotient
@@ -949,7 +948,7 @@ __global__ void __launch_bounds__(256) k3_hsum(const int32_t* __restrict__ uid_s
                            : zero;
             }
 #pragma unroll
-            for (int q = 0; q < kHLoads; ++q) {
+            for (int q = 0; q < 8; ++q) {
                 if (k + q >= n) break;
                 if (uq[q] != cur) {
                     flush(cur, acc);
