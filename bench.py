@@ -193,8 +193,9 @@ def max_over_ranks(world, x):
     return float(t.item())
 
 
-def kernel_traffic(name):
-    """Per-launch DRAM bytes from a committed ncu summary, if it matches the current source."""
+def kernel_traffic(name, precision, workload):
+    """Per-launch DRAM bytes from a committed ncu summary, if it was taken on the same kernel
+    variant (precision mode), the same workload and the current source."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
@@ -202,7 +203,7 @@ def kernel_traffic(name):
         rec = json.load(open(path)).get(name)
     except (OSError, ValueError):
         return None
-    if not rec:
+    if not rec or rec.get("precision", "fp32") != precision or rec.get("workload_name") != workload:
         return None
     src = os.path.join(ROOT, "tensor_train_compressed_mixed_b200", "csrc", rec["source"])
     if not os.path.exists(src):
@@ -376,7 +377,7 @@ def run_ours(args):
         peak = f_all / t_ideal / 1e12
         achieved = f_all / (per_step[dom] / 1e3) / 1e12
         roof = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None,
+                "frac": achieved / peak, "traffic": kernel_traffic(dom, args.precision, w.name),
                 "peak_source": f"work-weighted: {f_tc / 1e9:.1f} GFLOP of prefix-level products as {products} "
                                f"bf16 tensor-core product(s) each at the measured bf16 peak "
                                f"{BF16_PEAK_TFLOPS:.0f} TF/s, {f_rest / 1e9:.1f} GFLOP at the derived FP32 peak "
@@ -385,12 +386,12 @@ def run_ours(args):
         achieved = flops[dom] / (per_step[dom] / 1e3) / 1e12
         roof = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": FP32_PEAK_TFLOPS,
                 "unit": "TFLOP/s", "frac": achieved / FP32_PEAK_TFLOPS,
-                "traffic": kernel_traffic(dom), "peak_source": "derived: 148 SM x 128 FP32 lanes x 2 x 1.965 GHz"}
+                "traffic": kernel_traffic(dom, args.precision, w.name), "peak_source": "derived: 148 SM x 128 FP32 lanes x 2 x 1.965 GHz"}
     else:
         byts = {"bwd_rowsum": alg["b_rowsum"], "sgd": alg["b_train"] - alg["b_fwd"]}.get(dom)
         ach = byts / (per_step[dom] / 1e3) / 1e9 if byts else None
         roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": 6550.4, "unit": "GB/s",
-                "frac": ach / 6550.4 if ach else None, "traffic": kernel_traffic(dom),
+                "frac": ach / 6550.4 if ach else None, "traffic": kernel_traffic(dom, args.precision, w.name),
                 "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)"}
     t_roof_step = max((alg["f_fwd"] + (alg["f_bwd"] if train else 0)) / (FP32_PEAK_TFLOPS * 1e12),
                       (alg["b_train"] if train else alg["b_fwd"]) / 6550.4e9)
