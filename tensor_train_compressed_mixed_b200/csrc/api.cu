@@ -15,7 +15,7 @@ struct Layout {
         uniq_start, grp_start, bag_sorted;
     // specialised path only (zero when unused)
     size_t uid_at_pos, uid_sorted, rowbuf, pkeys[2], pvals[2], col_count, col_start, chunk_base,
-        hdr, chunks, tasks, grec, g12, dg12, g3t, bf1, bf2;
+        hdr, chunks, tasks, grec, g12, dg12, g3t, dg3t, bf1, bf2;
     int64_t chunk_cap, task_cap;
     size_t total;
 };
@@ -78,6 +78,7 @@ Layout make_layout(int key_bytes, int64_t L, int64_t B, const FastDims& f)
             y.dg12 = take((size_t)f.g12_floats * 4);
         }
         y.g3t = take((size_t)f.g3t_floats * 4);
+        y.dg3t = take((size_t)f.g3t_floats * 4);
         if (f.bf1_elems > 0) {
             y.bf1 = take((size_t)f.bf1_elems * 2);
             y.bf2 = take((size_t)f.bf2_elems * 2);
@@ -747,10 +748,23 @@ static int backward_impl(tt_emb_t h, const float* grad_out, tt_stream_t stream, 
         e = e == cudaSuccess ? cudaMemsetAsync(&pb.hdr->col_head, 0, sizeof(int32_t), s) : e;
         if (e == cudaSuccess && h->merged)
             e = cudaMemsetAsync(h->at(y.dg12), 0, sizeof(float) * (size_t)h->g12_off[h->T], s);
+        // the last cores' gradients accumulate in the transposed layout [n_3][r_2][d_3] (one
+        // row's contribution is one contiguous block) and are transposed back afterwards
+        float* dg3[kMaxT];
+        for (int t = 0; t < h->T; ++t) {
+            dg3[t] = vgp.g[t][2];
+            vgp.g[t][2] = (float*)h->at(y.dg3t) + h->g3t_off[t];
+        }
+        if (e == cudaSuccess) e = cudaMemsetAsync(h->at(y.dg3t), 0, sizeof(float) * (size_t)h->g3t_off[h->T], s);
         h->begin(TT_PHASE_BWD_FUSED, s);
         if (e == cudaSuccess) e = k3_backward(a, vgp, grad_out, s, &nl);
         h->end(s);
         h->begin(TT_PHASE_BWD_REDUCE, s);
+        if (e == cudaSuccess) {
+            const float* src[kMaxT];
+            for (int t = 0; t < h->T; ++t) src[t] = vgp.g[t][2];
+            e = k3_transpose_last_back(vcp, src, dg3, s, &nl);
+        }
         if (e == cudaSuccess && h->merged) e = launch_unmerge(h->merge_params(), h->d_status, s, &nl);
     } else {
         h->begin(TT_PHASE_BWD_FUSED, s);

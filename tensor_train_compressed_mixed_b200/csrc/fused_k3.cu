@@ -1090,7 +1090,9 @@ __device__ __forceinline__ void bwd_issue_a_tc(const CoreParams& cp, int t, int 
 
 // Per-row backward of a chunk with one warp per contiguous range of its distinct rows (rank 64,
 // d = (4, 4, 8)); lane l owns rho_2 in {2l, 2l + 1}.  For each row u of prefix p:
-//   dS_u[rho][a3] = sum_r C_p[r][rho] H_u[r][a3]    -> dG_3[rho, i3(u), a3] (vector reductions)
+//   dS_u[rho][a3] = sum_r C_p[r][rho] H_u[r][a3]    -> dG_3[rho, i3(u), a3] (vector reductions into
+//                                                      the transposed copy [i3][rho][a3]: one row's
+//                                                      2 KB contribution is contiguous)
 //   dC_p[r][rho] += sum_a3 H_u[r][a3] S_u[rho][a3]   (registers; into dCn when the prefix ends:
 //                                                      a plain store when the prefix lies inside
 //                                                      this warp's range, shared atomics if not)
@@ -1202,7 +1204,7 @@ __device__ __forceinline__ void bwd_rows_warp(const CoreParams& cp, int t, int m
         }
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-            float* dst = dG3 + ((int64_t)(2 * lane + q) * n3 + w.i3) * D3;
+            float* dst = dG3 + ((int64_t)w.i3 * R + 2 * lane + q) * D3;
             red_add_v4(dst, make_float4(ds[q][0], ds[q][1], ds[q][2], ds[q][3]));
             red_add_v4(dst + 4, make_float4(ds[q][4], ds[q][5], ds[q][6], ds[q][7]));
         }
@@ -1241,6 +1243,15 @@ __device__ __forceinline__ void warp_row_load1(const CoreParams& cp, int t, int 
     w.h = __ldcg(reinterpret_cast<const float4*>(rowbuf + (int64_t)w.u * D) + lane);
 }
 
+// the row range [lo, hi) of this warp's pair
+__device__ __forceinline__ void warp_pair_range(int total, int& lo, int& hi)
+{
+    constexpr int NPAIR = kBwdThreadsTC / 64;
+    const int pair = (int)(threadIdx.x >> 6);
+    lo = (int)((int64_t)total * pair / NPAIR);
+    hi = (int)((int64_t)total * (pair + 1) / NPAIR);
+}
+
 template <class S, typename K>
 __device__ __forceinline__ void bwd_rows_warp2(const CoreParams& cp, int t, int mb, int total, int cnt,
                                                const BwdMeta<S>& M, const K* __restrict__ uniq_keys,
@@ -1249,11 +1260,14 @@ __device__ __forceinline__ void bwd_rows_warp2(const CoreParams& cp, int t, int 
 {
     constexpr int R = S::R, N = S::N, D1 = S::D1, D2 = S::D2, D3 = S::D3, P = S::P;
     static_assert(R == 64 && D3 == 8 && P == 16 && S::D == 128, "warp row path: rank 64, d = (4, 4, 8)");
-    constexpr int NPAIR = kBwdThreadsTC / 64;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, pair = warp >> 1;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rho = (warp & 1) * 32 + lane;
-    const int lo = (int)((int64_t)total * pair / NPAIR), hi = (int)((int64_t)total * (pair + 1) / NPAIR);
+    int lo, hi;
+    warp_pair_range(total, lo, hi);
     if (lo >= hi) return;
+    WarpRow1 a, b;
+    warp_row_load1<S, K>(cp, t, mb, lo, cnt, rho, M, uniq_keys, rowbuf, n3, a);
+    if (lo + 1 < hi) warp_row_load1<S, K>(cp, t, mb, lo + 1, cnt, rho, M, uniq_keys, rowbuf, n3, b);
     float* hs = hslots + warp * 2 * P * D3;
     float c[P], o[P];
     int cur = -1;
@@ -1266,9 +1280,6 @@ __device__ __forceinline__ void bwd_rows_warp2(const CoreParams& cp, int t, int 
             else atomicAdd(d, o[r]);
         }
     };
-    WarpRow1 a, b;
-    warp_row_load1<S, K>(cp, t, mb, lo, cnt, rho, M, uniq_keys, rowbuf, n3, a);
-    if (lo + 1 < hi) warp_row_load1<S, K>(cp, t, mb, lo + 1, cnt, rho, M, uniq_keys, rowbuf, n3, b);
 #pragma unroll 1
     for (int kq = lo; kq < hi; ++kq) {
         const WarpRow1 w = a;
@@ -1303,7 +1314,7 @@ __device__ __forceinline__ void bwd_rows_warp2(const CoreParams& cp, int t, int 
             }
             o[r] = acc;
         }
-        float* dst = dG3 + ((int64_t)rho * n3 + w.i3) * D3;
+        float* dst = dG3 + ((int64_t)w.i3 * R + rho) * D3;
         red_add_v4(dst, make_float4(ds[0], ds[1], ds[2], ds[3]));
         red_add_v4(dst + 4, make_float4(ds[4], ds[5], ds[6], ds[7]));
     }
@@ -1389,7 +1400,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
         const uint32_t n2 = cp.n[t][1], n3 = cp.n[t][2];
         float* __restrict__ dG1 = gp.g[t][0];
         float* __restrict__ dG2 = gp.g[t][1];
-        float* __restrict__ dG3 = gp.g[t][2];
+        float* __restrict__ dG3 = gp.g[t][2];   // transposed layout [n3][R][D3]
         TT_PH_START();
 
         // B for the whole column group, and the first chunk's A
@@ -1579,7 +1590,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                         const int i3 = rr.i3[uu];
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
-                            red_add_v4(dG3 + ((int64_t)(rc * 4 + i) * n3 + i3) * D3 + cg * 4, o[i]);
+                            red_add_v4(dG3 + ((int64_t)i3 * R + rc * 4 + i) * D3 + cg * 4, o[i]);
                     }
                 }
 #ifdef TT_PROFILE_PHASES
@@ -1943,7 +1954,7 @@ __global__ void __launch_bounds__(256) k3_bf16_kernel(Bf16Job j)
 }
 
 struct TransposeJob {
-    int32_t T, R, D3, pad;
+    int32_t T, R, D3, back;   // back: src [n3][R][D3] -> dst [R][n3][D3]
     int64_t row_base[kMaxT + 1];   // prefix sums of n3 * R
     uint32_t n3[kMaxT];
     const float* src[kMaxT];
@@ -1960,8 +1971,9 @@ __global__ void __launch_bounds__(256) k3_transpose_last_kernel(TransposeJob tj,
         while (t + 1 < tj.T && tj.row_base[t + 1] <= q) ++t;
         const int64_t rq = q - tj.row_base[t];
         const int64_t i3 = rq / tj.R, rho = rq % tj.R;
-        const float4* src = reinterpret_cast<const float4*>(tj.src[t] + (rho * tj.n3[t] + i3) * tj.D3);
-        float4* dst = reinterpret_cast<float4*>(tj.dst[t] + (i3 * tj.R + rho) * tj.D3);
+        const int64_t core = (rho * tj.n3[t] + i3) * tj.D3, trans = (i3 * tj.R + rho) * tj.D3;
+        const float4* src = reinterpret_cast<const float4*>(tj.src[t] + (tj.back ? trans : core));
+        float4* dst = reinterpret_cast<float4*>(tj.dst[t] + (tj.back ? core : trans));
         for (int c = 0; c < tj.D3 / 4; ++c) dst[c] = __ldg(src + c);
     }
 }
@@ -2125,19 +2137,21 @@ cudaError_t k3_forward(const K3Args& a, float* out, cudaStream_t s, int* nl)
     return cudaErrorInvalidValue;
 }
 
-cudaError_t k3_transpose_last(const CoreParams& cp, float* const* dst, cudaStream_t s, int* nl)
+static cudaError_t transpose_last(const CoreParams& cp, const float* const* src, float* const* dst, bool back,
+                                  cudaStream_t s, int* nl)
 {
     TransposeJob tj;
     memset(&tj, 0, sizeof(tj));
     tj.T = cp.T;
     tj.R = cp.r[2];
     tj.D3 = cp.d[2];
+    tj.back = back ? 1 : 0;
     int64_t b = 0;
     for (int t = 0; t < cp.T; ++t) {
         tj.row_base[t] = b;
         b += (int64_t)cp.n[t][2] * tj.R;
         tj.n3[t] = cp.n[t][2];
-        tj.src[t] = cp.cores[t][2];
+        tj.src[t] = src[t];
         tj.dst[t] = dst[t];
     }
     tj.row_base[cp.T] = b;
@@ -2146,6 +2160,19 @@ cudaError_t k3_transpose_last(const CoreParams& cp, float* const* dst, cudaStrea
     k3_transpose_last_kernel<<<grid, 256, 0, s>>>(tj, nullptr);
     *nl += 1;
     return cudaGetLastError();
+}
+
+cudaError_t k3_transpose_last(const CoreParams& cp, float* const* dst, cudaStream_t s, int* nl)
+{
+    const float* src[kMaxT];
+    for (int t = 0; t < cp.T; ++t) src[t] = cp.cores[t][2];
+    return transpose_last(cp, src, dst, false, s, nl);
+}
+
+cudaError_t k3_transpose_last_back(const CoreParams& cp, const float* const* src, float* const* dst, cudaStream_t s,
+                                   int* nl)
+{
+    return transpose_last(cp, src, dst, true, s, nl);
 }
 
 cudaError_t k3_to_bf16(const CoreParams& cp, int terms, uint16_t* const* dst1, uint16_t* const* dst2,

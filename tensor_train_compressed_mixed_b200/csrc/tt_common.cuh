@@ -70,6 +70,8 @@ struct CoreParams {
 };
 
 struct GradPtrs {
+    // gradient buffers in the core layouts; the three-core specialised backward takes the last
+    // core's gradient in the transposed layout [n3][R][D3] instead
     float* g[kMaxT][kMaxK];
     // fused SGD (tt_emb_backward_sgd): the middle core is updated in place by the block that
     // reduces its column group, G_2[:, i_2] -= lr * dB, instead of writing dG_2
@@ -263,6 +265,9 @@ cudaError_t k3_to_bf16(const CoreParams& cp, int terms, uint16_t* const* dst1, u
 cudaError_t k3_forward(const K3Args& a, float* out, cudaStream_t s, int* nl);
 // last core [r][n_k][d_k] -> [n_k][r][d_k] into cp.last_t (before k3_forward / k3_backward)
 cudaError_t k3_transpose_last(const CoreParams& cp, float* const* dst, cudaStream_t s, int* nl);
+// [n3][R][D3] per table -> dst in the core layout [R][n3][D3] (gradients of the last cores)
+cudaError_t k3_transpose_last_back(const CoreParams& cp, const float* const* src, float* const* dst, cudaStream_t s,
+                                   int* nl);
 // upstream sums per distinct row (must run before k3_backward)
 cudaError_t k3_rowsum(const K3Args& a, const float* grad_out, cudaStream_t s, int* nl);
 cudaError_t k3_backward(const K3Args& a, const GradPtrs& gp, const float* grad_out, cudaStream_t s,
