@@ -1885,6 +1885,453 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
 }
 
 // ---------------------------------------------------------------------------
+// Tensor-core backward with transposed prefix products (rank 64, d = (4, 4, 8)).
+//
+// A chunk is kMPB2 = 16 prefixes of a column group, i.e. 64 rows m = (prefix, a_1) of A.
+//   C^T = B^T A^T   two M = 128 products (n = (a_2, rho_2) in [0, 128) and [128, 256)), N = 64,
+//                   K = R, left in tensor memory: lane n holds column n of C for every chunk row.
+//                   The warp of sub-partition s reads rho_2 = 32 (s mod 2) + l for a_2 in
+//                   {s / 2, s / 2 + 2} with one tcgen05.ld per prefix -- no copy of C through
+//                   shared memory.
+//   rows            the four warps of a quad (one per sub-partition) share each distinct row u of
+//                   prefix p; a lane holds C_p for its rho_2 and two a_2 (8 values) and adds
+//                     dS_u[rho][a3] += sum_{a1, its a2} C_p[(a1, a2)][rho] H_u[(a1, a2)][a3]
+//                                      (vector reductions into dG_3^T [i3][rho][a3])
+//                     dC_p[(a1, a2)][rho] += sum_a3 H_u[(a1, a2)][a3] S_u[rho][a3]
+//                   with the quads on contiguous row ranges and no block barrier between rows.
+//   dA = dC . B^T (M = 64, every row a chunk row), dB += A^T . dC over the column group.
+// ---------------------------------------------------------------------------
+constexpr int kMPB2 = 16;   // prefixes per chunk
+constexpr int kMB2 = 64;    // rows of A per chunk
+
+struct BwdMeta2 {
+    int u0[2][kMPB2];
+    int ucum[2][kMPB2 + 1];
+    int i1[2][kMPB2];
+    int cnt[2];
+    int task;
+    RowTable rows;
+    int4 rec[2][kMPB2];   // the next chunk's per-group records, prefetched
+};
+
+// chunk metadata into buffer mb (ends with a barrier), then asynchronous copies of the keys of
+// its first kKeyCap distinct rows into keys[mb] (they join the caller's next commit group)
+template <typename K>
+__device__ __forceinline__ void bwd2_meta(const int4* recs, int j0, int ccount, int mb, const K* __restrict__ uniq_keys,
+                                          BwdMeta2& M, K* keys)
+{
+    const int tid = threadIdx.x;
+    const int cnt = min(kMPB2, ccount - j0);
+    if (tid < 32) {
+        // one warp: records, exclusive scan of the row counts
+        const int4 g = tid < cnt ? recs[tid] : make_int4(0, 0, 0, 0);
+        int x = tid < kMPB2 ? g.y : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, x, o);
+            if (tid >= o) x += y;
+        }
+        if (tid < kMPB2) {
+            M.u0[mb][tid] = g.x;
+            M.ucum[mb][tid] = x - g.y;
+            M.i1[mb][tid] = g.z;
+        }
+        if (tid == kMPB2 - 1) M.ucum[mb][kMPB2] = x;
+        if (tid == 0) M.cnt[mb] = cnt;
+    }
+    __syncthreads();
+    const int nk = min(M.ucum[mb][kMPB2], kKeyCap);
+    for (int kq = tid; kq < nk; kq += (int)blockDim.x) {
+        const int j = prefix_of(M.ucum[mb], cnt, kq);
+        cp_async_key(keys + mb * kKeyCap + kq, uniq_keys + M.u0[mb][j] + (kq - M.ucum[mb][j]));
+    }
+}
+
+// the chunk's G_1 rows (NS bf16 terms) into 8 x 16-byte core matrices of kMB2 rows; one commit group
+template <int NS>
+__device__ __forceinline__ void bwd2_issue_a(const CoreParams& cp, int t, int mb, const BwdMeta2& M, uint16_t* Ab)
+{
+    constexpr int R = 64, MB = kMB2, D1 = 4, KC = R / 8;
+    const uint16_t* G1 = cp.bf1[t];
+    const int cnt = M.cnt[mb];
+    for (int q = threadIdx.x; q < NS * MB * KC; q += (int)blockDim.x) {
+        const int term = q / (MB * KC), r = q % (MB * KC);
+        const int m = (r / (8 * KC)) * 8 + (r & 7), kc = (r >> 3) % KC;   // 8 threads per core matrix
+        const int j = m / D1, a1 = m % D1;
+        uint16_t* dst = Ab + term * (MB * R) + ((m >> 3) * KC + kc) * 64 + (m & 7) * 8;
+        if (j < cnt) cp_async16(dst, G1 + ((int64_t)M.i1[mb][j] * D1 + a1) * (NS * R) + term * R + kc * 8);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    cp_async_commit();
+}
+
+// two 32 x 4 reads of tensor memory (lane i of the warp: row taddr lane + i, 4 columns each), and
+// the wait for both, in one statement so no use of the values can move above the wait
+__device__ __forceinline__ void tmem_ld4x2(uint32_t ta, uint32_t tb, float (&v)[8])
+{
+    uint32_t r[8];
+    asm volatile(
+        "{\n\ttcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%8];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%4, %5, %6, %7}, [%9];\n\t"
+        "tcgen05.wait::ld.sync.aligned;\n\t}"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+        : "r"(ta), "r"(tb)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+// 32 lanes x 16 consecutive columns, with the wait
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
+{
+    uint32_t r[16];
+    asm volatile(
+        "{\n\ttcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15}, [%16];\n\ttcgen05.wait::ld.sync.aligned;\n\t}"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <typename K>
+__device__ __forceinline__ void warp_row_load2(const CoreParams& cp, int t, int mb, int kq, int cnt, int rho,
+                                               const BwdMeta2& M, const K* __restrict__ uniq_keys,
+                                               const float* __restrict__ rowbuf, uint32_t n3, WarpRow1& w)
+{
+    constexpr int R = 64, D3 = 8, D = 128;
+    const int lane = threadIdx.x & 31;
+    if (kq < kKeyCap) {
+        w.u = M.rows.u[mb][kq];
+        w.j = M.rows.p[mb][kq];
+        w.i3 = M.rows.i3[mb][kq];
+    } else {
+        w.j = prefix_of(M.ucum[mb], cnt, kq);
+        w.u = M.u0[mb][w.j] + (kq - M.ucum[mb][w.j]);
+        w.i3 = (int)(key_row(uniq_keys[w.u], cp.ibits) % n3);
+    }
+    const float4* sp = reinterpret_cast<const float4*>(cp.last_t[t] + (int64_t)w.i3 * (R * D3) + rho * D3);
+    w.s[0] = __ldg(sp);
+    w.s[1] = __ldg(sp + 1);
+    // the four warps of the quad read the same row: through L1
+    w.h = __ldg(reinterpret_cast<const float4*>(rowbuf + (int64_t)w.u * D) + lane);
+}
+
+// the chunk's distinct rows by quads of warps (see above); tmem_c = the C^T accumulators
+template <typename K>
+__device__ __forceinline__ void bwd2_rows(const CoreParams& cp, int t, int mb, int total, int cnt, const BwdMeta2& M,
+                                          const K* __restrict__ uniq_keys, const float* __restrict__ rowbuf,
+                                          uint32_t tmem_c, float* dCn, float* __restrict__ dG3, uint32_t n3,
+                                          float* hslots)
+{
+    constexpr int R = 64, N = 256, D1 = 4, D2 = 4, D3 = 8, P = 16, MB = kMB2, NQ = kBwdThreadsTC / 128;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, sub = warp & 3, quad = warp >> 2;
+    const int rho = (sub & 1) * 32 + lane, a2a = sub >> 1;   // this warp's a_2: a2a and a2a + 2
+    const int lo = (int)((int64_t)total * quad / NQ), hi = (int)((int64_t)total * (quad + 1) / NQ);
+    if (lo >= hi) return;
+    const uint32_t tl = tmem_c + ((uint32_t)(32 * sub) << 16);
+    float* hs = hslots + warp * 2 * P * D3;
+    WarpRow1 a, b;
+    warp_row_load2<K>(cp, t, mb, lo, cnt, rho, M, uniq_keys, rowbuf, n3, a);
+    if (lo + 1 < hi) warp_row_load2<K>(cp, t, mb, lo + 1, cnt, rho, M, uniq_keys, rowbuf, n3, b);
+    float c[8], o[8];   // entry 2 a1 + g: a_2 = a2a + 2 g
+    int cur = -1;
+    auto flush = [&]() {
+        const bool whole = M.ucum[mb][cur] >= lo && M.ucum[mb][cur + 1] <= hi;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float* d = &dCn[swz_m<N>(cur * D1 + (i >> 1), (a2a + 2 * (i & 1)) * R + rho)];
+            if (whole) *d = o[i];
+            else atomicAdd(d, o[i]);
+        }
+    };
+#pragma unroll 1
+    for (int kq = lo; kq < hi; ++kq) {
+        const WarpRow1 w = a;
+        a = b;
+        if (kq + 2 < hi) warp_row_load2<K>(cp, t, mb, kq + 2, cnt, rho, M, uniq_keys, rowbuf, n3, b);
+        if (w.j != cur) {
+            if (cur >= 0) flush();
+            cur = w.j;
+            float v[8];   // columns m = 4 cur + a1 of the two accumulators
+            tmem_ld4x2(tl + (uint32_t)(cur * D1), tl + (uint32_t)(MB + cur * D1), v);
+#pragma unroll
+            for (int a1 = 0; a1 < 4; ++a1) {
+                c[2 * a1] = v[a1];
+                c[2 * a1 + 1] = v[4 + a1];
+                o[2 * a1] = 0.f;
+                o[2 * a1 + 1] = 0.f;
+            }
+        }
+        float* hb = hs + (kq & 1) * (P * D3);
+        reinterpret_cast<float4*>(hb)[lane] = w.h;
+        __syncwarp();
+        const float sv[8] = {w.s[0].x, w.s[0].y, w.s[0].z, w.s[0].w, w.s[1].x, w.s[1].y, w.s[1].z, w.s[1].w};
+        float ds[8];
+#pragma unroll
+        for (int a3 = 0; a3 < 8; ++a3) ds[a3] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int r = (i >> 1) * D2 + a2a + 2 * (i & 1);   // row (a1, a2) of H_u
+            const float4 h0 = *reinterpret_cast<const float4*>(hb + r * D3);
+            const float4 h1 = *reinterpret_cast<const float4*>(hb + r * D3 + 4);
+            const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+            float acc = o[i];
+#pragma unroll
+            for (int a3 = 0; a3 < 8; ++a3) {
+                ds[a3] = fmaf(c[i], hv[a3], ds[a3]);
+                acc = fmaf(hv[a3], sv[a3], acc);
+            }
+            o[i] = acc;
+        }
+        float* dst = dG3 + ((int64_t)w.i3 * R + rho) * D3;
+        red_add_v4(dst, make_float4(ds[0], ds[1], ds[2], ds[3]));
+        red_add_v4(dst + 4, make_float4(ds[4], ds[5], ds[6], ds[7]));
+    }
+    flush();
+}
+
+template <typename K, int NT>
+__global__ void __launch_bounds__(kBwdThreadsTC, 1)
+k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ uniq_keys,
+                  const int4* __restrict__ grec, const int32_t* __restrict__ col_count,
+                  const int32_t* __restrict__ col_start, PlanHeader* hdr, const float* __restrict__ rowbuf,
+                  int32_t* status)
+{
+    constexpr int R = 64, N = 256, D1 = 4, MPB = kMPB2, MB = kMB2, BT = kBwdThreadsTC;
+    constexpr int NS = NT == 3 ? 2 : 1;
+    constexpr int CB = BT / 128;   // column blocks per tensor-memory sub-partition
+    constexpr int DAQ = 4;         // dA accumulators in tensor-memory columns [N, N + DAQ R)
+    static_assert(NT == 1 || NT == 3, "tensor-core variants");
+    extern __shared__ __align__(16) float smem_f[];
+    __shared__ BwdMeta2 M;
+    __shared__ __align__(16) K s_keys[2 * kKeyCap];
+    __shared__ __align__(8) uint64_t s_mbar;
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_ok;
+    uint16_t* Bb = reinterpret_cast<uint16_t*>(smem_f);            // NS x (N x R): [n/8][rho/8][8][8]
+    uint16_t* Abt = Bb + NS * R * N;                                // [2][NS][MB x R]: [m/8][rho/8][8][8]
+    float* dCn = reinterpret_cast<float*>(Abt + 2 * NS * MB * R);   // [MB][N] swizzled; then NS x (MB x N) bf16
+    uint16_t* dCb = reinterpret_cast<uint16_t*>(dCn);
+    float* hslots = dCn + MB * N;                                   // [warps][2][P D3]
+    if (has_error(status)) return;
+    const int tid = threadIdx.x;
+    uint32_t parity = 0;
+    bool failed = false;
+    // tensor memory: columns [0, N) dB of the column group; [N, N + 2 MB) C^T, then [N, N + DAQ R) dA
+    if (tid < 32) tmem_alloc(&s_tmem, 2 * N);
+    if (tid == 0) mbar_init(&s_mbar, 1);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+
+    for (int iter = 0;; ++iter) {
+        if (tid == 0) M.task = next_task(pp.sched, &hdr->col_head, iter);
+        __syncthreads();
+        const int c = M.task;
+        if (c >= pp.ncols) break;
+        const int ccount = col_count[c];
+        if (ccount == 0) {
+            __syncthreads();
+            continue;
+        }
+        int t = 0;
+        while (t + 1 < cp.T && pp.col_base[t + 1] <= c) ++t;
+        const int i2 = c - pp.col_base[t];
+        const int cfirst = col_start[c];
+        const uint32_t n2 = cp.n[t][1], n3 = cp.n[t][2];
+        float* __restrict__ dG1 = gp.g[t][0];
+        float* __restrict__ dG2 = gp.g[t][1];
+        float* __restrict__ dG3 = gp.g[t][2];   // transposed layout [n3][R][D3]
+        TT_PH_START();
+        {
+            const uint16_t* src = cp.bf2[t] + (int64_t)i2 * (NS * R * N);
+            for (int q = tid; q < NS * R * N / 8; q += BT) cp_async16(Bb + q * 8, src + q * 8);
+        }
+        bwd2_meta<K>(grec + cfirst, 0, ccount, 0, uniq_keys, M, s_keys);
+        bwd2_issue_a<NS>(cp, t, 0, M, Abt);
+        TT_PH(8);
+
+        int mb = 0;
+        for (int j0 = 0; j0 < ccount; j0 += MPB, mb ^= 1) {
+            const int cnt = M.cnt[mb];
+            const uint16_t* Ab16 = Abt + mb * NS * MB * R;
+            cp_async_wait_all();   // B, this chunk's A rows and row keys
+            __syncthreads();
+            const int total = M.ucum[mb][MPB];
+            const bool more = j0 + MPB < ccount;
+            build_rows(M.rows, mb, M.ucum[mb], M.u0[mb], cnt, total, s_keys, cp.ibits, n3, BT);
+            if (more && tid < min(MPB, ccount - j0 - MPB)) cp_async16(&M.rec[mb ^ 1][tid], grec + cfirst + j0 + MPB + tid);
+            cp_async_commit();
+            for (int q = tid; q < MB * N / 4; q += BT)
+                reinterpret_cast<float4*>(dCn)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            fence_async_smem();
+            __syncthreads();
+            TT_PH(9);
+
+            // C^T = B^T A^T: A operand = the B tile read as M = n (K-major), B operand = the A tile
+            if (tid == 0) {
+                tc_fence_after();
+                constexpr uint32_t SBO = (R / 8) * 128;
+                const uint32_t a0 = smem_u32(Bb), b0 = smem_u32(Ab16);
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int k = 0; k < R / 16; ++k)
+                        tc_mma_terms<NT>(tmem + (uint32_t)(N + h * MB), umma_desc(a0 + h * 16 * SBO + k * 256, 128, SBO),
+                                         umma_desc(b0 + k * 256, 128, SBO), R * N * 2, MB * R * 2,
+                                         umma_idesc_bf16(128, MB), k > 0);
+            }
+            if (!tc_commit_wait(&s_mbar, parity, &s_ok)) {
+                failed = true;
+                break;
+            }
+            tc_fence_after();
+            TT_PH(10);
+
+            // next chunk's metadata and A rows go in flight while this chunk's rows are processed
+            if (more) {
+                cp_async_wait_all();   // its group records
+                __syncthreads();
+                bwd2_meta<K>(M.rec[mb ^ 1], j0 + MPB, ccount, mb ^ 1, uniq_keys, M, s_keys);
+                bwd2_issue_a<NS>(cp, t, mb ^ 1, M, Abt + (mb ^ 1) * NS * MB * R);
+            }
+            TT_PH(16);
+
+            bwd2_rows<K>(cp, t, mb, total, cnt, M, uniq_keys, rowbuf, tmem + (uint32_t)N, dCn, dG3, n3, hslots);
+            tc_fence_before();
+            __syncthreads();
+            TT_PH(12);
+
+            // dC -> NS bf16 terms in core matrices (MB rows, K = N), written over dCn once
+            {
+                constexpr int CPT = MB * N / 8 / BT;   // 16-byte chunks per thread
+                static_assert(CPT * BT * 8 == MB * N, "dC conversion tiling");
+                float v[CPT][8];
+#pragma unroll
+                for (int i = 0; i < CPT; ++i) {
+                    const int q = tid + i * BT;
+                    const int m = (q / (8 * (N / 8))) * 8 + (q & 7), nc = (q >> 3) % (N / 8);
+                    const float4 x0 = *reinterpret_cast<const float4*>(&dCn[swz_m<N>(m, nc * 8)]);
+                    const float4 x1 = *reinterpret_cast<const float4*>(&dCn[swz_m<N>(m, nc * 8 + 4)]);
+                    v[i][0] = x0.x; v[i][1] = x0.y; v[i][2] = x0.z; v[i][3] = x0.w;
+                    v[i][4] = x1.x; v[i][5] = x1.y; v[i][6] = x1.z; v[i][7] = x1.w;
+                }
+                __syncthreads();
+#pragma unroll
+                for (int i = 0; i < CPT; ++i) {
+                    const int q = tid + i * BT;
+                    const int m = (q / (8 * (N / 8))) * 8 + (q & 7), nc = (q >> 3) % (N / 8);
+                    uint16_t* dst = dCb + ((m >> 3) * (N / 8) + nc) * 64 + (m & 7) * 8;
+                    uint4 hi, lo;
+                    split_bf16x8(v[i], hi, lo);
+                    *reinterpret_cast<uint4*>(dst) = hi;
+                    if constexpr (NS == 2) *reinterpret_cast<uint4*>(dst + MB * N) = lo;
+                }
+            }
+            fence_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+                tc_fence_after();
+                const uint32_t c0 = smem_u32(dCb), b0 = smem_u32(Bb), a0 = smem_u32(Ab16);
+                // dA = dC . B^T: A = dC (K-major), B = the B tile viewed MN-major; the K range
+                // split over DAQ accumulators issued in turn
+#pragma unroll 1
+                for (int kk = 0; kk < N / 16 / DAQ; ++kk)
+#pragma unroll
+                    for (int q = 0; q < DAQ; ++q) {
+                        const int k = q * (N / 16 / DAQ) + kk;
+                        tc_mma_terms<NT>(tmem + (uint32_t)(N + q * R), umma_desc(c0 + k * 256, 128, (N / 8) * 128),
+                                         umma_desc_mn(b0 + k * 2 * (R / 8) * 128, 128, (R / 8) * 128),
+                                         MB * N * 2, R * N * 2, umma_idesc_bf16(MB, R, false, true), kk > 0);
+                    }
+                // dB += A^T . dC: A = the A tile viewed MN-major, B = dC viewed MN-major
+#pragma unroll
+                for (int k = 0; k < MB / 16; ++k)
+                    tc_mma_terms<NT>(tmem, umma_desc_mn(a0 + k * 2 * (R / 8) * 128, 128, (R / 8) * 128),
+                                     umma_desc_mn(c0 + k * 2 * (N / 8) * 128, 128, (N / 8) * 128),
+                                     MB * R * 2, MB * N * 2, umma_idesc_bf16(R, N, true, true), j0 > 0 || k > 0);
+            }
+            if (!tc_commit_wait(&s_mbar, parity, &s_ok)) {
+                failed = true;
+                break;
+            }
+            tc_fence_after();
+            TT_PH(13);
+            {
+                // dA rows m = 16 sub + lane (lane < 16), columns 16 qtr .. 16 qtr + 15, summed over the
+                // accumulators -> dG_1
+                const int warp = tid >> 5, lane = tid & 31, sub = warp & 3, qtr = warp >> 2;
+                const int m = 16 * sub + lane, p = m / D1, a1 = m % D1;
+                const uint32_t ta = tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)(N + qtr * 16);
+                float v[16];
+                tmem_ld16(ta, v);
+#pragma unroll 1
+                for (int q = 1; q < DAQ; ++q) {
+                    float x[16];
+                    tmem_ld16(ta + (uint32_t)(q * R), x);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] += x[i];
+                }
+                if (lane < 16 && p < cnt) {
+                    float* dst = dG1 + ((int64_t)M.i1[mb][p] * D1 + a1) * R + qtr * 16;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        red_add_v4(dst + 4 * j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+                }
+            }
+            tc_fence_before();
+            __syncthreads();   // dCn, the dC tile and the A buffer are reused by the next chunks
+            TT_PH(14);
+        }
+        if (failed) break;
+        {
+            // dG_2[:, i_2] = dB from tensor memory: rows rho_1 = 16 sub + lane (lane < 16)
+            tc_fence_after();
+            const int warp = tid >> 5, lane = tid & 31, sub = warp & 3, cblk = warp >> 2;
+            const int rho1 = 16 * sub + lane;
+#pragma unroll 1
+            for (int g = 0; g < N / CB / 32; ++g) {
+                const int c0 = cblk * (N / CB) + g * 32;
+                float v[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)c0, v);
+                if (lane < 16) {
+                    if (gp.fused) {   // sparse fused SGD: G_2[:, i_2] -= lr dB
+                        float* g2 = gp.upd1[t] + ((int64_t)rho1 * n2 + i2) * N + c0;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const float4 x = *reinterpret_cast<const float4*>(g2 + 4 * j);
+                            *reinterpret_cast<float4*>(g2 + 4 * j) =
+                                make_float4(x.x - gp.lr * v[4 * j], x.y - gp.lr * v[4 * j + 1],
+                                            x.z - gp.lr * v[4 * j + 2], x.w - gp.lr * v[4 * j + 3]);
+                        }
+                    } else {
+                        float* dst = dG2 + ((int64_t)rho1 * n2 + i2) * N + c0;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            *reinterpret_cast<float4*>(dst + 4 * j) =
+                                make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                    }
+                }
+            }
+            tc_fence_before();
+        }
+        __syncthreads();
+        TT_PH(15);
+    }
+    cp_async_wait_all();
+    if (failed && tid == 0) raise_error(status, TT_ERR_TIMEOUT, 103);
+    tc_fence_before();
+    __syncthreads();
+    if (tid < 32) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 2 * N);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // last core [R][n3][D3] -> [n3][R][D3]; one thread per (table, i3, rho) row of D3 floats
 // ---------------------------------------------------------------------------
 // bf16 operand copies for the tensor-core forward.  Items are 16-byte output chunks:
@@ -2052,12 +2499,32 @@ cudaError_t bwd_dispatch(const K3Args& a, const GradPtrs& gp, const float* g, cu
 {
     return a.key64 ? bwd_launch<S, uint64_t, 0>(a, gp, g, s, nl) : bwd_launch<S, uint32_t, 0>(a, gp, g, s, nl);
 }
-template <class S>
-cudaError_t bwd_dispatch_tc(const K3Args& a, const GradPtrs& gp, const float* g, cudaStream_t s, int* nl)
+// shared memory of the transposed-product backward: B tile, two A tiles, dC, per-warp H slots
+template <int NT>
+constexpr size_t bwd2_smem_bytes()
 {
-    if (a.tc == 3)
-        return a.key64 ? bwd_launch<S, uint64_t, 3>(a, gp, g, s, nl) : bwd_launch<S, uint32_t, 3>(a, gp, g, s, nl);
-    return a.key64 ? bwd_launch<S, uint64_t, 1>(a, gp, g, s, nl) : bwd_launch<S, uint32_t, 1>(a, gp, g, s, nl);
+    constexpr size_t NS = NT == 3 ? 2 : 1;
+    return NS * 64 * 256 * 2 + 2 * NS * kMB2 * 64 * 2 + (size_t)kMB2 * 256 * 4 + (kBwdThreadsTC / 32) * 2 * 128 * 4;
+}
+
+template <typename K, int NT>
+cudaError_t bwd2_launch(const K3Args& a, const GradPtrs& gp, cudaStream_t s, int* nl)
+{
+    const size_t smem = bwd2_smem_bytes<NT>();
+    cudaError_t e = cudaFuncSetAttribute(k3_bwd_tc2_kernel<K, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const PlanBuffers& pb = *a.pb;
+    k3_bwd_tc2_kernel<K, NT><<<a.grid, kBwdThreadsTC, smem, s>>>(
+        *a.cp, gp, *a.pp, (const K*)a.uniq_keys, a.grec, pb.col_count, pb.col_start, pb.hdr, a.rowbuf, a.status);
+    *nl += 1;
+    return cudaGetLastError();
+}
+
+// tensor-core backward (rank 64, d = (4, 4, 8)): the transposed-product kernel
+cudaError_t bwd_dispatch_tc(const K3Args& a, const GradPtrs& gp, cudaStream_t s, int* nl)
+{
+    if (a.tc == 3) return a.key64 ? bwd2_launch<uint64_t, 3>(a, gp, s, nl) : bwd2_launch<uint32_t, 3>(a, gp, s, nl);
+    return a.key64 ? bwd2_launch<uint64_t, 1>(a, gp, s, nl) : bwd2_launch<uint32_t, 1>(a, gp, s, nl);
 }
 
 template <class S, int NT>
@@ -2217,7 +2684,7 @@ cudaError_t k3_backward(const K3Args& a, const GradPtrs& gp, const float* grad_o
 {
     const CoreParams& cp = *a.cp;
     if (a.tc) {
-        if (k3_tc_bwd_supported(cp)) return bwd_dispatch_tc<S3<4, 4, 8, 64>>(a, gp, grad_out, s, nl);
+        if (k3_tc_bwd_supported(cp)) return bwd_dispatch_tc(a, gp, s, nl);
         return cudaErrorInvalidValue;
     }
 #define TT_BWD_CASE(Q1, Q2, Q3, QR) \
