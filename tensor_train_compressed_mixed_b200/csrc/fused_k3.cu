@@ -21,6 +21,11 @@
 //     and dB += A^T dC.  dB is reduced on chip over the whole column group and
 //     written once; dA and the last-slice gradients are reduced into the
 //     small, L2-resident gradient arrays with 16-byte vector reductions.
+//   * With the tensor-core precisions (d = (4,4,8), R in {32, 64}) the
+//     prefix-level products run as tcgen05 MMAs with fp32 accumulators in
+//     tensor memory: C = A . B in the forward; in the backward (R = 64) the
+//     transposed C^T = B^T A^T, which each warp reads straight from tensor
+//     memory, then dA = dC . B^T and dB += A^T . dC.
 #include <cuda_bf16.h>
 #include <string.h>
 
@@ -62,7 +67,7 @@ namespace {
 
 constexpr int kFwdThreads = 512;  // forward: 16 warps, at most 128 registers per thread
 constexpr int kBwdThreads = 256;  // backward, FP32 variant: 8 warps, up to 255 registers per thread
-constexpr int kBwdThreadsTC = 512; // backward, tensor-core variants: 16 warps, at most 128 registers
+constexpr int kBwdThreadsTC = 512; // backward, tensor-core kernel: 16 warps (4 per sub-partition), at most 128 registers
 constexpr int kNB = kPoolBags;    // bags per pooling task
 constexpr int kHChunk = 256;      // sorted lookups per upstream-sum warp
 constexpr int kSpinLimit = 1 << 22;
@@ -107,13 +112,6 @@ struct S3 {
     static constexpr size_t fwd_smem_floats_tc(int NS)
     {
         return (size_t)NS * ((size_t)R * N + (size_t)MF * R) / 2 + (size_t)MF * N + (size_t)FBUF * NUF * SU;
-    }
-    // tensor-core backward (rank 64): B and two A buffers as NS bf16 terms; dC's bf16 terms
-    // overwrite dCn
-    static constexpr size_t bwd_smem_floats_tc(int NS)
-    {
-        return (size_t)NS * R * N / 2 + (size_t)NS * MB * R + 2 * (size_t)MB * N + 2 * (size_t)NUB * P * D3 +
-               2 * (size_t)NUB * R * SR;
     }
     static constexpr size_t bwd_smem_floats()
     {
@@ -1067,27 +1065,6 @@ __device__ __forceinline__ void bwd_issue_batch(const CoreParams& cp, int t, int
     cp_async_commit();
 }
 
-// Tensor-core variant of bwd_issue_a: the chunk's G_1 rows (NS bf16 terms: hi tile, then
-// lo tile) into 8 x 16-byte core matrices of MB rows; one commit group.  The M = 64 MMAs
-// read 64 rows: rows MB..63 fall on the following tile, and the output rows they feed are
-// never read.
-template <class S, int NS>
-__device__ __forceinline__ void bwd_issue_a_tc(const CoreParams& cp, int t, int mb, const BwdMeta<S>& M, uint16_t* Ab)
-{
-    constexpr int R = S::R, MB = S::MB, D1 = S::D1, KC = R / 8;
-    const uint16_t* G1 = cp.bf1[t];
-    const int cnt = M.cnt[mb];
-    for (int q = threadIdx.x; q < NS * MB * KC; q += (int)blockDim.x) {
-        const int term = q / (MB * KC), r = q % (MB * KC);
-        const int m = (r / (8 * KC)) * 8 + (r & 7), kc = (r >> 3) % KC;   // 8 threads per core matrix
-        const int j = m / D1, a1 = m % D1;
-        uint16_t* dst = Ab + term * (MB * R) + ((m >> 3) * KC + kc) * 64 + (m & 7) * 8;
-        if (j < cnt) cp_async16(dst, G1 + ((int64_t)M.i1[mb][j] * D1 + a1) * (NS * R) + term * R + kc * 8);
-        else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-    }
-    cp_async_commit();
-}
-
 // Per-row backward of a chunk with one warp per contiguous range of its distinct rows (rank 64,
 // d = (4, 4, 8)); lane l owns rho_2 in {2l, 2l + 1}.  For each row u of prefix p:
 //   dS_u[rho][a3] = sum_r C_p[r][rho] H_u[r][a3]    -> dG_3[rho, i3(u), a3] (vector reductions into
@@ -1212,114 +1189,13 @@ __device__ __forceinline__ void bwd_rows_warp(const CoreParams& cp, int t, int m
     flush();
 }
 
-// The same per-row backward with 16 warps: a pair of warps shares each row range, warp 2p + h
-// taking rho_2 = 32 h + lane (one column per lane), so that C_p, dC_p, dS and the streamed rows fit
-// in 128 registers.  Both warps of a pair load the row's H (the second load hits L2).
+// One lane's share of a distinct row in the tensor-core backward (rank 64): its row of the last
+// slice and a quarter-row of H_u
 struct WarpRow1 {
     float4 s[2];   // S_u row rho (8 values)
     float4 h;      // H_u[4 lane .. 4 lane + 3]
     int u, j, i3;
 };
-
-template <class S, typename K>
-__device__ __forceinline__ void warp_row_load1(const CoreParams& cp, int t, int mb, int kq, int cnt, int rho,
-                                               const BwdMeta<S>& M, const K* __restrict__ uniq_keys,
-                                               const float* __restrict__ rowbuf, uint32_t n3, WarpRow1& w)
-{
-    constexpr int R = S::R, D3 = S::D3, D = S::D;
-    const int lane = threadIdx.x & 31;
-    if (kq < kKeyCap) {
-        w.u = M.rows.u[mb][kq];
-        w.j = M.rows.p[mb][kq];
-        w.i3 = M.rows.i3[mb][kq];
-    } else {
-        w.j = prefix_of(M.ucum[mb], cnt, kq);
-        w.u = M.u0[mb][w.j] + (kq - M.ucum[mb][w.j]);
-        w.i3 = (int)(key_row(uniq_keys[w.u], cp.ibits) % n3);
-    }
-    const float4* sp = reinterpret_cast<const float4*>(cp.last_t[t] + (int64_t)w.i3 * (R * D3) + rho * D3);
-    w.s[0] = __ldg(sp);
-    w.s[1] = __ldg(sp + 1);
-    w.h = __ldcg(reinterpret_cast<const float4*>(rowbuf + (int64_t)w.u * D) + lane);
-}
-
-// the row range [lo, hi) of this warp's pair
-__device__ __forceinline__ void warp_pair_range(int total, int& lo, int& hi)
-{
-    constexpr int NPAIR = kBwdThreadsTC / 64;
-    const int pair = (int)(threadIdx.x >> 6);
-    lo = (int)((int64_t)total * pair / NPAIR);
-    hi = (int)((int64_t)total * (pair + 1) / NPAIR);
-}
-
-template <class S, typename K>
-__device__ __forceinline__ void bwd_rows_warp2(const CoreParams& cp, int t, int mb, int total, int cnt,
-                                               const BwdMeta<S>& M, const K* __restrict__ uniq_keys,
-                                               const float* __restrict__ rowbuf, const float* Cn, float* dCn,
-                                               float* __restrict__ dG3, uint32_t n3, float* hslots)
-{
-    constexpr int R = S::R, N = S::N, D1 = S::D1, D2 = S::D2, D3 = S::D3, P = S::P;
-    static_assert(R == 64 && D3 == 8 && P == 16 && S::D == 128, "warp row path: rank 64, d = (4, 4, 8)");
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int rho = (warp & 1) * 32 + lane;
-    int lo, hi;
-    warp_pair_range(total, lo, hi);
-    if (lo >= hi) return;
-    WarpRow1 a, b;
-    warp_row_load1<S, K>(cp, t, mb, lo, cnt, rho, M, uniq_keys, rowbuf, n3, a);
-    if (lo + 1 < hi) warp_row_load1<S, K>(cp, t, mb, lo + 1, cnt, rho, M, uniq_keys, rowbuf, n3, b);
-    float* hs = hslots + warp * 2 * P * D3;
-    float c[P], o[P];
-    int cur = -1;
-    auto flush = [&]() {
-        const bool whole = M.ucum[mb][cur] >= lo && M.ucum[mb][cur + 1] <= hi;
-#pragma unroll
-        for (int r = 0; r < P; ++r) {
-            float* d = &dCn[swz_m<N>(cur * D1 + r / D2, (r % D2) * R + rho)];
-            if (whole) *d = o[r];
-            else atomicAdd(d, o[r]);
-        }
-    };
-#pragma unroll 1
-    for (int kq = lo; kq < hi; ++kq) {
-        const WarpRow1 w = a;
-        a = b;
-        if (kq + 2 < hi) warp_row_load1<S, K>(cp, t, mb, kq + 2, cnt, rho, M, uniq_keys, rowbuf, n3, b);
-        if (w.j != cur) {
-            if (cur >= 0) flush();
-            cur = w.j;
-#pragma unroll
-            for (int r = 0; r < P; ++r) {
-                c[r] = Cn[swz_m<N>(cur * D1 + r / D2, (r % D2) * R + rho)];
-                o[r] = 0.f;
-            }
-        }
-        float* hb = hs + (kq & 1) * (P * D3);
-        reinterpret_cast<float4*>(hb)[lane] = w.h;
-        __syncwarp();
-        const float sv[8] = {w.s[0].x, w.s[0].y, w.s[0].z, w.s[0].w, w.s[1].x, w.s[1].y, w.s[1].z, w.s[1].w};
-        float ds[8];
-#pragma unroll
-        for (int a3 = 0; a3 < 8; ++a3) ds[a3] = 0.f;
-#pragma unroll
-        for (int r = 0; r < P; ++r) {
-            const float4 h0 = *reinterpret_cast<const float4*>(hb + r * D3);
-            const float4 h1 = *reinterpret_cast<const float4*>(hb + r * D3 + 4);
-            const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-            float acc = o[r];
-#pragma unroll
-            for (int a3 = 0; a3 < 8; ++a3) {
-                ds[a3] = fmaf(c[r], hv[a3], ds[a3]);
-                acc = fmaf(hv[a3], sv[a3], acc);
-            }
-            o[r] = acc;
-        }
-        float* dst = dG3 + ((int64_t)w.i3 * R + rho) * D3;
-        red_add_v4(dst, make_float4(ds[0], ds[1], ds[2], ds[3]));
-        red_add_v4(dst + 4, make_float4(ds[4], ds[5], ds[6], ds[7]));
-    }
-    flush();
-}
 
 // one thread issues, the others wait at the barrier; false (all threads) when the wait ran out
 __device__ __forceinline__ bool tc_commit_wait(uint64_t* bar, uint32_t& parity, int* s_ok)
@@ -1333,8 +1209,8 @@ __device__ __forceinline__ bool tc_commit_wait(uint64_t* bar, uint32_t& parity, 
     return *s_ok != 0;
 }
 
-template <class S, typename K, int NT>
-__global__ void __launch_bounds__(NT > 0 ? kBwdThreadsTC : kBwdThreads, 1)
+template <class S, typename K>
+__global__ void __launch_bounds__(kBwdThreads, 1)
 k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ uniq_keys,
               const int4* __restrict__ grec, const int32_t* __restrict__ col_count,
               const int32_t* __restrict__ col_start, PlanHeader* hdr, const float* __restrict__ rowbuf,
@@ -1345,43 +1221,18 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
     extern __shared__ __align__(16) float smem_f[];
     __shared__ BwdMeta<S> M;
     __shared__ __align__(16) K s_keys[2 * kKeyCap];   // keys of each chunk buffer's first rows
-    __shared__ __align__(8) uint64_t s_mbar;
-    __shared__ uint32_t s_tmem;
-    __shared__ int s_ok;
-    // tensor-core variants: MMA row count 64 (the MB chunk rows, then rows nobody reads) and
-    // bf16 operand tiles of NS terms each (NT = 3 products for two terms)
-    constexpr bool TC = NT > 0;
-    constexpr int NS = NT == 3 ? 2 : 1;
-    constexpr int MT = TC ? 64 : MB;
-    constexpr int BT = TC ? kBwdThreadsTC : kBwdThreads;   // threads of this variant
-    constexpr int CB = BT / 128;                           // column blocks per tensor-memory sub-partition
-    constexpr int DAQ = 4;   // dA accumulators in tensor-memory columns [N, N + DAQ R)
+    constexpr int BT = kBwdThreads;
     // per-row backward by warps over contiguous row ranges (rank 64, d = (4, 4, 8)); other
     // shapes use barrier-synchronised batches of NUB rows
     constexpr bool WARP_ROWS = R == 64 && D1 == 4 && D2 == 4 && D3 == 8;
-    static_assert(!TC || (R == 64 && MB == 32 && N == 256 && DAQ * R <= N), "tensor-core backward: rank 64, d_2 = 4");
-    float* Bs = smem_f;                    // [R][N] swizzled (key row/4)            (fp32 variant)
-    uint16_t* Bb = reinterpret_cast<uint16_t*>(smem_f);   // NS x (N x R) bf16 core matrices (tensor cores)
-    float* As = smem_f + (TC ? NS * R * N / 2 : R * N);   // [2][MB][R] fp32 swizzled, or [2][NS][MB x R] bf16
-    uint16_t* Abt = reinterpret_cast<uint16_t*>(As);
-    float* Cn = As + (TC ? NS * MB * R : 2 * MB * R);     // [MB][N] swizzled (key row)
-    float* dCn = Cn + MB * N;              // [MB][N] swizzled (key row); tensor cores: then NS x (MB x N) bf16
-    uint16_t* dCb = reinterpret_cast<uint16_t*>(dCn);
+    float* Bs = smem_f;                    // [R][N] swizzled (key row/4)
+    float* As = smem_f + R * N;            // [2][MB][R] swizzled
+    float* Cn = As + 2 * MB * R;           // [MB][N] swizzled (key row)
+    float* dCn = Cn + MB * N;              // [MB][N] swizzled (key row)
     float* Hs = dCn + MB * N;              // [2][NUB][P][D3]
     float* Ss = Hs + 2 * NUB * P * D3;     // [2][NUB][R][SR]
     if (has_error(status)) return;
     const int tid = threadIdx.x;
-    uint32_t tmem = 0, parity = 0;
-    bool failed = false;
-    if constexpr (TC) {
-        // tensor memory: columns [0, N) hold dB of the current column group, [N, 2N) C and then dA
-        if (tid < 32) tmem_alloc(&s_tmem, 2 * N);
-        if (tid == 0) mbar_init(&s_mbar, 1);
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        tmem = s_tmem;
-    }
 
     for (int iter = 0;; ++iter) {
         if (tid == 0) M.task = next_task(pp.sched, &hdr->col_head, iter);
@@ -1404,10 +1255,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
         TT_PH_START();
 
         // B for the whole column group, and the first chunk's A
-        if constexpr (TC) {
-            const uint16_t* src = cp.bf2[t] + (int64_t)i2 * (NS * R * N);
-            for (int q = tid; q < NS * R * N / 8; q += BT) cp_async16(Bb + q * 8, src + q * 8);
-        } else {
+        {
             const float* G2 = cp.cores[t][1] + (int64_t)i2 * N;
             const int64_t rs = (int64_t)n2 * N;
             for (int q = tid; q < R * N / 4; q += BT) {
@@ -1416,25 +1264,23 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             }
         }
         bwd_meta<S, K>(grec + cfirst, 0, ccount, 0, uniq_keys, M, s_keys);
-        if constexpr (TC) bwd_issue_a_tc<S, NS>(cp, t, 0, M, Abt);
-        else bwd_issue_a<S>(cp, t, 0, M, As);
+        bwd_issue_a<S>(cp, t, 0, M, As);
         TT_PH(8);
 
-        constexpr int XR = TC ? 1 : DBR, XC = TC ? 4 : DBC;   // register dB (FP32 variant only)
-        constexpr int NCH = XC / 4;
-        constexpr int TNB = N / XC;
+        // dB of the column group in registers: DBR rows x DBC columns per thread
+        constexpr int NCH = DBC / 4;
+        constexpr int TNB = N / DBC;
         const int tnb = tid % TNB, trb = tid / TNB;
-        float dB[XR][XC];
+        float dB[DBR][DBC];
 #pragma unroll
-        for (int i = 0; i < XR; ++i)
+        for (int i = 0; i < DBR; ++i)
 #pragma unroll
-            for (int j = 0; j < XC; ++j) dB[i][j] = 0.f;
+            for (int j = 0; j < DBC; ++j) dB[i][j] = 0.f;
 
         int mb = 0;
         for (int j0 = 0; j0 < ccount; j0 += MPB, mb ^= 1) {
             const int cnt = M.cnt[mb];
             const float* Ab = As + mb * MB * R;
-            const uint16_t* Ab16 = Abt + mb * NS * MB * R;
             cp_async_wait_all();   // B, this chunk's A rows and row keys (usually prefetched long ago)
             __syncthreads();
             const int total = M.ucum[mb][MPB];
@@ -1451,43 +1297,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             __syncthreads();
             TT_PH(9);
 
-            if constexpr (TC) {
-                // C_all = A . B on the tensor cores (M = 64, N, K = R) into tensor-memory columns
-                // [N, 2N), then rows < MB into Cn (sub-partitions 0 and 1)
-                fence_async_smem();
-                __syncthreads();
-                if (tid == 0) {
-                    tc_fence_after();
-                    constexpr uint32_t SBO = (R / 8) * 128;
-                    const uint32_t a0 = smem_u32(Ab16), b0 = smem_u32(Bb);
-#pragma unroll
-                    for (int k = 0; k < R / 16; ++k)
-                        tc_mma_terms<NT>(tmem + N, umma_desc(a0 + k * 256, 128, SBO), umma_desc(b0 + k * 256, 128, SBO),
-                                         MB * R * 2, R * N * 2, umma_idesc_bf16(MT, N), k > 0);
-                }
-                if (!tc_commit_wait(&s_mbar, parity, &s_ok)) {
-                    failed = true;
-                    break;
-                }
-                tc_fence_after();
-                const int warp = tid >> 5, lane = tid & 31, sub = warp & 3, cblk = warp >> 2;
-                if (sub < 2) {   // rows 16 sub + lane (lane < 16), column block cblk of CB
-                    const int m = 16 * sub + lane;
-#pragma unroll 1
-                    for (int g = 0; g < N / CB / 32; ++g) {
-                        const int c0 = cblk * (N / CB) + g * 32;
-                        float v[32];
-                        tmem_ld32(tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)(N + c0), v);
-                        if (lane < 16) {
-#pragma unroll
-                            for (int j = 0; j < 8; ++j)
-                                *reinterpret_cast<float4*>(&Cn[swz_m<N>(m, c0 + 4 * j)]) =
-                                    make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-                        }
-                    }
-                }
-                tc_fence_before();
-            } else {
+            {
                 // C_all = A . B  (MB x N): thread tile 4 rows x 8 cols
                 constexpr int TN = N / 8;
                 int tm, tn;   // tm < MB / 4
@@ -1532,16 +1342,11 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                 cp_async_wait_all();   // its group records (and this chunk's first batch)
                 __syncthreads();
                 bwd_meta<S, K>(M.rec[mb ^ 1], j0 + MPB, ccount, mb ^ 1, uniq_keys, M, s_keys);
-                if constexpr (TC) bwd_issue_a_tc<S, NS>(cp, t, mb ^ 1, M, Abt + (mb ^ 1) * NS * MB * R);
-                else bwd_issue_a<S>(cp, t, mb ^ 1, M, As + (mb ^ 1) * MB * R);
+                bwd_issue_a<S>(cp, t, mb ^ 1, M, As + (mb ^ 1) * MB * R);
             }
             TT_PH(16);
 
-            if constexpr (WARP_ROWS && BT == 512) {
-                bwd_rows_warp2<S, K>(cp, t, mb, total, cnt, M, uniq_keys, rowbuf, Cn, dCn, dG3, n3, Ss);
-                __syncthreads();
-                TT_PH(12);
-            } else if constexpr (WARP_ROWS) {
+            if constexpr (WARP_ROWS) {
                 bwd_rows_warp<S, K>(cp, t, mb, total, cnt, M, uniq_keys, rowbuf, Cn, dCn, dG3, n3, Hs);
                 __syncthreads();
                 TT_PH(12);
@@ -1644,92 +1449,6 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                 TT_PH(12);
             }
 
-            if constexpr (TC) {
-                // dC -> NS bf16 terms in core matrices (MB rows, K = N), written over dCn once
-                // every thread holds its share in registers; then on the tensor cores
-                //   dA = dC . B^T   (M = 64, N = R, K = N) into columns [N, N + R)
-                //   dB += A^T . dC  (M = R, N, K = MB)     into columns [0, N), over the column group
-                {
-                    constexpr int CPT = MB * N / 8 / BT;   // 16-byte chunks per thread
-                    static_assert(CPT * BT * 8 == MB * N, "dC conversion tiling");
-                    // chunk q: core matrix (m / 8, nc), row m % 8 = q % 8: 8 consecutive threads
-                    // write one contiguous 128-byte core matrix
-                    float v[CPT][8];
-#pragma unroll
-                    for (int i = 0; i < CPT; ++i) {
-                        const int q = tid + i * BT;
-                        const int m = (q / (8 * (N / 8))) * 8 + (q & 7), nc = (q >> 3) % (N / 8);
-                        const float4 x0 = *reinterpret_cast<const float4*>(&dCn[swz_m<N>(m, nc * 8)]);
-                        const float4 x1 = *reinterpret_cast<const float4*>(&dCn[swz_m<N>(m, nc * 8 + 4)]);
-                        v[i][0] = x0.x; v[i][1] = x0.y; v[i][2] = x0.z; v[i][3] = x0.w;
-                        v[i][4] = x1.x; v[i][5] = x1.y; v[i][6] = x1.z; v[i][7] = x1.w;
-                    }
-                    __syncthreads();
-#pragma unroll
-                    for (int i = 0; i < CPT; ++i) {
-                        const int q = tid + i * BT;
-                        const int m = (q / (8 * (N / 8))) * 8 + (q & 7), nc = (q >> 3) % (N / 8);
-                        uint16_t* dst = dCb + ((m >> 3) * (N / 8) + nc) * 64 + (m & 7) * 8;
-                        uint4 hi, lo;
-                        split_bf16x8(v[i], hi, lo);
-                        *reinterpret_cast<uint4*>(dst) = hi;
-                        if constexpr (NS == 2) *reinterpret_cast<uint4*>(dst + MB * N) = lo;
-                    }
-                }
-                fence_async_smem();
-                __syncthreads();
-                if (tid == 0) {
-                    tc_fence_after();
-                    const uint32_t c0 = smem_u32(dCb), b0 = smem_u32(Bb), a0 = smem_u32(Ab16);
-                    // dA: A = dC (K-major: 8-row groups 16 N bytes apart), B = B viewed MN-major.
-                    // The K range is split over DAQ accumulators (columns N + q R) issued in turn,
-                    // so the small M = 64 x N = R products do not form one serial chain.
-#pragma unroll 1
-                    for (int kk = 0; kk < N / 16 / DAQ; ++kk)
-#pragma unroll
-                        for (int q = 0; q < DAQ; ++q) {
-                            const int k = q * (N / 16 / DAQ) + kk;
-                            tc_mma_terms<NT>(tmem + N + q * R, umma_desc(c0 + k * 256, 128, (N / 8) * 128),
-                                             umma_desc_mn(b0 + k * 2 * (R / 8) * 128, 128, (R / 8) * 128),
-                                             MB * N * 2, R * N * 2, umma_idesc_bf16(MT, R, false, true), kk > 0);
-                        }
-                    // dB: A = A^T (MN-major over the A tile), B = dC viewed MN-major
-#pragma unroll
-                    for (int k = 0; k < MB / 16; ++k)
-                        tc_mma_terms<NT>(tmem, umma_desc_mn(a0 + k * 2 * (R / 8) * 128, 128, (R / 8) * 128),
-                                         umma_desc_mn(c0 + k * 2 * (N / 8) * 128, 128, (N / 8) * 128),
-                                         MB * R * 2, MB * N * 2, umma_idesc_bf16(R, N, true, true), j0 > 0 || k > 0);
-                }
-                if (!tc_commit_wait(&s_mbar, parity, &s_ok)) {
-                    failed = true;
-                    break;
-                }
-                tc_fence_after();
-                TT_PH(13);
-                const int warp = tid >> 5, lane = tid & 31, sub = warp & 3, half = warp >> 2;
-                if (sub < 2 && half < 2) {   // dA rows 16 sub + lane, columns half * R / 2 .., summed over the accumulators
-                    const int m = 16 * sub + lane, p = m / D1, a1 = m % D1;
-                    float v[32];
-                    tmem_ld32(tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)(N + half * 32), v);
-#pragma unroll 1
-                    for (int q = 1; q < DAQ; ++q) {
-                        float x[32];
-                        tmem_ld32(tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)(N + q * R + half * 32), x);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] += x[i];
-                    }
-                    if (lane < 16 && p < cnt) {
-                        float* dst = dG1 + ((int64_t)M.i1[mb][p] * D1 + a1) * R + half * 32;
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            red_add_v4(dst + 4 * j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
-                    }
-                }
-                tc_fence_before();
-                __syncthreads();   // dCn, the dC tile and the A buffer are reused by the next chunks
-                TT_PH(14);
-                // (the FP32 variant follows)
-            } else {
             // dA[m][rho1] = sum_n dC[m][n] B[rho1][n] -> dG_1; tiles 4 m x 4 rho1, the n range split
             // between the two halves of the block and combined through shared memory
             {
@@ -1810,40 +1529,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
             }
             __syncthreads();   // dCn, Ab and the partial buffer are reused by the next chunk
             TT_PH(14);
-            }
         }
-        if (failed) break;
-        if constexpr (TC) {
-            // dG_2[:, i_2] = dB from tensor memory: rows rho_1 = 16 sub + lane (lane < 16), half the columns
-            tc_fence_after();
-            const int warp = tid >> 5, lane = tid & 31, sub = warp & 3, cblk = warp >> 2;
-            const int rho1 = 16 * sub + lane;
-#pragma unroll 1
-            for (int g = 0; g < N / CB / 32; ++g) {
-                const int c0 = cblk * (N / CB) + g * 32;
-                float v[32];
-                tmem_ld32(tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)c0, v);
-                if (lane < 16) {
-                    if (gp.fused) {   // sparse fused SGD: G_2[:, i_2] -= lr dB
-                        float* g2 = gp.upd1[t] + ((int64_t)rho1 * n2 + i2) * N + c0;
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const float4 x = *reinterpret_cast<const float4*>(g2 + 4 * j);
-                            *reinterpret_cast<float4*>(g2 + 4 * j) =
-                                make_float4(x.x - gp.lr * v[4 * j], x.y - gp.lr * v[4 * j + 1],
-                                            x.z - gp.lr * v[4 * j + 2], x.w - gp.lr * v[4 * j + 3]);
-                        }
-                    } else {
-                        float* dst = dG2 + ((int64_t)rho1 * n2 + i2) * N + c0;
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            *reinterpret_cast<float4*>(dst + 4 * j) =
-                                make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-                    }
-                }
-            }
-            tc_fence_before();
-        } else {
         // the column group is complete: dG_2[:, i_2] = dB (this block owns the slice)
 #pragma unroll
         for (int i = 0; i < DBR; ++i) {
@@ -1868,20 +1554,10 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
                         make_float4(dB[i][ch * 4], dB[i][ch * 4 + 1], dB[i][ch * 4 + 2], dB[i][ch * 4 + 3]);
             }
         }
-        }
         __syncthreads();
         TT_PH(15);
     }
     cp_async_wait_all();
-    if constexpr (TC) {
-        if (failed && tid == 0) raise_error(status, TT_ERR_TIMEOUT, 101);
-        tc_fence_before();
-        __syncthreads();
-        if (tid < 32) {
-            tc_fence_after();
-            tmem_dealloc(tmem, 2 * N);
-        }
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -2434,10 +2110,10 @@ constexpr size_t fwd_smem_bytes()
 {
     return sizeof(float) * (NT == 0 ? S::fwd_smem_floats() : S::fwd_smem_floats_tc(NT == 3 ? 2 : 1));
 }
-template <class S, int NT>
+template <class S>
 constexpr size_t bwd_smem_bytes()
 {
-    return sizeof(float) * (NT == 0 ? S::bwd_smem_floats() : S::bwd_smem_floats_tc(NT == 3 ? 2 : 1));
+    return sizeof(float) * S::bwd_smem_floats();
 }
 
 template <class S, typename K, int NT>
@@ -2467,15 +2143,15 @@ cudaError_t rowsum_launch(const K3Args& a, const float* grad_out, cudaStream_t s
     return cudaGetLastError();
 }
 
-template <class S, typename K, int NT>
+template <class S, typename K>
 cudaError_t bwd_launch(const K3Args& a, const GradPtrs& gp, const float* grad_out, cudaStream_t s, int* nl)
 {
     (void)grad_out;
-    const size_t smem = bwd_smem_bytes<S, NT>();
-    cudaError_t e = cudaFuncSetAttribute(k3_bwd_kernel<S, K, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = bwd_smem_bytes<S>();
+    cudaError_t e = cudaFuncSetAttribute(k3_bwd_kernel<S, K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const PlanBuffers& pb = *a.pb;
-    k3_bwd_kernel<S, K, NT><<<a.grid, NT > 0 ? kBwdThreadsTC : kBwdThreads, smem, s>>>(
+    k3_bwd_kernel<S, K><<<a.grid, kBwdThreads, smem, s>>>(
         *a.cp, gp, *a.pp, (const K*)a.uniq_keys, a.grec, pb.col_count, pb.col_start, pb.hdr, a.rowbuf,
         a.status);
     *nl += 1;
@@ -2497,7 +2173,7 @@ cudaError_t fwd_dispatch_tc(const K3Args& a, float* out, cudaStream_t s, int* nl
 template <class S>
 cudaError_t bwd_dispatch(const K3Args& a, const GradPtrs& gp, const float* g, cudaStream_t s, int* nl)
 {
-    return a.key64 ? bwd_launch<S, uint64_t, 0>(a, gp, g, s, nl) : bwd_launch<S, uint32_t, 0>(a, gp, g, s, nl);
+    return a.key64 ? bwd_launch<S, uint64_t>(a, gp, g, s, nl) : bwd_launch<S, uint32_t>(a, gp, g, s, nl);
 }
 // shared memory of the transposed-product backward: B tile, two A tiles, dC, per-warp H slots
 template <int NT>
@@ -2541,9 +2217,9 @@ template <class S>
 int occ_bwd()
 {
     const size_t smem = sizeof(float) * S::bwd_smem_floats();
-    cudaFuncSetAttribute(k3_bwd_kernel<S, uint32_t, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(k3_bwd_kernel<S, uint32_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k3_bwd_kernel<S, uint32_t, 0>, kBwdThreads, smem) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k3_bwd_kernel<S, uint32_t>, kBwdThreads, smem) !=
         cudaSuccess)
         return 1;
     return n > 0 ? n : 1;
