@@ -1778,8 +1778,10 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
     constexpr int R = 64, N = 256, D1 = 4, MPB = kMPB2, MB = kMB2, BT = kBwdThreadsTC;
     constexpr int NS = NT == 3 ? 2 : 1;
     constexpr int CB = BT / 128;   // column blocks per tensor-memory sub-partition
-    constexpr int DAQ = 4;         // dA accumulators in tensor-memory columns [N, N + DAQ R)
+    constexpr int DAQ = 2;         // dA accumulators in tensor-memory columns [N + 2 MB, N + 2 MB + DAQ R)
+    constexpr uint32_t TDA = N + 2 * MB;
     static_assert(NT == 1 || NT == 3, "tensor-core variants");
+    static_assert(TDA + DAQ * R <= 2 * N, "tensor-memory columns");
     extern __shared__ __align__(16) float smem_f[];
     __shared__ BwdMeta2 M;
     __shared__ __align__(16) K s_keys[2 * kKeyCap];
@@ -1795,7 +1797,9 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
     const int tid = threadIdx.x;
     uint32_t parity = 0;
     bool failed = false;
-    // tensor memory: columns [0, N) dB of the column group; [N, N + 2 MB) C^T, then [N, N + DAQ R) dA
+    // tensor memory: columns [0, N) dB of the column group, [N, N + 2 MB) C^T, [TDA, TDA + DAQ R) dA.
+    // A chunk's dA and dB products are waited for by the commit after the next chunk's C^T
+    // product (or at the end of the column): they run while the next chunk's row table is built.
     if (tid < 32) tmem_alloc(&s_tmem, 2 * N);
     if (tid == 0) mbar_init(&s_mbar, 1);
     tc_fence_before();
@@ -1829,6 +1833,29 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
         bwd2_meta<K>(grec + cfirst, 0, ccount, 0, uniq_keys, M, s_keys);
         bwd2_issue_a<NS>(cp, t, 0, M, Abt);
         TT_PH(8);
+        // dA of a chunk whose products are complete -> dG_1: rows m = 16 sub + lane (lane < 16),
+        // columns 16 qtr .. 16 qtr + 15, summed over the accumulators
+        auto read_dA = [&](int pmb, int pcnt) {
+            const int warp = tid >> 5, lane = tid & 31, sub = warp & 3, qtr = warp >> 2;
+            const int m = 16 * sub + lane, p = m / D1, a1 = m % D1;
+            const uint32_t ta = tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)(TDA + qtr * 16);
+            float v[16];
+            tmem_ld16(ta, v);
+#pragma unroll 1
+            for (int q = 1; q < DAQ; ++q) {
+                float x[16];
+                tmem_ld16(ta + (uint32_t)(q * R), x);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] += x[i];
+            }
+            if (lane < 16 && p < pcnt) {
+                float* dst = dG1 + ((int64_t)M.i1[pmb][p] * D1 + a1) * R + qtr * 16;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    red_add_v4(dst + 4 * j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+            }
+        };
+        int pmb = -1, pcnt = 0;   // the chunk whose dA / dB products are in flight
 
         int mb = 0;
         for (int j0 = 0; j0 < ccount; j0 += MPB, mb ^= 1) {
@@ -1841,8 +1868,6 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
             build_rows(M.rows, mb, M.ucum[mb], M.u0[mb], cnt, total, s_keys, cp.ibits, n3, BT);
             if (more && tid < min(MPB, ccount - j0 - MPB)) cp_async16(&M.rec[mb ^ 1][tid], grec + cfirst + j0 + MPB + tid);
             cp_async_commit();
-            for (int q = tid; q < MB * N / 4; q += BT)
-                reinterpret_cast<float4*>(dCn)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
             fence_async_smem();
             __syncthreads();
             TT_PH(9);
@@ -1860,11 +1885,16 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
                                          umma_desc(b0 + k * 256, 128, SBO), R * N * 2, MB * R * 2,
                                          umma_idesc_bf16(128, MB), k > 0);
             }
-            if (!tc_commit_wait(&s_mbar, parity, &s_ok)) {
+            if (!tc_commit_wait(&s_mbar, parity, &s_ok)) {   // also the previous chunk's dA and dB
                 failed = true;
                 break;
             }
             tc_fence_after();
+            if (pmb >= 0) read_dA(pmb, pcnt);
+            for (int q = tid; q < MB * N / 4; q += BT)   // the previous chunk's dC tile is no longer read
+                reinterpret_cast<float4*>(dCn)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            tc_fence_before();
+            __syncthreads();
             TT_PH(10);
 
             // next chunk's metadata and A rows go in flight while this chunk's rows are processed
@@ -1919,7 +1949,7 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
 #pragma unroll
                     for (int q = 0; q < DAQ; ++q) {
                         const int k = q * (N / 16 / DAQ) + kk;
-                        tc_mma_terms<NT>(tmem + (uint32_t)(N + q * R), umma_desc(c0 + k * 256, 128, (N / 8) * 128),
+                        tc_mma_terms<NT>(tmem + (uint32_t)(TDA + q * R), umma_desc(c0 + k * 256, 128, (N / 8) * 128),
                                          umma_desc_mn(b0 + k * 2 * (R / 8) * 128, 128, (R / 8) * 128),
                                          MB * N * 2, R * N * 2, umma_idesc_bf16(MB, R, false, true), kk > 0);
                     }
@@ -1930,39 +1960,18 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
                                      umma_desc_mn(c0 + k * 2 * (N / 8) * 128, 128, (N / 8) * 128),
                                      MB * R * 2, MB * N * 2, umma_idesc_bf16(R, N, true, true), j0 > 0 || k > 0);
             }
-            if (!tc_commit_wait(&s_mbar, parity, &s_ok)) {
-                failed = true;
-                break;
-            }
-            tc_fence_after();
+            pmb = mb;
+            pcnt = cnt;
             TT_PH(13);
-            {
-                // dA rows m = 16 sub + lane (lane < 16), columns 16 qtr .. 16 qtr + 15, summed over the
-                // accumulators -> dG_1
-                const int warp = tid >> 5, lane = tid & 31, sub = warp & 3, qtr = warp >> 2;
-                const int m = 16 * sub + lane, p = m / D1, a1 = m % D1;
-                const uint32_t ta = tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)(N + qtr * 16);
-                float v[16];
-                tmem_ld16(ta, v);
-#pragma unroll 1
-                for (int q = 1; q < DAQ; ++q) {
-                    float x[16];
-                    tmem_ld16(ta + (uint32_t)(q * R), x);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] += x[i];
-                }
-                if (lane < 16 && p < cnt) {
-                    float* dst = dG1 + ((int64_t)M.i1[mb][p] * D1 + a1) * R + qtr * 16;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        red_add_v4(dst + 4 * j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
-                }
-            }
-            tc_fence_before();
-            __syncthreads();   // dCn, the dC tile and the A buffer are reused by the next chunks
-            TT_PH(14);
         }
         if (failed) break;
+        if (!tc_commit_wait(&s_mbar, parity, &s_ok)) {   // the column's last dA and dB
+            failed = true;
+            break;
+        }
+        tc_fence_after();
+        read_dA(pmb, pcnt);
+        TT_PH(14);
         {
             // dG_2[:, i_2] = dB from tensor memory: rows rho_1 = 16 sub + lane (lane < 16)
             tc_fence_after();
