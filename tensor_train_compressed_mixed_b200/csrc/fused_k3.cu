@@ -859,9 +859,13 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
                 TT_PH(3);
             }
         }
-        __threadfence();
+        // publish the chunk's rows: the barrier orders every thread's row stores before thread
+        // 0's device-scope fence (cumulative), which precedes the counter increment
         __syncthreads();
-        if (tid == 0) atomicAdd(&hdr->done[M.t[mb]], 1);
+        if (tid == 0) {
+            __threadfence();
+            atomicAdd(&hdr->done[M.t[mb]], 1);
+        }
         q = qn;
         staged = next_chunk;
         if (next_chunk) mb ^= 1;
