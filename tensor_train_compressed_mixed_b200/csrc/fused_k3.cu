@@ -906,7 +906,6 @@ __global__ void __launch_bounds__(256) k3_hzero(const int32_t* __restrict__ uid_
 template <int D>
 __global__ void __launch_bounds__(256) k3_hsum(const int32_t* __restrict__ uid_sorted,
                                                const int32_t* __restrict__ bag_sorted,
-                                               const int32_t* __restrict__ uniq_start,
                                                const float* __restrict__ grad_out, int64_t L, int64_t B,
                                                float inv_b, int T, float* __restrict__ rowbuf,
                                                const int32_t* status)
@@ -921,18 +920,27 @@ __global__ void __launch_bounds__(256) k3_hsum(const int32_t* __restrict__ uid_s
     const int64_t TD = (int64_t)T * D;
     const bool active = lane < LB;
     const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
-    int cur = uid_sorted[c0];
+    // only the segment's first and last rows can continue past its edges: those (zeroed by
+    // k3_hzero) receive vector reductions, every other row one plain store
+    const int first_u = uid_sorted[c0], last_u = uid_sorted[c1 - 1];
+    const bool cut_lo = c0 > 0 && uid_sorted[c0 - 1] == first_u;
+    const bool cut_hi = c1 < L && uid_sorted[c1] == last_u;
+    int cur = first_u;
     float4 acc = zero;
     auto flush = [&](int u, float4 a) {
         if (!active) return;
         float* dst = rowbuf + (int64_t)u * D + lane * 4;
-        if (uniq_start[u] >= c0 && uniq_start[u + 1] <= c1) *reinterpret_cast<float4*>(dst) = a;
-        else red_add_v4(dst, a);
+        if ((u == first_u && cut_lo) || (u == last_u && cut_hi)) red_add_v4(dst, a);
+        else *reinterpret_cast<float4*>(dst) = a;
     };
+    // the row and bag ids of the next 32 lookups are loaded one group ahead
+    int myu = c0 + lane < c1 ? uid_sorted[c0 + lane] : -1;
+    int myb = c0 + lane < c1 ? bag_sorted[c0 + lane] : 0;
     for (int64_t base = c0; base < c1; base += 32) {
         const int n = (int)min64(32, c1 - base);
-        const int myu = lane < n ? uid_sorted[base + lane] : -1;
-        const int myb = lane < n ? bag_sorted[base + lane] : 0;
+        const int64_t nx = base + 32 + lane;
+        const int nu = nx < c1 ? uid_sorted[nx] : -1;
+        const int nb = nx < c1 ? bag_sorted[nx] : 0;
         for (int k = 0; k < n; k += 8) {
             float4 v[8];
             int uq[8];
@@ -960,6 +968,8 @@ __global__ void __launch_bounds__(256) k3_hsum(const int32_t* __restrict__ uid_s
                 acc = f4add(acc, v[q]);
             }
         }
+        myu = nu;
+        myb = nb;
     }
     flush(cur, acc);
 }
@@ -2150,7 +2160,7 @@ cudaError_t rowsum_launch(const K3Args& a, const float* grad_out, cudaStream_t s
     const int64_t nwarps = ceil_div(L, kHChunk);
     k3_hzero<D><<<148, 256, 0, s>>>(a.uid_sorted, L, a.rowbuf, a.status);
     k3_hsum<D><<<(unsigned)ceil_div(nwarps * 32, 256), 256, 0, s>>>(
-        a.uid_sorted, a.bag_sorted, a.uniq_start, grad_out, L, a.cp->B, (float)(1.0 / (double)a.cp->B), a.cp->T,
+        a.uid_sorted, a.bag_sorted, grad_out, L, a.cp->B, (float)(1.0 / (double)a.cp->B), a.cp->T,
         a.rowbuf, a.status);
     *nl += 2;
     return cudaGetLastError();
