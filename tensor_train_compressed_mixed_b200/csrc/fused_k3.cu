@@ -903,6 +903,17 @@ __global__ void __launch_bounds__(256) k3_hzero(const int32_t* __restrict__ uid_
     }
 }
 
+// grad_out row of global bag g = t B + b (table t < 64): row b T + t, in units of D floats (B T
+// rows of D >= 64 floats fit in device memory, so the row number fits in 32 bits); the quotient
+// t comes from a float estimate corrected to the exact value
+__device__ __forceinline__ uint32_t grad_row_of_bag(int g, int64_t B, float inv_b, int T)
+{
+    int t = __float2int_rz(__int2float_rz(g) * inv_b);
+    if ((int64_t)t * B > g) --t;
+    else if ((int64_t)(t + 1) * B <= g) ++t;
+    return (uint32_t)((g - (int64_t)t * B) * T + t);
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) k3_hsum(const int32_t* __restrict__ uid_sorted,
                                                const int32_t* __restrict__ bag_sorted,
@@ -917,9 +928,9 @@ __global__ void __launch_bounds__(256) k3_hsum(const int32_t* __restrict__ uid_s
     const int64_t c0 = warp * kHChunk;
     if (c0 >= L) return;
     const int64_t c1 = min64(L, c0 + kHChunk);
-    const int64_t TD = (int64_t)T * D;
     const bool active = lane < LB;
     const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4* g4 = reinterpret_cast<const float4*>(grad_out) + (active ? lane : 0);
     // only the segment's first and last rows can continue past its edges: those (zeroed by
     // k3_hzero) receive vector reductions, every other row one plain store
     const int first_u = uid_sorted[c0], last_u = uid_sorted[c1 - 1];
@@ -933,29 +944,30 @@ __global__ void __launch_bounds__(256) k3_hsum(const int32_t* __restrict__ uid_s
         if ((u == first_u && cut_lo) || (u == last_u && cut_hi)) red_add_v4(dst, a);
         else *reinterpret_cast<float4*>(dst) = a;
     };
-    // the row and bag ids of the next 32 lookups are loaded one group ahead
-    int myu = c0 + lane < c1 ? uid_sorted[c0 + lane] : -1;
-    int myb = c0 + lane < c1 ? bag_sorted[c0 + lane] : 0;
+    // each lane owns one of the next 32 lookups: its row id and its grad_out row, computed once
+    // (lane-parallel) one group ahead of the gathers, which then broadcast them
+    int myu = -1;
+    uint32_t myr = 0;
+    if (c0 + lane < c1) {
+        myu = uid_sorted[c0 + lane];
+        myr = grad_row_of_bag(bag_sorted[c0 + lane], B, inv_b, T);
+    }
     for (int64_t base = c0; base < c1; base += 32) {
         const int n = (int)min64(32, c1 - base);
         const int64_t nx = base + 32 + lane;
-        const int nu = nx < c1 ? uid_sorted[nx] : -1;
-        const int nb = nx < c1 ? bag_sorted[nx] : 0;
+        int nu = -1, nbag = 0;
+        if (nx < c1) {
+            nu = uid_sorted[nx];
+            nbag = bag_sorted[nx];
+        }
         for (int k = 0; k < n; k += 8) {
             float4 v[8];
             int uq[8];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 uq[q] = __shfl_sync(kFull, myu, k + q);
-                const int bag = __shfl_sync(kFull, myb, k + q);
-                // table t = bag / B (t < 64): a float estimate, corrected to the exact quotient
-                int t = __float2int_rz(__int2float_rz(bag) * inv_b);
-                if ((int64_t)t * B > bag) --t;
-                else if ((int64_t)(t + 1) * B <= bag) ++t;
-                const int64_t b = bag - (int64_t)t * B;
-                v[q] = (active && k + q < n)
-                           ? __ldg(reinterpret_cast<const float4*>(grad_out + b * TD + (int64_t)t * D) + lane)
-                           : zero;
+                const uint32_t r = __shfl_sync(kFull, myr, k + q);
+                v[q] = (active && k + q < n) ? __ldg(g4 + (size_t)r * (D / 4)) : zero;
             }
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
@@ -969,7 +981,7 @@ __global__ void __launch_bounds__(256) k3_hsum(const int32_t* __restrict__ uid_s
             }
         }
         myu = nu;
-        myb = nb;
+        myr = nx < c1 ? grad_row_of_bag(nbag, B, inv_b, T) : 0u;
     }
     flush(cur, acc);
 }
