@@ -677,6 +677,9 @@ __device__ void fwd_pool(const CoreParams& cp, int ptask, int nP, const int32_t*
                          int* s_flag)
 {
     constexpr int D = S::D, LB = D / 4, BPW = 32 / LB;
+    // row gathers in flight per lane: 16 below rank 64; at rank 64 the kernel's register budget
+    // is held by the tensor-core phases and 8 is faster
+    constexpr int kPoolLoads = S::R >= 64 ? 8 : 16;
     const int t = ptask / nP, jb = ptask % nP;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     TT_PH_START();
@@ -710,16 +713,16 @@ __device__ void fwd_pool(const CoreParams& cp, int ptask, int nP, const int32_t*
         for (int64_t base = l0; base < l1; base += LB) {
             const int n = (int)min64(LB, l1 - base);
             const int myu = sl < n ? uid_at_pos[base + sl] : 0;   // row ids of up to LB lookups
-            for (int k = 0; k < n; k += 8) {
-                float4 v[8];
+            for (int k = 0; k < n; k += kPoolLoads) {
+                float4 v[kPoolLoads];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
+                for (int q = 0; q < kPoolLoads; ++q) {
                     const int u = __shfl_sync(smask, myu, (k + q) & (LB - 1), LB);
                     v[q] = (k + q < n) ? __ldcg(reinterpret_cast<const float4*>(rowbuf + (int64_t)u * D + col))
                                        : zero;
                 }
 #pragma unroll
-                for (int q = 0; q < 8; ++q)   // lookup order: the sum is the same for every schedule
+                for (int q = 0; q < kPoolLoads; ++q)   // lookup order: the sum is the same for every schedule
                     if (k + q < n) acc = f4add(acc, v[q]);
             }
         }
@@ -1925,8 +1928,9 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
 
             // next chunk's metadata and A rows go in flight while this chunk's rows are processed
             if (more) {
-                cp_async_wait_all();   // its group records
-                __syncthreads();
+                // its group records: copied by the warp-0 threads that read them in bwd2_meta, so
+                // each thread's own wait suffices
+                cp_async_wait_all();
                 bwd2_meta<K>(M.rec[mb ^ 1], j0 + MPB, ccount, mb ^ 1, uniq_keys, M, s_keys);
                 bwd2_issue_a<NS>(cp, t, mb ^ 1, M, Abt + (mb ^ 1) * NS * MB * R);
             }
