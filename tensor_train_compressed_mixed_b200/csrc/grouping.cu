@@ -96,7 +96,7 @@ cudaError_t launch_make_keys(const KeyParams& kp, bool key64, const int64_t* ind
 //            match + per-warp counters, warps in tile order), staged in
 //            shared memory by digit, then written out coalesced at
 //            digit base + tile base + rank
-// A tile is 256 threads x 8 keys; warp w owns keys [w*256, (w+1)*256) of
+// A tile is 256 threads x kSortItems keys; warp w owns keys [w*32*kSortItems, (w+1)*32*kSortItems) of
 // the tile, visited in (item, lane) order, which is input order.
 // ---------------------------------------------------------------------------
 template <typename K>

@@ -171,7 +171,7 @@ __device__ __forceinline__ T block256_exclusive_scan(T v, T* total, T* s_tmp)
 // Host-side launchers (stream-ordered, no host synchronisation).
 // ---------------------------------------------------------------------------
 
-constexpr int kSortItems = 8;
+constexpr int kSortItems = 12;
 constexpr int kSortTile = 256 * kSortItems;
 constexpr int kScanTile = 256 * 16;
 
