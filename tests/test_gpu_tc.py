@@ -190,3 +190,23 @@ def test_rank64_training_chunks_beyond_row_table(precision_name, tol):
     upd = oracle.sgd(w.cores, want, 0.01)
     for j in range(w.num_cores):
         assert core_grad_err(new[0][j], upd[0][j]) <= tol, j
+
+
+@pytest.mark.parametrize("precision_name,tol", [("TT_PREC_FP32", FP32_TOL), ("TT_PREC_FP32_SPLIT_TC", FP32_TOL),
+                                                ("TT_PREC_BF16_TC", BF16_TOL)])
+def test_rank64_training_with_64bit_keys(precision_name, tol):
+    """Three tables of 1.1e9 rows: 31 row bits + 2 table bits do not fit a 32-bit key, so
+    the sort, the segmentation and the fused kernels run their 64-bit key variants."""
+    from tensor_train_compressed_mixed_b200 import abi
+    w = random_workload(963, (4, 4, 8), (1, 64, 64, 1), [(1100, 1000, 1000)] * 3, batch=64,
+                        pooling={"kind": "uniform", "lo": 1, "hi": 8}, with_grad=True)
+    _, out, grads, new = gpu_train_step(w, options=_opts(getattr(abi, precision_name)), lr=0.01)
+    assert output_err(out, oracle.workload_forward(w), w.dim) <= tol
+    want = oracle.workload_backward(w)
+    for t in range(w.num_tables):
+        for j in range(w.num_cores):
+            assert core_grad_err(grads[t][j], want[t][j]) <= tol, (t, j)
+    upd = oracle.sgd(w.cores, want, 0.01)
+    for t in range(w.num_tables):
+        for j in range(w.num_cores):
+            assert core_grad_err(new[t][j], upd[t][j]) <= tol, (t, j)
