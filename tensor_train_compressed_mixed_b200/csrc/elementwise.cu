@@ -1,5 +1,5 @@
 // Elementwise kernels over the T*k core buffers of a handle: zero fill of the
-// gradient buffers and the SGD step G <- G - lr * dG (spec training
+// gradient buffers and the SGD step G <- G - lr * dG (the benchmark's training
 // step; the FlowTT pages leave the optimiser open, plain SGD is the reading).
 // One launch covers every buffer: block x finds its buffer by binary search
 // over the per-buffer chunk prefix sums and handles one 8192-float chunk,
