@@ -380,7 +380,8 @@ def run_ours(args):
                 "frac": achieved / peak, "traffic": kernel_traffic(dom, args.precision, w.name),
                 "peak_source": f"work-weighted: {f_tc / 1e9:.1f} GFLOP of prefix-level products as {products} "
                                f"bf16 tensor-core product(s) each at the measured bf16 peak "
-                               f"{BF16_PEAK_TFLOPS:.0f} TF/s, {f_rest / 1e9:.1f} GFLOP at the derived FP32 peak "
+                               f"{BF16_PEAK_TFLOPS:.0f} TF/s (burst figure: the step runs at the maximum SM clock, "
+                               f"see clocks), {f_rest / 1e9:.1f} GFLOP at the derived FP32 peak "
                                f"{FP32_PEAK_TFLOPS:.1f} TF/s"}
     elif dom in flops:
         achieved = flops[dom] / (per_step[dom] / 1e3) / 1e12
