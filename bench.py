@@ -23,6 +23,7 @@ import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 import numpy as np
@@ -31,8 +32,50 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "pooled TT lookups/sec fwd and fwd+bwd at batch 32768; % of roofline"
-FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # FFMA lanes x 2 flops x max SM clock
-BF16_PEAK_TFLOPS = 1644.9   # cuBLAS bf16 GEMM, burst, measured on this B200 pool (MEASURED_PEAKS.json)
+# FP32 FFMA peak, derived from the unit counts and the maximum SM clock (148 SMs x 128 FP32
+# lanes x 2 flops x 1.965 GHz): the kernels are bound by plain FP32 arithmetic, for which no
+# measured peak is recorded.
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+# used only when MEASURED_PEAKS.json (written per machine next to this file) is absent
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def _find_number(obj, names):
+    """First numeric value stored under one of `names` anywhere in a nested JSON object."""
+    if isinstance(obj, dict):
+        for n in names:
+            v = obj.get(n)
+            if isinstance(v, (int, float)) and not isinstance(v, bool):
+                return float(v)
+        for v in obj.values():
+            x = _find_number(v, names)
+            if x is not None:
+                return x
+    elif isinstance(obj, list):
+        for v in obj:
+            x = _find_number(v, names)
+            if x is not None:
+                return x
+    return None
+
+
+def measured_peaks():
+    """HBM copy bandwidth (GB/s) and dense bf16 GEMM throughput (TF/s, burst) of this machine's
+    B200, from MEASURED_PEAKS.json when present; otherwise the fallback figures."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    data = None
+    if os.path.exists(path):
+        try:
+            data = json.load(open(path))
+        except (OSError, ValueError):
+            data = None
+    hbm = _find_number(data, ("hbm_gbs",)) if data is not None else None
+    bf16 = _find_number(data, ("bf16_tflops",)) if data is not None else None
+    return {"hbm_gbs": hbm if hbm else FALLBACK_HBM_GBS,
+            "hbm_source": "of measured (MEASURED_PEAKS.json hbm_gbs)" if hbm else "of fallback",
+            "bf16_tflops": bf16 if bf16 else FALLBACK_BF16_TFLOPS,
+            "bf16_source": "of measured (MEASURED_PEAKS.json bf16_tflops, burst)" if bf16 else "of fallback"}
 
 
 def parse_args():
@@ -54,6 +97,8 @@ def parse_args():
                         "tensor cores; auto = split where the shape has tensor-core kernels, else fp32")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extra-fwd", action="store_true",
+                   help="skip the forward of the 26-table rank-32 workload that the default run adds")
     p.add_argument("--cpu-seconds", type=float, default=15.0,
                    help="target CPU time of the oracle sample")
     return p.parse_args()
@@ -112,28 +157,81 @@ def algorithmic(w, U, G):
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock and throttle reasons sampled during the timed region.
+
+    NVML is polled from a thread every 10 ms (the timed region of a default run lasts well
+    under a second, too short for nvidia-smi's 200 ms period); nvidia-smi is the fallback."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
     def __init__(self, device_index: int):
         self.idx = device_index
         self.proc = None
         self.path = None
+        self.thread = None
+        self.samples = []
+        self.stop_flag = threading.Event()
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            p = torch.cuda.get_device_properties(self.idx)
+            bus = "%08x:%02x:%02x.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.idx)
+
+    def _poll(self, nv, h):
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.stop_flag.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), smax, int(get_reasons(h))))
+            except Exception:
+                break
+            time.sleep(0.01)
 
     def start(self):
+        try:
+            nv, h = self._nvml_handle()
+            self.thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self.thread.start()
+            self.source = "nvml, 10 ms"
+            time.sleep(0.05)
+            return
+        except Exception:
+            self.thread = None
         fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
         os.close(fd)
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi, 50 ms"
         except OSError:
             self.proc = None
         time.sleep(0.3)
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=5)
+            rows = self.samples
+            if not rows:
+                return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
+            reasons = sorted({name for _, _, bits in rows for b, name in self.REASONS.items() if bits & b})
+            return {"sm_mhz": statistics.median(float(r[0]) for r in rows),
+                    "sm_max_mhz": float(max(r[1] for r in rows)), "reasons": reasons,
+                    "samples": len(rows), "source": self.source}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -149,30 +247,37 @@ class ClockSampler:
                     rows.append(parts)
         os.unlink(self.path)
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
         sm = [float(x[0]) for x in rows if x[0].replace(".", "").isdigit()]
         mx = [float(x[1]) for x in rows if x[1].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for x in rows for i in range(4) if x[4 + i] == "Active"})
         return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows),
+                "source": self.source}
 
 
 # ---------------------------------------------------------------------------
 # distributed plumbing
 # ---------------------------------------------------------------------------
-def dist_init(n):
+def dist_init(n, backend=None):
+    """Joins the process group of a torchrun launch (NCCL on GPUs; gloo when torch has no
+    CUDA device, which the CPU tests use).  Returns (world, rank, local rank)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    cuda = torch.cuda.is_available()
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
-    elif torch.cuda.is_available():
+        backend = backend or ("nccl" if cuda else "gloo")
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300), **kw)
+    elif cuda:
         torch.cuda.set_device(0)
     return world, rank, local
 
@@ -188,14 +293,26 @@ def max_over_ranks(world, x):
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def kernel_traffic(name, precision, workload):
-    """Per-launch DRAM bytes from a committed ncu summary, if it was taken on the same kernel
-    variant (precision mode), the same workload and the current source."""
+def dist_teardown(world):
+    """Last collective step of every rank: a barrier, then the process group is destroyed once."""
+    if world > 1:
+        import torch.distributed as dist
+        if dist.is_initialized():
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+def kernel_traffic(name, precision, config, lookups):
+    """Per-launch DRAM bytes of a fused kernel from a committed single-kernel ncu capture
+    (profiles/ncu_traffic.json), taken on a smaller batch of the same workload and the same
+    kernel variant (precision mode) with the current kernel source, scaled to this launch by
+    the number of lookups it processes; None when no such capture exists."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
@@ -203,13 +320,15 @@ def kernel_traffic(name, precision, workload):
         rec = json.load(open(path)).get(name)
     except (OSError, ValueError):
         return None
-    if not rec or rec.get("precision", "fp32") != precision or rec.get("workload_name") != workload:
+    if not rec or rec.get("precision", "fp32") != precision or rec.get("config") != config:
         return None
     src = os.path.join(ROOT, "tensor_train_compressed_mixed_b200", "csrc", rec["source"])
     if not os.path.exists(src):
         return None
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return rec["dram_bytes_per_launch"] if sha == rec.get("source_sha") else None
+    if sha != rec.get("source_sha") or not rec.get("lookups"):
+        return None
+    return rec["dram_bytes_per_launch"] * lookups / rec["lookups"]
 
 
 # ---------------------------------------------------------------------------
@@ -278,6 +397,91 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 
 
+def kernel_roofline(kernel, ms, alg, precision, w, peaks, config):
+    """Roofline record of one fused kernel from its per-launch device time `ms`.
+
+    The fused kernels are bound by arithmetic.  Where part of a kernel's algorithmic work
+    runs on the tensor cores (the prefix-level products in the bf16 and split modes), the
+    peak is the work-weighted combination of the two pipes: ideal time = F_tc x products /
+    P_bf16 + F_fp32 / P_fp32, three tensor-core products per algorithmic one in split mode."""
+    flops = {"fwd_fused": alg["f_fwd"], "bwd_fused": alg["f_bwd_kernel"]}
+    tc_work = {}
+    if precision in ("bf16", "split"):
+        tc_work["fwd_fused"] = alg["f_fwd_prefix"]
+        if len(w.d) == 3 and w.r[1] == 64:
+            tc_work["bwd_fused"] = 2.0 * alg["f_fwd_prefix"]
+    traffic = kernel_traffic(kernel, precision, config, w.num_lookups)
+    p_bf16 = peaks["bf16_tflops"]
+    if kernel in tc_work:
+        f_all = flops[kernel]
+        f_tc = tc_work[kernel]
+        f_rest = f_all - f_tc
+        products = 3 if precision == "split" else 1
+        t_ideal = products * f_tc / (p_bf16 * 1e12) + f_rest / (FP32_PEAK_TFLOPS * 1e12)
+        peak = f_all / t_ideal / 1e12
+        achieved = f_all / (ms / 1e3) / 1e12
+        return {"bound": "alu", "kernel": kernel, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "peak_source": f"work-weighted: {f_tc / 1e9:.1f} GFLOP of prefix-level products as {products} "
+                               f"bf16 tensor-core product(s) each at the bf16 peak {p_bf16:.0f} TF/s "
+                               f"{peaks['bf16_source']}, {f_rest / 1e9:.1f} GFLOP at the FP32 peak "
+                               f"{FP32_PEAK_TFLOPS:.1f} TF/s derived from 148 SM x 128 lanes x 2 x 1.965 GHz"}
+    if kernel in flops:
+        achieved = flops[kernel] / (ms / 1e3) / 1e12
+        return {"bound": "alu", "kernel": kernel, "achieved": achieved, "peak": FP32_PEAK_TFLOPS,
+                "unit": "TFLOP/s", "frac": achieved / FP32_PEAK_TFLOPS, "traffic": traffic,
+                "peak_source": "derived: 148 SM x 128 FP32 lanes x 2 x 1.965 GHz"}
+    byts = {"bwd_rowsum": alg["b_rowsum"], "sgd": alg["b_train"] - alg["b_fwd"]}.get(kernel)
+    ach = byts / (ms / 1e3) / 1e9 if byts else None
+    hbm = peaks["hbm_gbs"]
+    return {"bound": "hbm", "kernel": kernel, "achieved": ach, "peak": hbm, "unit": "GB/s",
+            "frac": ach / hbm if ach else None, "traffic": traffic,
+            "peak_source": f"HBM copy bandwidth {peaks['hbm_source']}"}
+
+
+def time_rank32_forward(args, world, rank, dev, peaks, barrier_fn, max_fn):
+    """Forward pass of the 26-table, rank-32, batch-32768 workload on its own handle, timed
+    like the main step (CUDA events, max over ranks), with the fused kernel's roofline."""
+    import torch
+    from tensor_train_compressed_mixed_b200 import abi, from_workload
+    from workloads import config_workload
+    w3 = config_workload(3, with_grad=False, shard=rank)
+    opts = abi.tt_emb_default_options()
+    opts.precision = abi.TT_PREC_FP32_SPLIT_TC
+    emb3, cores3, idx3, off3 = from_workload(w3, device=dev, options=opts, with_grads=False)
+    out3 = torch.empty(w3.batch, w3.num_tables * w3.dim, dtype=torch.float32, device=dev)
+    emb3.reserve(w3.num_lookups, w3.batch)
+    for _ in range(args.warmup):
+        emb3.forward(idx3, off3, w3.batch, out3)
+    emb3.sync()
+    seg = emb3.segmentation()
+    alg3 = algorithmic(w3, seg["num_unique"], seg["num_groups"])
+    abi.tt_emb_enable_timing(emb3.handle, True)
+    barrier_fn(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        emb3.forward(idx3, off3, w3.batch, out3)
+    e1.record()
+    torch.cuda.synchronize()
+    emb3.sync()
+    barrier_fn(world)
+    ms = max_fn(world, e0.elapsed_time(e1)) / args.steps
+    ph, _ = abi.tt_emb_phase_times(emb3.handle)
+    abi.tt_emb_enable_timing(emb3.handle, False)
+    fused_ms = ph["fwd_fused"] / args.steps
+    t_roof = max(alg3["f_fwd"] / (FP32_PEAK_TFLOPS * 1e12), alg3["b_fwd"] / (peaks["hbm_gbs"] * 1e9))
+    rec = {"workload": w3.name, "precision": "split", "lookups": w3.num_lookups,
+           "value": world * w3.num_lookups / (ms / 1e3), "unit": "lookups/s", "ms": ms,
+           "roofline_frac": t_roof / (ms / 1e3), "phases_ms": {k: v / args.steps for k, v in ph.items() if v},
+           "fused_roofline": kernel_roofline("fwd_fused", fused_ms, alg3, "split", w3, peaks, 3)}
+    emb3.close()
+    del cores3, idx3, off3, out3
+    torch.cuda.empty_cache()
+    return rec
+
+
 def run_ours(args):
     import torch
     from tensor_train_compressed_mixed_b200 import abi, dp, from_workload
@@ -285,6 +489,7 @@ def run_ours(args):
 
     world, rank, local = dist_init(args.gpus)
     dev = torch.device("cuda", local)
+    peaks = measured_peaks()
     # every rank draws its own batch of the same workload (rank 0's is the single-GPU one)
     w = config_workload(args.config, batch=args.batch, tables=args.tables, with_grad=True, shard=rank)
     if args.precision == "auto":
@@ -306,6 +511,7 @@ def run_ours(args):
     L, B, T, D = w.num_lookups, w.batch, w.num_tables, w.dim
     out = torch.empty(B, T * D, dtype=torch.float32, device=dev)
     emb.reserve(L, B)
+    ws_bytes = abi.tt_emb_workspace_size(emb.handle, L, B)
 
     sgd = args.config == 4
     fused_sgd = sgd and not dp_train   # data parallel: the gradients are exchanged before SGD
@@ -358,45 +564,10 @@ def run_ours(args):
     # --- dominant kernel roofline (device times from the timed region) ---
     per_step = {k: v / args.steps for k, v in ph.items()}
     dom = max(per_step, key=per_step.get)
-    flops = {"fwd_fused": alg["f_fwd"], "bwd_fused": alg["f_bwd_kernel"]}
-    # tensor-core share of each fused kernel's algorithmic work in bf16 mode: the forward's
-    # prefix step; at rank 64 also the backward's two prefix-level gradient products
-    tc_work = {}
-    if args.precision in ("bf16", "split"):
-        tc_work["fwd_fused"] = alg["f_fwd_prefix"]
-        if len(w.d) == 3 and w.r[1] == 64:
-            tc_work["bwd_fused"] = 2.0 * alg["f_fwd_prefix"]
-    if dom in tc_work:
-        # tensor-core work and FP32 work: the peak is their work-weighted combination
-        # (ideal time = F_tc / P_tc + F_fp32 / P_fp32)
-        f_all = flops[dom]
-        f_tc = tc_work[dom]
-        f_rest = f_all - f_tc
-        products = 3 if args.precision == "split" else 1   # tensor-core products per algorithmic one
-        t_ideal = products * f_tc / (BF16_PEAK_TFLOPS * 1e12) + f_rest / (FP32_PEAK_TFLOPS * 1e12)
-        peak = f_all / t_ideal / 1e12
-        achieved = f_all / (per_step[dom] / 1e3) / 1e12
-        roof = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": kernel_traffic(dom, args.precision, w.name),
-                "peak_source": f"work-weighted: {f_tc / 1e9:.1f} GFLOP of prefix-level products as {products} "
-                               f"bf16 tensor-core product(s) each at the measured bf16 peak "
-                               f"{BF16_PEAK_TFLOPS:.0f} TF/s (burst figure: the step runs at the maximum SM clock, "
-                               f"see clocks), {f_rest / 1e9:.1f} GFLOP at the derived FP32 peak "
-                               f"{FP32_PEAK_TFLOPS:.1f} TF/s"}
-    elif dom in flops:
-        achieved = flops[dom] / (per_step[dom] / 1e3) / 1e12
-        roof = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": FP32_PEAK_TFLOPS,
-                "unit": "TFLOP/s", "frac": achieved / FP32_PEAK_TFLOPS,
-                "traffic": kernel_traffic(dom, args.precision, w.name), "peak_source": "derived: 148 SM x 128 FP32 lanes x 2 x 1.965 GHz"}
-    else:
-        byts = {"bwd_rowsum": alg["b_rowsum"], "sgd": alg["b_train"] - alg["b_fwd"]}.get(dom)
-        ach = byts / (per_step[dom] / 1e3) / 1e9 if byts else None
-        roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": 6550.4, "unit": "GB/s",
-                "frac": ach / 6550.4 if ach else None, "traffic": kernel_traffic(dom, args.precision, w.name),
-                "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)"}
+    roof = kernel_roofline(dom, per_step[dom], alg, args.precision, w, peaks, args.config)
     t_roof_step = max((alg["f_fwd"] + (alg["f_bwd"] if train else 0)) / (FP32_PEAK_TFLOPS * 1e12),
-                      (alg["b_train"] if train else alg["b_fwd"]) / 6550.4e9)
-    t_roof_fwd = max(alg["f_fwd"] / (FP32_PEAK_TFLOPS * 1e12), alg["b_fwd"] / 6550.4e9)
+                      (alg["b_train"] if train else alg["b_fwd"]) / (peaks["hbm_gbs"] * 1e9))
+    t_roof_fwd = max(alg["f_fwd"] / (FP32_PEAK_TFLOPS * 1e12), alg["b_fwd"] / (peaks["hbm_gbs"] * 1e9))
 
     # --- end to end through the public API with host buffers ---
     # Every step copies its inputs from pinned host memory and reads its pooled output
@@ -474,6 +645,17 @@ def run_ours(args):
                "d2h_bytes_per_step": 4 * B * T * D, "ms_per_step": ms_e2e,
                "copies": "pinned host buffers, double-buffered on two copy streams, overlapped with compute"}
 
+    # --- forward of the 26-table rank-32 workload (the forward-only configuration) ---
+    extra = None
+    if args.config == 4 and args.batch is None and args.tables is None and not args.no_extra_fwd:
+        extra = time_rank32_forward(args, world, rank, dev, peaks, barrier, max_over_ranks)
+
+    mem = {"workspace_bytes": ws_bytes,
+           "core_bytes": int(sum(c.numel() for tab in cores for c in tab) * 4),
+           "peak_allocated_bytes": int(torch.cuda.max_memory_allocated(dev)),
+           "note": "workspace sized by tt_emb_workspace_size for this batch; peak over the whole run, "
+                   "inputs, outputs, cores and gradients included"}
+
     # --- CPU oracle on a bounded sample (rank 0, one GPU only) ---
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -515,16 +697,16 @@ def run_ours(args):
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clk,
+            "memory": mem,
+            "peaks": {"hbm_gbs": peaks["hbm_gbs"], "hbm": peaks["hbm_source"],
+                      "bf16_tflops": peaks["bf16_tflops"], "bf16": peaks["bf16_source"],
+                      "fp32_tflops": FP32_PEAK_TFLOPS, "fp32": "derived from unit counts and the maximum SM clock"},
         }
+        if extra is not None:
+            line["fwd_rank32"] = extra
         print(json.dumps(line), flush=True)
     emb.close()
-    if world > 1:
-        import torch.distributed as dist
-        barrier(world)
-        dist.destroy_process_group()
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    dist_teardown(world)
     return 0
 
 
