@@ -116,12 +116,16 @@ typedef struct {
     int32_t reserved[10];    /* must be zero */
 } tt_emb_options;
 
-/* Fills *opt with the defaults. */
+/* Fills *opt with the defaults (scheduler STEAL_L2, prefix grouping, fp32 pipes).  The
+ * options select among the pages' design points: FlowTT section 3.4 (scheduling), section 4
+ * "Prefix-Based Reuse over Exact Deduplication" (grouping). */
 void tt_emb_default_options(tt_emb_options* opt);
 
 /*
  * Creates a handle for T tables sharing k, d and r (host call, no device work
- * besides allocating the 256-byte device status block).
+ * besides allocating the 256-byte device status block).  The table is the TT
+ * format of FlowTT section 2.4 "Problem Definition" (cores [r_{j-1}][n_j][d_j][r_j],
+ * r_0 = r_k = 1) and of the TT-Rec abstract (TT-EmbeddingBag).
  *   num_tables   T, 1..TT_EMB_MAX_TABLES
  *   num_cores    k, 1..TT_EMB_MAX_CORES
  *   n_factors    host int64 [T][k]: n_j of each table, each >= 1; the product of
@@ -139,7 +143,7 @@ int tt_emb_create(int32_t num_tables, int32_t num_cores, const int64_t* n_factor
 
 /*
  * Registers the cores (and optionally the gradient buffers) by borrowing
- * device pointers.  Host arrays of T*k device pointers, table-major
+ * device pointers (FlowTT section 2.4: the TT cores G_j that replace the table).  Host arrays of T*k device pointers, table-major
  * (entry t*k + j is core j of table t, float32 [r_{j-1}][n_j][d_j][r_j],
  * 16-byte aligned).  core_grads may be NULL for inference; when given, each
  * buffer has the shape of its core and is overwritten by tt_emb_backward.
@@ -150,21 +154,30 @@ int tt_emb_set_cores(tt_emb_t h, float* const* cores, float* const* core_grads);
 
 /*
  * Device workspace needed for batches of at most max_lookups lookups and
- * batch bags per table (host call).  *bytes receives the size.
+ * batch bags per table (host call).  *bytes receives the size.  It holds the
+ * grouping of FlowTT section 3.3 (sort buffers, distinct rows, prefix groups) and
+ * the plan of section 3.4, plus the row checkpoint of the fused kernels; FlowTT
+ * section 5 reports peak memory, which this figure bounds for the library's part.
+ * Returns TT_OK or TT_ERR_ARG (null handle or pointer, negative sizes,
+ * max_lookups >= 2^31 - 1).
  */
 int tt_emb_workspace_size(tt_emb_t h, int64_t max_lookups, int64_t batch, size_t* bytes);
 
 /*
  * Registers caller-owned device workspace (256-byte aligned) of `bytes` bytes,
  * sized for (max_lookups, batch) by tt_emb_workspace_size.  The workspace
- * holds the segmentation between a forward and its backward; it must not be
- * shared by two handles that run at the same time.
+ * holds the segmentation between a forward and its backward (FlowTT section 3.2:
+ * the backward reverses the forward's flow); it must not be shared by two
+ * handles that run at the same time.  Returns TT_OK, TT_ERR_ARG (null or
+ * misaligned pointer, bad sizes) or TT_ERR_WORKSPACE (bytes below the size asked).
  */
 int tt_emb_set_workspace(tt_emb_t h, void* workspace, size_t bytes, int64_t max_lookups,
                          int64_t batch);
 
 /*
- * Forward pass: out[b][t*D + c] = sum over bag (t, b) of row_t(i)[c] (float32,
+ * Forward pass (FlowTT section 3.3 grouping, section 3.2 fused execution "C = A.B,
+ * then E = C.D, followed by pooling", section 3.4 persistent scheduling):
+ * out[b][t*D + c] = sum over bag (t, b) of row_t(i)[c] (float32,
  * fp32 accumulation).  Enqueues on `stream`: index validation, digit/key
  * extraction, radix sort, unique + prefix run-length grouping, and the fused
  * gather + pooling kernel.
@@ -173,13 +186,17 @@ int tt_emb_set_workspace(tt_emb_t h, void* workspace, size_t bytes, int64_t max_
  *             offsets[T*batch] = num_lookups
  *   out       device float32 [batch][T*D], overwritten (empty bags give 0)
  * num_lookups and batch must not exceed the workspace's sizes.  The
- * segmentation is kept in the workspace for tt_emb_backward.
+ * segmentation is kept in the workspace for tt_emb_backward.  Host errors:
+ * TT_ERR_ARG, TT_ERR_STATE (no cores), TT_ERR_WORKSPACE, TT_ERR_CUDA (a launch
+ * failed); device errors (TT_ERR_INDEX_RANGE, TT_ERR_OFFSETS, TT_ERR_TIMEOUT)
+ * surface at tt_emb_sync.
  */
 int tt_emb_forward(tt_emb_t h, const int64_t* indices, const int64_t* offsets,
                    int64_t num_lookups, int64_t batch, float* out, tt_stream_t stream);
 
 /*
- * Backward pass of the last forward on this handle: overwrites the registered
+ * Backward pass of the last forward on this handle (FlowTT section 3.2: "the
+ * backward path reverses this structure"): overwrites the registered
  * core_grads with dL/dG_j for L = sum <grad_out, out> (zero for slices no
  * lookup touched).  grad_out: device float32 [batch][T*D] of the last forward's
  * batch.  Reuses the forward's segmentation (no re-sort).  Returns
@@ -187,7 +204,10 @@ int tt_emb_forward(tt_emb_t h, const int64_t* indices, const int64_t* offsets,
  */
 int tt_emb_backward(tt_emb_t h, const float* grad_out, tt_stream_t stream);
 
-/* SGD step on every registered core: G <- G - lr * dG (float32, elementwise). */
+/* SGD step on every registered core: G <- G - lr * dG (float32, elementwise).  The
+ * training step the pages time (FlowTT section 4, training latency) ends with an
+ * optimiser step; the pages name none, so this is plain SGD without momentum.
+ * Returns TT_OK, TT_ERR_ARG, TT_ERR_STATE (cores or gradients missing) or TT_ERR_CUDA. */
 int tt_emb_sgd_update(tt_emb_t h, float lr, tt_stream_t stream);
 
 /*
@@ -206,9 +226,10 @@ int tt_emb_sgd_update(tt_emb_t h, float lr, tt_stream_t stream);
 int tt_emb_backward_sgd(tt_emb_t h, const float* grad_out, float lr, tt_stream_t stream);
 
 /*
- * Test and inspection hook: device views of the last forward's segmentation,
- * valid until the next forward on the handle.  Synchronises the stream of the
- * last call to read the counts.
+ * Test and inspection hook: device views of the last forward's segmentation
+ * (FlowTT section 3.3: sorted indices, unique extraction, prefix run-length
+ * groups), valid until the next forward on the handle.  Synchronises the stream
+ * of the last call to read the counts.  TT_ERR_STATE without a forward.
  */
 typedef struct {
     int64_t num_lookups;        /* L */
@@ -237,11 +258,23 @@ int tt_emb_copy_segmentation(tt_emb_t h, void* sorted_keys, int32_t* perm, void*
 /*
  * Waits for the handle's work on the stream of its last call and returns the
  * first device-side error recorded since the last tt_emb_sync (then clears it),
- * or TT_ERR_CUDA if the stream itself failed.
+ * or TT_ERR_CUDA if the stream itself failed.  The device errors are the input
+ * checks of the grouping step (FlowTT section 3.3) and the bounded waits of the
+ * persistent scheduler (section 3.4).
  */
 int tt_emb_sync(tt_emb_t h);
 
-/* Message for a status code (static storage). */
+/*
+ * The most recent failure on this handle, then cleared: the code of the last
+ * call on it that returned an error (host-detected), or of a device error that
+ * tt_emb_sync reported, whichever came last; TT_OK when nothing failed since the
+ * handle was created or since the previous tt_emb_last_error.  Host call; it
+ * never waits for the device (use tt_emb_sync for that).  A null handle gives
+ * TT_ERR_ARG.
+ */
+int tt_emb_last_error(tt_emb_t h);
+
+/* Message for a status code (static storage, never null). */
 const char* tt_emb_error_string(int code);
 
 /* Destroys the handle (host + its status block).  NULL is ignored. */
@@ -272,9 +305,14 @@ int tt_emb_enable_timing(tt_emb_t h, int enable);
 int tt_emb_phase_times(tt_emb_t h, double* ms, int64_t* launches);
 
 /*
- * tt_emb_forward_noalloc -- the forward pass (same contract and result as
- * tt_emb_forward) for callers that cannot allocate device memory.  The paper
+ * tt_emb_forward_noalloc -- the forward pass (same arguments and output contract
+ * as tt_emb_forward) for callers that cannot allocate device memory.  The paper
  * has no counterpart; this is a deployment variant of this library.
+ *
+ * Arithmetic: it always runs the shape-generic FP32 kernels, whatever the
+ * handle's precision option, so its output matches tt_emb_forward within the
+ * parity tolerance (1e-4 normwise per pooled row), not bit for bit; on a handle
+ * in TT_PREC_BF16_TC mode it is the more exact of the two.
  *
  * Who needs it: hosts that give an embedded library neither an allocator nor
  * a workspace (plugin interfaces with fixed buffers), processes that forbid
@@ -291,8 +329,15 @@ int tt_emb_phase_times(tt_emb_t h, double* ms, int64_t* launches);
  *   - num_lookups above TT_EMB_NOALLOC_MAX_LOOKUPS (262144) is rejected with
  *     TT_ERR_WORKSPACE before any work is enqueued.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and keeps it; make that
- *     first call before any stream capture.
+ *     (cudaGetSymbolAddress, with that device current) and keeps it.  With
+ *     CUDA's lazy module loading (the default since CUDA 12.2) that lookup is
+ *     also what loads the library's module holding the array, which reserves its
+ *     16 MiB on that device at that moment and can fail if the device is full.
+ *     So make the first call at start-up, before serving and before any stream
+ *     capture; a call with num_lookups = 0 does the set-up (it only zero-fills
+ *     `out`).
+ *   - The handle's device (the one current at tt_emb_create) must be current;
+ *     otherwise the call returns TT_ERR_STATE before enqueuing anything.
  *   - Every call, on every handle and stream, shares the one array, which keeps
  *     the previous call's contents (the call clears what must start at zero).
  *     Calls that overlap on the GPU race: order them (one stream, or events).
@@ -304,6 +349,35 @@ int tt_emb_phase_times(tt_emb_t h, double* ms, int64_t* launches);
 
 int tt_emb_forward_noalloc(tt_emb_t h, const int64_t* indices, const int64_t* offsets,
                            int64_t num_lookups, int64_t batch, float* out, tt_stream_t stream);
+
+/*
+ * Test hook for failure detection (no GPU fault is involved).  Arms one
+ * injected failure of a bounded device wait; it is consumed by the next call
+ * that runs the wait:
+ *   TT_INJECT_POOL_WAIT      next tt_emb_forward on the shape-specialised path:
+ *                            every pooling task waits for one more finished
+ *                            chunk of its table than there is, polling at most
+ *                            `spin_limit` times (0 = the library's default)
+ *                            before it records TT_ERR_TIMEOUT and returns.
+ *   TT_INJECT_MMA_WAIT_FWD   next tt_emb_forward in a tensor-core precision: the
+ *   TT_INJECT_MMA_WAIT_BWD   (or next backward's) first tensor-core completion
+ *                            wait reports that it ran out once the products have
+ *                            completed, so the kernel takes its timeout exit
+ *                            (copies drained, tensor memory freed) and records
+ *                            TT_ERR_TIMEOUT.
+ *   TT_INJECT_NONE           disarms.
+ * The error surfaces at tt_emb_sync like any device error; the handle is then
+ * usable again.  Returns TT_OK, TT_ERR_ARG or TT_ERR_UNSUPPORTED (the handle has
+ * no such wait: generic kernels, or no tensor-core precision).
+ */
+typedef enum {
+    TT_INJECT_NONE = 0,
+    TT_INJECT_POOL_WAIT = 1,
+    TT_INJECT_MMA_WAIT_FWD = 2,
+    TT_INJECT_MMA_WAIT_BWD = 3
+} tt_inject;
+
+int tt_emb_debug_inject(tt_emb_t h, int32_t what, int32_t spin_limit);
 
 /* ABI version of the loaded library (TT_EMB_ABI_VERSION). */
 int tt_emb_abi_version(void);

@@ -22,6 +22,7 @@ TT_ERR_WORKSPACE, TT_ERR_STATE, TT_ERR_CUDA, TT_ERR_TIMEOUT, TT_ERR_UNSUPPORTED 
 TT_SCHED_STATIC, TT_SCHED_STEAL, TT_SCHED_STEAL_L2 = 0, 1, 2
 TT_GROUP_PREFIX, TT_GROUP_UNIQUE_ONLY = 0, 1
 TT_PREC_FP32, TT_PREC_BF16_TC, TT_PREC_FP32_SPLIT_TC = 0, 1, 2
+TT_INJECT_NONE, TT_INJECT_POOL_WAIT, TT_INJECT_MMA_WAIT_FWD, TT_INJECT_MMA_WAIT_BWD = 0, 1, 2, 3
 MAX_TABLES, MAX_CORES = 64, 4
 
 
@@ -74,6 +75,8 @@ _SIGS = {
                             ctypes.POINTER(ctypes.c_int64)], ctypes.c_int),
     "tt_emb_forward_noalloc": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                 ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
+    "tt_emb_last_error": ([ctypes.c_void_p], ctypes.c_int),
+    "tt_emb_debug_inject": ([ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32], ctypes.c_int),
     "tt_emb_destroy": ([ctypes.c_void_p], None),
 }
 
@@ -256,6 +259,16 @@ def tt_emb_phase_times(h):
     n = ctypes.c_int64()
     _check(lib().tt_emb_phase_times(h, ms, ctypes.byref(n)), "tt_emb_phase_times")
     return dict(zip(PHASES, list(ms))), int(n.value)
+
+
+def tt_emb_last_error(h) -> int:
+    """The most recent failure recorded on the handle (a status code), then cleared."""
+    return int(lib().tt_emb_last_error(h))
+
+
+def tt_emb_debug_inject(h, what: int, spin_limit: int = 0):
+    """Test hook: arms one injected failure of a bounded device wait (TT_INJECT_*)."""
+    _check(lib().tt_emb_debug_inject(h, int(what), int(spin_limit)), "tt_emb_debug_inject")
 
 
 def tt_emb_destroy(h):

@@ -136,6 +136,8 @@ struct tt_emb_handle {
     bool timing = false;
     double phase_ms[TT_EMB_NUM_PHASES] = {};
     int64_t launches = 0;
+    int last_error = TT_OK;           // tt_emb_last_error
+    int inject = TT_INJECT_NONE, inject_spin = 0;   // tt_emb_debug_inject, armed until consumed
     struct Interval { int phase; cudaEvent_t a, b; };
     std::vector<Interval> pending;
     std::vector<cudaEvent_t> pool;
@@ -375,6 +377,20 @@ struct tt_emb_handle {
 
 static int cuda_status(cudaError_t e) { return e == cudaSuccess ? TT_OK : TT_ERR_CUDA; }
 
+// records a failed call on the handle for tt_emb_last_error
+static int note(tt_emb_t h, int rc)
+{
+    if (h && rc != TT_OK) h->last_error = rc;
+    return rc;
+}
+
+namespace tt {
+// device the handle was created on (tt_emb_forward_noalloc checks it is current)
+int handle_device(tt_emb_t h) { return h ? h->device : -1; }
+// records a failed call of an entry point defined in another file
+int record_error(tt_emb_t h, int rc) { return note(h, rc); }
+}  // namespace tt
+
 extern "C" {
 
 int tt_emb_abi_version(void) { return TT_EMB_ABI_VERSION; }
@@ -550,7 +566,7 @@ int tt_emb_create(int32_t num_tables, int32_t num_cores, const int64_t* n_factor
     return TT_OK;
 }
 
-int tt_emb_set_cores(tt_emb_t h, float* const* cores, float* const* core_grads)
+static int tt_emb_set_cores_impl(tt_emb_t h, float* const* cores, float* const* core_grads)
 {
     if (!h || !cores) return TT_ERR_ARG;
     const int n = h->T * h->k;
@@ -567,7 +583,7 @@ int tt_emb_set_cores(tt_emb_t h, float* const* cores, float* const* core_grads)
     return TT_OK;
 }
 
-int tt_emb_workspace_size(tt_emb_t h, int64_t max_lookups, int64_t batch, size_t* bytes)
+static int tt_emb_workspace_size_impl(tt_emb_t h, int64_t max_lookups, int64_t batch, size_t* bytes)
 {
     if (!h || !bytes || max_lookups < 0 || batch < 1) return TT_ERR_ARG;
     if (max_lookups >= (int64_t)INT32_MAX) return TT_ERR_ARG;
@@ -575,7 +591,7 @@ int tt_emb_workspace_size(tt_emb_t h, int64_t max_lookups, int64_t batch, size_t
     return TT_OK;
 }
 
-int tt_emb_set_workspace(tt_emb_t h, void* workspace, size_t bytes, int64_t max_lookups,
+static int tt_emb_set_workspace_impl(tt_emb_t h, void* workspace, size_t bytes, int64_t max_lookups,
                          int64_t batch)
 {
     if (!h || !workspace || max_lookups < 0 || batch < 1) return TT_ERR_ARG;
@@ -592,7 +608,7 @@ int tt_emb_set_workspace(tt_emb_t h, void* workspace, size_t bytes, int64_t max_
     return TT_OK;
 }
 
-int tt_emb_forward(tt_emb_t h, const int64_t* indices, const int64_t* offsets, int64_t num_lookups,
+static int tt_emb_forward_impl(tt_emb_t h, const int64_t* indices, const int64_t* offsets, int64_t num_lookups,
                    int64_t batch, float* out, tt_stream_t stream)
 {
     if (!h || !offsets || !out || num_lookups < 0 || batch < 1) return TT_ERR_ARG;
@@ -689,6 +705,12 @@ int tt_emb_forward(tt_emb_t h, const int64_t* indices, const int64_t* offsets, i
             }
             e = k3_to_bf16(cp, h->tc == 3 ? 2 : 1, d1, d2, s, &nl);
         }
+        if (h->inject == TT_INJECT_POOL_WAIT || (h->inject == TT_INJECT_MMA_WAIT_FWD && h->tc)) {
+            cp.inj_pool = h->inject == TT_INJECT_POOL_WAIT;
+            cp.inj_mma = h->inject == TT_INJECT_MMA_WAIT_FWD;
+            cp.inj_spin = h->inject_spin;
+            h->inject = TT_INJECT_NONE;
+        }
         K3Args a = h->k3_args(&cp, &pp, &pb, offsets, L, false);
         if (e == cudaSuccess) e = k3_forward(a, out, s, &nl);
     } else {
@@ -735,7 +757,11 @@ static int backward_impl(tt_emb_t h, const float* grad_out, tt_stream_t stream, 
         PlanBuffers pb = h->plan_buffers(sb);
         pb.sorted_groups = h->plan_sorted_groups;
         GradPtrs vgp;
-        const CoreParams vcp = h->view_cores(h->fwd_B, &vgp);
+        CoreParams vcp = h->view_cores(h->fwd_B, &vgp);
+        if (h->inject == TT_INJECT_MMA_WAIT_BWD) {
+            vcp.inj_mma = 1;
+            h->inject = TT_INJECT_NONE;
+        }
         if (fused) {
             vgp.fused = 1;
             vgp.lr = lr;
@@ -779,14 +805,14 @@ static int backward_impl(tt_emb_t h, const float* grad_out, tt_stream_t stream, 
     return cuda_status(e);
 }
 
-int tt_emb_backward(tt_emb_t h, const float* grad_out, tt_stream_t stream)
+static int tt_emb_backward_impl(tt_emb_t h, const float* grad_out, tt_stream_t stream)
 {
     if (!h || !grad_out) return TT_ERR_ARG;
     if (!h->have_fwd || !h->have_grads || !h->have_cores) return TT_ERR_STATE;
     return backward_impl(h, grad_out, stream, false, 0.f);
 }
 
-int tt_emb_backward_sgd(tt_emb_t h, const float* grad_out, float lr, tt_stream_t stream)
+static int tt_emb_backward_sgd_impl(tt_emb_t h, const float* grad_out, float lr, tt_stream_t stream)
 {
     if (!h || !grad_out) return TT_ERR_ARG;
     if (!h->have_fwd || !h->have_grads || !h->have_cores) return TT_ERR_STATE;
@@ -804,7 +830,7 @@ int tt_emb_backward_sgd(tt_emb_t h, const float* grad_out, float lr, tt_stream_t
     return cuda_status(e);
 }
 
-int tt_emb_sgd_update(tt_emb_t h, float lr, tt_stream_t stream)
+static int tt_emb_sgd_update_impl(tt_emb_t h, float lr, tt_stream_t stream)
 {
     if (!h) return TT_ERR_ARG;
     if (!h->have_cores || !h->have_grads) return TT_ERR_STATE;
@@ -823,21 +849,21 @@ int tt_emb_sync(tt_emb_t h)
 {
     if (!h) return TT_ERR_ARG;
     cudaStream_t s = h->used_stream ? h->last_stream : (cudaStream_t)0;
-    if (cudaStreamSynchronize(s) != cudaSuccess) return TT_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return note(h, TT_ERR_CUDA);
     h->fold();
     int32_t st[2] = {0, 0};
     if (cudaMemcpyAsync(st, h->d_status, sizeof(st), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess)
-        return TT_ERR_CUDA;
+        return note(h, TT_ERR_CUDA);
     if (st[0] != 0) {
         if (cudaMemsetAsync(h->d_status, 0, 256, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
-            return TT_ERR_CUDA;
-        return st[0];
+            return note(h, TT_ERR_CUDA);
+        return note(h, st[0]);
     }
     return TT_OK;
 }
 
-int tt_emb_get_segmentation(tt_emb_t h, tt_seg_view* v)
+static int tt_emb_get_segmentation_impl(tt_emb_t h, tt_seg_view* v)
 {
     if (!h || !v) return TT_ERR_ARG;
     if (!h->have_fwd) return TT_ERR_STATE;
@@ -861,7 +887,7 @@ int tt_emb_get_segmentation(tt_emb_t h, tt_seg_view* v)
     return TT_OK;
 }
 
-int tt_emb_copy_segmentation(tt_emb_t h, void* sorted_keys, int32_t* perm, void* uniq_keys,
+static int tt_emb_copy_segmentation_impl(tt_emb_t h, void* sorted_keys, int32_t* perm, void* uniq_keys,
                              int32_t* uniq_start, int32_t* grp_start, int32_t* bag_sorted)
 {
     tt_seg_view v;
@@ -879,7 +905,7 @@ int tt_emb_copy_segmentation(tt_emb_t h, void* sorted_keys, int32_t* perm, void*
     return cuda_status(e);
 }
 
-int tt_emb_enable_timing(tt_emb_t h, int enable)
+static int tt_emb_enable_timing_impl(tt_emb_t h, int enable)
 {
     if (!h) return TT_ERR_ARG;
     h->fold();
@@ -889,11 +915,86 @@ int tt_emb_enable_timing(tt_emb_t h, int enable)
     return TT_OK;
 }
 
-int tt_emb_phase_times(tt_emb_t h, double* ms, int64_t* launches)
+static int tt_emb_phase_times_impl(tt_emb_t h, double* ms, int64_t* launches)
 {
     if (!h || !ms) return TT_ERR_ARG;
     for (int i = 0; i < TT_EMB_NUM_PHASES; ++i) ms[i] = h->phase_ms[i];
     if (launches) *launches = h->launches;
+    return TT_OK;
+}
+
+// Public entry points: the implementations above, with failures recorded for tt_emb_last_error.
+int tt_emb_set_cores(tt_emb_t h, float* const* cores, float* const* core_grads)
+{
+    return note(h, tt_emb_set_cores_impl(h, cores, core_grads));
+}
+int tt_emb_workspace_size(tt_emb_t h, int64_t max_lookups, int64_t batch, size_t* bytes)
+{
+    return note(h, tt_emb_workspace_size_impl(h, max_lookups, batch, bytes));
+}
+int tt_emb_set_workspace(tt_emb_t h, void* workspace, size_t bytes, int64_t max_lookups, int64_t batch)
+{
+    return note(h, tt_emb_set_workspace_impl(h, workspace, bytes, max_lookups, batch));
+}
+int tt_emb_forward(tt_emb_t h, const int64_t* indices, const int64_t* offsets, int64_t num_lookups,
+                   int64_t batch, float* out, tt_stream_t stream)
+{
+    return note(h, tt_emb_forward_impl(h, indices, offsets, num_lookups, batch, out, stream));
+}
+int tt_emb_backward(tt_emb_t h, const float* grad_out, tt_stream_t stream)
+{
+    return note(h, tt_emb_backward_impl(h, grad_out, stream));
+}
+int tt_emb_backward_sgd(tt_emb_t h, const float* grad_out, float lr, tt_stream_t stream)
+{
+    return note(h, tt_emb_backward_sgd_impl(h, grad_out, lr, stream));
+}
+int tt_emb_sgd_update(tt_emb_t h, float lr, tt_stream_t stream)
+{
+    return note(h, tt_emb_sgd_update_impl(h, lr, stream));
+}
+int tt_emb_get_segmentation(tt_emb_t h, tt_seg_view* v)
+{
+    return note(h, tt_emb_get_segmentation_impl(h, v));
+}
+int tt_emb_copy_segmentation(tt_emb_t h, void* sorted_keys, int32_t* perm, void* uniq_keys,
+                             int32_t* uniq_start, int32_t* grp_start, int32_t* bag_sorted)
+{
+    return note(h, tt_emb_copy_segmentation_impl(h, sorted_keys, perm, uniq_keys, uniq_start, grp_start,
+                                                 bag_sorted));
+}
+int tt_emb_enable_timing(tt_emb_t h, int enable) { return note(h, tt_emb_enable_timing_impl(h, enable)); }
+int tt_emb_phase_times(tt_emb_t h, double* ms, int64_t* launches)
+{
+    return note(h, tt_emb_phase_times_impl(h, ms, launches));
+}
+
+int tt_emb_last_error(tt_emb_t h)
+{
+    if (!h) return TT_ERR_ARG;
+    const int rc = h->last_error;
+    h->last_error = TT_OK;
+    return rc;
+}
+
+int tt_emb_debug_inject(tt_emb_t h, int32_t what, int32_t spin_limit)
+{
+    if (!h || spin_limit < 0) return note(h, TT_ERR_ARG);
+    switch (what) {
+    case TT_INJECT_NONE: break;
+    case TT_INJECT_POOL_WAIT:
+        if (!h->fast) return note(h, TT_ERR_UNSUPPORTED);
+        break;
+    case TT_INJECT_MMA_WAIT_FWD:
+        if (!h->tc) return note(h, TT_ERR_UNSUPPORTED);
+        break;
+    case TT_INJECT_MMA_WAIT_BWD:
+        if (!h->tc || !k3_tc_bwd_supported(h->view_params())) return note(h, TT_ERR_UNSUPPORTED);
+        break;
+    default: return note(h, TT_ERR_ARG);
+    }
+    h->inject = what;
+    h->inject_spin = spin_limit;
     return TT_OK;
 }
 

@@ -159,12 +159,14 @@ cudaError_t launch_forward_generic(const CoreParams& cp, bool key64, const void*
     const int g = (int)(max_groups < grid ? max_groups : grid);
     if (g <= 0) return cudaSuccess;
     if (key64) {
-        cudaFuncSetAttribute(k_fwd_generic<uint64_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        const cudaError_t ea = cudaFuncSetAttribute(k_fwd_generic<uint64_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (ea != cudaSuccess) return ea;
         k_fwd_generic<uint64_t><<<g, 256, smem, s>>>(cp, (const uint64_t*)uniq_keys, uniq_start,
                                                      grp_start, bag_sorted, counters, (int)inter,
                                                      out, status);
     } else {
-        cudaFuncSetAttribute(k_fwd_generic<uint32_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        const cudaError_t ea = cudaFuncSetAttribute(k_fwd_generic<uint32_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (ea != cudaSuccess) return ea;
         k_fwd_generic<uint32_t><<<g, 256, smem, s>>>(cp, (const uint32_t*)uniq_keys, uniq_start,
                                                      grp_start, bag_sorted, counters, (int)inter,
                                                      out, status);
@@ -322,12 +324,14 @@ cudaError_t launch_backward_generic(const CoreParams& cp, const GradPtrs& gp, bo
     const int g = (int)(max_groups < grid ? max_groups : grid);
     if (g <= 0) return cudaSuccess;
     if (key64) {
-        cudaFuncSetAttribute(k_bwd_generic<uint64_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        const cudaError_t ea = cudaFuncSetAttribute(k_bwd_generic<uint64_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (ea != cudaSuccess) return ea;
         k_bwd_generic<uint64_t><<<g, 256, smem, s>>>(cp, gp, (const uint64_t*)uniq_keys, uniq_start,
                                                      grp_start, bag_sorted, counters, (int)dcap,
                                                      (int)sum, grad_out, status);
     } else {
-        cudaFuncSetAttribute(k_bwd_generic<uint32_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        const cudaError_t ea = cudaFuncSetAttribute(k_bwd_generic<uint32_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (ea != cudaSuccess) return ea;
         k_bwd_generic<uint32_t><<<g, 256, smem, s>>>(cp, gp, (const uint32_t*)uniq_keys, uniq_start,
                                                      grp_start, bag_sorted, counters, (int)dcap,
                                                      (int)sum, grad_out, status);

@@ -548,7 +548,7 @@ __device__ __forceinline__ void tc_mma_terms(uint32_t tmem_d, uint64_t adesc, ui
 // threads) when the completion wait ran out.
 template <class S, int NT>
 __device__ __forceinline__ bool fwd_gemm_tc(const FwdSmem<S>& sm, uint32_t tmem, uint64_t* bar, uint32_t& parity,
-                                            int* s_ok)
+                                            int* s_ok, bool inject_fail)
 {
     constexpr int R = S::R, N = S::N, MF = S::MF;
     static_assert(MF == 64 || MF == 128, "tensor-core M is 64 or 128");
@@ -566,7 +566,8 @@ __device__ __forceinline__ bool fwd_gemm_tc(const FwdSmem<S>& sm, uint32_t tmem,
             tc_mma_terms<NT>(tmem, umma_desc(a0 + k * 256, 128, SBO), umma_desc(b0 + k * 256, 128, SBO),
                              MF * R * 2, R * N * 2, idesc, k > 0);
         tc_commit(bar);
-        *s_ok = mbar_wait(bar, parity) ? 1 : 0;
+        // an injected failure (test hook) is reported only after the products completed
+        *s_ok = (mbar_wait(bar, parity) && !inject_fail) ? 1 : 0;
     }
     __syncthreads();
     parity ^= 1u;
@@ -684,11 +685,17 @@ __device__ void fwd_pool(const CoreParams& cp, int ptask, int nP, const int32_t*
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     TT_PH_START();
     if (tid == 0) {
-        const int want = hdr->nC[t];
+        // injected failure (test hook): wait for one chunk more than the table has
+        const int want = hdr->nC[t] + (cp.inj_pool ? 1 : 0);
+        const int limit = cp.inj_spin > 0 ? cp.inj_spin : kSpinLimit;
         int it = 0, ok = 1;
         while (*reinterpret_cast<volatile int*>(&hdr->done[t]) < want) {
-            if (++it > kSpinLimit) {
+            if (++it > limit) {
                 raise_error(status, TT_ERR_TIMEOUT, t);
+                ok = 0;
+                break;
+            }
+            if ((it & 63) == 0 && has_error(status)) {   // another block failed: stop waiting
                 ok = 0;
                 break;
             }
@@ -815,7 +822,7 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
         if (total > 0) fwd_issue_batch<S, K>(cp, mb, 0, 0, uniq_keys, M, sm, s_keys);
         TT_PH(0);
         if constexpr (TC) {
-            if (!fwd_gemm_tc<S, NT>(sm, tmem, &s_mbar, parity, &s_ok)) {
+            if (!fwd_gemm_tc<S, NT>(sm, tmem, &s_mbar, parity, &s_ok, cp.inj_mma != 0)) {
                 if (tid == 0) raise_error(status, TT_ERR_TIMEOUT, 100);
                 break;
             }
@@ -1227,11 +1234,12 @@ struct WarpRow1 {
 };
 
 // one thread issues, the others wait at the barrier; false (all threads) when the wait ran out
-__device__ __forceinline__ bool tc_commit_wait(uint64_t* bar, uint32_t& parity, int* s_ok)
+// (or, with inject_fail, a test hook, once the products have completed)
+__device__ __forceinline__ bool tc_commit_wait(uint64_t* bar, uint32_t& parity, int* s_ok, bool inject_fail = false)
 {
     if (threadIdx.x == 0) {
         tc_commit(bar);
-        *s_ok = mbar_wait(bar, parity) ? 1 : 0;
+        *s_ok = (mbar_wait(bar, parity) && !inject_fail) ? 1 : 0;
     }
     __syncthreads();
     parity ^= 1u;
@@ -1914,7 +1922,7 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
                                          umma_desc(b0 + k * 256, 128, SBO), R * N * 2, MB * R * 2,
                                          umma_idesc_bf16(128, MB), k > 0);
             }
-            if (!tc_commit_wait(&s_mbar, parity, &s_ok)) {   // also the previous chunk's dA and dB
+            if (!tc_commit_wait(&s_mbar, parity, &s_ok, cp.inj_mma != 0)) {   // also the previous chunk's dA and dB
                 failed = true;
                 break;
             }

@@ -67,6 +67,11 @@ struct CoreParams {
     // tiles (n = (a_2, rho_2) rows x K = rho_1, 8 x 8 core matrices) in bf16, built by k3_to_bf16
     const uint16_t* bf1[kMaxT];
     const uint16_t* bf2[kMaxT];
+    // failure injection (tt_emb_debug_inject; zero in normal calls): inj_pool = 1 makes every
+    // pooling wait want one finished chunk more than its table has; inj_mma = 1 makes the
+    // first tensor-core completion wait report a timeout after the products completed;
+    // inj_spin > 0 replaces the pooling wait's iteration limit
+    int32_t inj_pool, inj_mma, inj_spin, inj_pad;
 };
 
 struct GradPtrs {

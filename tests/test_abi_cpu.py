@@ -109,3 +109,9 @@ def test_tensor_core_precisions_reject_other_shapes(n, d, r):
         with pytest.raises(abi.TTEmbError) as e:
             abi.tt_emb_create(n, rows, d, r, o)
         assert e.value.code == abi.TT_ERR_SHAPE
+
+
+def test_handle_free_calls_reject_a_null_handle():
+    assert abi.lib().tt_emb_last_error(None) == abi.TT_ERR_ARG
+    assert abi.lib().tt_emb_debug_inject(None, abi.TT_INJECT_POOL_WAIT, 0) == abi.TT_ERR_ARG
+    assert abi.lib().tt_emb_sync(None) == abi.TT_ERR_ARG
