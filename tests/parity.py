@@ -10,12 +10,49 @@ and the result x,
     err = max_e |x_e - y_e| / max_e |y_e|,
 and the reported error is the largest over groups.  A group whose reference
 is all zeros (an empty bag, an untouched slice) must come out exactly zero.
+
+Beside it, every comparison also computes the elementwise metric with a floor,
+    err_e = max_e |x_e - y_e| / max(|y_e|, 1e-3 max_group |y|),
+which weighs every element by its own size down to a thousandth of its group's
+largest.  The bounds (1e-4, 2e-2) apply to the normwise metric; when the
+environment variable TT_PARITY_REPORT names a file, each comparison appends one
+JSON line with both metrics (test, kind, normwise, elementwise_floor), so the
+elementwise figures are on record for every case.
 """
 from __future__ import annotations
+
+import json
+import os
 
 import numpy as np
 
 FP32_TOL = 1e-4
+FLOOR = 1e-3
+
+
+def floor_elementwise_err(got, want, axis_groups, floor=FLOOR):
+    """Elementwise relative error with a per-group floor of `floor` x the group's max |y|."""
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    if want.size == 0:
+        return 0.0
+    scale = np.max(np.abs(want), axis=axis_groups, keepdims=True)
+    denom = np.maximum(np.abs(want), floor * scale)
+    diff = np.abs(got - want)
+    zero = denom == 0
+    if np.any(zero & (diff != 0)):
+        return float("inf")
+    return float(np.max(np.where(zero, 0.0, diff / np.where(zero, 1.0, denom))))
+
+
+def _report(kind, normwise, elementwise):
+    path = os.environ.get("TT_PARITY_REPORT")
+    if not path:
+        return
+    rec = {"test": os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0], "kind": kind,
+           "normwise": normwise, "elementwise_floor": elementwise}
+    with open(path, "a") as f:
+        f.write(json.dumps(rec) + "\n")
 
 
 def grouped_rel_err(got, want, axis_groups):
@@ -36,13 +73,18 @@ def grouped_rel_err(got, want, axis_groups):
 def output_err(got, want, D):
     """Per bag row: out is [B, T*D]; each (b, t) block of D values is one group."""
     B = want.shape[0]
-    return grouped_rel_err(np.asarray(got).reshape(B, -1, D), np.asarray(want).reshape(B, -1, D),
-                           (2,))
+    g = np.asarray(got).reshape(B, -1, D)
+    y = np.asarray(want).reshape(B, -1, D)
+    e = grouped_rel_err(g, y, (2,))
+    _report("pooled rows", e, floor_elementwise_err(g, y, (2,)))
+    return e
 
 
 def core_grad_err(got, want):
     """Per digit slice: a core is [r0, n, d, r1]; G[:, i] is one group."""
-    return grouped_rel_err(got, want, (0, 2, 3))
+    e = grouped_rel_err(got, want, (0, 2, 3))
+    _report("core slices", e, floor_elementwise_err(got, want, (0, 2, 3)))
+    return e
 
 
 def gpu_forward(w, options=None, device="cuda", with_grads=None):

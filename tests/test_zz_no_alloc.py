@@ -8,7 +8,10 @@ fixed 16 MiB device array and this entry point allocates nothing.  These tests
 call it through the C ABI and check it against tt_emb_forward (the entry point
 with a caller workspace), within the parity tolerance, on consecutive calls
 whose inputs differ, so stale scratch contents from one call cannot leak into
-the next.
+the next.  They also check that warmed calls leave the device's allocated and
+free memory unchanged, that the wide (64-bit) sort keys of eight 1e9-row tables
+work, and that a backward after this forward is refused (its grouping is not
+kept).
 """
 import pytest
 import torch
@@ -49,11 +52,46 @@ def test_noalloc_forward_matches_forward_on_consecutive_calls():
 
 
 def test_noalloc_forward_with_wide_keys_and_four_cores():
-    w = config_workload(5, batch=256, tables=2, with_grad=False)    # 64-bit keys, k = 4
+    # eight tables of 1e9 rows: 30 row bits + 3 table bits, so the sort keys take 64 bits
+    w = config_workload(5, batch=256, tables=8, with_grad=False)
     emb, cores, idx, off = from_workload(w, with_grads=False)
     want = _reference(emb, idx, off, w.batch)
+    assert emb.segmentation()["sorted_keys"].dtype.itemsize == 8
+    assert idx.numel() <= abi.NOALLOC_MAX_LOOKUPS
     for _ in range(2):
         assert output_err(_noalloc(emb, idx, off, w.batch), want, w.dim) <= FP32_TOL
+
+
+def test_noalloc_call_allocates_no_device_memory():
+    w = config_workload(3, batch=512, tables=4, with_grad=False)
+    emb, cores, idx, off = from_workload(w, with_grads=False)
+    out = torch.empty(w.batch, emb.T * emb.D, device="cuda")
+    # first call on the device: looks up the scratch (and loads its module); not measured
+    abi.tt_emb_forward_noalloc(emb.handle, idx, off, w.batch, out)
+    emb.sync()
+    torch.cuda.synchronize()
+    used0 = torch.cuda.memory_allocated()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        abi.tt_emb_forward_noalloc(emb.handle, idx, off, w.batch, out)
+    emb.sync()
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated() == used0
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+
+
+def test_backward_after_a_noalloc_forward_is_refused():
+    w = config_workload(4, batch=16, tables=2, with_grad=True)
+    emb, cores, idx, off = from_workload(w, with_grads=True)
+    g = torch.from_numpy(w.grad_out).cuda()
+    emb.forward(idx, off, w.batch)
+    out = torch.empty(w.batch, emb.T * emb.D, device="cuda")
+    abi.tt_emb_forward_noalloc(emb.handle, idx, off, w.batch, out)
+    with pytest.raises(abi.TTEmbError) as e:
+        abi.tt_emb_backward(emb.handle, g)
+    assert e.value.code == abi.TT_ERR_STATE
+    emb.sync()
 
 
 def test_noalloc_rejects_batches_above_its_capacity():
