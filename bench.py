@@ -439,6 +439,33 @@ def kernel_roofline(kernel, ms, alg, precision, w, peaks, config):
             "peak_source": f"HBM copy bandwidth {peaks['hbm_source']}"}
 
 
+def balance_report(records, cap):
+    """Per fused kernel: busy time per SM (block start to end, minus time in bounded waits),
+    its max and mean over SMs, and the kernel span, from the probe records of one step."""
+    import numpy as np
+    r = records.view(2, cap, 4).cpu().numpy().astype(np.int64)
+    out = {}
+    for slot, name in ((0, "fwd_fused"), (1, "bwd_fused")):
+        rec = r[slot]
+        rec = rec[rec[:, 1] > 0]
+        if rec.size == 0:
+            continue
+        sm = rec[:, 0] & 0xffffffff
+        tasks = rec[:, 0] >> 32
+        busy = rec[:, 2] - rec[:, 1] - rec[:, 3]
+        per_sm = {}
+        for s_, b_ in zip(sm.tolist(), busy.tolist()):
+            per_sm[s_] = per_sm.get(s_, 0) + b_
+        v = np.array(list(per_sm.values()), dtype=np.float64) / 1e6
+        out[name] = {"blocks": int(rec.shape[0]), "sms": int(len(per_sm)),
+                     "span_ms": float(rec[:, 2].max() - rec[:, 1].min()) / 1e6,
+                     "busy_max_ms": float(v.max()), "busy_mean_ms": float(v.mean()),
+                     "max_over_mean": float(v.max() / v.mean()) if v.mean() > 0 else None,
+                     "wait_mean_ms": float(rec[:, 3].mean()) / 1e6,
+                     "tasks_max": int(tasks.max()), "tasks_mean": float(tasks.mean())}
+    return out
+
+
 def time_rank32_forward(args, world, rank, dev, peaks, barrier_fn, max_fn):
     """Forward pass of the 26-table, rank-32, batch-32768 workload on its own handle, timed
     like the main step (CUDA events, max over ranks), with the fused kernel's roofline."""
@@ -560,6 +587,15 @@ def run_ours(args):
 
     # --- forward only ---
     ms_fwd = timed(lambda: emb.forward(idx, off, B, out), args.steps) / args.steps
+
+    # --- SM balance: one more step, untimed, with the scheduler probe on ---
+    cap = 4096
+    probe = torch.zeros(2 * cap * 4, dtype=torch.int64, device=dev)
+    abi.tt_emb_set_probe(emb.handle, probe, cap)
+    step()
+    emb.sync()
+    abi.tt_emb_set_probe(emb.handle, None, 0)
+    balance = balance_report(probe, cap)
 
     # --- dominant kernel roofline (device times from the timed region) ---
     per_step = {k: v / args.steps for k, v in ph.items()}
@@ -698,6 +734,7 @@ def run_ours(args):
             "gpu_launches": launches,
             "clocks": clk,
             "memory": mem,
+            "balance": balance,
             "peaks": {"hbm_gbs": peaks["hbm_gbs"], "hbm": peaks["hbm_source"],
                       "bf16_tflops": peaks["bf16_tflops"], "bf16": peaks["bf16_source"],
                       "fp32_tflops": FP32_PEAK_TFLOPS, "fp32": "derived from unit counts and the maximum SM clock"},

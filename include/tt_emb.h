@@ -351,6 +351,18 @@ int tt_emb_forward_noalloc(tt_emb_t h, const int64_t* indices, const int64_t* of
                            int64_t num_lookups, int64_t batch, float* out, tt_stream_t stream);
 
 /*
+ * Balance probe of the persistent scheduler (FlowTT section 2.4: skewed prefix frequencies
+ * create load imbalance; section 3.4 balances it).  While `records` is set, every block of
+ * the fused forward kernel (slot 0) and of the fused backward kernel (slot 1) writes one
+ * record of 4 uint64 at records[(slot * max_blocks + block) * 4]: SM id | tasks << 32, the
+ * block's start and end on the GPU's global timer (ns), and the nanoseconds it spent in
+ * bounded waits (pooling tasks waiting for their table).  Blocks >= max_blocks write nothing;
+ * each launch overwrites its slot.  records: device memory of 2 * max_blocks * 4 uint64,
+ * 8-byte aligned, owned by the caller; NULL turns the probe off.  Returns TT_OK or TT_ERR_ARG.
+ */
+int tt_emb_set_probe(tt_emb_t h, uint64_t* records, int32_t max_blocks);
+
+/*
  * Test hook for failure detection (no GPU fault is involved).  Arms one
  * injected failure of a bounded device wait; it is consumed by the next call
  * that runs the wait:

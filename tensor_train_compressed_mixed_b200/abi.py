@@ -76,6 +76,7 @@ _SIGS = {
     "tt_emb_forward_noalloc": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                 ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
     "tt_emb_last_error": ([ctypes.c_void_p], ctypes.c_int),
+    "tt_emb_set_probe": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32], ctypes.c_int),
     "tt_emb_debug_inject": ([ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32], ctypes.c_int),
     "tt_emb_destroy": ([ctypes.c_void_p], None),
 }
@@ -264,6 +265,13 @@ def tt_emb_phase_times(h):
 def tt_emb_last_error(h) -> int:
     """The most recent failure recorded on the handle (a status code), then cleared."""
     return int(lib().tt_emb_last_error(h))
+
+
+def tt_emb_set_probe(h, records, max_blocks: int):
+    """Balance probe: records is a CUDA int64 tensor of 2 * max_blocks * 4 entries, or None."""
+    import torch
+    ptr = ctypes.c_void_p(0) if records is None else _dev_ptr(records, torch.int64, "records")
+    _check(lib().tt_emb_set_probe(h, ptr, int(max_blocks) if records is not None else 0), "tt_emb_set_probe")
 
 
 def tt_emb_debug_inject(h, what: int, spin_limit: int = 0):

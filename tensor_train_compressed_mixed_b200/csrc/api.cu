@@ -14,9 +14,10 @@ struct Layout {
     size_t counters, keys[2], vals[2], bag_of_pos, hist, digit_total, partials, uniq_keys,
         uniq_start, grp_start, bag_sorted;
     // specialised path only (zero when unused)
-    size_t uid_at_pos, uid_sorted, rowbuf, pkeys[2], pvals[2], col_count, col_start, chunk_base,
-        hdr, chunks, tasks, grec, g12, dg12, g3t, dg3t, bf1, bf2;
-    int64_t chunk_cap, task_cap;
+    size_t uid_at_pos, uid_sorted, rowbuf, pkeys[2], pvals[2], col_count, col_rows, col_order, col_start, chunk_base,
+        hdr, chunks, grec, crow, sub_base, slot_of, subs, claim, own_head, steal_tail, exhausted, slot_flag,
+        ckpt, g12, dg12, g3t, dg3t, bf1, bf2;
+    int64_t chunk_cap, sub_cap, slot_cap;
     size_t total;
 };
 
@@ -65,14 +66,27 @@ Layout make_layout(int key_bytes, int64_t L, int64_t B, const FastDims& f)
         y.pvals[0] = take(Lz * 4);
         y.pvals[1] = take(Lz * 4);
         y.col_count = take(((size_t)f.ncols + 1) * 4);
+        y.col_rows = take(((size_t)f.ncols + 1) * 4);
+        y.col_order = take(((size_t)f.ncols + 1) * 4);
         y.col_start = take(((size_t)f.ncols + 1) * 4);
         y.chunk_base = take(((size_t)f.ncols + 1) * 4);
         y.hdr = take(sizeof(PlanHeader));
         y.chunk_cap = (int64_t)f.ncols + ceil_div((int64_t)Lz, f.MP) + 1;
         y.chunks = take((size_t)y.chunk_cap * sizeof(int4));
-        y.task_cap = y.chunk_cap + (int64_t)f.T * ceil_div(B, kPoolBags);
-        y.tasks = take((size_t)y.task_cap * 4);
         y.grec = take(Lz * sizeof(int4));
+        // forward subtasks: every chunk once, plus one per kSplitRows distinct rows of split chunks
+        y.sub_cap = y.chunk_cap + ceil_div((int64_t)Lz, kSplitRows) + 1;
+        y.slot_cap = min64(kCkptSlots, ceil_div((int64_t)Lz, kSplitRows) + 1);
+        y.crow = take((size_t)y.chunk_cap * 4);
+        y.sub_base = take(((size_t)y.chunk_cap + 1) * 4);
+        y.slot_of = take((size_t)y.chunk_cap * 4);
+        y.subs = take((size_t)y.sub_cap * sizeof(int4));
+        y.claim = take((size_t)y.sub_cap * 4);
+        y.own_head = take((size_t)kMaxGrid * 4);
+        y.steal_tail = take((size_t)kMaxGrid * 4);
+        y.exhausted = take((size_t)kMaxGrid * 4);
+        y.slot_flag = take((size_t)y.slot_cap * 4);
+        y.ckpt = take((size_t)y.slot_cap * kCkptFloats * 4);
         if (f.g12_floats > 0) {
             y.g12 = take((size_t)f.g12_floats * 4);
             y.dg12 = take((size_t)f.g12_floats * 4);
@@ -138,6 +152,8 @@ struct tt_emb_handle {
     int64_t launches = 0;
     int last_error = TT_OK;           // tt_emb_last_error
     int inject = TT_INJECT_NONE, inject_spin = 0;   // tt_emb_debug_inject, armed until consumed
+    unsigned long long* probe = nullptr;              // tt_emb_set_probe
+    int32_t probe_cap = 0;
     struct Interval { int phase; cudaEvent_t a, b; };
     std::vector<Interval> pending;
     std::vector<cudaEvent_t> pool;
@@ -280,10 +296,22 @@ struct tt_emb_handle {
         pp.NB = kPoolBags;
         pp.ncols = ncols;
         pp.sched = opt.sched;
+        pp.grid = fwd_grid();
+        pp.slot_cap = (int32_t)lay.slot_cap;
         for (int t = 0; t < T; ++t)
             for (int j = 0; j < 3; ++j) pp.n[t][j] = (uint32_t)vn[t][j];
         for (int t = 0; t <= T; ++t) pp.col_base[t] = col_base[t];
         return pp;
+    }
+    // persistent blocks of the fused forward: the option, else one wave (owner ranges need it at plan time)
+    mutable int fwd_grid_cache = 0;
+    int fwd_grid() const
+    {
+        if (fwd_grid_cache == 0) {
+            const int g = opt.grid > 0 ? opt.grid : num_sms * k3_blocks_per_sm(view_params(), false, tc != 0);
+            fwd_grid_cache = g < kMaxGrid ? g : kMaxGrid;
+        }
+        return fwd_grid_cache;
     }
     int64_t core_floats(int t, int j) const { return (int64_t)r[j] * n[t][j] * d[j] * r[j + 1]; }
 
@@ -339,12 +367,23 @@ struct tt_emb_handle {
         pb.sort.hist = lookup_sort.hist ? lookup_sort.hist : (uint32_t*)at(lay.hist);
         pb.sort.digit_total = lookup_sort.digit_total ? lookup_sort.digit_total : (uint32_t*)at(lay.digit_total);
         pb.col_count = (int32_t*)at(lay.col_count);
+        pb.col_rows = (int32_t*)at(lay.col_rows);
+        pb.col_order = (int32_t*)at(lay.col_order);
         pb.col_start = (int32_t*)at(lay.col_start);
         pb.chunk_base = (int32_t*)at(lay.chunk_base);
         pb.hdr = (PlanHeader*)at(lay.hdr);
         pb.chunks = (int4*)at(lay.chunks);
-        pb.tasks = (int32_t*)at(lay.tasks);
         pb.grec = (int4*)at(lay.grec);
+        pb.crow = (int32_t*)at(lay.crow);
+        pb.sub_base = (int32_t*)at(lay.sub_base);
+        pb.slot_of = (int32_t*)at(lay.slot_of);
+        pb.subs = (int4*)at(lay.subs);
+        pb.claim = (int32_t*)at(lay.claim);
+        pb.own_head = (int32_t*)at(lay.own_head);
+        pb.steal_tail = (int32_t*)at(lay.steal_tail);
+        pb.exhausted = (int32_t*)at(lay.exhausted);
+        pb.slot_flag = (int32_t*)at(lay.slot_flag);
+        pb.ckpt = (float*)at(lay.ckpt);
         return pb;
     }
 
@@ -369,7 +408,8 @@ struct tt_emb_handle {
         a.rowbuf = (float*)at(lay.rowbuf);
         a.L = L;
         a.tc = (tc && (!backward || k3_tc_bwd_supported(*cp))) ? tc : 0;
-        a.grid = opt.grid > 0 ? opt.grid : num_sms * k3_blocks_per_sm(*cp, backward, a.tc != 0);
+        a.grid = backward ? (opt.grid > 0 ? opt.grid : num_sms * k3_blocks_per_sm(*cp, true, a.tc != 0))
+                          : fwd_grid();
         a.status = d_status;
         return a;
     }
@@ -705,6 +745,9 @@ static int tt_emb_forward_impl(tt_emb_t h, const int64_t* indices, const int64_t
             }
             e = k3_to_bf16(cp, h->tc == 3 ? 2 : 1, d1, d2, s, &nl);
         }
+        cp.probe = h->probe;
+        cp.probe_slot = 0;
+        cp.probe_cap = h->probe_cap;
         if (h->inject == TT_INJECT_POOL_WAIT || (h->inject == TT_INJECT_MMA_WAIT_FWD && h->tc)) {
             cp.inj_pool = h->inject == TT_INJECT_POOL_WAIT;
             cp.inj_mma = h->inject == TT_INJECT_MMA_WAIT_FWD;
@@ -762,6 +805,9 @@ static int backward_impl(tt_emb_t h, const float* grad_out, tt_stream_t stream, 
             vcp.inj_mma = 1;
             h->inject = TT_INJECT_NONE;
         }
+        vcp.probe = h->probe;
+        vcp.probe_slot = 1;
+        vcp.probe_cap = h->probe_cap;
         if (fused) {
             vgp.fused = 1;
             vgp.lr = lr;
@@ -975,6 +1021,15 @@ int tt_emb_last_error(tt_emb_t h)
     const int rc = h->last_error;
     h->last_error = TT_OK;
     return rc;
+}
+
+int tt_emb_set_probe(tt_emb_t h, uint64_t* records, int32_t max_blocks)
+{
+    if (!h || max_blocks < 0 || (records && max_blocks == 0)) return note(h, TT_ERR_ARG);
+    if (records && ((uintptr_t)records & 7)) return note(h, TT_ERR_ARG);
+    h->probe = (unsigned long long*)records;
+    h->probe_cap = records ? max_blocks : 0;
+    return TT_OK;
 }
 
 int tt_emb_debug_inject(tt_emb_t h, int32_t what, int32_t spin_limit)

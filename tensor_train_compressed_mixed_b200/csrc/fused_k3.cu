@@ -337,14 +337,15 @@ struct RowTable {
 };
 
 template <class S>
-struct FwdMeta {   // shared-memory metadata of a chunk (double buffered)
+struct FwdMeta {   // shared-memory metadata of a subtask (double buffered)
     int u0[2][S::MPF];
     int ucum[2][S::MPF + 1];
     int i1[2][S::MPF];
     int cnt[2], t[2], i2[2];
-    int bu[2][S::NUF], bp[2][S::NUF], bi3[2][S::NUF];
+    int cid[2], rb[2], re[2], slot[2];   // chunk, its distinct rows [rb, re), checkpoint slot
     int task[2];
     int flag;
+    int ck;                              // checkpoint decision of the current subtask
     RowTable rows;
 };
 
@@ -356,19 +357,21 @@ __device__ __forceinline__ int prefix_of(const int* ucum, int cnt, int kq)
     return j;
 }
 
-// The chunk's row table: for its first kKeyCap distinct rows, the row id, the prefix slot and
-// the last digit, computed once per chunk by all threads from the staged keys (which must have
-// landed and be visible).  Batches inside the table then need no per-batch metadata pass.
+// The row table of distinct rows base .. base + kKeyCap of a chunk (at most `total`): the row
+// id, the prefix slot and the last digit, computed once by all threads from the staged keys
+// (which must have landed and be visible).  Batches inside the table then need no per-batch
+// metadata pass.
 template <typename K>
 __device__ __forceinline__ void build_rows(RowTable& rt, int mb, const int* ucum, const int* u0, int cnt, int total,
-                                           const K* keys, int ibits, uint32_t n3, int nthreads)
+                                           const K* keys, int ibits, uint32_t n3, int nthreads, int base = 0)
 {
-    const int n = min(total, kKeyCap);
-    for (int kq = threadIdx.x; kq < n; kq += nthreads) {
+    const int n = min(total - base, kKeyCap);
+    for (int i = threadIdx.x; i < n; i += nthreads) {
+        const int kq = base + i;
         const int j = prefix_of(ucum, cnt, kq);
-        rt.u[mb][kq] = u0[j] + (kq - ucum[j]);
-        rt.p[mb][kq] = j;
-        rt.i3[mb][kq] = (int)(key_row(keys[mb * kKeyCap + kq], ibits) % n3);
+        rt.u[mb][i] = u0[j] + (kq - ucum[j]);
+        rt.p[mb][i] = j;
+        rt.i3[mb][i] = (int)(key_row(keys[mb * kKeyCap + i], ibits) % n3);
     }
 }
 // Rows k0 .. k0 + nb of chunk buffer mb: the row table when it covers them, else the batch's own
@@ -385,16 +388,16 @@ __device__ __forceinline__ RowRef batch_rows(const RowTable& rt, int mb, int k0,
     return RowRef{bu, bp, bi3};
 }
 
-// Metadata of chunk `cid` into buffer mb (all threads call; ends with a barrier), and
-// asynchronous copies of the keys of its first kKeyCap distinct rows into keys[mb]; those
-// join the caller's next commit group (the chunk's A/B copies).
+// Metadata of subtask `sub` = (chunk, first row, end row, slot) into buffer mb (all threads
+// call; ends with a barrier), and asynchronous copies of the keys of its distinct rows (at most
+// kKeyCap) into keys[mb]; those join the caller's next commit group (the chunk's A/B copies).
 template <class S, typename K>
-__device__ __forceinline__ void fwd_meta(const CoreParams& cp, int cid, int mb, const K* __restrict__ uniq_keys,
+__device__ __forceinline__ void fwd_meta(const CoreParams& cp, int4 sub, int mb, const K* __restrict__ uniq_keys,
                                          const int4* __restrict__ grec, const int4* __restrict__ chunks,
                                          FwdMeta<S>& M, K* keys)
 {
     const int tid = threadIdx.x;
-    const int4 ch = chunks[cid];
+    const int4 ch = chunks[sub.x];
     if (tid < S::MPF) {
         const int4 g = tid < ch.y ? grec[ch.x + tid] : make_int4(0, 0, 0, 0);
         M.u0[mb][tid] = g.x;
@@ -405,6 +408,10 @@ __device__ __forceinline__ void fwd_meta(const CoreParams& cp, int cid, int mb, 
         M.cnt[mb] = ch.y;
         M.t[mb] = ch.z;
         M.i2[mb] = ch.w;
+        M.cid[mb] = sub.x;
+        M.rb[mb] = sub.y;
+        M.re[mb] = sub.z;
+        M.slot[mb] = sub.w;
     }
     __syncthreads();
     if (tid == 0) {
@@ -417,10 +424,11 @@ __device__ __forceinline__ void fwd_meta(const CoreParams& cp, int cid, int mb, 
         M.ucum[mb][S::MPF] = run;
     }
     __syncthreads();
-    const int nk = min(M.ucum[mb][S::MPF], kKeyCap);
-    for (int kq = tid; kq < nk; kq += kFwdThreads) {
+    const int nk = min(sub.z - sub.y, kKeyCap);
+    for (int i = tid; i < nk; i += kFwdThreads) {
+        const int kq = sub.y + i;
         const int j = prefix_of(M.ucum[mb], M.cnt[mb], kq);
-        cp_async_key(keys + mb * kKeyCap + kq, uniq_keys + M.u0[mb][j] + (kq - M.ucum[mb][j]));
+        cp_async_key(keys + mb * kKeyCap + i, uniq_keys + M.u0[mb][j] + (kq - M.ucum[mb][j]));
     }
 }
 
@@ -595,52 +603,35 @@ __device__ __forceinline__ bool fwd_gemm_tc(const FwdSmem<S>& sm, uint32_t tmem,
     return true;
 }
 
-// distinct rows k0..k0+nb of the chunk into batch buffer bb; issues their last slices (one
-// commit group).  Row keys come from the chunk's staged keys (landed and made visible by the
-// caller) for the first kKeyCap rows, from global memory beyond.
-template <class S, typename K>
-__device__ __forceinline__ void fwd_issue_batch(const CoreParams& cp, int mb, int k0, int bb,
-                                                const K* __restrict__ uniq_keys, FwdMeta<S>& M,
-                                                const FwdSmem<S>& sm, const K* keys)
+// Distinct rows i0 .. i0 + NUF of the subtask in buffer mb (indices local to the subtask, inside
+// its row table) into batch buffer bb: issues their last slices (one commit group).
+template <class S>
+__device__ __forceinline__ void fwd_issue_batch(const CoreParams& cp, int mb, int i0, int bb, const FwdMeta<S>& M,
+                                                const FwdSmem<S>& sm)
 {
     constexpr int R = S::R, D3 = S::D3;
     const int tid = threadIdx.x;
-    const int total = M.ucum[mb][S::MPF];
-    const int nb = min(S::NUF, total - k0);
-    const int t = M.t[mb];
-    const uint32_t n3 = cp.n[t][2];
-    if (k0 + nb > kKeyCap) {   // beyond the row table: this batch's metadata
-        if (tid < nb) {
-            const int kq = k0 + tid;
-            const int j = prefix_of(M.ucum[mb], M.cnt[mb], kq);
-            const int u = M.u0[mb][j] + (kq - M.ucum[mb][j]);
-            const K key = kq < kKeyCap ? keys[mb * kKeyCap + kq] : uniq_keys[u];
-            M.bu[bb][tid] = u;
-            M.bp[bb][tid] = j;
-            M.bi3[bb][tid] = (int)(key_row(key, cp.ibits) % n3);
-        }
-        __syncthreads();
-    }
-    const RowRef rr = batch_rows(M.rows, mb, k0, nb, M.bu[bb], M.bp[bb], M.bi3[bb]);
-    const float* G3t = cp.last_t[t];   // [n3][R][D3]: one row's slice is contiguous
+    const int nb = min(S::NUF, M.re[mb] - M.rb[mb] - i0);
+    const int* i3 = M.rows.i3[mb] + i0;
+    const float* G3t = cp.last_t[M.t[mb]];   // [n3][R][D3]: one row's slice is contiguous
     float* Ss = sm.Ss + (size_t)bb * S::NUF * S::SU;
     for (int q = tid; q < nb * R * (D3 / 4); q += kFwdThreads) {
         const int uu = q / (R * (D3 / 4)), rem = q % (R * (D3 / 4));
-        cp_async16(&Ss[uu * S::SU + rem * 4], G3t + (int64_t)rr.i3[uu] * (R * D3) + rem * 4);
+        cp_async16(&Ss[uu * S::SU + rem * 4], G3t + (int64_t)i3[uu] * (R * D3) + rem * 4);
     }
     cp_async_commit();
 }
 
 // E_u = C_p . S_u for the batch in buffer bb; tile: rows (a1, a2 = 2h, 2h+1) x 4 columns of a3
 template <class S>
-__device__ __forceinline__ void fwd_batch_compute(int mb, int k0, int nb, int bb, const FwdMeta<S>& M,
+__device__ __forceinline__ void fwd_batch_compute(int mb, int i0, int nb, int bb, const FwdMeta<S>& M,
                                                   const FwdSmem<S>& sm, float* __restrict__ rowbuf)
 {
     constexpr int R = S::R, N = S::N, D1 = S::D1, D2 = S::D2, D3 = S::D3;
     const int tid = threadIdx.x;
     const int uu = tid / S::TPU;
     if (uu >= nb) return;
-    const RowRef rr = batch_rows(M.rows, mb, k0, nb, M.bu[bb], M.bp[bb], M.bi3[bb]);
+    const RowRef rr{M.rows.u[mb] + i0, M.rows.p[mb] + i0, M.rows.i3[mb] + i0};
     const int rem = tid % S::TPU;
     const int a1 = rem / (2 * (D3 / 4)), h = (rem / (D3 / 4)) % 2, cg = rem % (D3 / 4);
     const int m = rr.p[uu] * D1 + a1;
@@ -675,7 +666,7 @@ template <class S>
 __device__ void fwd_pool(const CoreParams& cp, int ptask, int nP, const int32_t* __restrict__ uid_at_pos,
                          const int64_t* __restrict__ offsets, PlanHeader* hdr,
                          const float* __restrict__ rowbuf, float* __restrict__ out, int32_t* status,
-                         int* s_flag)
+                         int* s_flag, unsigned long long* wait_ns)
 {
     constexpr int D = S::D, LB = D / 4, BPW = 32 / LB;
     // row gathers in flight per lane: 16 below rank 64; at rank 64 the kernel's register budget
@@ -685,7 +676,8 @@ __device__ void fwd_pool(const CoreParams& cp, int ptask, int nP, const int32_t*
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     TT_PH_START();
     if (tid == 0) {
-        // injected failure (test hook): wait for one chunk more than the table has
+        // injected failure (test hook): wait for one subtask more than the table has
+        const unsigned long long w0 = cp.probe ? global_ns() : 0ull;
         const int want = hdr->nC[t] + (cp.inj_pool ? 1 : 0);
         const int limit = cp.inj_spin > 0 ? cp.inj_spin : kSpinLimit;
         int it = 0, ok = 1;
@@ -703,6 +695,7 @@ __device__ void fwd_pool(const CoreParams& cp, int ptask, int nP, const int32_t*
         }
         __threadfence();
         s_flag[0] = ok;
+        if (cp.probe) *wait_ns += global_ns() - w0;
     }
     __syncthreads();
     TT_PH(4);
@@ -739,22 +732,125 @@ __device__ void fwd_pool(const CoreParams& cp, int ptask, int nP, const int32_t*
     TT_PH(5);
 }
 
-// Persistent forward.  Software pipeline per chunk: wait for its A/B copies,
-// GEMM, then fetch the next task and, if it is a chunk, prefetch its
-// metadata and A/B rows (As and Bs are free once the GEMM is done) while this
-// chunk's distinct rows are contracted batch by batch (double-buffered last
-// slices when shared memory allows).
+// ---------------------------------------------------------------------------
+// Forward scheduler (FlowTT section 3.4).  Subtasks (row ranges of chunks, in column order)
+// are split into one contiguous owner range per persistent block.  A block takes its own
+// subtasks front to back; in the stealing modes it then takes subtasks of other blocks that
+// have not started, from the back of their ranges (so a thief and the owner meet in the middle
+// and each subtask is claimed exactly once), and finally pooling tasks from a shared queue.
+// Thread 0 only.  Returns a subtask index, -2 - p for pooling task p, or -1 when done.
+// ---------------------------------------------------------------------------
+struct FwdSched {
+    const int4* subs;
+    int32_t* claim;
+    int32_t* own_head;
+    int32_t* steal_tail;
+    int32_t* exhausted;
+    int32_t* slot_flag;
+    float* ckpt;
+};
+
+__device__ __forceinline__ int fwd_next(const FwdSched& fs, PlanHeader* hdr, int sched, int S, int npool, int& phase,
+                                        int& vk)
+{
+    const int G = (int)gridDim.x, b = (int)blockIdx.x;
+    if (phase == 0) {
+        const int h = atomicAdd(&fs.own_head[b], 1);
+        if (h < owner_start(S, b + 1, G) && atomicExch(&fs.claim[h], 1) == 0) return h;
+        phase = sched == TT_SCHED_STATIC ? 2 : 1;
+        vk = 1;
+    }
+    if (phase == 1) {
+        while (vk < G) {
+            const int v = b + vk < G ? b + vk : b + vk - G;
+            if (*reinterpret_cast<volatile int*>(&fs.exhausted[v]) == 0) {
+                const int t = atomicSub(&fs.steal_tail[v], 1) - 1;
+                if (t >= owner_start(S, v, G) && atomicExch(&fs.claim[t], 1) == 0) return t;   // again from v next time
+                *reinterpret_cast<volatile int*>(&fs.exhausted[v]) = 1;
+            }
+            ++vk;
+        }
+        phase = 2;
+    }
+    const int p = atomicAdd(&hdr->pool_head, 1);
+    return p < npool ? -2 - p : -1;
+}
+
+// L2 checkpoint of a split chunk's C tile (TT_SCHED_STEAL_L2; FlowTT section 3.2 / 3.4: shared
+// intermediates kept in L2 for reuse between blocks).  Flag protocol per slot: 0 empty, 1 being
+// written (the block that won the compare-and-swap), 2 ready (release after a device fence).
+constexpr int kCkptPolls = 64;   // bounded wait for a slot another block is writing; then recompute
+
+__device__ __forceinline__ int ld_acquire(const int32_t* p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release(int32_t* p, int v)
+{
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t l2_evict_last_policy()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ void st_v4_hint(float* p, float4 v, uint64_t pol)
+{
+    asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(v.x), "f"(v.y),
+                 "f"(v.z), "f"(v.w), "l"(pol)
+                 : "memory");
+}
+
+// Thread 0: 1 when slot `slot` holds a ready C tile (waiting a bounded number of polls while
+// another block writes it), else 0.
+__device__ __forceinline__ int ckpt_ready(const FwdSched& fs, int slot)
+{
+    int f = ld_acquire(&fs.slot_flag[slot]);
+    for (int it = 0; f == 1 && it < kCkptPolls; ++it) {
+        __nanosleep(200);
+        f = ld_acquire(&fs.slot_flag[slot]);
+    }
+    return f == 2;
+}
+
+// All threads: the tile (MF x N floats, the shared-memory layout as is) from / to the slot.
+template <class S>
+__device__ __forceinline__ void ckpt_load(const FwdSched& fs, int slot, float* Cn)
+{
+    static_assert(S::MF * S::N == kCkptFloats, "checkpoint slot holds one C tile");
+    const float4* src = reinterpret_cast<const float4*>(fs.ckpt + (size_t)slot * (S::MF * S::N));
+    float4* dst = reinterpret_cast<float4*>(Cn);
+    for (int q = threadIdx.x; q < S::MF * S::N / 4; q += kFwdThreads) dst[q] = __ldcg(src + q);
+}
+template <class S>
+__device__ __forceinline__ void ckpt_store(const FwdSched& fs, int slot, const float* Cn)
+{
+    static_assert(S::MF * S::N == kCkptFloats, "checkpoint slot holds one C tile");
+    float4* dst = reinterpret_cast<float4*>(fs.ckpt + (size_t)slot * (S::MF * S::N));
+    const float4* src = reinterpret_cast<const float4*>(Cn);
+    const uint64_t pol = l2_evict_last_policy();
+    for (int q = threadIdx.x; q < S::MF * S::N / 4; q += kFwdThreads) st_v4_hint(reinterpret_cast<float*>(dst + q), src[q], pol);
+}
+
+// Persistent forward.  Software pipeline per subtask: wait for its A/B copies (none when the
+// previous subtask was of the same chunk: its C is still in shared memory), the chunk's C
+// (GEMM, or the L2 checkpoint a block published), then fetch the next task and, if it is a
+// subtask, prefetch its metadata and A/B rows while this subtask's distinct rows are contracted
+// batch by batch (double-buffered last slices when shared memory allows).
 template <class S, typename K, int NT>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
               const int4* __restrict__ grec, const int32_t* __restrict__ uid_at_pos,
               const int64_t* __restrict__ offsets, const int4* __restrict__ chunks,
-              const int32_t* __restrict__ tasks, PlanHeader* hdr,
+              FwdSched fs, PlanHeader* hdr,
               float* __restrict__ rowbuf, float* __restrict__ out, int32_t* status)
 {
     extern __shared__ __align__(16) float smem_f[];
     __shared__ FwdMeta<S> M;
-    __shared__ __align__(16) K s_keys[2 * kKeyCap];   // keys of each chunk buffer's first rows
+    __shared__ __align__(16) K s_keys[2 * kKeyCap];   // keys of each buffer's distinct rows
     __shared__ __align__(8) uint64_t s_mbar;
     __shared__ uint32_t s_tmem;
     __shared__ int s_ok;
@@ -763,6 +859,9 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
     constexpr int NS = NT == 3 ? 2 : 1;   // bf16 terms stored per operand element
     FwdSmem<S> sm;
     const int tid = threadIdx.x;
+    const unsigned long long pr_t0 = cp.probe ? global_ns() : 0ull;
+    unsigned long long pr_wait = 0;
+    int pr_tasks = 0;
     uint32_t tmem = 0, parity = 0;
     if constexpr (TC) {
         // one bf16 term takes half the room of an fp32 operand, two terms the same room
@@ -783,93 +882,127 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
         sm.Cn = sm.As + S::MF * S::R;
     }
     sm.Ss = sm.Cn + S::MF * S::N;
-    const int ntasks = hdr->ntasks, nP = hdr->nP;
-    int iter = 0;
-    int cur_t = -1, cur_i2 = -1;   // column of the B now in (or on its way to) Bs
+    const int nS = hdr->nsub, nP = hdr->nP, npool = cp.T * nP;
+    const bool use_ckpt = sched == TT_SCHED_STEAL_L2;
+    int phase = 0, vk = 1;   // scheduler state (thread 0)
+    int cur_t = -1, cur_i2 = -1;   // column of the B now in (or on its way to) the B tile
+    int cur_cid = -1;              // chunk whose C tile is in shared memory
     int mb = 0;
     bool staged = false;
-    if (tid == 0) M.task[0] = next_task(sched, &hdr->queue_head, iter);
-    ++iter;
+    if (tid == 0) M.task[0] = fwd_next(fs, hdr, sched, nS, npool, phase, vk);
     __syncthreads();
     int q = M.task[0];
-    while (q < ntasks) {
-        const int tv = tasks[q];
-        if (tv < 0) {
-            fwd_pool<S>(cp, -1 - tv, nP, uid_at_pos, offsets, hdr, rowbuf, out, status, &M.flag);
+    while (q != -1) {
+        if (q <= -2) {
+            fwd_pool<S>(cp, -2 - q, nP, uid_at_pos, offsets, hdr, rowbuf, out, status, &M.flag, &pr_wait);
+            ++pr_tasks;
             __syncthreads();
-            if (tid == 0) M.task[0] = next_task(sched, &hdr->queue_head, iter);
-            ++iter;
+            if (tid == 0) M.task[0] = fwd_next(fs, hdr, sched, nS, npool, phase, vk);
             __syncthreads();
             q = M.task[0];
             staged = false;
             continue;
         }
         TT_PH_START();
+        ++pr_tasks;
         if (!staged) {
-            fwd_meta<S, K>(cp, tv, mb, uniq_keys, grec, chunks, M, s_keys);
-            if constexpr (TC) fwd_issue_ab_tc<S, NS>(cp, mb, M, sm, cur_t, cur_i2);
-            else fwd_issue_ab<S>(cp, mb, M, sm, cur_t, cur_i2);
-        }
-        if (tid == 0) M.task[1] = next_task(sched, &hdr->queue_head, iter);   // result used after the GEMM
-        ++iter;
-        cp_async_wait_all();   // the chunk's A/B rows and row keys (usually prefetched long ago)
-        __syncthreads();
-        const int total = M.ucum[mb][S::MPF];
-        build_rows(M.rows, mb, M.ucum[mb], M.u0[mb], M.cnt[mb], total, s_keys, cp.ibits, cp.n[M.t[mb]][2],
-                   kFwdThreads);
-        __syncthreads();
-        // the first batch of last slices is in flight during the GEMM
-        if (total > 0) fwd_issue_batch<S, K>(cp, mb, 0, 0, uniq_keys, M, sm, s_keys);
-        TT_PH(0);
-        if constexpr (TC) {
-            if (!fwd_gemm_tc<S, NT>(sm, tmem, &s_mbar, parity, &s_ok, cp.inj_mma != 0)) {
-                if (tid == 0) raise_error(status, TT_ERR_TIMEOUT, 100);
-                break;
+            const int4 sub = fs.subs[q];
+            fwd_meta<S, K>(cp, sub, mb, uniq_keys, grec, chunks, M, s_keys);
+            if (sub.x != cur_cid) {
+                if constexpr (TC) fwd_issue_ab_tc<S, NS>(cp, mb, M, sm, cur_t, cur_i2);
+                else fwd_issue_ab<S>(cp, mb, M, sm, cur_t, cur_i2);
+            } else {
+                cp_async_commit();   // the row keys alone
             }
-        } else {
-            fwd_gemm<S>(sm);
+        }
+        if (tid == 0) M.task[1] = fwd_next(fs, hdr, sched, nS, npool, phase, vk);   // used after the C step
+        cp_async_wait_all();   // the subtask's A/B rows and row keys (usually prefetched long ago)
+        __syncthreads();
+        const int nrows = M.re[mb] - M.rb[mb];
+        build_rows(M.rows, mb, M.ucum[mb], M.u0[mb], M.cnt[mb], M.re[mb], s_keys, cp.ibits, cp.n[M.t[mb]][2],
+                   kFwdThreads, M.rb[mb]);
+        __syncthreads();
+        // the first batch of last slices is in flight during the C step
+        if (nrows > 0) fwd_issue_batch<S>(cp, mb, 0, 0, M, sm);
+        TT_PH(0);
+        const int cid = M.cid[mb], slot = M.slot[mb];
+        if (cid != cur_cid) {
+            // C of this chunk: the checkpoint when another block has published it, else the GEMM
+            if (tid == 0) M.ck = (use_ckpt && slot >= 0) ? ckpt_ready(fs, slot) : 0;
+            __syncthreads();
+            if (M.ck) {
+                ckpt_load<S>(fs, slot, sm.Cn);
+            } else {
+                if constexpr (TC) {
+                    if (!fwd_gemm_tc<S, NT>(sm, tmem, &s_mbar, parity, &s_ok, cp.inj_mma != 0)) {
+                        if (tid == 0) raise_error(status, TT_ERR_TIMEOUT, 100);
+                        break;
+                    }
+                } else {
+                    fwd_gemm<S>(sm);
+                }
+                if (use_ckpt && slot >= 0) {   // publish once: the block that wins the slot writes it
+                    __syncthreads();
+                    if (tid == 0) M.ck = atomicCAS(&fs.slot_flag[slot], 0, 1) == 0;
+                    __syncthreads();
+                    if (M.ck) {
+                        ckpt_store<S>(fs, slot, sm.Cn);
+                        __syncthreads();
+                        if (tid == 0) {
+                            __threadfence();
+                            st_release(&fs.slot_flag[slot], 2);
+                        }
+                    }
+                }
+            }
+            cur_cid = cid;
         }
         __syncthreads();
         TT_PH(1);
         const int qn = M.task[1];
-        const bool next_chunk = qn < ntasks && tasks[qn] >= 0;
-        if (next_chunk) {
-            fwd_meta<S, K>(cp, tasks[qn], mb ^ 1, uniq_keys, grec, chunks, M, s_keys);
-            if constexpr (TC) fwd_issue_ab_tc<S, NS>(cp, mb ^ 1, M, sm, cur_t, cur_i2);
-            else fwd_issue_ab<S>(cp, mb ^ 1, M, sm, cur_t, cur_i2);
+        const bool next_sub = qn >= 0;
+        if (next_sub) {
+            const int4 nsub = fs.subs[qn];
+            fwd_meta<S, K>(cp, nsub, mb ^ 1, uniq_keys, grec, chunks, M, s_keys);
+            if (nsub.x != cur_cid) {
+                if constexpr (TC) fwd_issue_ab_tc<S, NS>(cp, mb ^ 1, M, sm, cur_t, cur_i2);
+                else fwd_issue_ab<S>(cp, mb ^ 1, M, sm, cur_t, cur_i2);
+            } else {
+                cp_async_commit();
+            }
         }
-        // distinct rows of this chunk, in batches of NUF (commit groups in flight: the batch,
-        // then possibly the next chunk's A/B, then possibly the next batch)
+        // distinct rows of this subtask, in batches of NUF (commit groups in flight: the batch,
+        // then possibly the next subtask's A/B, then possibly the next batch)
         if (S::FBUF == 2) {
-            for (int k0 = 0, b = 0; k0 < total; k0 += S::NUF, b ^= 1) {
-                const bool more = k0 + S::NUF < total;
+            for (int i0 = 0, b = 0; i0 < nrows; i0 += S::NUF, b ^= 1) {
+                const bool more = i0 + S::NUF < nrows;
                 if (more) {
-                    fwd_issue_batch<S, K>(cp, mb, k0 + S::NUF, b ^ 1, uniq_keys, M, sm, s_keys);
+                    fwd_issue_batch<S>(cp, mb, i0 + S::NUF, b ^ 1, M, sm);
                     cp_async_wait<1>();
-                } else if (k0 == 0 && next_chunk) {
+                } else if (i0 == 0 && next_sub) {
                     cp_async_wait<1>();
                 } else {
                     cp_async_wait_all();
                 }
                 __syncthreads();
                 TT_PH(2);
-                fwd_batch_compute<S>(mb, k0, min(S::NUF, total - k0), b, M, sm, rowbuf);
+                fwd_batch_compute<S>(mb, i0, min(S::NUF, nrows - i0), b, M, sm, rowbuf);
                 __syncthreads();
                 TT_PH(3);
             }
         } else {
-            for (int k0 = 0; k0 < total; k0 += S::NUF) {
-                if (k0 > 0) fwd_issue_batch<S, K>(cp, mb, k0, 0, uniq_keys, M, sm, s_keys);
-                if (k0 == 0 && next_chunk) cp_async_wait<1>();
+            for (int i0 = 0; i0 < nrows; i0 += S::NUF) {
+                if (i0 > 0) fwd_issue_batch<S>(cp, mb, i0, 0, M, sm);
+                if (i0 == 0 && next_sub) cp_async_wait<1>();
                 else cp_async_wait_all();
                 __syncthreads();
                 TT_PH(2);
-                fwd_batch_compute<S>(mb, k0, min(S::NUF, total - k0), 0, M, sm, rowbuf);
+                fwd_batch_compute<S>(mb, i0, min(S::NUF, nrows - i0), 0, M, sm, rowbuf);
                 __syncthreads();
                 TT_PH(3);
             }
         }
-        // publish the chunk's rows: the barrier orders every thread's row stores before thread
+        // publish the subtask's rows: the barrier orders every thread's row stores before thread
         // 0's device-scope fence (cumulative), which precedes the counter increment
         __syncthreads();
         if (tid == 0) {
@@ -877,8 +1010,8 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
             atomicAdd(&hdr->done[M.t[mb]], 1);
         }
         q = qn;
-        staged = next_chunk;
-        if (next_chunk) mb ^= 1;
+        staged = next_sub;
+        if (next_sub) mb ^= 1;
     }
     cp_async_wait_all();
     if constexpr (TC) {
@@ -889,6 +1022,7 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
             tmem_dealloc(tmem, (uint32_t)S::N);
         }
     }
+    probe_write(cp, pr_t0, pr_tasks, pr_wait);
 }
 
 // ---------------------------------------------------------------------------
@@ -1250,8 +1384,8 @@ template <class S, typename K>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ uniq_keys,
               const int4* __restrict__ grec, const int32_t* __restrict__ col_count,
-              const int32_t* __restrict__ col_start, PlanHeader* hdr, const float* __restrict__ rowbuf,
-              int32_t* status)
+              const int32_t* __restrict__ col_start, const int32_t* __restrict__ col_order, PlanHeader* hdr,
+              const float* __restrict__ rowbuf, int32_t* status)
 {
     constexpr int R = S::R, N = S::N, MB = S::MB, MPB = S::MPB, D1 = S::D1, D2 = S::D2, D3 = S::D3,
                   P = S::P, NUB = S::NUB, DBR = S::DBR, DBC = S::DBC, SR = S::SR;
@@ -1271,11 +1405,15 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
     if (has_error(status)) return;
     const int tid = threadIdx.x;
 
+    const unsigned long long pr_t0 = cp.probe ? global_ns() : 0ull;
+    int pr_tasks = 0;
+    const int ncols_busy = hdr->ncols_busy;   // the column queue (see k_plan_order)
     for (int iter = 0;; ++iter) {
         if (tid == 0) M.task = next_task(pp.sched, &hdr->col_head, iter);
         __syncthreads();
-        const int c = M.task;
-        if (c >= pp.ncols) break;
+        if (M.task >= ncols_busy) break;
+        const int c = col_order[M.task];
+        ++pr_tasks;
         const int ccount = col_count[c];
         if (ccount == 0) {
             __syncthreads();
@@ -1595,6 +1733,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
         TT_PH(15);
     }
     cp_async_wait_all();
+    probe_write(cp, pr_t0, pr_tasks, 0ull);
 }
 
 // ---------------------------------------------------------------------------
@@ -1731,12 +1870,21 @@ __device__ __forceinline__ void warp_row_load2(const CoreParams& cp, int t, int 
     w.h = __ldg(reinterpret_cast<const float4*>(rowbuf + (int64_t)w.u * D) + lane);
 }
 
-// the chunk's distinct rows by quads of warps (see above); tmem_c = the C^T accumulators
+__device__ __forceinline__ void named_bar(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// the chunk's distinct rows by quads of warps (see above); tmem_c = the C^T accumulators.
+// Warps s and s + 2 of a quad hold the same rho_2 and complementary a_2, so each has half of
+// dS_u[rho][.]: the second passes its half through shared memory (pslots, double-buffered by
+// row parity, one named barrier per row and pair) and the first issues the reductions, one
+// per (rho, row) instead of two.
 template <typename K>
 __device__ __forceinline__ void bwd2_rows(const CoreParams& cp, int t, int mb, int total, int cnt, const BwdMeta2& M,
                                           const K* __restrict__ uniq_keys, const float* __restrict__ rowbuf,
                                           uint32_t tmem_c, float* dCn, float* __restrict__ dG3, uint32_t n3,
-                                          float* hslots)
+                                          float* hslots, float* pslots)
 {
     constexpr int R = 64, N = 256, D1 = 4, D2 = 4, D3 = 8, P = 16, MB = kMB2, NQ = kBwdThreadsTC / 128;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, sub = warp & 3, quad = warp >> 2;
@@ -1745,6 +1893,8 @@ __device__ __forceinline__ void bwd2_rows(const CoreParams& cp, int t, int mb, i
     if (lo >= hi) return;
     const uint32_t tl = tmem_c + ((uint32_t)(32 * sub) << 16);
     float* hs = hslots + warp * 2 * P * D3;
+    const int pair = quad * 2 + (sub & 1);            // named barrier 1 + pair (0 is __syncthreads)
+    float* ps = pslots + pair * (2 * 32 * 8) + lane * 8;
     WarpRow1 a, b;
     warp_row_load2<K>(cp, t, mb, lo, cnt, rho, M, uniq_keys, rowbuf, n3, a);
     if (lo + 1 < hi) warp_row_load2<K>(cp, t, mb, lo + 1, cnt, rho, M, uniq_keys, rowbuf, n3, b);
@@ -1798,9 +1948,19 @@ __device__ __forceinline__ void bwd2_rows(const CoreParams& cp, int t, int mb, i
             }
             o[i] = acc;
         }
-        float* dst = dG3 + ((int64_t)w.i3 * R + rho) * D3;
-        red_add_v4(dst, make_float4(ds[0], ds[1], ds[2], ds[3]));
-        red_add_v4(dst + 4, make_float4(ds[4], ds[5], ds[6], ds[7]));
+        float* slot = ps + (kq & 1) * (32 * 8);
+        if (sub >= 2) {
+            reinterpret_cast<float4*>(slot)[0] = make_float4(ds[0], ds[1], ds[2], ds[3]);
+            reinterpret_cast<float4*>(slot)[1] = make_float4(ds[4], ds[5], ds[6], ds[7]);
+        }
+        named_bar(1 + pair, 64);
+        if (sub < 2) {
+            const float4 p0 = reinterpret_cast<const float4*>(slot)[0];
+            const float4 p1 = reinterpret_cast<const float4*>(slot)[1];
+            float* dst = dG3 + ((int64_t)w.i3 * R + rho) * D3;
+            red_add_v4(dst, make_float4(ds[0] + p0.x, ds[1] + p0.y, ds[2] + p0.z, ds[3] + p0.w));
+            red_add_v4(dst + 4, make_float4(ds[4] + p1.x, ds[5] + p1.y, ds[6] + p1.z, ds[7] + p1.w));
+        }
     }
     flush();
 }
@@ -1809,8 +1969,8 @@ template <typename K, int NT>
 __global__ void __launch_bounds__(kBwdThreadsTC, 1)
 k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ uniq_keys,
                   const int4* __restrict__ grec, const int32_t* __restrict__ col_count,
-                  const int32_t* __restrict__ col_start, PlanHeader* hdr, const float* __restrict__ rowbuf,
-                  int32_t* status)
+                  const int32_t* __restrict__ col_start, const int32_t* __restrict__ col_order, PlanHeader* hdr,
+                  const float* __restrict__ rowbuf, int32_t* status)
 {
     constexpr int R = 64, N = 256, D1 = 4, MPB = kMPB2, MB = kMB2, BT = kBwdThreadsTC;
     constexpr int NS = NT == 3 ? 2 : 1;
@@ -1830,6 +1990,7 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
     float* dCn = reinterpret_cast<float*>(Abt + 2 * NS * MB * R);   // [MB][N] swizzled; then NS x (MB x N) bf16
     uint16_t* dCb = reinterpret_cast<uint16_t*>(dCn);
     float* hslots = dCn + MB * N;                                   // [warps][2][P D3]
+    float* pslots = hslots + (BT / 32) * 2 * 128;                   // [warp pairs][2][32][8] dS halves
     if (has_error(status)) return;
     const int tid = threadIdx.x;
     uint32_t parity = 0;
@@ -1844,11 +2005,15 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
     tc_fence_after();
     const uint32_t tmem = s_tmem;
 
+    const unsigned long long pr_t0 = cp.probe ? global_ns() : 0ull;
+    int pr_tasks = 0;
+    const int ncols_busy = hdr->ncols_busy;   // the column queue (see k_plan_order)
     for (int iter = 0;; ++iter) {
         if (tid == 0) M.task = next_task(pp.sched, &hdr->col_head, iter);
         __syncthreads();
-        const int c = M.task;
-        if (c >= pp.ncols) break;
+        if (M.task >= ncols_busy) break;
+        const int c = col_order[M.task];
+        ++pr_tasks;
         const int ccount = col_count[c];
         if (ccount == 0) {
             __syncthreads();
@@ -1944,7 +2109,8 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
             }
             TT_PH(16);
 
-            bwd2_rows<K>(cp, t, mb, total, cnt, M, uniq_keys, rowbuf, tmem + (uint32_t)N, dCn, dG3, n3, hslots);
+            bwd2_rows<K>(cp, t, mb, total, cnt, M, uniq_keys, rowbuf, tmem + (uint32_t)N, dCn, dG3, n3, hslots,
+                         pslots);
             tc_fence_before();
             __syncthreads();
             TT_PH(12);
@@ -2052,6 +2218,7 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
         tc_fence_after();
         tmem_dealloc(tmem, 2 * N);
     }
+    probe_write(cp, pr_t0, pr_tasks, 0ull);
 }
 
 // ---------------------------------------------------------------------------
@@ -2170,9 +2337,11 @@ cudaError_t fwd_launch(const K3Args& a, float* out, cudaStream_t s, int* nl)
     cudaError_t e = cudaFuncSetAttribute(k3_fwd_kernel<S, K, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const PlanBuffers& pb = *a.pb;
+    if (a.grid != a.pp->grid || a.grid > kMaxGrid) return cudaErrorInvalidConfiguration;
+    const FwdSched fs{pb.subs, pb.claim, pb.own_head, pb.steal_tail, pb.exhausted, pb.slot_flag, pb.ckpt};
     k3_fwd_kernel<S, K, NT><<<a.grid, kFwdThreads, smem, s>>>(
         *a.cp, a.pp->sched, (const K*)a.uniq_keys, a.grec, a.uid_at_pos, a.offsets,
-        pb.chunks, pb.tasks, pb.hdr, a.rowbuf, out, a.status);
+        pb.chunks, fs, pb.hdr, a.rowbuf, out, a.status);
     *nl += 1;
     return cudaGetLastError();
 }
@@ -2199,8 +2368,8 @@ cudaError_t bwd_launch(const K3Args& a, const GradPtrs& gp, const float* grad_ou
     if (e != cudaSuccess) return e;
     const PlanBuffers& pb = *a.pb;
     k3_bwd_kernel<S, K><<<a.grid, kBwdThreads, smem, s>>>(
-        *a.cp, gp, *a.pp, (const K*)a.uniq_keys, a.grec, pb.col_count, pb.col_start, pb.hdr, a.rowbuf,
-        a.status);
+        *a.cp, gp, *a.pp, (const K*)a.uniq_keys, a.grec, pb.col_count, pb.col_start, pb.col_order, pb.hdr,
+        a.rowbuf, a.status);
     *nl += 1;
     return cudaGetLastError();
 }
@@ -2227,7 +2396,8 @@ template <int NT>
 constexpr size_t bwd2_smem_bytes()
 {
     constexpr size_t NS = NT == 3 ? 2 : 1;
-    return NS * 64 * 256 * 2 + 2 * NS * kMB2 * 64 * 2 + (size_t)kMB2 * 256 * 4 + (kBwdThreadsTC / 32) * 2 * 128 * 4;
+    return NS * 64 * 256 * 2 + 2 * NS * kMB2 * 64 * 2 + (size_t)kMB2 * 256 * 4 + (kBwdThreadsTC / 32) * 2 * 128 * 4 +
+           (kBwdThreadsTC / 64) * 2 * 32 * 8 * 4;
 }
 
 template <typename K, int NT>
@@ -2238,7 +2408,8 @@ cudaError_t bwd2_launch(const K3Args& a, const GradPtrs& gp, cudaStream_t s, int
     if (e != cudaSuccess) return e;
     const PlanBuffers& pb = *a.pb;
     k3_bwd_tc2_kernel<K, NT><<<a.grid, kBwdThreadsTC, smem, s>>>(
-        *a.cp, gp, *a.pp, (const K*)a.uniq_keys, a.grec, pb.col_count, pb.col_start, pb.hdr, a.rowbuf, a.status);
+        *a.cp, gp, *a.pp, (const K*)a.uniq_keys, a.grec, pb.col_count, pb.col_start, pb.col_order, pb.hdr,
+        a.rowbuf, a.status);
     *nl += 1;
     return cudaGetLastError();
 }

@@ -11,11 +11,14 @@
 //   2. stable-sorts the groups by column (so each column's groups stay in
 //      canonical order and results do not depend on the schedule),
 //   3. scans the column counts into column starts and chunk bases,
-//   4. writes one record per chunk (at most MP groups of one column) and the
-//      task queue: compute chunks and pooling tasks, table-major, with each
-//      table's pooling placed after the next table's compute chunks so the
-//      pooled rows are still in L2 when they are gathered (TT_SCHED_STEAL_L2),
-//      or all pooling after all compute (other modes).
+//   4. writes one record per chunk (at most MP groups of one column) with its
+//      distinct-row total,
+//   5. splits chunks of more than kSplitRows distinct rows into row-range
+//      subtasks (the stealing granule of FlowTT section 3.4), numbers the
+//      split chunks' checkpoint slots (TT_SCHED_STEAL_L2), and gives every
+//      persistent block of the forward an owner range: an equal share of the
+//      subtasks, contiguous in column order (the static prefix mapping the
+//      pages start from).  Pooling tasks (NB bags of one table) follow.
 #include "tt_common.cuh"
 
 namespace tt {
@@ -43,6 +46,7 @@ __global__ void __launch_bounds__(256) k_plan_keys(PlanParams pp, const K* __res
                                                    uint32_t* __restrict__ pkeys,
                                                    int32_t* __restrict__ pvals,
                                                    int32_t* __restrict__ col_count,
+                                                   int32_t* __restrict__ col_rows,
                                                    const int32_t* status)
 {
     if (has_error(status)) return;
@@ -51,11 +55,52 @@ __global__ void __launch_bounds__(256) k_plan_keys(PlanParams pp, const K* __res
          g += (int64_t)gridDim.x * blockDim.x) {
         int t;
         uint32_t ic, i1;
-        group_col(pp, (uint64_t)uniq_keys[grp_start[g]], &t, &ic, &i1);
+        const int u0 = grp_start[g];
+        group_col(pp, (uint64_t)uniq_keys[u0], &t, &ic, &i1);
         const uint32_t col = (uint32_t)pp.col_base[t] + ic;
         pkeys[g] = col;
         pvals[g] = (int32_t)g;
         atomicAdd(&col_count[col], 1);
+        atomicAdd(&col_rows[col], grp_start[g + 1] - u0);
+    }
+}
+
+// One block: the backward's column queue.  TT_SCHED_STATIC: every column in index order (the
+// static round robin of the backward).  Stealing modes: the non-empty columns, costliest
+// first (cost ~ distinct rows + 4 x prefix groups, bucketed by its power of two), so the
+// dynamic queue hands out the long column groups before the short ones.
+__global__ void __launch_bounds__(1024) k_plan_order(PlanParams pp, const int32_t* __restrict__ col_count,
+                                                    const int32_t* __restrict__ col_rows,
+                                                    int32_t* __restrict__ col_order, PlanHeader* __restrict__ hdr,
+                                                    const int32_t* status)
+{
+    __shared__ int32_t s_hist[32], s_pos[32];
+    if (has_error(status)) return;
+    const int tid = threadIdx.x;
+    if (pp.sched == TT_SCHED_STATIC) {
+        for (int c = tid; c < pp.ncols; c += 1024) col_order[c] = c;
+        if (tid == 0) hdr->ncols_busy = pp.ncols;
+        return;
+    }
+    if (tid < 32) s_hist[tid] = 0;
+    __syncthreads();
+    for (int c = tid; c < pp.ncols; c += 1024) {
+        const int cost = col_rows[c] + 4 * col_count[c];
+        if (cost > 0) atomicAdd(&s_hist[31 - __clz(cost)], 1);
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int run = 0;
+        for (int b = 31; b >= 0; --b) {
+            s_pos[b] = run;
+            run += s_hist[b];
+        }
+        hdr->ncols_busy = run;
+    }
+    __syncthreads();
+    for (int c = tid; c < pp.ncols; c += 1024) {
+        const int cost = col_rows[c] + 4 * col_count[c];
+        if (cost > 0) col_order[atomicAdd(&s_pos[31 - __clz(cost)], 1)] = c;
     }
 }
 
@@ -115,33 +160,9 @@ __global__ void __launch_bounds__(1024) k_plan_cols(PlanParams pp,
     if (threadIdx.x == 0) {
         col_start[pp.ncols] = s_carry[0];
         chunk_base[pp.ncols] = s_carry[1];
-        const int nP = (int)((pp.B + pp.NB - 1) / pp.NB);
-        int q = 0;
-        // task layout: C(t) chunks, then (interleaved mode) P(t-1) after C(t)
-        for (int t = 0; t < pp.T; ++t) {
-            const int c0 = chunk_base[pp.col_base[t]], c1 = chunk_base[pp.col_base[t + 1]];
-            hdr->chunk_first[t] = c0;
-            hdr->nC[t] = c1 - c0;
-            hdr->task_base_C[t] = q;
-            q += c1 - c0;
-            if (pp.sched == TT_SCHED_STEAL_L2 && t >= 1) {
-                hdr->task_base_P[t - 1] = q;
-                q += nP;
-            }
-        }
-        if (pp.sched == TT_SCHED_STEAL_L2) {
-            hdr->task_base_P[pp.T - 1] = q;
-            q += nP;
-        } else {
-            for (int t = 0; t < pp.T; ++t) {
-                hdr->task_base_P[t] = q;
-                q += nP;
-            }
-        }
-        hdr->nP = nP;
-        hdr->ntasks = q;
+        hdr->nP = (int)((pp.B + pp.NB - 1) / pp.NB);
         hdr->nchunks = s_carry[1];
-        hdr->queue_head = 0;
+        hdr->pool_head = 0;
         hdr->col_head = 0;
     }
     if (threadIdx.x < pp.T) hdr->done[threadIdx.x] = 0;
@@ -152,9 +173,8 @@ __global__ void __launch_bounds__(256) k_plan_chunks(PlanParams pp, const WsCoun
                                                      const int32_t* __restrict__ col_count,
                                                      const int32_t* __restrict__ col_start,
                                                      const int32_t* __restrict__ chunk_base,
-                                                     const PlanHeader* __restrict__ hdr,
-                                                     int4* __restrict__ chunks,
-                                                     int32_t* __restrict__ tasks,
+                                                     const int4* __restrict__ grec,
+                                                     int4* __restrict__ chunks, int32_t* __restrict__ crow,
                                                      const int32_t* status)
 {
     if (has_error(status)) return;
@@ -169,13 +189,102 @@ __global__ void __launch_bounds__(256) k_plan_chunks(PlanParams pp, const WsCoun
         while (t + 1 < pp.T && (uint32_t)pp.col_base[t + 1] <= c) ++t;
         const int cid = chunk_base[c] + r / pp.MP;
         const int cnt = min(pp.MP, col_count[c] - r);
+        int rows = 0;
+        for (int q = 0; q < cnt; ++q) rows += grec[i + q].y;
         chunks[cid] = make_int4((int)i, cnt, t, (int)(c - (uint32_t)pp.col_base[t]));
-        tasks[hdr->task_base_C[t] + (cid - hdr->chunk_first[t])] = cid;
+        crow[cid] = rows;
     }
-    const int nP = hdr->nP;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)pp.T * nP; i += stride) {
-        const int t = (int)(i / nP), j = (int)(i % nP);
-        tasks[hdr->task_base_P[t] + j] = -1 - (t * nP + j);
+}
+
+
+// One block: subtask bases and checkpoint slots of every chunk (an exclusive scan of the
+// subtask counts and of the split flags), subtasks per table, and the owner ranges.
+__global__ void __launch_bounds__(1024) k_plan_split(PlanParams pp, const int32_t* __restrict__ crow,
+                                                    const int32_t* __restrict__ chunk_base,
+                                                    int32_t* __restrict__ sub_base, int32_t* __restrict__ slot_of,
+                                                    PlanHeader* __restrict__ hdr, int32_t* __restrict__ own_head,
+                                                    int32_t* __restrict__ steal_tail,
+                                                    int32_t* __restrict__ exhausted, const int32_t* status)
+{
+    __shared__ int32_t s_w[2][32];
+    if (has_error(status)) return;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int nch = hdr->nchunks;
+    const int per = (nch + 1023) / 1024;
+    const int lo = min(nch, tid * per), hi = min(nch, lo + per);
+    int ns = 0, np = 0;
+    for (int c = lo; c < hi; ++c) {
+        const int k = subtasks_of(crow[c]);
+        ns += k;
+        np += k > 1;
+    }
+    int x[2] = {ns, np};
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, x[q], o);
+            if (lane >= o) x[q] += y;
+        }
+        if (lane == 31) s_w[q][wid] = x[q];
+    }
+    __syncthreads();
+    if (wid == 0) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            int w = s_w[q][lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(kFull, w, o);
+                if (lane >= o) w += y;
+            }
+            s_w[q][lane] = w;
+        }
+    }
+    __syncthreads();
+    int rs = (wid ? s_w[0][wid - 1] : 0) + x[0] - ns;
+    int rp = (wid ? s_w[1][wid - 1] : 0) + x[1] - np;
+    const bool ckpt = pp.sched == TT_SCHED_STEAL_L2;
+    for (int c = lo; c < hi; ++c) {
+        const int k = subtasks_of(crow[c]);
+        sub_base[c] = rs;
+        slot_of[c] = (ckpt && k > 1 && rp < pp.slot_cap) ? rp : -1;
+        rs += k;
+        rp += k > 1;
+    }
+    const int S = s_w[0][31];
+    if (tid == 0) {
+        sub_base[nch] = S;
+        hdr->nsub = S;
+        hdr->nslots = ckpt ? min(s_w[1][31], pp.slot_cap) : 0;
+    }
+    __syncthreads();
+    if (tid < pp.T)
+        hdr->nC[tid] = sub_base[chunk_base[pp.col_base[tid + 1]]] - sub_base[chunk_base[pp.col_base[tid]]];
+    for (int b = tid; b < pp.grid; b += 1024) {
+        own_head[b] = owner_start(S, b, pp.grid);
+        steal_tail[b] = owner_start(S, b + 1, pp.grid);
+        exhausted[b] = 0;
+    }
+}
+
+// Subtask records: chunk c's rows split into n near-equal row ranges; claims and the
+// checkpoint flags start at zero.
+__global__ void __launch_bounds__(256) k_plan_subs(const PlanHeader* __restrict__ hdr, const int32_t* __restrict__ crow,
+                                                   const int32_t* __restrict__ sub_base,
+                                                   const int32_t* __restrict__ slot_of, int4* __restrict__ subs,
+                                                   int32_t* __restrict__ claim, int32_t* __restrict__ slot_flag,
+                                                   const int32_t* status)
+{
+    if (has_error(status)) return;
+    const int nch = hdr->nchunks;
+    for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < nch; c += gridDim.x * blockDim.x) {
+        const int base = sub_base[c], n = sub_base[c + 1] - base, R = crow[c], slot = slot_of[c];
+        for (int q = 0; q < n; ++q) {
+            subs[base + q] = make_int4(c, (int)((int64_t)R * q / n), (int)((int64_t)R * (q + 1) / n), slot);
+            claim[base + q] = 0;
+        }
+        if (slot >= 0) slot_flag[slot] = 0;
     }
 }
 
@@ -207,16 +316,17 @@ cudaError_t launch_plan(const PlanParams& pp, bool key64, const void* uniq_keys,
                         PlanBuffers& pb, int32_t* status, cudaStream_t s, int* nl)
 {
     cudaError_t e = cudaMemsetAsync(pb.col_count, 0, sizeof(int32_t) * (size_t)pp.ncols, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(pb.col_rows, 0, sizeof(int32_t) * (size_t)pp.ncols, s);
     if (e != cudaSuccess) return e;
     const int grid = 148 * 4;
     if (key64)
         k_plan_keys<uint64_t><<<grid, 256, 0, s>>>(pp, (const uint64_t*)uniq_keys, grp_start, counters,
                                                    (uint32_t*)pb.sort.keys[0], pb.sort.vals[0],
-                                                   pb.col_count, status);
+                                                   pb.col_count, pb.col_rows, status);
     else
         k_plan_keys<uint32_t><<<grid, 256, 0, s>>>(pp, (const uint32_t*)uniq_keys, grp_start, counters,
                                                    (uint32_t*)pb.sort.keys[0], pb.sort.vals[0],
-                                                   pb.col_count, status);
+                                                   pb.col_count, pb.col_rows, status);
     *nl += 1;
     int bits = 1;
     while ((1u << bits) < (uint32_t)pp.ncols) ++bits;
@@ -226,15 +336,20 @@ cudaError_t launch_plan(const PlanParams& pp, bool key64, const void* uniq_keys,
     if (e != cudaSuccess) return e;
     pb.sorted_groups = pb.sort.vals[which];
     k_plan_cols<<<1, 1024, 0, s>>>(pp, pb.col_count, pb.col_start, pb.chunk_base, pb.hdr, status);
-    k_plan_chunks<<<grid, 256, 0, s>>>(pp, counters, (const uint32_t*)pb.sort.keys[which], pb.col_count,
-                                       pb.col_start, pb.chunk_base, pb.hdr, pb.chunks, pb.tasks, status);
+    k_plan_order<<<1, 1024, 0, s>>>(pp, pb.col_count, pb.col_rows, pb.col_order, pb.hdr, status);
     if (key64)
         k_plan_grec<uint64_t><<<grid, 256, 0, s>>>(pp, counters, pb.sorted_groups, grp_start,
                                                    (const uint64_t*)uniq_keys, pb.grec, status);
     else
         k_plan_grec<uint32_t><<<grid, 256, 0, s>>>(pp, counters, pb.sorted_groups, grp_start,
                                                    (const uint32_t*)uniq_keys, pb.grec, status);
-    *nl += 3;
+    k_plan_chunks<<<grid, 256, 0, s>>>(pp, counters, (const uint32_t*)pb.sort.keys[which], pb.col_count,
+                                       pb.col_start, pb.chunk_base, pb.grec, pb.chunks, pb.crow, status);
+    k_plan_split<<<1, 1024, 0, s>>>(pp, pb.crow, pb.chunk_base, pb.sub_base, pb.slot_of, pb.hdr, pb.own_head,
+                                    pb.steal_tail, pb.exhausted, status);
+    k_plan_subs<<<grid, 256, 0, s>>>(pb.hdr, pb.crow, pb.sub_base, pb.slot_of, pb.subs, pb.claim, pb.slot_flag,
+                                     status);
+    *nl += 7;
     return cudaGetLastError();
 }
 

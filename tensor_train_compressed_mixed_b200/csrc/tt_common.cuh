@@ -72,7 +72,37 @@ struct CoreParams {
     // first tensor-core completion wait report a timeout after the products completed;
     // inj_spin > 0 replaces the pooling wait's iteration limit
     int32_t inj_pool, inj_mma, inj_spin, inj_pad;
+    // balance probe (tt_emb_set_probe; null in normal calls): each block of a fused kernel
+    // writes one record of kProbeWords words at probe[(probe_slot * probe_cap + block) * 4]
+    unsigned long long* probe;
+    int32_t probe_slot, probe_cap;
 };
+
+// Balance probe record of one block of a fused kernel: SM id | tasks << 32, start and end
+// (global timer, ns), nanoseconds spent waiting (pooling waits for unfinished tables).
+constexpr int kProbeWords = 4;
+__device__ __forceinline__ unsigned long long global_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ unsigned sm_id()
+{
+    unsigned id;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(id));
+    return id;
+}
+__device__ __forceinline__ void probe_write(const CoreParams& cp, unsigned long long t0, int tasks,
+                                            unsigned long long wait_ns)
+{
+    if (cp.probe == nullptr || (int)blockIdx.x >= cp.probe_cap || threadIdx.x != 0) return;
+    unsigned long long* r = cp.probe + ((size_t)cp.probe_slot * cp.probe_cap + blockIdx.x) * kProbeWords;
+    r[0] = (unsigned long long)sm_id() | ((unsigned long long)(unsigned)tasks << 32);
+    r[1] = t0;
+    r[2] = global_ns();
+    r[3] = wait_ns;
+}
 
 struct GradPtrs {
     // gradient buffers in the core layouts; the three-core specialised backward takes the last
@@ -111,33 +141,58 @@ struct PlanParams {
     int32_t NB;                      // bags per pooling task
     int32_t ncols;                   // sum over tables of n_{col_digit}
     int32_t sched;                   // tt_sched_mode
+    int32_t grid;                    // persistent blocks of the fused forward (owner ranges)
+    int32_t slot_cap;                // checkpoint slots for split chunks (TT_SCHED_STEAL_L2)
     uint32_t n[kMaxT][kMaxK];
     int32_t col_base[kMaxT + 1];     // first column of each table
 };
 
+// Distinct rows per forward subtask: chunks with more rows are split into row ranges of at
+// most this many (FlowTT section 3.4's chunks of long prefix groups, the stealing granule).
+constexpr int kSplitRows = 256;
+constexpr int kMaxGrid = 4096;       // persistent blocks the scheduler arrays hold
+constexpr int kCkptFloats = 16384;   // one forward C tile (MF x N = 16384 floats for every shape)
+constexpr int64_t kCkptSlots = 2048; // checkpoint slots at most (128 MB, about the size of L2)
+// subtasks of a chunk of `rows` distinct rows; first subtask owned by block b of G (of S)
+__host__ __device__ __forceinline__ int subtasks_of(int rows)
+{
+    return rows > kSplitRows ? (rows + kSplitRows - 1) / kSplitRows : 1;
+}
+__host__ __device__ __forceinline__ int owner_start(int S, int b, int G) { return (int)((int64_t)S * b / G); }
+
 // Device-side plan header (workspace).  Queue cursors and per-table
 // completion counters are reset by the planner on every forward.
 struct PlanHeader {
-    int32_t ntasks, nchunks, nP, pad0;
-    int32_t queue_head, col_head, pad1, pad2;
-    int32_t nC[kMaxT];             // compute chunks per table
-    int32_t chunk_first[kMaxT];    // first chunk id of each table
-    int32_t task_base_C[kMaxT];    // queue position of each table's first chunk
-    int32_t task_base_P[kMaxT];    // queue position of each table's first pooling task
-    int32_t done[kMaxT];           // finished compute chunks per table
+    int32_t nsub, nchunks, nP, nslots;   // forward subtasks, chunks, pooling tasks per table, used slots
+    int32_t pool_head, col_head, ncols_busy, pad2;   // ncols_busy: columns with work (backward queue)
+    int32_t nC[kMaxT];             // forward subtasks per table (pooling of t waits for all of them)
+    int32_t done[kMaxT];           // finished forward subtasks per table
 };
 
 struct PlanBuffers {
     SortBuffers sort;              // uint32 column keys / group ids, ping-pong
     int32_t* sorted_groups;        // set by launch_plan: group ids in column order
     int32_t* col_count;            // [ncols]
+    int32_t* col_rows;             // [ncols] distinct rows of each column
+    int32_t* col_order;            // [ncols] backward column queue: non-empty columns, costliest first
     int32_t* col_start;            // [ncols + 1]
     int32_t* chunk_base;           // [ncols + 1]
     PlanHeader* hdr;
     int4* chunks;                  // (first sorted position, groups, table, column digit)
-    int32_t* tasks;                // >= 0: chunk id; < 0: pooling task -1 - (t * nP + j)
     int4* grec;                    // [G] per sorted group position: (first distinct row, rows,
                                    //     first digit i_1, 0), so chunk metadata is one load
+    // forward subtask scheduler (FlowTT section 3.4): chunks split into row ranges, each
+    // block owning a contiguous range of subtasks, claims, and the C checkpoint slots
+    int32_t* crow;                 // [chunks] distinct rows of each chunk
+    int32_t* sub_base;             // [chunks + 1] first subtask of each chunk
+    int32_t* slot_of;              // [chunks] checkpoint slot of a split chunk, or -1
+    int4* subs;                    // [subtasks] (chunk, first row, end row, slot)
+    int32_t* claim;                // [subtasks] 1 once a block has taken the subtask
+    int32_t* own_head;             // [kMaxGrid] next own subtask of each block
+    int32_t* steal_tail;           // [kMaxGrid] one past the last subtask not yet stolen
+    int32_t* exhausted;            // [kMaxGrid] hint: the block's range is fully claimed
+    int32_t* slot_flag;            // [slot_cap] 0 empty, 1 being written, 2 ready
+    float* ckpt;                   // [slot_cap][16384] the forward C tile of a split chunk
 };
 
 // ---------------------------------------------------------------------------

@@ -189,3 +189,72 @@ def test_generic_and_specialised_paths_agree(cfg, batch, tables):
     for t in range(w.num_tables):
         for j in range(w.num_cores):
             assert core_grad_err(grads_f[t][j], grads_g[t][j]) <= FP32_TOL, (t, j)
+
+
+def _hot_prefix_workload(cfg, batch, seed):
+    """Lookups concentrated on 32 prefixes (i_1 < 16, i_2 < 2) of each table, every last digit
+    possible: chunks of thousands of distinct rows, split into many subtasks, so stealing and
+    the C checkpoint of split chunks are exercised."""
+    from workloads.gen import Workload
+    base = config_workload(cfg, batch=batch, tables=2, with_grad=True)
+    rng = np.random.default_rng(seed)
+    T, B = base.num_tables, base.batch
+    sizes = rng.integers(1, 48, size=T * B)
+    offsets = np.zeros(T * B + 1, dtype=np.int64)
+    np.cumsum(sizes, out=offsets[1:])
+    idx = []
+    for t in range(T):
+        n1, n2, n3 = base.n[t]
+        m = int(sizes[t * B:(t + 1) * B].sum())
+        row = (rng.integers(0, 16, m) * n2 + rng.integers(0, 2, m)) * n3 + rng.integers(0, n3, m)
+        idx.append(np.minimum(row, base.n_rows[t] - 1).astype(np.int64))
+    return Workload(name="hot_prefixes", d=base.d, r=base.r, n=base.n, n_rows=base.n_rows, batch=B,
+                    indices=np.concatenate(idx), offsets=offsets, cores=base.cores,
+                    grad_out=base.grad_out, train=True)
+
+
+@pytest.mark.parametrize("cfg,prec", [(3, "fp32"), (4, "split"), (3, "split")])
+def test_split_chunks_stealing_and_checkpoint_give_identical_rows(cfg, prec):
+    from tensor_train_compressed_mixed_b200 import abi
+    w = _hot_prefix_workload(cfg, 1024, 40 + cfg)
+    want = oracle.workload_forward(w)
+    ref = None
+    for sched in (abi.TT_SCHED_STATIC, abi.TT_SCHED_STEAL, abi.TT_SCHED_STEAL_L2):
+        for grid in (1, 3, 7, 0):
+            o = abi.tt_emb_default_options()
+            o.sched, o.grid = sched, grid
+            o.precision = abi.TT_PREC_FP32 if prec == "fp32" else abi.TT_PREC_FP32_SPLIT_TC
+            emb, cores, out = gpu_forward(w, options=o)
+            got = out.cpu().numpy()
+            emb.close()
+            if ref is None:
+                ref = got
+                assert output_err(got, want, w.dim) <= FP32_TOL
+            assert np.array_equal(got, ref), (sched, grid)
+
+
+def test_balance_probe_counts_every_task():
+    import torch
+    from tensor_train_compressed_mixed_b200 import abi
+    w = _hot_prefix_workload(4, 512, 7)
+    o = abi.tt_emb_default_options()
+    o.precision = abi.TT_PREC_FP32_SPLIT_TC
+    o.grid = 6
+    emb, cores, out = gpu_forward(w, options=o, with_grads=True)
+    cap = 16
+    rec = torch.zeros(2 * cap * 4, dtype=torch.int64, device="cuda")
+    abi.tt_emb_set_probe(emb.handle, rec, cap)
+    emb.forward(torch.from_numpy(w.indices).cuda(), torch.from_numpy(w.offsets).cuda(), w.batch, out)
+    emb.backward(torch.from_numpy(w.grad_out).cuda())
+    emb.sync()
+    abi.tt_emb_set_probe(emb.handle, None, 0)
+    r = rec.view(2, cap, 4).cpu().numpy()
+    fwd, bwd = r[0][:6], r[1]
+    assert (fwd[:, 1] > 0).all() and (fwd[:, 2] >= fwd[:, 1]).all()
+    assert not r[0][6:].any()                              # blocks beyond the grid: no record
+    n_pool = w.num_tables * ((w.batch + 63) // 64)
+    assert int((fwd[:, 0] >> 32).sum()) >= n_pool + 1       # every pooling task and >= 1 subtask
+    seg = emb.segmentation()
+    assert (bwd[:, 1] > 0).sum() >= 1
+    assert int((bwd[:, 0] >> 32).sum()) <= seg["num_groups"]   # columns taken, at most one per group
+    assert output_err(out.cpu().numpy(), oracle.workload_forward(w), w.dim) <= FP32_TOL
