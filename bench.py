@@ -95,6 +95,8 @@ def parse_args():
                    help="prefix-level products: fp32 on the FP32 pipes; split = fp32-accurate on the "
                         "tcgen05 tensor cores (two bf16 terms per value, three products); bf16 on the "
                         "tensor cores; auto = split where the shape has tensor-core kernels, else fp32")
+    p.add_argument("--generic", action="store_true",
+                   help="force the shape-generic kernels (comparison and profiling runs)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extra-fwd", action="store_true",
@@ -530,6 +532,10 @@ def run_ours(args):
     opts.grouping = abi.TT_GROUP_PREFIX if args.grouping == "prefix" else abi.TT_GROUP_UNIQUE_ONLY
     opts.precision = {"fp32": abi.TT_PREC_FP32, "split": abi.TT_PREC_FP32_SPLIT_TC,
                       "bf16": abi.TT_PREC_BF16_TC}[args.precision]
+    if args.generic:
+        opts.force_generic = 1
+        opts.precision = abi.TT_PREC_FP32
+        args.precision = "fp32"
     # data-parallel training: the core gradients of all ranks are summed (one NCCL
     # all-reduce over a flat buffer) before the SGD step
     dp_train = world > 1 and train

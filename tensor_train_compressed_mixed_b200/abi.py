@@ -15,7 +15,8 @@ import os
 import numpy as np
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libttemb.so")
+# TTEMB_LIB names another build of the same library (e.g. a variant compiled for a comparison)
+LIB_PATH = os.environ.get("TTEMB_LIB") or os.path.join(PKG, "libttemb.so")
 
 TT_OK, TT_ERR_ARG, TT_ERR_SHAPE, TT_ERR_INDEX_RANGE, TT_ERR_OFFSETS = 0, 1, 2, 3, 4
 TT_ERR_WORKSPACE, TT_ERR_STATE, TT_ERR_CUDA, TT_ERR_TIMEOUT, TT_ERR_UNSUPPORTED = 5, 6, 7, 8, 9
