@@ -109,8 +109,10 @@ typedef enum {
 typedef struct {
     int32_t sched;           /* tt_sched_mode, default TT_SCHED_STEAL_L2 */
     int32_t grouping;        /* tt_group_mode, default TT_GROUP_PREFIX */
-    int32_t chunk;           /* rows per stealable chunk of a prefix group; 0 = library default */
-    int32_t grid;            /* persistent blocks; 0 = one wave on the current device */
+    int32_t chunk;           /* distinct rows per stealable subtask of the fused forward, 1..256;
+                                0 = 256 (longer chunks of prefix groups are split) */
+    int32_t grid;            /* persistent blocks; 0 = one wave on the current device (the fused forward
+                                never runs more than one resident wave) */
     int32_t force_generic;   /* 1: run the shape-generic kernels even where a specialised path exists */
     int32_t precision;       /* tt_precision, default TT_PREC_FP32 */
     int32_t reserved[10];    /* must be zero */

@@ -28,6 +28,7 @@ struct FastDims {
     int64_t g12_floats;   // merged first cores of four-core tables (0 otherwise)
     int64_t g3t_floats;   // transposed copies of the last cores
     int64_t bf1_elems, bf2_elems;   // bf16 operand copies of G_1 and G_2 (tensor-core forward)
+    int split;                      // distinct rows per forward subtask at most
 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -75,8 +76,8 @@ Layout make_layout(int key_bytes, int64_t L, int64_t B, const FastDims& f)
         y.chunks = take((size_t)y.chunk_cap * sizeof(int4));
         y.grec = take(Lz * sizeof(int4));
         // forward subtasks: every chunk once, plus one per kSplitRows distinct rows of split chunks
-        y.sub_cap = y.chunk_cap + ceil_div((int64_t)Lz, kSplitRows) + 1;
-        y.slot_cap = min64(kCkptSlots, ceil_div((int64_t)Lz, kSplitRows) + 1);
+        y.sub_cap = y.chunk_cap + ceil_div((int64_t)Lz, f.split) + 1;
+        y.slot_cap = min64(kCkptSlots, ceil_div((int64_t)Lz, f.split) + 1);
         y.crow = take((size_t)y.chunk_cap * 4);
         y.sub_base = take(((size_t)y.chunk_cap + 1) * 4);
         y.slot_of = take((size_t)y.chunk_cap * 4);
@@ -214,6 +215,7 @@ struct tt_emb_handle {
         f.g3t_floats = g3t_off[T];
         f.bf1_elems = tc ? bf1_off[T] : 0;
         f.bf2_elems = tc ? bf2_off[T] : 0;
+        f.split = opt.chunk > 0 ? opt.chunk : kSplitRows;
         return f;
     }
     // three-core view of the shapes (identity for three-core tables), without core pointers
@@ -298,6 +300,7 @@ struct tt_emb_handle {
         pp.sched = opt.sched;
         pp.grid = fwd_grid();
         pp.slot_cap = (int32_t)lay.slot_cap;
+        pp.split_rows = opt.chunk > 0 ? opt.chunk : kSplitRows;
         for (int t = 0; t < T; ++t)
             for (int j = 0; j < 3; ++j) pp.n[t][j] = (uint32_t)vn[t][j];
         for (int t = 0; t <= T; ++t) pp.col_base[t] = col_base[t];
@@ -308,7 +311,10 @@ struct tt_emb_handle {
     int fwd_grid() const
     {
         if (fwd_grid_cache == 0) {
-            const int g = opt.grid > 0 ? opt.grid : num_sms * k3_blocks_per_sm(view_params(), false, tc != 0);
+            // at most one resident wave: a pooling task waits for subtasks owned by other blocks,
+            // which must all be running
+            const int wave = num_sms * k3_blocks_per_sm(view_params(), false, tc != 0);
+            const int g = opt.grid > 0 && opt.grid < wave ? opt.grid : wave;
             fwd_grid_cache = g < kMaxGrid ? g : kMaxGrid;
         }
         return fwd_grid_cache;
@@ -480,7 +486,7 @@ int tt_emb_create(int32_t num_tables, int32_t num_cores, const int64_t* n_factor
             return TT_ERR_ARG;
         if (o.sched < TT_SCHED_STATIC || o.sched > TT_SCHED_STEAL_L2) return TT_ERR_ARG;
         if (o.grouping < TT_GROUP_PREFIX || o.grouping > TT_GROUP_UNIQUE_ONLY) return TT_ERR_ARG;
-        if (o.chunk < 0 || o.grid < 0) return TT_ERR_ARG;
+        if (o.chunk < 0 || o.chunk > kSplitRows || o.grid < 0) return TT_ERR_ARG;
     }
     const int k = num_cores;
     if (ranks[0] != 1 || ranks[k] != 1) return TT_ERR_SHAPE;

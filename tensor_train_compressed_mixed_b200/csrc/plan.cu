@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(1024) k_plan_split(PlanParams pp, const int32_
     const int lo = min(nch, tid * per), hi = min(nch, lo + per);
     int ns = 0, np = 0;
     for (int c = lo; c < hi; ++c) {
-        const int k = subtasks_of(crow[c]);
+        const int k = subtasks_of(crow[c], pp.split_rows);
         ns += k;
         np += k > 1;
     }
@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(1024) k_plan_split(PlanParams pp, const int32_
     int rp = (wid ? s_w[1][wid - 1] : 0) + x[1] - np;
     const bool ckpt = pp.sched == TT_SCHED_STEAL_L2;
     for (int c = lo; c < hi; ++c) {
-        const int k = subtasks_of(crow[c]);
+        const int k = subtasks_of(crow[c], pp.split_rows);
         sub_base[c] = rs;
         slot_of[c] = (ckpt && k > 1 && rp < pp.slot_cap) ? rp : -1;
         rs += k;

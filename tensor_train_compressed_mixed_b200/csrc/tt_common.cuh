@@ -143,20 +143,22 @@ struct PlanParams {
     int32_t sched;                   // tt_sched_mode
     int32_t grid;                    // persistent blocks of the fused forward (owner ranges)
     int32_t slot_cap;                // checkpoint slots for split chunks (TT_SCHED_STEAL_L2)
+    int32_t split_rows;              // distinct rows per forward subtask at most (1 .. kSplitRows)
     uint32_t n[kMaxT][kMaxK];
     int32_t col_base[kMaxT + 1];     // first column of each table
 };
 
-// Distinct rows per forward subtask: chunks with more rows are split into row ranges of at
-// most this many (FlowTT section 3.4's chunks of long prefix groups, the stealing granule).
+// Distinct rows per forward subtask at most (the default; tt_emb_options.chunk may lower it):
+// chunks with more rows are split into row ranges of at most this many (FlowTT section 3.4's
+// chunks of long prefix groups, the stealing granule).  It may not exceed the row table.
 constexpr int kSplitRows = 256;
 constexpr int kMaxGrid = 4096;       // persistent blocks the scheduler arrays hold
 constexpr int kCkptFloats = 16384;   // one forward C tile (MF x N = 16384 floats for every shape)
 constexpr int64_t kCkptSlots = 2048; // checkpoint slots at most (128 MB, about the size of L2)
 // subtasks of a chunk of `rows` distinct rows; first subtask owned by block b of G (of S)
-__host__ __device__ __forceinline__ int subtasks_of(int rows)
+__host__ __device__ __forceinline__ int subtasks_of(int rows, int split)
 {
-    return rows > kSplitRows ? (rows + kSplitRows - 1) / kSplitRows : 1;
+    return rows > split ? (rows + split - 1) / split : 1;
 }
 __host__ __device__ __forceinline__ int owner_start(int S, int b, int G) { return (int)((int64_t)S * b / G); }
 

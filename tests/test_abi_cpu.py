@@ -82,6 +82,12 @@ def test_create_rejects_bad_options_on_host():
     with pytest.raises(abi.TTEmbError) as e:
         abi.tt_emb_create([[2, 3]], [6], [2, 2], [1, 4, 1], o)
     assert e.value.code == abi.TT_ERR_ARG
+    for chunk in (-1, 257):   # subtask size: 1..256 distinct rows (0 = default)
+        o = abi.tt_emb_default_options()
+        o.chunk = chunk
+        with pytest.raises(abi.TTEmbError) as e:
+            abi.tt_emb_create([[2, 3]], [6], [2, 2], [1, 4, 1], o)
+        assert e.value.code == abi.TT_ERR_ARG
 
 
 def test_null_handle_calls_fail_cleanly():
