@@ -15,7 +15,7 @@ struct Layout {
         uniq_start, grp_start, bag_sorted;
     // specialised path only (zero when unused)
     size_t uid_at_pos, uid_sorted, rowbuf, pkeys[2], pvals[2], col_count, col_rows, col_order, col_start, chunk_base,
-        hdr, chunks, grec, crow, sub_base, slot_of, subs, claim, own_head, steal_tail, exhausted, slot_flag,
+        hdr, chunks, grec, crow, sub_base, slot_of, subs, deque, exhausted, slot_flag,
         ckpt, g12, dg12, g3t, dg3t, bf1, bf2;
     int64_t chunk_cap, sub_cap, slot_cap;
     size_t total;
@@ -82,9 +82,7 @@ Layout make_layout(int key_bytes, int64_t L, int64_t B, const FastDims& f)
         y.sub_base = take(((size_t)y.chunk_cap + 1) * 4);
         y.slot_of = take((size_t)y.chunk_cap * 4);
         y.subs = take((size_t)y.sub_cap * sizeof(int4));
-        y.claim = take((size_t)y.sub_cap * 4);
-        y.own_head = take((size_t)kMaxGrid * 4);
-        y.steal_tail = take((size_t)kMaxGrid * 4);
+        y.deque = take((size_t)kMaxGrid * 8);
         y.exhausted = take((size_t)kMaxGrid * 4);
         y.slot_flag = take((size_t)y.slot_cap * 4);
         y.ckpt = take((size_t)y.slot_cap * kCkptFloats * 4);
@@ -384,9 +382,7 @@ struct tt_emb_handle {
         pb.sub_base = (int32_t*)at(lay.sub_base);
         pb.slot_of = (int32_t*)at(lay.slot_of);
         pb.subs = (int4*)at(lay.subs);
-        pb.claim = (int32_t*)at(lay.claim);
-        pb.own_head = (int32_t*)at(lay.own_head);
-        pb.steal_tail = (int32_t*)at(lay.steal_tail);
+        pb.deque = (unsigned long long*)at(lay.deque);
         pb.exhausted = (int32_t*)at(lay.exhausted);
         pb.slot_flag = (int32_t*)at(lay.slot_flag);
         pb.ckpt = (float*)at(lay.ckpt);

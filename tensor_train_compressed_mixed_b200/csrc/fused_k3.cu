@@ -669,9 +669,7 @@ __device__ void fwd_pool(const CoreParams& cp, int ptask, int nP, const int32_t*
                          int* s_flag, unsigned long long* wait_ns)
 {
     constexpr int D = S::D, LB = D / 4, BPW = 32 / LB;
-    // row gathers in flight per lane: 16 below rank 64; at rank 64 the kernel's register budget
-    // is held by the tensor-core phases and 8 is faster
-    constexpr int kPoolLoads = S::R >= 64 ? 8 : 16;
+    constexpr int kPoolLoads = 16;   // row gathers in flight per lane
     const int t = ptask / nP, jb = ptask % nP;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     TT_PH_START();
@@ -736,27 +734,30 @@ __device__ void fwd_pool(const CoreParams& cp, int ptask, int nP, const int32_t*
 // Forward scheduler (FlowTT section 3.4).  Subtasks (row ranges of chunks, in column order)
 // are split into one contiguous owner range per persistent block.  A block takes its own
 // subtasks front to back; in the stealing modes it then takes subtasks of other blocks that
-// have not started, from the back of their ranges (so a thief and the owner meet in the middle
-// and each subtask is claimed exactly once), and finally pooling tasks from a shared queue.
+// have not started, from the back of their ranges, and finally pooling tasks from a shared
+// queue.  Each block's remaining range is one 64-bit word, (head + kDequeBias) << 32 |
+// (tail + kDequeBias): the owner takes `head` by adding 1 << 32, a thief takes `tail - 1` by
+// adding -1, and the one atomic of each tells whether the range still held a subtask, so every
+// subtask runs exactly once.  The bias keeps both halves positive: tails fall at most once per
+// failed steal per block below the range start.
 // Thread 0 only.  Returns a subtask index, -2 - p for pooling task p, or -1 when done.
 // ---------------------------------------------------------------------------
 struct FwdSched {
     const int4* subs;
-    int32_t* claim;
-    int32_t* own_head;
-    int32_t* steal_tail;
-    int32_t* exhausted;
+    unsigned long long* deque;   // [grid] (head, tail) of each block's owner range
+    int32_t* exhausted;          // [grid] hint: the range has no subtask left
     int32_t* slot_flag;
     float* ckpt;
 };
 
-__device__ __forceinline__ int fwd_next(const FwdSched& fs, PlanHeader* hdr, int sched, int S, int npool, int& phase,
+__device__ __forceinline__ int fwd_next(const FwdSched& fs, PlanHeader* hdr, int sched, int npool, int& phase,
                                         int& vk)
 {
     const int G = (int)gridDim.x, b = (int)blockIdx.x;
     if (phase == 0) {
-        const int h = atomicAdd(&fs.own_head[b], 1);
-        if (h < owner_start(S, b + 1, G) && atomicExch(&fs.claim[h], 1) == 0) return h;
+        const unsigned long long old = atomicAdd(&fs.deque[b], 1ull << 32);
+        const int h = (int)(old >> 32) - kDequeBias, t = (int)(old & 0xffffffffull) - kDequeBias;
+        if (h < t) return h;
         phase = sched == TT_SCHED_STATIC ? 2 : 1;
         vk = 1;
     }
@@ -764,8 +765,9 @@ __device__ __forceinline__ int fwd_next(const FwdSched& fs, PlanHeader* hdr, int
         while (vk < G) {
             const int v = b + vk < G ? b + vk : b + vk - G;
             if (*reinterpret_cast<volatile int*>(&fs.exhausted[v]) == 0) {
-                const int t = atomicSub(&fs.steal_tail[v], 1) - 1;
-                if (t >= owner_start(S, v, G) && atomicExch(&fs.claim[t], 1) == 0) return t;   // again from v next time
+                const unsigned long long old = atomicAdd(&fs.deque[v], ~0ull);   // tail - 1
+                const int h = (int)(old >> 32) - kDequeBias, t = (int)(old & 0xffffffffull) - kDequeBias;
+                if (t - 1 >= h) return t - 1;   // again from v next time
                 *reinterpret_cast<volatile int*>(&fs.exhausted[v]) = 1;
             }
             ++vk;
@@ -882,14 +884,14 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
         sm.Cn = sm.As + S::MF * S::R;
     }
     sm.Ss = sm.Cn + S::MF * S::N;
-    const int nS = hdr->nsub, nP = hdr->nP, npool = cp.T * nP;
+    const int nP = hdr->nP, npool = cp.T * nP;
     const bool use_ckpt = sched == TT_SCHED_STEAL_L2;
     int phase = 0, vk = 1;   // scheduler state (thread 0)
     int cur_t = -1, cur_i2 = -1;   // column of the B now in (or on its way to) the B tile
     int cur_cid = -1;              // chunk whose C tile is in shared memory
     int mb = 0;
     bool staged = false;
-    if (tid == 0) M.task[0] = fwd_next(fs, hdr, sched, nS, npool, phase, vk);
+    if (tid == 0) M.task[0] = fwd_next(fs, hdr, sched, npool, phase, vk);
     __syncthreads();
     int q = M.task[0];
     while (q != -1) {
@@ -897,7 +899,7 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
             fwd_pool<S>(cp, -2 - q, nP, uid_at_pos, offsets, hdr, rowbuf, out, status, &M.flag, &pr_wait);
             ++pr_tasks;
             __syncthreads();
-            if (tid == 0) M.task[0] = fwd_next(fs, hdr, sched, nS, npool, phase, vk);
+            if (tid == 0) M.task[0] = fwd_next(fs, hdr, sched, npool, phase, vk);
             __syncthreads();
             q = M.task[0];
             staged = false;
@@ -915,7 +917,7 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
                 cp_async_commit();   // the row keys alone
             }
         }
-        if (tid == 0) M.task[1] = fwd_next(fs, hdr, sched, nS, npool, phase, vk);   // used after the C step
+        if (tid == 0) M.task[1] = fwd_next(fs, hdr, sched, npool, phase, vk);   // used after the C step
         cp_async_wait_all();   // the subtask's A/B rows and row keys (usually prefetched long ago)
         __syncthreads();
         const int nrows = M.re[mb] - M.rb[mb];
@@ -928,9 +930,12 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
         const int cid = M.cid[mb], slot = M.slot[mb];
         if (cid != cur_cid) {
             // C of this chunk: the checkpoint when another block has published it, else the GEMM
-            if (tid == 0) M.ck = (use_ckpt && slot >= 0) ? ckpt_ready(fs, slot) : 0;
-            __syncthreads();
-            if (M.ck) {
+            const bool ck_slot = use_ckpt && slot >= 0;   // uniform: slot comes from shared memory
+            if (ck_slot) {
+                if (tid == 0) M.ck = ckpt_ready(fs, slot);
+                __syncthreads();
+            }
+            if (ck_slot && M.ck) {
                 ckpt_load<S>(fs, slot, sm.Cn);
             } else {
                 if constexpr (TC) {
@@ -941,7 +946,7 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
                 } else {
                     fwd_gemm<S>(sm);
                 }
-                if (use_ckpt && slot >= 0) {   // publish once: the block that wins the slot writes it
+                if (ck_slot) {   // publish once: the block that wins the slot writes it
                     __syncthreads();
                     if (tid == 0) M.ck = atomicCAS(&fs.slot_flag[slot], 0, 1) == 0;
                     __syncthreads();
@@ -1870,21 +1875,23 @@ __device__ __forceinline__ void warp_row_load2(const CoreParams& cp, int t, int 
     w.h = __ldg(reinterpret_cast<const float4*>(rowbuf + (int64_t)w.u * D) + lane);
 }
 
-__device__ __forceinline__ void named_bar(int id, int nthreads)
+// two fp32 fused multiply-adds in one instruction (fma.rn.f32x2): d.lo += a.lo * b.lo,
+// d.hi += a.hi * b.hi, each rounded as an fp32 fmaf
+__device__ __forceinline__ uint64_t pack2(float lo, float hi)
 {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+    return ((uint64_t)__float_as_uint(hi) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ void ffma2(uint64_t& d, uint64_t a, uint64_t b)
+{
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
 }
 
-// the chunk's distinct rows by quads of warps (see above); tmem_c = the C^T accumulators.
-// Warps s and s + 2 of a quad hold the same rho_2 and complementary a_2, so each has half of
-// dS_u[rho][.]: the second passes its half through shared memory (pslots, double-buffered by
-// row parity, one named barrier per row and pair) and the first issues the reductions, one
-// per (rho, row) instead of two.
+// the chunk's distinct rows by quads of warps (see above); tmem_c = the C^T accumulators
 template <typename K>
 __device__ __forceinline__ void bwd2_rows(const CoreParams& cp, int t, int mb, int total, int cnt, const BwdMeta2& M,
                                           const K* __restrict__ uniq_keys, const float* __restrict__ rowbuf,
                                           uint32_t tmem_c, float* dCn, float* __restrict__ dG3, uint32_t n3,
-                                          float* hslots, float* pslots)
+                                          float* hslots)
 {
     constexpr int R = 64, N = 256, D1 = 4, D2 = 4, D3 = 8, P = 16, MB = kMB2, NQ = kBwdThreadsTC / 128;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, sub = warp & 3, quad = warp >> 2;
@@ -1893,8 +1900,6 @@ __device__ __forceinline__ void bwd2_rows(const CoreParams& cp, int t, int mb, i
     if (lo >= hi) return;
     const uint32_t tl = tmem_c + ((uint32_t)(32 * sub) << 16);
     float* hs = hslots + warp * 2 * P * D3;
-    const int pair = quad * 2 + (sub & 1);            // named barrier 1 + pair (0 is __syncthreads)
-    float* ps = pslots + pair * (2 * 32 * 8) + lane * 8;
     WarpRow1 a, b;
     warp_row_load2<K>(cp, t, mb, lo, cnt, rho, M, uniq_keys, rowbuf, n3, a);
     if (lo + 1 < hi) warp_row_load2<K>(cp, t, mb, lo + 1, cnt, rho, M, uniq_keys, rowbuf, n3, b);
@@ -1931,36 +1936,30 @@ __device__ __forceinline__ void bwd2_rows(const CoreParams& cp, int t, int mb, i
         reinterpret_cast<float4*>(hb)[lane] = w.h;
         __syncwarp();
         const float sv[8] = {w.s[0].x, w.s[0].y, w.s[0].z, w.s[0].w, w.s[1].x, w.s[1].y, w.s[1].z, w.s[1].w};
-        float ds[8];
-#pragma unroll
-        for (int a3 = 0; a3 < 8; ++a3) ds[a3] = 0.f;
+        uint64_t ds2[4] = {0ull, 0ull, 0ull, 0ull};   // dS_u[rho][a3] as (even, odd) a3 pairs
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int r = (i >> 1) * D2 + a2a + 2 * (i & 1);   // row (a1, a2) of H_u
             const float4 h0 = *reinterpret_cast<const float4*>(hb + r * D3);
             const float4 h1 = *reinterpret_cast<const float4*>(hb + r * D3 + 4);
             const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+            const uint64_t cc = pack2(c[i], c[i]);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) ffma2(ds2[k], cc, pack2(hv[2 * k], hv[2 * k + 1]));
             float acc = o[i];
 #pragma unroll
-            for (int a3 = 0; a3 < 8; ++a3) {
-                ds[a3] = fmaf(c[i], hv[a3], ds[a3]);
-                acc = fmaf(hv[a3], sv[a3], acc);
-            }
+            for (int a3 = 0; a3 < 8; ++a3) acc = fmaf(hv[a3], sv[a3], acc);
             o[i] = acc;
         }
-        float* slot = ps + (kq & 1) * (32 * 8);
-        if (sub >= 2) {
-            reinterpret_cast<float4*>(slot)[0] = make_float4(ds[0], ds[1], ds[2], ds[3]);
-            reinterpret_cast<float4*>(slot)[1] = make_float4(ds[4], ds[5], ds[6], ds[7]);
+        float ds[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            ds[2 * k] = __uint_as_float((uint32_t)ds2[k]);
+            ds[2 * k + 1] = __uint_as_float((uint32_t)(ds2[k] >> 32));
         }
-        named_bar(1 + pair, 64);
-        if (sub < 2) {
-            const float4 p0 = reinterpret_cast<const float4*>(slot)[0];
-            const float4 p1 = reinterpret_cast<const float4*>(slot)[1];
-            float* dst = dG3 + ((int64_t)w.i3 * R + rho) * D3;
-            red_add_v4(dst, make_float4(ds[0] + p0.x, ds[1] + p0.y, ds[2] + p0.z, ds[3] + p0.w));
-            red_add_v4(dst + 4, make_float4(ds[4] + p1.x, ds[5] + p1.y, ds[6] + p1.z, ds[7] + p1.w));
-        }
+        float* dst = dG3 + ((int64_t)w.i3 * R + rho) * D3;
+        red_add_v4(dst, make_float4(ds[0], ds[1], ds[2], ds[3]));
+        red_add_v4(dst + 4, make_float4(ds[4], ds[5], ds[6], ds[7]));
     }
     flush();
 }
@@ -1990,7 +1989,6 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
     float* dCn = reinterpret_cast<float*>(Abt + 2 * NS * MB * R);   // [MB][N] swizzled; then NS x (MB x N) bf16
     uint16_t* dCb = reinterpret_cast<uint16_t*>(dCn);
     float* hslots = dCn + MB * N;                                   // [warps][2][P D3]
-    float* pslots = hslots + (BT / 32) * 2 * 128;                   // [warp pairs][2][32][8] dS halves
     if (has_error(status)) return;
     const int tid = threadIdx.x;
     uint32_t parity = 0;
@@ -2109,8 +2107,7 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
             }
             TT_PH(16);
 
-            bwd2_rows<K>(cp, t, mb, total, cnt, M, uniq_keys, rowbuf, tmem + (uint32_t)N, dCn, dG3, n3, hslots,
-                         pslots);
+            bwd2_rows<K>(cp, t, mb, total, cnt, M, uniq_keys, rowbuf, tmem + (uint32_t)N, dCn, dG3, n3, hslots);
             tc_fence_before();
             __syncthreads();
             TT_PH(12);
@@ -2338,7 +2335,7 @@ cudaError_t fwd_launch(const K3Args& a, float* out, cudaStream_t s, int* nl)
     if (e != cudaSuccess) return e;
     const PlanBuffers& pb = *a.pb;
     if (a.grid != a.pp->grid || a.grid > kMaxGrid) return cudaErrorInvalidConfiguration;
-    const FwdSched fs{pb.subs, pb.claim, pb.own_head, pb.steal_tail, pb.exhausted, pb.slot_flag, pb.ckpt};
+    const FwdSched fs{pb.subs, pb.deque, pb.exhausted, pb.slot_flag, pb.ckpt};
     k3_fwd_kernel<S, K, NT><<<a.grid, kFwdThreads, smem, s>>>(
         *a.cp, a.pp->sched, (const K*)a.uniq_keys, a.grec, a.uid_at_pos, a.offsets,
         pb.chunks, fs, pb.hdr, a.rowbuf, out, a.status);
@@ -2396,8 +2393,7 @@ template <int NT>
 constexpr size_t bwd2_smem_bytes()
 {
     constexpr size_t NS = NT == 3 ? 2 : 1;
-    return NS * 64 * 256 * 2 + 2 * NS * kMB2 * 64 * 2 + (size_t)kMB2 * 256 * 4 + (kBwdThreadsTC / 32) * 2 * 128 * 4 +
-           (kBwdThreadsTC / 64) * 2 * 32 * 8 * 4;
+    return NS * 64 * 256 * 2 + 2 * NS * kMB2 * 64 * 2 + (size_t)kMB2 * 256 * 4 + (kBwdThreadsTC / 32) * 2 * 128 * 4;
 }
 
 template <typename K, int NT>

@@ -202,8 +202,8 @@ __global__ void __launch_bounds__(256) k_plan_chunks(PlanParams pp, const WsCoun
 __global__ void __launch_bounds__(1024) k_plan_split(PlanParams pp, const int32_t* __restrict__ crow,
                                                     const int32_t* __restrict__ chunk_base,
                                                     int32_t* __restrict__ sub_base, int32_t* __restrict__ slot_of,
-                                                    PlanHeader* __restrict__ hdr, int32_t* __restrict__ own_head,
-                                                    int32_t* __restrict__ steal_tail,
+                                                    PlanHeader* __restrict__ hdr,
+                                                    unsigned long long* __restrict__ deque,
                                                     int32_t* __restrict__ exhausted, const int32_t* status)
 {
     __shared__ int32_t s_w[2][32];
@@ -262,28 +262,26 @@ __global__ void __launch_bounds__(1024) k_plan_split(PlanParams pp, const int32_
     if (tid < pp.T)
         hdr->nC[tid] = sub_base[chunk_base[pp.col_base[tid + 1]]] - sub_base[chunk_base[pp.col_base[tid]]];
     for (int b = tid; b < pp.grid; b += 1024) {
-        own_head[b] = owner_start(S, b, pp.grid);
-        steal_tail[b] = owner_start(S, b + 1, pp.grid);
+        const unsigned long long h = (unsigned long long)(owner_start(S, b, pp.grid) + kDequeBias);
+        const unsigned long long t = (unsigned long long)(owner_start(S, b + 1, pp.grid) + kDequeBias);
+        deque[b] = (h << 32) | t;
         exhausted[b] = 0;
     }
 }
 
-// Subtask records: chunk c's rows split into n near-equal row ranges; claims and the
-// checkpoint flags start at zero.
+// Subtask records: chunk c's rows split into n near-equal row ranges; the checkpoint flags
+// start at zero.
 __global__ void __launch_bounds__(256) k_plan_subs(const PlanHeader* __restrict__ hdr, const int32_t* __restrict__ crow,
                                                    const int32_t* __restrict__ sub_base,
                                                    const int32_t* __restrict__ slot_of, int4* __restrict__ subs,
-                                                   int32_t* __restrict__ claim, int32_t* __restrict__ slot_flag,
-                                                   const int32_t* status)
+                                                   int32_t* __restrict__ slot_flag, const int32_t* status)
 {
     if (has_error(status)) return;
     const int nch = hdr->nchunks;
     for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < nch; c += gridDim.x * blockDim.x) {
         const int base = sub_base[c], n = sub_base[c + 1] - base, R = crow[c], slot = slot_of[c];
-        for (int q = 0; q < n; ++q) {
+        for (int q = 0; q < n; ++q)
             subs[base + q] = make_int4(c, (int)((int64_t)R * q / n), (int)((int64_t)R * (q + 1) / n), slot);
-            claim[base + q] = 0;
-        }
         if (slot >= 0) slot_flag[slot] = 0;
     }
 }
@@ -345,10 +343,9 @@ cudaError_t launch_plan(const PlanParams& pp, bool key64, const void* uniq_keys,
                                                    (const uint32_t*)uniq_keys, pb.grec, status);
     k_plan_chunks<<<grid, 256, 0, s>>>(pp, counters, (const uint32_t*)pb.sort.keys[which], pb.col_count,
                                        pb.col_start, pb.chunk_base, pb.grec, pb.chunks, pb.crow, status);
-    k_plan_split<<<1, 1024, 0, s>>>(pp, pb.crow, pb.chunk_base, pb.sub_base, pb.slot_of, pb.hdr, pb.own_head,
-                                    pb.steal_tail, pb.exhausted, status);
-    k_plan_subs<<<grid, 256, 0, s>>>(pb.hdr, pb.crow, pb.sub_base, pb.slot_of, pb.subs, pb.claim, pb.slot_flag,
-                                     status);
+    k_plan_split<<<1, 1024, 0, s>>>(pp, pb.crow, pb.chunk_base, pb.sub_base, pb.slot_of, pb.hdr, pb.deque,
+                                    pb.exhausted, status);
+    k_plan_subs<<<grid, 256, 0, s>>>(pb.hdr, pb.crow, pb.sub_base, pb.slot_of, pb.subs, pb.slot_flag, status);
     *nl += 7;
     return cudaGetLastError();
 }

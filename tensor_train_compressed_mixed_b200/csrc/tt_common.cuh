@@ -153,6 +153,7 @@ struct PlanParams {
 // chunks of long prefix groups, the stealing granule).  It may not exceed the row table.
 constexpr int kSplitRows = 256;
 constexpr int kMaxGrid = 4096;       // persistent blocks the scheduler arrays hold
+constexpr int kDequeBias = 1 << 30;  // offset of both halves of a block's (head, tail) word
 constexpr int kCkptFloats = 16384;   // one forward C tile (MF x N = 16384 floats for every shape)
 constexpr int64_t kCkptSlots = 2048; // checkpoint slots at most (128 MB, about the size of L2)
 // subtasks of a chunk of `rows` distinct rows; first subtask owned by block b of G (of S)
@@ -189,9 +190,7 @@ struct PlanBuffers {
     int32_t* sub_base;             // [chunks + 1] first subtask of each chunk
     int32_t* slot_of;              // [chunks] checkpoint slot of a split chunk, or -1
     int4* subs;                    // [subtasks] (chunk, first row, end row, slot)
-    int32_t* claim;                // [subtasks] 1 once a block has taken the subtask
-    int32_t* own_head;             // [kMaxGrid] next own subtask of each block
-    int32_t* steal_tail;           // [kMaxGrid] one past the last subtask not yet stolen
+    unsigned long long* deque;     // [kMaxGrid] (head + bias) << 32 | (tail + bias) of each owner range
     int32_t* exhausted;            // [kMaxGrid] hint: the block's range is fully claimed
     int32_t* slot_flag;            // [slot_cap] 0 empty, 1 being written, 2 ready
     float* ckpt;                   // [slot_cap][16384] the forward C tile of a split chunk
