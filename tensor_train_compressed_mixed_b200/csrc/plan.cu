@@ -66,42 +66,95 @@ __global__ void __launch_bounds__(256) k_plan_keys(PlanParams pp, const K* __res
 }
 
 // One block: the backward's column queue.  TT_SCHED_STATIC: every column in index order (the
-// static round robin of the backward).  Stealing modes: the non-empty columns, costliest
-// first (cost ~ distinct rows + 4 x prefix groups, bucketed by its power of two), so the
-// dynamic queue hands out the long column groups before the short ones.
+// static round robin of the backward).  Stealing modes: the non-empty columns, heavy ones first
+// (cost = distinct rows + 4 x prefix groups above twice the mean), each part in index order, so
+// the dynamic queue starts the long column groups early while blocks working at the same time
+// stay on neighbouring columns of one table (its gradient rows and last slices shared in L2).
+// Each thread takes a contiguous range of columns; a block scan of the per-range counts gives
+// every column its position (stable).
 __global__ void __launch_bounds__(1024) k_plan_order(PlanParams pp, const int32_t* __restrict__ col_count,
                                                     const int32_t* __restrict__ col_rows,
                                                     int32_t* __restrict__ col_order, PlanHeader* __restrict__ hdr,
                                                     const int32_t* status)
 {
-    __shared__ int32_t s_hist[32], s_pos[32];
+    __shared__ long long s_sum[32];
+    __shared__ int s_w[2][32];
     if (has_error(status)) return;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     if (pp.sched == TT_SCHED_STATIC) {
         for (int c = tid; c < pp.ncols; c += 1024) col_order[c] = c;
         if (tid == 0) hdr->ncols_busy = pp.ncols;
         return;
     }
-    if (tid < 32) s_hist[tid] = 0;
-    __syncthreads();
-    for (int c = tid; c < pp.ncols; c += 1024) {
-        const int cost = col_rows[c] + 4 * col_count[c];
-        if (cost > 0) atomicAdd(&s_hist[31 - __clz(cost)], 1);
+    const int per = (pp.ncols + 1023) / 1024;
+    const int lo = min(pp.ncols, tid * per), hi = min(pp.ncols, lo + per);
+    auto cost = [&](int c) { return (long long)col_rows[c] + 4ll * col_count[c]; };
+    // mean cost of the non-empty columns
+    long long sum = 0;
+    int busy = 0;
+    for (int c = lo; c < hi; ++c) {
+        const long long k = cost(c);
+        sum += k;
+        busy += k > 0;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        sum += __shfl_xor_sync(kFull, sum, o);
+        busy += __shfl_xor_sync(kFull, busy, o);
+    }
+    if (lane == 0) {
+        s_sum[wid] = sum;
+        s_w[0][wid] = busy;
     }
     __syncthreads();
-    if (tid == 0) {
-        int run = 0;
-        for (int b = 31; b >= 0; --b) {
-            s_pos[b] = run;
-            run += s_hist[b];
+    long long tot = 0;
+    int nbusy = 0;
+    for (int w = 0; w < 32; ++w) {
+        tot += s_sum[w];
+        nbusy += s_w[0][w];
+    }
+    __syncthreads();
+    const long long heavy = nbusy > 0 ? 2 * tot / nbusy : 0;   // cost above this: a heavy column
+    // stable two-way partition of the non-empty columns: heavy first
+    int nh = 0, nl = 0;
+    for (int c = lo; c < hi; ++c) {
+        const long long k = cost(c);
+        nh += k > heavy;
+        nl += k > 0 && k <= heavy;
+    }
+    int x[2] = {nh, nl};
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, x[q], o);
+            if (lane >= o) x[q] += y;
         }
-        hdr->ncols_busy = run;
+        if (lane == 31) s_w[q][wid] = x[q];
     }
     __syncthreads();
-    for (int c = tid; c < pp.ncols; c += 1024) {
-        const int cost = col_rows[c] + 4 * col_count[c];
-        if (cost > 0) col_order[atomicAdd(&s_pos[31 - __clz(cost)], 1)] = c;
+    if (wid == 0) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            int v = s_w[q][lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(kFull, v, o);
+                if (lane >= o) v += y;
+            }
+            s_w[q][lane] = v;
+        }
     }
+    __syncthreads();
+    const int H = s_w[0][31];
+    int ph = (wid ? s_w[0][wid - 1] : 0) + x[0] - nh;
+    int pl = H + (wid ? s_w[1][wid - 1] : 0) + x[1] - nl;
+    for (int c = lo; c < hi; ++c) {
+        const long long k = cost(c);
+        if (k > heavy) col_order[ph++] = c;
+        else if (k > 0) col_order[pl++] = c;
+    }
+    if (tid == 0) hdr->ncols_busy = H + s_w[1][31];
 }
 
 // One block: column starts, chunk bases and the task layout.

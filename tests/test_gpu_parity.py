@@ -141,13 +141,6 @@ def test_scheduler_modes_and_grids_give_identical_rows(cfg):
         for grid in (1, 2, 5, 0):
             got = _forward_with(w, sched, grid)
             assert np.array_equal(got, ref), (sched, grid)
-    for chunk in (1, 32, 100, 256):   # subtask sizes: the rows are the same bits
-        o = abi.tt_emb_default_options()
-        o.chunk, o.grid = chunk, 7
-        o.precision = abi.TT_PREC_FP32 if prec == "fp32" else abi.TT_PREC_FP32_SPLIT_TC
-        emb, cores, out = gpu_forward(w, options=o)
-        assert np.array_equal(out.cpu().numpy(), ref), chunk
-        emb.close()
 
 
 @pytest.mark.parametrize("sched", [0, 1, 2])
@@ -238,6 +231,13 @@ def test_split_chunks_stealing_and_checkpoint_give_identical_rows(cfg, prec):
                 ref = got
                 assert output_err(got, want, w.dim) <= FP32_TOL
             assert np.array_equal(got, ref), (sched, grid)
+    for chunk in (1, 32, 100, 256):   # subtask sizes: the rows are the same bits
+        o = abi.tt_emb_default_options()
+        o.chunk, o.grid = chunk, 7
+        o.precision = abi.TT_PREC_FP32 if prec == "fp32" else abi.TT_PREC_FP32_SPLIT_TC
+        emb, cores, out = gpu_forward(w, options=o)
+        assert np.array_equal(out.cpu().numpy(), ref), chunk
+        emb.close()
 
 
 def test_balance_probe_counts_every_task():
