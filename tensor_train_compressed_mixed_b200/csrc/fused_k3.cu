@@ -1014,6 +1014,7 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
             __threadfence();
             atomicAdd(&hdr->done[M.t[mb]], 1);
         }
+        TT_PH(6);
         q = qn;
         staged = next_sub;
         if (next_sub) mb ^= 1;
@@ -1414,6 +1415,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
     int pr_tasks = 0;
     const int ncols_busy = hdr->ncols_busy;   // the column queue (see k_plan_order)
     for (int iter = 0;; ++iter) {
+        TT_PH_START();
         if (tid == 0) M.task = next_task(pp.sched, &hdr->col_head, iter);
         __syncthreads();
         if (M.task >= ncols_busy) break;
@@ -1432,7 +1434,7 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
         float* __restrict__ dG1 = gp.g[t][0];
         float* __restrict__ dG2 = gp.g[t][1];
         float* __restrict__ dG3 = gp.g[t][2];   // transposed layout [n3][R][D3]
-        TT_PH_START();
+        TT_PH(17);
 
         // B for the whole column group, and the first chunk's A
         {
@@ -2007,6 +2009,7 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
     int pr_tasks = 0;
     const int ncols_busy = hdr->ncols_busy;   // the column queue (see k_plan_order)
     for (int iter = 0;; ++iter) {
+        TT_PH_START();
         if (tid == 0) M.task = next_task(pp.sched, &hdr->col_head, iter);
         __syncthreads();
         if (M.task >= ncols_busy) break;
@@ -2025,7 +2028,7 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
         float* __restrict__ dG1 = gp.g[t][0];
         float* __restrict__ dG2 = gp.g[t][1];
         float* __restrict__ dG3 = gp.g[t][2];   // transposed layout [n3][R][D3]
-        TT_PH_START();
+        TT_PH(17);
         {
             const uint16_t* src = cp.bf2[t] + (int64_t)i2 * (NS * R * N);
             for (int q = tid; q < NS * R * N / 8; q += BT) cp_async16(Bb + q * 8, src + q * 8);
@@ -2127,6 +2130,7 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
                     v[i][4] = x1.x; v[i][5] = x1.y; v[i][6] = x1.z; v[i][7] = x1.w;
                 }
                 __syncthreads();
+                TT_PH(18);
 #pragma unroll
                 for (int i = 0; i < CPT; ++i) {
                     const int q = tid + i * BT;
@@ -2140,6 +2144,7 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
             }
             fence_async_smem();
             __syncthreads();
+            TT_PH(19);
             if (tid == 0) {
                 tc_fence_after();
                 const uint32_t c0 = smem_u32(dCb), b0 = smem_u32(Bb), a0 = smem_u32(Ab16);
