@@ -452,7 +452,8 @@ def balance_report(records, cap):
         rec = rec[rec[:, 1] > 0]
         if rec.size == 0:
             continue
-        sm = rec[:, 0] & 0xffffffff
+        sm = rec[:, 0] & 0xffff
+        ckpt = (rec[:, 0] >> 16) & 0xffff
         tasks = rec[:, 0] >> 32
         busy = rec[:, 2] - rec[:, 1] - rec[:, 3]
         per_sm = {}
@@ -464,7 +465,8 @@ def balance_report(records, cap):
                      "busy_max_ms": float(v.max()), "busy_mean_ms": float(v.mean()),
                      "max_over_mean": float(v.max() / v.mean()) if v.mean() > 0 else None,
                      "wait_mean_ms": float(rec[:, 3].mean()) / 1e6,
-                     "tasks_max": int(tasks.max()), "tasks_mean": float(tasks.mean())}
+                     "tasks_max": int(tasks.max()), "tasks_mean": float(tasks.mean()),
+                     "checkpoint_loads": int(ckpt.sum())}
     return out
 
 

@@ -356,7 +356,8 @@ int tt_emb_forward_noalloc(tt_emb_t h, const int64_t* indices, const int64_t* of
  * Balance probe of the persistent scheduler (FlowTT section 2.4: skewed prefix frequencies
  * create load imbalance; section 3.4 balances it).  While `records` is set, every block of
  * the fused forward kernel (slot 0) and of the fused backward kernel (slot 1) writes one
- * record of 4 uint64 at records[(slot * max_blocks + block) * 4]: SM id | tasks << 32, the
+ * record of 4 uint64 at records[(slot * max_blocks + block) * 4]: SM id (bits 0-15) | the
+ * number of C tiles the block read from an L2 checkpoint slot (bits 16-31) | tasks << 32, the
  * block's start and end on the GPU's global timer (ns), and the nanoseconds it spent in
  * bounded waits (pooling tasks waiting for their table).  Blocks >= max_blocks write nothing;
  * each launch overwrites its slot.  records: device memory of 2 * max_blocks * 4 uint64,

@@ -863,7 +863,7 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
     const int tid = threadIdx.x;
     const unsigned long long pr_t0 = cp.probe ? global_ns() : 0ull;
     unsigned long long pr_wait = 0;
-    int pr_tasks = 0;
+    int pr_tasks = 0, pr_ckpt = 0;
     uint32_t tmem = 0, parity = 0;
     if constexpr (TC) {
         // one bf16 term takes half the room of an fp32 operand, two terms the same room
@@ -937,6 +937,7 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
             }
             if (ck_slot && M.ck) {
                 ckpt_load<S>(fs, slot, sm.Cn);
+                ++pr_ckpt;
             } else {
                 if constexpr (TC) {
                     if (!fwd_gemm_tc<S, NT>(sm, tmem, &s_mbar, parity, &s_ok, cp.inj_mma != 0)) {
@@ -1028,7 +1029,7 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
             tmem_dealloc(tmem, (uint32_t)S::N);
         }
     }
-    probe_write(cp, pr_t0, pr_tasks, pr_wait);
+    probe_write(cp, pr_t0, pr_tasks, pr_wait, pr_ckpt);
 }
 
 // ---------------------------------------------------------------------------

@@ -78,8 +78,9 @@ struct CoreParams {
     int32_t probe_slot, probe_cap;
 };
 
-// Balance probe record of one block of a fused kernel: SM id | tasks << 32, start and end
-// (global timer, ns), nanoseconds spent waiting (pooling waits for unfinished tables).
+// Balance probe record of one block of a fused kernel: SM id | C tiles read from a checkpoint
+// slot << 16 | tasks << 32, start and end (global timer, ns), nanoseconds spent waiting (pooling
+// waits for unfinished tables).
 constexpr int kProbeWords = 4;
 __device__ __forceinline__ unsigned long long global_ns()
 {
@@ -94,11 +95,12 @@ __device__ __forceinline__ unsigned sm_id()
     return id;
 }
 __device__ __forceinline__ void probe_write(const CoreParams& cp, unsigned long long t0, int tasks,
-                                            unsigned long long wait_ns)
+                                            unsigned long long wait_ns, int ckpt_loads = 0)
 {
     if (cp.probe == nullptr || (int)blockIdx.x >= cp.probe_cap || threadIdx.x != 0) return;
     unsigned long long* r = cp.probe + ((size_t)cp.probe_slot * cp.probe_cap + blockIdx.x) * kProbeWords;
-    r[0] = (unsigned long long)sm_id() | ((unsigned long long)(unsigned)tasks << 32);
+    r[0] = (unsigned long long)(sm_id() & 0xffffu) | ((unsigned long long)(min(ckpt_loads, 0xffff)) << 16) |
+           ((unsigned long long)(unsigned)tasks << 32);
     r[1] = t0;
     r[2] = global_ns();
     r[3] = wait_ns;
