@@ -1009,12 +1009,10 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
             }
         }
         // publish the subtask's rows: the barrier orders every thread's row stores before thread
-        // 0's device-scope fence (cumulative), which precedes the counter increment
+        // 0's release reduction (cumulative at device scope), which the pooling tasks acquire
         __syncthreads();
-        if (tid == 0) {
-            __threadfence();
-            atomicAdd(&hdr->done[M.t[mb]], 1);
-        }
+        if (tid == 0)
+            asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(&hdr->done[M.t[mb]]) : "memory");
         TT_PH(6);
         q = qn;
         staged = next_sub;
