@@ -279,13 +279,45 @@ cudaError_t radix_sort_pairs(bool key64, int64_t n, int bits, SortBuffers& sb, i
 //   write    per tile: block scan; each flagged lookup writes its run start
 //            (uniq_start, uniq_keys, grp_start); every lookup writes its bag
 // ---------------------------------------------------------------------------
+// The 16 consecutive sorted keys of one thread (l = base .. base + 15) and the key before them.
+// Runs that lie inside [0, L) are read with 16-byte loads (the key arrays are 256-byte aligned and
+// base is a multiple of 16 keys); a ragged last run reads key by key.
 template <typename K>
-__device__ __forceinline__ uint64_t seg_flags(const K* __restrict__ keys, int64_t l,
-                                              const KeyParams& kp)
+__device__ __forceinline__ void load_run16(const K* __restrict__ keys, int64_t base, int64_t L, K (&k)[16], K& kprev)
 {
-    const K k = keys[l];
+    if (base + 16 <= L) {
+        const uint4* p = reinterpret_cast<const uint4*>(keys + base);
+        if constexpr (sizeof(K) == 4) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint4 v = p[i];
+                k[4 * i] = v.x;
+                k[4 * i + 1] = v.y;
+                k[4 * i + 2] = v.z;
+                k[4 * i + 3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint4 v = p[i];
+                k[2 * i] = ((uint64_t)v.y << 32) | v.x;
+                k[2 * i + 1] = ((uint64_t)v.w << 32) | v.z;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) k[j] = base + j < L ? keys[base + j] : K(0);
+    }
+    kprev = base > 0 && base <= L ? keys[base - 1] : K(0);
+}
+
+// Segment flags of sorted position l from its key k and the previous key q: bit 0 = first
+// lookup of a distinct key, bit 32 = first distinct key of a prefix group (new table, or a new
+// row / n_k; every distinct key in unique-only grouping).
+template <typename K>
+__device__ __forceinline__ uint64_t seg_flags_kq(K k, K q, int64_t l, const KeyParams& kp)
+{
     if (l == 0) return 1ull | (1ull << 32);
-    const K q = keys[l - 1];
     if (k == q) return 0ull;
     if (kp.unique_only) return 1ull | (1ull << 32);
     const uint32_t t = (uint32_t)(k >> kp.ibits), tq = (uint32_t)(q >> kp.ibits);
@@ -304,10 +336,12 @@ __global__ void __launch_bounds__(256) k_seg_reduce(KeyParams kp, const K* __res
     __shared__ uint64_t s_tmp[8];
     if (has_error(status)) return;
     const int64_t base = (int64_t)blockIdx.x * kScanTile + (int64_t)threadIdx.x * 16;
+    K k[16], kprev;
+    load_run16(keys, base, kp.L, k, kprev);
     uint64_t acc = 0;
-#pragma unroll 4
+#pragma unroll
     for (int j = 0; j < 16; ++j)
-        if (base + j < kp.L) acc += seg_flags(keys, base + j, kp);
+        if (base + j < kp.L) acc += seg_flags_kq(k[j], j ? k[j - 1] : kprev, base + j, kp);
     uint64_t tot;
     block256_exclusive_scan<uint64_t>(acc, &tot, s_tmp);
     if (threadIdx.x == 0) partials[blockIdx.x] = tot;
@@ -368,35 +402,71 @@ __global__ void __launch_bounds__(256) k_seg_write(KeyParams kp, const K* __rest
     __shared__ uint64_t s_tmp[8];
     if (has_error(status)) return;
     const int64_t base = (int64_t)blockIdx.x * kScanTile + (int64_t)threadIdx.x * 16;
+    const bool full = base + 16 <= kp.L;
+    // every load first (independent, vectorised where the run is whole), then the scan and stores
+    K k[16], kprev;
+    load_run16(keys, base, kp.L, k, kprev);
+    int32_t pv[16], bg[16];
+    if (full) {
+        const int4* pp = reinterpret_cast<const int4*>(perm + base);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int4 v = pp[i];
+            pv[4 * i] = v.x;
+            pv[4 * i + 1] = v.y;
+            pv[4 * i + 2] = v.z;
+            pv[4 * i + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) pv[j] = base + j < kp.L ? perm[base + j] : 0;
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) bg[j] = base + j < kp.L ? bag_of_pos[pv[j]] : 0;
     uint64_t f[16];
     uint64_t acc = 0;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-        f[j] = (base + j < kp.L) ? seg_flags(keys, base + j, kp) : 0ull;
+        f[j] = base + j < kp.L ? seg_flags_kq(k[j], j ? k[j - 1] : kprev, base + j, kp) : 0ull;
         acc += f[j];
     }
     uint64_t tot;
     uint64_t run = partials[blockIdx.x] + block256_exclusive_scan<uint64_t>(acc, &tot, s_tmp);
+    int32_t us[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
         const int64_t l = base + j;
-        if (l >= kp.L) break;
+        const bool in = l < kp.L;
         const uint32_t uid = (uint32_t)(run & 0xffffffffull);  // distinct keys before l
         const uint32_t gid = (uint32_t)(run >> 32);
-        if (f[j] & 1ull) {
+        if (in && (f[j] & 1ull)) {
             uniq_start[uid] = (int32_t)l;
-            uniq_keys[uid] = keys[l];
+            uniq_keys[uid] = k[j];
             if (f[j] >> 32) grp_start[gid] = (int32_t)uid;
         }
         run += f[j];
-        const int32_t pl = perm[l];
-        bag_sorted[l] = bag_of_pos[pl];
-        const int32_t my_uid = (int32_t)(run & 0xffffffffull) - 1;  // inclusive count - 1
-        if (uid_at_pos) uid_at_pos[pl] = my_uid;
-        if (uid_sorted) uid_sorted[l] = my_uid;
+        us[j] = (int32_t)(run & 0xffffffffull) - 1;   // inclusive count - 1
+        if (in && uid_at_pos) uid_at_pos[pv[j]] = us[j];
         if (l == kp.L - 1) {
             uniq_start[(uint32_t)(run & 0xffffffffull)] = (int32_t)kp.L;
             grp_start[(uint32_t)(run >> 32)] = (int32_t)(run & 0xffffffffull);
+        }
+    }
+    if (full) {
+        int4* bs = reinterpret_cast<int4*>(bag_sorted + base);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) bs[i] = make_int4(bg[4 * i], bg[4 * i + 1], bg[4 * i + 2], bg[4 * i + 3]);
+        if (uid_sorted) {
+            int4* ps = reinterpret_cast<int4*>(uid_sorted + base);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) ps[i] = make_int4(us[4 * i], us[4 * i + 1], us[4 * i + 2], us[4 * i + 3]);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            if (base + j >= kp.L) break;
+            bag_sorted[base + j] = bg[j];
+            if (uid_sorted) uid_sorted[base + j] = us[j];
         }
     }
 }
