@@ -263,13 +263,30 @@ __global__ void __launch_bounds__(1024) k_plan_split(PlanParams pp, const int32_
     if (has_error(status)) return;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int nch = hdr->nchunks;
-    const int per = (nch + 1023) / 1024;
+    // a multiple of 4 chunks per thread, so each range starts 16-byte aligned (crow is 256-byte
+    // aligned) and is read four row counts per load
+    const int per = ((nch + 1023) / 1024 + 3) & ~3;
     const int lo = min(nch, tid * per), hi = min(nch, lo + per);
+    auto rows4 = [&](int c, int (&r)[4]) {
+        if (c + 4 <= hi) {
+            const int4 v = *reinterpret_cast<const int4*>(crow + c);
+            r[0] = v.x; r[1] = v.y; r[2] = v.z; r[3] = v.w;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) r[i] = c + i < hi ? crow[c + i] : 0;
+        }
+    };
     int ns = 0, np = 0;
-    for (int c = lo; c < hi; ++c) {
-        const int k = subtasks_of(crow[c], pp.split_rows);
-        ns += k;
-        np += k > 1;
+    for (int c = lo; c < hi; c += 4) {
+        int r[4];
+        rows4(c, r);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if (c + i >= hi) break;
+            const int k = subtasks_of(r[i], pp.split_rows);
+            ns += k;
+            np += k > 1;
+        }
     }
     int x[2] = {ns, np};
 #pragma unroll
@@ -298,12 +315,18 @@ __global__ void __launch_bounds__(1024) k_plan_split(PlanParams pp, const int32_
     int rs = (wid ? s_w[0][wid - 1] : 0) + x[0] - ns;
     int rp = (wid ? s_w[1][wid - 1] : 0) + x[1] - np;
     const bool ckpt = pp.sched == TT_SCHED_STEAL_L2;
-    for (int c = lo; c < hi; ++c) {
-        const int k = subtasks_of(crow[c], pp.split_rows);
-        sub_base[c] = rs;
-        slot_of[c] = (ckpt && k > 1 && rp < pp.slot_cap) ? rp : -1;
-        rs += k;
-        rp += k > 1;
+    for (int c = lo; c < hi; c += 4) {
+        int r[4];
+        rows4(c, r);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if (c + i >= hi) break;
+            const int k = subtasks_of(r[i], pp.split_rows);
+            sub_base[c + i] = rs;
+            slot_of[c + i] = (ckpt && k > 1 && rp < pp.slot_cap) ? rp : -1;
+            rs += k;
+            rp += k > 1;
+        }
     }
     const int S = s_w[0][31];
     if (tid == 0) {
