@@ -577,8 +577,6 @@ __device__ __forceinline__ bool fwd_gemm_tc(const FwdSmem<S>& sm, uint32_t tmem,
     static_assert(MF == 64 || MF == 128, "tensor-core M is 64 or 128");
     static_assert(kFwdThreads == 512, "16 warps: 4 sub-partitions x 4 column blocks");
     const int tid = threadIdx.x;
-    fence_async_smem();
-    __syncthreads();
     if (tid == 0) {
         tc_fence_after();
         constexpr uint32_t SBO = (R / 8) * 128;
@@ -633,6 +631,26 @@ __device__ __forceinline__ void fwd_issue_batch(const CoreParams& cp, int mb, in
     for (int q = tid; q < nb * R * (D3 / 4); q += kFwdThreads) {
         const int uu = q / (R * (D3 / 4)), rem = q % (R * (D3 / 4));
         cp_async16(&Ss[uu * S::SU + rem * 4], G3t + (int64_t)i3[uu] * (R * D3) + rem * 4);
+    }
+    cp_async_commit();
+}
+
+// As fwd_issue_batch for the subtask's first batch, with each row's last digit taken from the
+// staged keys instead of the row table (which is built while these copies run)
+template <class S, typename K>
+__device__ __forceinline__ void fwd_issue_batch_keys(const CoreParams& cp, int mb, const FwdMeta<S>& M,
+                                                     const FwdSmem<S>& sm, const K* keys)
+{
+    constexpr int R = S::R, D3 = S::D3;
+    const int tid = threadIdx.x;
+    const int nb = min(S::NUF, M.re[mb] - M.rb[mb]);
+    const uint32_t n3 = cp.n[M.t[mb]][2];
+    const float* G3t = cp.last_t[M.t[mb]];   // [n3][R][D3]: one row's slice is contiguous
+    float* Ss = sm.Ss;
+    for (int q = tid; q < nb * R * (D3 / 4); q += kFwdThreads) {
+        const int uu = q / (R * (D3 / 4)), rem = q % (R * (D3 / 4));
+        const uint32_t i3 = key_row(keys[mb * kKeyCap + uu], cp.ibits) % n3;
+        cp_async16(&Ss[uu * S::SU + rem * 4], G3t + (int64_t)i3 * (R * D3) + rem * 4);
     }
     cp_async_commit();
 }
@@ -934,13 +952,14 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
         }
         if (tid == 0) M.task[1] = fwd_next(fs, hdr, sched, npool, phase, vk);   // used after the C step
         cp_async_wait_all();   // the subtask's A/B rows and row keys (usually prefetched long ago)
+        fence_async_smem();    // A/B tiles: read by the tensor cores after the barrier
         __syncthreads();
         const int nrows = M.re[mb] - M.rb[mb];
+        // the first batch of last slices is in flight during the C step (last digits from the keys)
+        if (nrows > 0) fwd_issue_batch_keys<S, K>(cp, mb, M, sm, s_keys);
+        // the row table; read by the batches, which come after the C step's barriers
         build_rows(M.rows, mb, M.ucum[mb], M.u0[mb], M.cnt[mb], M.re[mb], s_keys, cp.ibits, cp.n[M.t[mb]][2],
                    kFwdThreads, M.rb[mb]);
-        __syncthreads();
-        // the first batch of last slices is in flight during the C step
-        if (nrows > 0) fwd_issue_batch<S>(cp, mb, 0, 0, M, sm);
         TT_PH(0);
         const int cid = M.cid[mb], slot = M.slot[mb];
         if (cid != cur_cid) {
