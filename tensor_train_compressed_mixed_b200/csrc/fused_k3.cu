@@ -398,45 +398,30 @@ __device__ __forceinline__ void fwd_meta(const CoreParams& cp, int4 sub, int mb,
 {
     const int tid = threadIdx.x;
     const int4 ch = chunks[sub.x];
-    if (tid < 32) {
-        // one warp: the group records and the exclusive scan of their row counts, E per lane
-        constexpr int E = (S::MPF + 31) / 32;
-        int4 g[E];
-        int cnt[E], sum = 0;
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-            const int j = tid * E + e;
-            g[e] = j < ch.y ? grec[ch.x + j] : make_int4(0, 0, 0, 0);
-            cnt[e] = j < S::MPF ? g[e].y : 0;
-            sum += cnt[e];
+    if (tid < S::MPF) {
+        const int4 g = tid < ch.y ? grec[ch.x + tid] : make_int4(0, 0, 0, 0);
+        M.u0[mb][tid] = g.x;
+        M.ucum[mb][tid] = g.y;
+        M.i1[mb][tid] = g.z;
+    }
+    if (tid == 0) {
+        M.cnt[mb] = ch.y;
+        M.t[mb] = ch.z;
+        M.i2[mb] = ch.w;
+        M.cid[mb] = sub.x;
+        M.rb[mb] = sub.y;
+        M.re[mb] = sub.z;
+        M.slot[mb] = sub.w;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int run = 0;
+        for (int j = 0; j < S::MPF; ++j) {
+            const int v = M.ucum[mb][j];
+            M.ucum[mb][j] = run;
+            run += v;
         }
-        int x = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(kFull, x, o);
-            if (tid >= o) x += y;
-        }
-        int run = x - sum;
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-            const int j = tid * E + e;
-            if (j < S::MPF) {
-                M.u0[mb][j] = g[e].x;
-                M.ucum[mb][j] = run;
-                M.i1[mb][j] = g[e].z;
-            }
-            run += cnt[e];
-        }
-        if (tid == 31) M.ucum[mb][S::MPF] = x;
-        if (tid == 0) {
-            M.cnt[mb] = ch.y;
-            M.t[mb] = ch.z;
-            M.i2[mb] = ch.w;
-            M.cid[mb] = sub.x;
-            M.rb[mb] = sub.y;
-            M.re[mb] = sub.z;
-            M.slot[mb] = sub.w;
-        }
+        M.ucum[mb][S::MPF] = run;
     }
     __syncthreads();
     const int nk = min(sub.z - sub.y, kKeyCap);
