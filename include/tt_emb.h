@@ -380,12 +380,6 @@ int tt_emb_set_probe(tt_emb_t h, uint64_t* records, int32_t max_blocks);
  *                            completed, so the kernel takes its timeout exit
  *                            (copies drained, tensor memory freed) and records
  *                            TT_ERR_TIMEOUT.
- *   TT_INJECT_SORT_WAIT      next tt_emb_forward with more than 3072 lookups:
- *                            in the first pass of the lookup sort, the first
- *                            tile never publishes its digit counts, so the next
- *                            tile's look-back polls at most `spin_limit` times
- *                            (0 = 4096) before it records TT_ERR_TIMEOUT and
- *                            the rest of the call returns at once.
  *   TT_INJECT_NONE           disarms.
  * The error surfaces at tt_emb_sync like any device error; the handle is then
  * usable again.  Returns TT_OK, TT_ERR_ARG or TT_ERR_UNSUPPORTED (the handle has
@@ -395,8 +389,7 @@ typedef enum {
     TT_INJECT_NONE = 0,
     TT_INJECT_POOL_WAIT = 1,
     TT_INJECT_MMA_WAIT_FWD = 2,
-    TT_INJECT_MMA_WAIT_BWD = 3,
-    TT_INJECT_SORT_WAIT = 4
+    TT_INJECT_MMA_WAIT_BWD = 3
 } tt_inject;
 
 int tt_emb_debug_inject(tt_emb_t h, int32_t what, int32_t spin_limit);

@@ -23,7 +23,7 @@ TT_ERR_WORKSPACE, TT_ERR_STATE, TT_ERR_CUDA, TT_ERR_TIMEOUT, TT_ERR_UNSUPPORTED 
 TT_SCHED_STATIC, TT_SCHED_STEAL, TT_SCHED_STEAL_L2 = 0, 1, 2
 TT_GROUP_PREFIX, TT_GROUP_UNIQUE_ONLY = 0, 1
 TT_PREC_FP32, TT_PREC_BF16_TC, TT_PREC_FP32_SPLIT_TC = 0, 1, 2
-TT_INJECT_NONE, TT_INJECT_POOL_WAIT, TT_INJECT_MMA_WAIT_FWD, TT_INJECT_MMA_WAIT_BWD, TT_INJECT_SORT_WAIT = 0, 1, 2, 3, 4
+TT_INJECT_NONE, TT_INJECT_POOL_WAIT, TT_INJECT_MMA_WAIT_FWD, TT_INJECT_MMA_WAIT_BWD = 0, 1, 2, 3
 MAX_TABLES, MAX_CORES = 64, 4
 
 

@@ -11,7 +11,7 @@ using namespace tt;
 namespace {
 
 struct Layout {
-    size_t counters, keys[2], vals[2], bag_of_pos, look[2], ghist, partials, uniq_keys,
+    size_t counters, keys[2], vals[2], bag_of_pos, hist, digit_total, partials, uniq_keys,
         uniq_start, grp_start, bag_sorted;
     // specialised path only (zero when unused)
     size_t uid_at_pos, uid_sorted, rowbuf, pkeys[2], pvals[2], col_count, col_rows, col_order, col_start, chunk_base,
@@ -51,9 +51,8 @@ Layout make_layout(int key_bytes, int64_t L, int64_t B, const FastDims& f)
     y.vals[0] = take(Lz * 4);
     y.vals[1] = take(Lz * 4);
     y.bag_of_pos = take(Lz * 4);
-    y.look[0] = take(256 * tiles * 8);
-    y.look[1] = take(256 * tiles * 8);
-    y.ghist = take(kSortGhistBytes);
+    y.hist = take(256 * tiles * 4);
+    y.digit_total = take(256 * 4);
     y.partials = take((size_t)ceil_div((int64_t)Lz, kScanTile) * 8);
     y.uniq_keys = take(Lz * key_bytes);
     y.uniq_start = take((Lz + 1) * 4);
@@ -361,7 +360,7 @@ struct tt_emb_handle {
 
     int32_t* plan_sorted_groups = nullptr;  // set by the last forward's plan
 
-    PlanBuffers plan_buffers()
+    PlanBuffers plan_buffers(const SortBuffers& lookup_sort)
     {
         PlanBuffers pb;
         memset(&pb, 0, sizeof(pb));
@@ -369,10 +368,8 @@ struct tt_emb_handle {
         pb.sort.keys[1] = at(lay.pkeys[1]);
         pb.sort.vals[0] = (int32_t*)at(lay.pvals[0]);
         pb.sort.vals[1] = (int32_t*)at(lay.pvals[1]);
-        pb.sort.look[0] = (uint64_t*)at(lay.look[0]);
-        pb.sort.look[1] = (uint64_t*)at(lay.look[1]);
-        pb.sort.ghist = (uint32_t*)at(lay.ghist);
-        pb.sort.inject_spin = 0;
+        pb.sort.hist = lookup_sort.hist ? lookup_sort.hist : (uint32_t*)at(lay.hist);
+        pb.sort.digit_total = lookup_sort.digit_total ? lookup_sort.digit_total : (uint32_t*)at(lay.digit_total);
         pb.col_count = (int32_t*)at(lay.col_count);
         pb.col_rows = (int32_t*)at(lay.col_rows);
         pb.col_order = (int32_t*)at(lay.col_order);
@@ -690,14 +687,8 @@ static int tt_emb_forward_impl(tt_emb_t h, const int64_t* indices, const int64_t
     sb.keys[1] = h->at(y.keys[1]);
     sb.vals[0] = (int32_t*)h->at(y.vals[0]);
     sb.vals[1] = (int32_t*)h->at(y.vals[1]);
-    sb.look[0] = (uint64_t*)h->at(y.look[0]);
-    sb.look[1] = (uint64_t*)h->at(y.look[1]);
-    sb.ghist = (uint32_t*)h->at(y.ghist);
-    sb.inject_spin = 0;
-    if (h->inject == TT_INJECT_SORT_WAIT && L > kSortTile) {
-        sb.inject_spin = h->inject_spin > 0 ? h->inject_spin : 4096;
-        h->inject = TT_INJECT_NONE;
-    }
+    sb.hist = (uint32_t*)h->at(y.hist);
+    sb.digit_total = (uint32_t*)h->at(y.digit_total);
 
     int nl = 0;
     h->begin(TT_PHASE_FWD_KEYS, s);
@@ -732,7 +723,7 @@ static int tt_emb_forward_impl(tt_emb_t h, const int64_t* indices, const int64_t
     cp.B = batch;
     if (e == cudaSuccess && h->fast) {
         pp = h->plan_params(batch);
-        pb = h->plan_buffers();
+        pb = h->plan_buffers(sb);
         e = launch_plan(pp, h->key64, h->at(y.uniq_keys), (const int32_t*)h->at(y.grp_start), counters, L,
                         pb, h->d_status, s, &nl);
         h->plan_sorted_groups = pb.sorted_groups;
@@ -806,7 +797,9 @@ static int backward_impl(tt_emb_t h, const float* grad_out, tt_stream_t stream, 
     nl = 0;
     if (h->fast) {
         PlanParams pp = h->plan_params(h->fwd_B);
-        PlanBuffers pb = h->plan_buffers();
+        SortBuffers sb;
+        memset(&sb, 0, sizeof(sb));
+        PlanBuffers pb = h->plan_buffers(sb);
         pb.sorted_groups = h->plan_sorted_groups;
         GradPtrs vgp;
         CoreParams vcp = h->view_cores(h->fwd_B, &vgp);
@@ -1055,7 +1048,6 @@ int tt_emb_debug_inject(tt_emb_t h, int32_t what, int32_t spin_limit)
     case TT_INJECT_MMA_WAIT_BWD:
         if (!h->tc || !k3_tc_bwd_supported(h->view_params())) return note(h, TT_ERR_UNSUPPORTED);
         break;
-    case TT_INJECT_SORT_WAIT: break;
     default: return note(h, TT_ERR_ARG);
     }
     h->inject = what;
@@ -1126,10 +1118,8 @@ int forward_with_scratch(tt_emb_t h, char* scratch, size_t scratch_bytes, const 
     sb.keys[1] = at(y.keys[1]);
     sb.vals[0] = (int32_t*)at(y.vals[0]);
     sb.vals[1] = (int32_t*)at(y.vals[1]);
-    sb.look[0] = (uint64_t*)at(y.look[0]);
-    sb.look[1] = (uint64_t*)at(y.look[1]);
-    sb.ghist = (uint32_t*)at(y.ghist);
-    sb.inject_spin = 0;
+    sb.hist = (uint32_t*)at(y.hist);
+    sb.digit_total = (uint32_t*)at(y.digit_total);
     int nl = 0;
     e = launch_make_keys(kp, h->key64, indices, offsets, sb.keys[0], sb.vals[0], bag_of_pos,
                          h->d_status, s, &nl);

@@ -88,87 +88,83 @@ cudaError_t launch_make_keys(const KeyParams& kp, bool key64, const int64_t* ind
 }
 
 // ---------------------------------------------------------------------------
-// Stable LSD radix sort, 8 bits per pass: one histogram kernel per sort and
-// one kernel per pass.
-//   hist_all  the digit counts of every pass in one read of the keys (the
-//             count of a digit over the whole array does not depend on the
-//             order the earlier passes leave), and the zeroing of the first
-//             pass's look-back words
-//   onesweep  per tile of kSortTile keys, tiles numbered in the order blocks
-//             start (an atomic counter): the stable rank of each key among
-//             equal digits (warp match + per-warp counters, warps in tile
-//             order); the tile's count of every digit published at once; the
-//             count of each digit over all earlier tiles found by decoupled
-//             look-back (Merrill and Garland, "Single-pass Parallel Prefix Scan
-//             with Decoupled Look-back", NVIDIA technical report NVR-2016-002);
-//             keys staged in shared memory by digit, then written out coalesced
-//             at digit base + earlier tiles + rank
-// A tile is 256 threads x kSortItems keys; warp w owns keys
-// [w*32*kSortItems, (w+1)*32*kSortItems) of the tile, visited in (item, lane)
-// order, which is input order, so equal digits keep input order.
-//
-// Look-back words (one per tile and digit, 64 bits): bits 62-63 = 1 when the
-// low bits hold the tile's own count, 2 when they hold the inclusive count
-// over tiles 0..t, 0 while the tile has published nothing.  A block only
-// waits for tiles with smaller numbers, which blocks that started before it
-// hold, so the wait always ends; it is bounded all the same (kLookbackLimit
-// polls, then TT_ERR_TIMEOUT), and it stops when another block has failed.
-// Pass p reads the words of buffer p & 1 and zeroes, for its own tile, the
-// words of the other buffer, which pass p + 1 reads.
+// Stable LSD radix sort, 8 bits per pass, three kernels per pass:
+//   hist     per-tile digit counts, stored digit-major: hist[d * tiles + tile]
+//   colscan  one block per digit: exclusive scan of its row over tiles, and
+//            the digit's total
+//   scatter  per tile: stable rank of each key among equal digits (warp
+//            match + per-warp counters, warps in tile order), staged in
+//            shared memory by digit, then written out coalesced at
+//            digit base + tile base + rank
+// A tile is 256 threads x kSortItems keys; warp w owns keys [w*32*kSortItems, (w+1)*32*kSortItems) of
+// the tile, visited in (item, lane) order, which is input order.
 // ---------------------------------------------------------------------------
-constexpr uint64_t kLbOwn = 1ull << 62, kLbIncl = 2ull << 62, kLbCount = (1ull << 62) - 1;
-constexpr int kLookbackLimit = 1 << 22;
-
-__device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v)
-{
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p)
-{
-    uint64_t v;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-
 template <typename K>
-__global__ void __launch_bounds__(256) k_radix_hist_all(const K* __restrict__ kin, int64_t n,
-                                                        const int64_t* __restrict__ dev_n, int passes,
-                                                        uint32_t* __restrict__ ghist, uint64_t* __restrict__ look0,
-                                                        int64_t look_words, const int32_t* status)
+__global__ void __launch_bounds__(256) k_radix_hist(const K* __restrict__ kin, int64_t n,
+                                                    const int64_t* __restrict__ dev_n, int shift,
+                                                    uint32_t* __restrict__ hist, int tiles,
+                                                    const int32_t* status)
 {
-    __shared__ uint32_t s_cnt[kSortPassMax][256];
+    __shared__ uint32_t s_cnt[256];
     if (has_error(status)) return;
     if (dev_n) n = min64(n, *dev_n);
-    const int tid = threadIdx.x, lane = tid & 31;
-    const int64_t stride = (int64_t)gridDim.x * 256;
-    for (int64_t i = (int64_t)blockIdx.x * 256 + tid; i < look_words; i += stride) look0[i] = 0ull;
-    for (int i = tid; i < kSortPassMax * 256; i += 256) (&s_cnt[0][0])[i] = 0u;
+    s_cnt[threadIdx.x] = 0;
     __syncthreads();
-    // whole warps walk the keys; a lane past the end counts nothing (digit 256)
-    for (int64_t base = (int64_t)blockIdx.x * 256; base < n; base += stride) {
-        const int64_t e = base + tid;
-        const bool valid = e < n;
-        const K k = valid ? kin[e] : K(0);
-        for (int p = 0; p < passes; ++p) {
-            const int d = valid ? (int)((uint32_t)(k >> (8 * p)) & 255u) : 256;
-            const unsigned peers = __match_any_sync(kFull, d);
-            // one shared-memory add per distinct digit of the warp, by its lowest lane
-            if (valid && (peers & ((1u << lane) - 1u)) == 0) atomicAdd(&s_cnt[p][d], (uint32_t)__popc(peers));
+    const int64_t base = (int64_t)blockIdx.x * kSortTile;
+    const int cnt = (int)min64(kSortTile, n - base);
+    for (int e = threadIdx.x; e < cnt; e += 256)
+        atomicAdd(&s_cnt[(uint32_t)(kin[base + e] >> shift) & 255u], 1u);
+    __syncthreads();
+    hist[(int64_t)threadIdx.x * tiles + blockIdx.x] = s_cnt[threadIdx.x];
+}
+
+__global__ void __launch_bounds__(1024) k_radix_colscan(uint32_t* __restrict__ hist, int tiles,
+                                                       uint32_t* __restrict__ digit_total,
+                                                       const int32_t* status)
+{
+    __shared__ uint32_t s_w[32];
+    if (has_error(status)) return;
+    uint32_t* row = hist + (int64_t)blockIdx.x * tiles;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    uint32_t carry = 0;
+    for (int b0 = 0; b0 < tiles; b0 += 1024) {
+        const int i = b0 + threadIdx.x;
+        const uint32_t v = i < tiles ? row[i] : 0u;
+        uint32_t x = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            uint32_t y = __shfl_up_sync(kFull, x, o);
+            if (lane >= o) x += y;
         }
+        if (lane == 31) s_w[wid] = x;
+        __syncthreads();
+        if (wid == 0) {
+            uint32_t w = s_w[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                uint32_t y = __shfl_up_sync(kFull, w, o);
+                if (lane >= o) w += y;
+            }
+            s_w[lane] = w;
+        }
+        __syncthreads();
+        const uint32_t excl = carry + (wid ? s_w[wid - 1] : 0u) + x - v;
+        if (i < tiles) row[i] = excl;
+        carry += s_w[31];
+        __syncthreads();
     }
-    __syncthreads();
-    for (int p = 0; p < passes; ++p)
-        if (s_cnt[p][tid]) atomicAdd(&ghist[p * 256 + tid], s_cnt[p][tid]);
+    if (threadIdx.x == 0) digit_total[blockIdx.x] = carry;
 }
 
 template <typename K>
-__global__ void __launch_bounds__(256) k_radix_onesweep(const K* __restrict__ kin, const int32_t* __restrict__ vin,
-                                                        K* __restrict__ kout, int32_t* __restrict__ vout, int64_t n,
-                                                        const int64_t* __restrict__ dev_n, int shift,
-                                                        const uint32_t* __restrict__ ghist, uint64_t* look,
-                                                        uint64_t* __restrict__ look_next, int* tile_counter,
-                                                        int inject_spin, int32_t* status)
+__global__ void __launch_bounds__(256) k_radix_scatter(const K* __restrict__ kin,
+                                                       const int32_t* __restrict__ vin,
+                                                       K* __restrict__ kout, int32_t* __restrict__ vout,
+                                                       int64_t n, const int64_t* __restrict__ dev_n,
+                                                       int shift,
+                                                       const uint32_t* __restrict__ hist,
+                                                       const uint32_t* __restrict__ digit_total,
+                                                       int tiles, const int32_t* status)
 {
     __shared__ uint32_t s_wcnt[8][256];
     __shared__ uint32_t s_tile_start[256];
@@ -176,38 +172,33 @@ __global__ void __launch_bounds__(256) k_radix_onesweep(const K* __restrict__ ki
     __shared__ uint32_t s_tmp[8];
     __shared__ K s_keys[kSortTile];
     __shared__ int32_t s_vals[kSortTile];
-    __shared__ int s_tile;
+    if (has_error(status)) return;
 
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    if (tid == 0) s_tile = atomicAdd(tile_counter, 1);
-    __syncthreads();
-    const int tile = s_tile;
-    if (look_next) look_next[(int64_t)tile * 256 + tid] = 0ull;
-    if (has_error(status)) return;
     if (dev_n) n = min64(n, *dev_n);
-    const int64_t base = (int64_t)tile * kSortTile;
+    const int64_t base = (int64_t)blockIdx.x * kSortTile;
     const int cnt = (int)min64(kSortTile, n - base);
-    if (cnt <= 0) return;   // only tiles after every tile that holds keys
+    if (cnt <= 0) return;
+    for (int i = tid; i < 8 * 256; i += 256) (&s_wcnt[0][0])[i] = 0;
+    {
+        uint32_t tot;
+        const uint32_t dbase = block256_exclusive_scan<uint32_t>(digit_total[tid], &tot, s_tmp);
+        s_gbase[tid] = dbase + hist[(int64_t)tid * tiles + blockIdx.x];
+    }
+    __syncthreads();
 
-    // the tile's keys and positions, all loads issued before the ranking
     K key[kSortItems];
     int32_t val[kSortItems];
-    const int sub = wid * 32 * kSortItems;
-#pragma unroll
-    for (int j = 0; j < kSortItems; ++j) {
-        const int e = sub + j * 32 + lane;
-        key[j] = e < cnt ? kin[base + e] : K(0);
-        val[j] = e < cnt ? vin[base + e] : 0;
-    }
-    for (int i = tid; i < 8 * 256; i += 256) (&s_wcnt[0][0])[i] = 0;
-    __syncthreads();
-
     uint32_t rank[kSortItems];
     int dig[kSortItems];
+    const int sub = wid * 32 * kSortItems;
     const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
     for (int j = 0; j < kSortItems; ++j) {
-        const bool valid = sub + j * 32 + lane < cnt;
+        const int e = sub + j * 32 + lane;
+        const bool valid = e < cnt;
+        key[j] = valid ? kin[base + e] : K(0);
+        val[j] = valid ? vin[base + e] : 0;
         dig[j] = valid ? (int)((uint32_t)(key[j] >> shift) & 255u) : 256;
         const unsigned peers = __match_any_sync(kFull, dig[j]);
         const uint32_t pre = valid ? s_wcnt[wid][dig[j]] : 0u;
@@ -217,7 +208,6 @@ __global__ void __launch_bounds__(256) k_radix_onesweep(const K* __restrict__ ki
         __syncwarp();
     }
     __syncthreads();
-    uint32_t own;   // this tile's count of digit tid
     {
         uint32_t run = 0;
 #pragma unroll
@@ -226,47 +216,10 @@ __global__ void __launch_bounds__(256) k_radix_onesweep(const K* __restrict__ ki
             s_wcnt[w][tid] = run;
             run += c;
         }
-        own = run;
-    }
-    // publish the tile's counts; the first tile's are already inclusive
-    uint64_t* my = look + (int64_t)tile * 256 + tid;
-    const bool withhold = inject_spin > 0 && tile == 0;   // test hook: the first tile never publishes
-    if (!withhold) st_relaxed_u64(my, (tile == 0 ? kLbIncl : kLbOwn) | own);
-    {
         uint32_t tot;
-        s_tile_start[tid] = block256_exclusive_scan<uint32_t>(own, &tot, s_tmp);
+        s_tile_start[tid] = block256_exclusive_scan<uint32_t>(run, &tot, s_tmp);
     }
-    // decoupled look-back: this digit's count over all earlier tiles
-    uint64_t before = 0;
-    bool ok = true;
-    {
-        const int limit = inject_spin > 0 ? inject_spin : kLookbackLimit;
-        int polls = 0;
-        for (int tp = tile - 1; tp >= 0;) {
-            const uint64_t v = ld_relaxed_u64(look + (int64_t)tp * 256 + tid);
-            const uint64_t flag = v >> 62;
-            if (flag == 0) {
-                if (++polls > limit || ((polls & 63) == 0 && has_error(status))) {
-                    ok = false;
-                    break;
-                }
-                __nanosleep(32);
-                continue;
-            }
-            before += v & kLbCount;
-            if (flag == 2) break;
-            --tp;
-        }
-    }
-    if (tile > 0 && ok) st_relaxed_u64(my, kLbIncl | (before + own));
-    if (__syncthreads_or(!ok)) {
-        if (tid == 0) raise_error(status, TT_ERR_TIMEOUT, 200 + tile);
-        return;
-    }
-    {
-        uint32_t tot;
-        s_gbase[tid] = block256_exclusive_scan<uint32_t>(ghist[tid], &tot, s_tmp) + (uint32_t)before;
-    }
+    __syncthreads();
 #pragma unroll
     for (int j = 0; j < kSortItems; ++j) {
         if (dig[j] < 256) {
@@ -290,22 +243,16 @@ static cudaError_t radix_sort_t(int64_t n, int bits, SortBuffers& sb, int* which
                                 cudaStream_t s, int* nl, const int64_t* dev_n)
 {
     const int tiles = (int)ceil_div(n, kSortTile);
-    const int passes = (bits + 7) / 8;
-    int* counters = reinterpret_cast<int*>(sb.ghist + kSortPassMax * 256);
-    cudaError_t e = cudaMemsetAsync(sb.ghist, 0, kSortGhistBytes, s);
-    if (e != cudaSuccess) return e;
-    const int hgrid = (int)min64(ceil_div(n, 256), 148 * 8);
-    k_radix_hist_all<K><<<hgrid, 256, 0, s>>>((const K*)sb.keys[0], n, dev_n, passes, sb.ghist, sb.look[0],
-                                              (int64_t)tiles * 256, status);
-    *nl += 1;
     int cur = 0;
-    for (int p = 0; p < passes; ++p) {
-        k_radix_onesweep<K><<<tiles, 256, 0, s>>>((const K*)sb.keys[cur], sb.vals[cur], (K*)sb.keys[cur ^ 1],
-                                                  sb.vals[cur ^ 1], n, dev_n, 8 * p, sb.ghist + p * 256,
-                                                  sb.look[p & 1], p + 1 < passes ? sb.look[(p + 1) & 1] : nullptr,
-                                                  counters + p, p == 0 ? sb.inject_spin : 0, status);
+    for (int shift = 0; shift < bits; shift += 8) {
+        const K* kin = (const K*)sb.keys[cur];
+        k_radix_hist<K><<<tiles, 256, 0, s>>>(kin, n, dev_n, shift, sb.hist, tiles, status);
+        k_radix_colscan<<<256, 1024, 0, s>>>(sb.hist, tiles, sb.digit_total, status);
+        k_radix_scatter<K><<<tiles, 256, 0, s>>>(kin, sb.vals[cur], (K*)sb.keys[cur ^ 1],
+                                                 sb.vals[cur ^ 1], n, dev_n, shift, sb.hist,
+                                                 sb.digit_total, tiles, status);
         cur ^= 1;
-        *nl += 1;
+        *nl += 3;
     }
     *which = cur;
     return cudaGetLastError();
@@ -314,11 +261,10 @@ static cudaError_t radix_sort_t(int64_t n, int bits, SortBuffers& sb, int* which
 cudaError_t radix_sort_pairs(bool key64, int64_t n, int bits, SortBuffers& sb, int* which,
                              int32_t* status, cudaStream_t s, int* nl, const int64_t* dev_n)
 {
-    if (n <= 0 || bits <= 0) {
+    if (n <= 0) {
         *which = 0;
         return cudaSuccess;
     }
-    if (bits > 8 * kSortPassMax) return cudaErrorInvalidValue;
     return key64 ? radix_sort_t<uint64_t>(n, bits, sb, which, status, s, nl, dev_n)
                  : radix_sort_t<uint32_t>(n, bits, sb, which, status, s, nl, dev_n);
 }

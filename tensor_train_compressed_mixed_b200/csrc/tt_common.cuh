@@ -131,10 +131,8 @@ constexpr int kElemChunk = 8192;             // floats per block of an elementwi
 struct SortBuffers {
     void* keys[2];        // ping-pong key arrays (uint32 or uint64)
     int32_t* vals[2];     // ping-pong positions
-    uint64_t* look[2];    // [tiles * 256] look-back words of alternate passes
-    uint32_t* ghist;      // [kSortPassMax * 256] digit counts of every pass, then kSortPassMax tile counters
-    int inject_spin;      // test hook: > 0 = the first pass's first tile withholds its counts, and the
-                          // look-back polls at most this many times
+    uint32_t* hist;       // [256 * tiles]
+    uint32_t* digit_total;// [256]
 };
 
 // Parameters of the column-group planner and of the specialised kernels.
@@ -238,8 +236,6 @@ __device__ __forceinline__ T block256_exclusive_scan(T v, T* total, T* s_tmp)
 
 constexpr int kSortItems = 12;
 constexpr int kSortTile = 256 * kSortItems;
-constexpr int kSortPassMax = 8;   // 8-bit digits of keys up to 64 bits
-constexpr size_t kSortGhistBytes = (size_t)kSortPassMax * 256 * 4 + kSortPassMax * 4;
 constexpr int kScanTile = 256 * 16;
 
 __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }

@@ -144,29 +144,6 @@ def test_tensor_core_wait_timeout_exit_path(stage):
             assert core_grad_err(got, want[t][j]) <= FP32_TOL, (t, j)
 
 
-@pytest.mark.parametrize("path", ["fused", "generic"])
-def test_sort_lookback_timeout_is_reported_and_handle_recovers(path):
-    """The lookup sort's decoupled look-back: the first tile of the first pass withholds its
-    digit counts, the next tile gives up after its poll limit, and the call reports
-    TT_ERR_TIMEOUT; the next forward (several sort tiles) matches the oracle."""
-    if path == "fused":
-        w, emb, idx, off = _fast_handle(batch=256)
-    else:
-        w = random_workload(95, (2, 2, 2), (1, 3, 3, 1), [(16, 16, 16)], [4096], batch=2000,
-                            pooling={"kind": "uniform", "lo": 1, "hi": 8})
-        emb, cores, idx, off = from_workload(w, with_grads=True)
-    assert idx.numel() > 2 * 3072
-    want = oracle.workload_forward(w)
-    abi.tt_emb_debug_inject(emb.handle, abi.TT_INJECT_SORT_WAIT, 1000)
-    emb.forward(idx, off, w.batch)
-    with pytest.raises(abi.TTEmbError) as e:
-        emb.sync()
-    assert e.value.code == abi.TT_ERR_TIMEOUT
-    out = emb.forward(idx, off, w.batch)
-    emb.sync()
-    assert output_err(out.cpu().numpy(), want, w.dim) <= FP32_TOL
-
-
 def test_injection_needs_a_wait_of_that_kind():
     w = random_workload(93, (2, 2), (1, 3, 1), [(4, 4)], batch=4)
     emb, cores, idx, off = from_workload(w, with_grads=True)    # generic kernels: no such waits
