@@ -1404,6 +1404,22 @@ __device__ __forceinline__ bool tc_commit_wait(uint64_t* bar, uint32_t& parity, 
     return *s_ok != 0;
 }
 
+// as tc_commit_wait, and when wait2 also the completion of phase parity2 of bar2 (products
+// other threads committed there); parity2 flips with it
+__device__ __forceinline__ bool tc_commit_wait2(uint64_t* bar, uint32_t& parity, uint64_t* bar2, uint32_t& parity2,
+                                                bool wait2, int* s_ok, bool inject_fail = false)
+{
+    if (threadIdx.x == 0) {
+        tc_commit(bar);
+        const bool ok = mbar_wait(bar, parity) && (!wait2 || mbar_wait(bar2, parity2));
+        *s_ok = (ok && !inject_fail) ? 1 : 0;
+    }
+    __syncthreads();
+    parity ^= 1u;
+    if (wait2) parity2 ^= 1u;
+    return *s_ok != 0;
+}
+
 template <class S, typename K>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ uniq_keys,
@@ -1776,7 +1792,8 @@ k3_bwd_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict__ u
 //                                      (vector reductions into dG_3^T [i3][rho][a3])
 //                     dC_p[(a1, a2)][rho] += sum_a3 H_u[(a1, a2)][a3] S_u[rho][a3]
 //                   with the quads on contiguous row ranges and no block barrier between rows.
-//   dA = dC . B^T (M = 64, every row a chunk row), dB += A^T . dC over the column group.
+//   dA = dC . B^T (M = 64, every row a chunk row), dB += A^T . dC over the column group; the
+//                   two dA accumulators and dB are issued by three threads of different warps.
 // ---------------------------------------------------------------------------
 constexpr int kMPB2 = 16;   // prefixes per chunk
 constexpr int kMB2 = 64;    // rows of A per chunk
@@ -2002,6 +2019,7 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
     __shared__ BwdMeta2 M;
     __shared__ __align__(16) K s_keys[2 * kKeyCap];
     __shared__ __align__(8) uint64_t s_mbar;
+    __shared__ __align__(8) uint64_t s_mbar2;   // a chunk's dA and dB products, committed by three threads
     __shared__ uint32_t s_tmem;
     __shared__ int s_ok;
     uint16_t* Bb = reinterpret_cast<uint16_t*>(smem_f);            // NS x (N x R): [n/8][rho/8][8][8]
@@ -2014,14 +2032,22 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
     uint32_t parity = 0;
     bool failed = false;
     // tensor memory: columns [0, N) dB of the column group, [N, N + 2 MB) C^T, [TDA, TDA + DAQ R) dA.
-    // A chunk's dA and dB products are waited for by the commit after the next chunk's C^T
-    // product (or at the end of the column): they run while the next chunk's row table is built.
+    // A chunk's dA and dB products are waited for with the next chunk's C^T product (or at the end
+    // of the column): they run while the next chunk's row table is built. They are issued by
+    // three threads in different warps (two dA accumulators and dB), because one thread issuing
+    // all sixty small products in a row holds the block at its next barrier; each of the three
+    // commits to s_mbar2.
     if (tid < 32) tmem_alloc(&s_tmem, 2 * N);
-    if (tid == 0) mbar_init(&s_mbar, 1);
+    if (tid == 0) {
+        mbar_init(&s_mbar, 1);
+        mbar_init(&s_mbar2, 3);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s_tmem;
+    uint32_t parity2 = 0;
+    bool pend2 = false;   // a chunk's dA / dB products committed to s_mbar2 and not yet waited for
 
     const unsigned long long pr_t0 = cp.probe ? global_ns() : 0ull;
     int pr_tasks = 0;
@@ -2106,10 +2132,11 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
                                          umma_desc(b0 + k * 256, 128, SBO), R * N * 2, MB * R * 2,
                                          umma_idesc_bf16(128, MB), k > 0);
             }
-            if (!tc_commit_wait(&s_mbar, parity, &s_ok, cp.inj_mma != 0)) {   // also the previous chunk's dA and dB
-                failed = true;
+            if (!tc_commit_wait2(&s_mbar, parity, &s_mbar2, parity2, pend2, &s_ok, cp.inj_mma != 0)) {
+                failed = true;   // (the wait also covers the previous chunk's dA and dB)
                 break;
             }
+            pend2 = false;
             tc_fence_after();
             if (pmb >= 0) read_dA(pmb, pcnt);
             for (int q = tid; q < MB * N / 4; q += BT)   // the previous chunk's dC tile is no longer read
@@ -2163,36 +2190,45 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
             fence_async_smem();
             __syncthreads();
             TT_PH(19);
-            if (tid == 0) {
+            // lane 0 of warps 0 .. DAQ - 1 issues dA accumulator q = warp, lane 0 of warp DAQ issues
+            // dB; each commits its products to s_mbar2 (count DAQ + 1)
+            static_assert(DAQ == 2, "three issuing threads");
+            if ((tid & 31) == 0 && (tid >> 5) <= DAQ) {
                 tc_fence_after();
+                const int q = tid >> 5;
                 const uint32_t c0 = smem_u32(dCb), b0 = smem_u32(Bb), a0 = smem_u32(Ab16);
-                // dA = dC . B^T: A = dC (K-major), B = the B tile viewed MN-major; the K range
-                // split over DAQ accumulators issued in turn
+                if (q < DAQ) {
+                    // dA = dC . B^T: A = dC (K-major), B = the B tile viewed MN-major; accumulator q
+                    // takes the K range [q N / DAQ, (q + 1) N / DAQ)
 #pragma unroll 1
-                for (int kk = 0; kk < N / 16 / DAQ; ++kk)
-#pragma unroll
-                    for (int q = 0; q < DAQ; ++q) {
+                    for (int kk = 0; kk < N / 16 / DAQ; ++kk) {
                         const int k = q * (N / 16 / DAQ) + kk;
                         tc_mma_terms<NT>(tmem + (uint32_t)(TDA + q * R), umma_desc(c0 + k * 256, 128, (N / 8) * 128),
                                          umma_desc_mn(b0 + k * 2 * (R / 8) * 128, 128, (R / 8) * 128),
                                          MB * N * 2, R * N * 2, umma_idesc_bf16(MB, R, false, true), kk > 0);
                     }
-                // dB += A^T . dC: A = the A tile viewed MN-major, B = dC viewed MN-major
+                } else {
+                    // dB += A^T . dC: A = the A tile viewed MN-major, B = dC viewed MN-major
 #pragma unroll
-                for (int k = 0; k < MB / 16; ++k)
-                    tc_mma_terms<NT>(tmem, umma_desc_mn(a0 + k * 2 * (R / 8) * 128, 128, (R / 8) * 128),
-                                     umma_desc_mn(c0 + k * 2 * (N / 8) * 128, 128, (N / 8) * 128),
-                                     MB * R * 2, MB * N * 2, umma_idesc_bf16(R, N, true, true), j0 > 0 || k > 0);
+                    for (int k = 0; k < MB / 16; ++k)
+                        tc_mma_terms<NT>(tmem, umma_desc_mn(a0 + k * 2 * (R / 8) * 128, 128, (R / 8) * 128),
+                                         umma_desc_mn(c0 + k * 2 * (N / 8) * 128, 128, (N / 8) * 128),
+                                         MB * R * 2, MB * N * 2, umma_idesc_bf16(R, N, true, true),
+                                         j0 > 0 || k > 0);
+                }
+                tc_commit(&s_mbar2);
             }
+            pend2 = true;
             pmb = mb;
             pcnt = cnt;
             TT_PH(13);
         }
         if (failed) break;
-        if (!tc_commit_wait(&s_mbar, parity, &s_ok)) {   // the column's last dA and dB
+        if (!tc_commit_wait2(&s_mbar, parity, &s_mbar2, parity2, pend2, &s_ok)) {   // the column's last dA and dB
             failed = true;
             break;
         }
+        pend2 = false;
         tc_fence_after();
         read_dA(pmb, pcnt);
         TT_PH(14);
