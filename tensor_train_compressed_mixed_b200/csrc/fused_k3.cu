@@ -1404,19 +1404,23 @@ __device__ __forceinline__ bool tc_commit_wait(uint64_t* bar, uint32_t& parity, 
     return *s_ok != 0;
 }
 
-// as tc_commit_wait, and when wait2 also the completion of phase parity2 of bar2 (products
-// other threads committed there); parity2 flips with it
+// as tc_commit_wait, and when wait2 also the completion of phase parity2 of bar2, and with bar3 the
+// completion of phase *parity3 of bar3 (products other threads committed there); the parities of
+// the barriers waited for flip
 __device__ __forceinline__ bool tc_commit_wait2(uint64_t* bar, uint32_t& parity, uint64_t* bar2, uint32_t& parity2,
-                                                bool wait2, int* s_ok, bool inject_fail = false)
+                                                bool wait2, int* s_ok, bool inject_fail = false,
+                                                uint64_t* bar3 = nullptr, uint32_t* parity3 = nullptr)
 {
     if (threadIdx.x == 0) {
         tc_commit(bar);
-        const bool ok = mbar_wait(bar, parity) && (!wait2 || mbar_wait(bar2, parity2));
+        const bool ok = mbar_wait(bar, parity) && (!wait2 || mbar_wait(bar2, parity2)) &&
+                        (bar3 == nullptr || mbar_wait(bar3, *parity3));
         *s_ok = (ok && !inject_fail) ? 1 : 0;
     }
     __syncthreads();
     parity ^= 1u;
     if (wait2) parity2 ^= 1u;
+    if (bar3) *parity3 ^= 1u;
     return *s_ok != 0;
 }
 
@@ -2020,6 +2024,7 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
     __shared__ __align__(16) K s_keys[2 * kKeyCap];
     __shared__ __align__(8) uint64_t s_mbar;
     __shared__ __align__(8) uint64_t s_mbar2;   // a chunk's dA and dB products, committed by three threads
+    __shared__ __align__(8) uint64_t s_mbar3;   // the second half of a chunk's C^T product
     __shared__ uint32_t s_tmem;
     __shared__ int s_ok;
     uint16_t* Bb = reinterpret_cast<uint16_t*>(smem_f);            // NS x (N x R): [n/8][rho/8][8][8]
@@ -2041,12 +2046,13 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
     if (tid == 0) {
         mbar_init(&s_mbar, 1);
         mbar_init(&s_mbar2, 3);
+        mbar_init(&s_mbar3, 1);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s_tmem;
-    uint32_t parity2 = 0;
+    uint32_t parity2 = 0, parity3 = 0;
     bool pend2 = false;   // a chunk's dA / dB products committed to s_mbar2 and not yet waited for
 
     const unsigned long long pr_t0 = cp.probe ? global_ns() : 0ull;
@@ -2120,19 +2126,21 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
             TT_PH(9);
 
             // C^T = B^T A^T: A operand = the B tile read as M = n (K-major), B operand = the A tile
-            if (tid == 0) {
+            // half h = 0 by thread 0 (committed by tc_commit_wait2), h = 1 by lane 0 of warp 2 (s_mbar3)
+            if (tid == 0 || tid == 64) {
                 tc_fence_after();
                 constexpr uint32_t SBO = (R / 8) * 128;
                 const uint32_t a0 = smem_u32(Bb), b0 = smem_u32(Ab16);
+                const int h = tid == 0 ? 0 : 1;
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
-#pragma unroll
-                    for (int k = 0; k < R / 16; ++k)
-                        tc_mma_terms<NT>(tmem + (uint32_t)(N + h * MB), umma_desc(a0 + h * 16 * SBO + k * 256, 128, SBO),
-                                         umma_desc(b0 + k * 256, 128, SBO), R * N * 2, MB * R * 2,
-                                         umma_idesc_bf16(128, MB), k > 0);
+                for (int k = 0; k < R / 16; ++k)
+                    tc_mma_terms<NT>(tmem + (uint32_t)(N + h * MB), umma_desc(a0 + h * 16 * SBO + k * 256, 128, SBO),
+                                     umma_desc(b0 + k * 256, 128, SBO), R * N * 2, MB * R * 2,
+                                     umma_idesc_bf16(128, MB), k > 0);
+                if (h == 1) tc_commit(&s_mbar3);
             }
-            if (!tc_commit_wait2(&s_mbar, parity, &s_mbar2, parity2, pend2, &s_ok, cp.inj_mma != 0)) {
+            if (!tc_commit_wait2(&s_mbar, parity, &s_mbar2, parity2, pend2, &s_ok, cp.inj_mma != 0, &s_mbar3,
+                                 &parity3)) {
                 failed = true;   // (the wait also covers the previous chunk's dA and dB)
                 break;
             }
