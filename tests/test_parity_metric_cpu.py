@@ -19,6 +19,6 @@ def test_elementwise_metric_uses_each_element_down_to_the_floor():
     x[0, 2] -= 2e-4                       # 1e-4 of that element
     assert np.isclose(floor_elementwise_err(x, y, (1,)), 1e-4)
     x = y.copy()
-    x[0, 1] += 4e-7                       # tiny element: judged against the floor 4e-3
+    x[0, 1] += 4e-7                       # tiny element: compared with the floor 4e-3
     assert np.isclose(floor_elementwise_err(x, y, (1,)), 4e-7 / 4e-3)
     assert floor_elementwise_err(y, y, (1,)) == 0.0
