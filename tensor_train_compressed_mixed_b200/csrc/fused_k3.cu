@@ -289,11 +289,14 @@ __device__ __forceinline__ void split_bf16x8(const float (&v)[8], uint4& hi, uin
     uint32_t h[4], l[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * i]), h1 = __float2bfloat16_rn(v[2 * i + 1]);
-        const __nv_bfloat16 l0 = __float2bfloat16_rn(v[2 * i] - __bfloat162float(h0));
-        const __nv_bfloat16 l1 = __float2bfloat16_rn(v[2 * i + 1] - __bfloat162float(h1));
-        h[i] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-        l[i] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+        // two values per conversion; a bf16 widens to fp32 exactly by a 16-bit shift
+        const __nv_bfloat162 hh = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        const uint32_t hb = *reinterpret_cast<const uint32_t*>(&hh);
+        const float r0 = v[2 * i] - __uint_as_float(hb << 16);
+        const float r1 = v[2 * i + 1] - __uint_as_float(hb & 0xffff0000u);
+        const __nv_bfloat162 ll = __floats2bfloat162_rn(r0, r1);
+        h[i] = hb;
+        l[i] = *reinterpret_cast<const uint32_t*>(&ll);
     }
     hi = make_uint4(h[0], h[1], h[2], h[3]);
     lo = make_uint4(l[0], l[1], l[2], l[3]);
