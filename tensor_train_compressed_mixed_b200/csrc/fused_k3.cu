@@ -761,7 +761,9 @@ __device__ void fwd_pool(const CoreParams& cp, int ptask, int nP, const int32_t*
 // adding -1, and the one atomic of each tells whether the range still held a subtask, so every
 // subtask runs exactly once.  The bias keeps both halves positive: tails fall at most once per
 // failed steal per block below the range start.
-// Thread 0 only.  Returns a subtask index, -2 - p for pooling task p, or -1 when done.
+// One thread only (lane 0 of warp 1: thread 0 issues the tensor-core products, and a queue
+// atomic on it would delay them).  Returns a subtask index, -2 - p for pooling task p, or -1
+// when done.
 // ---------------------------------------------------------------------------
 struct FwdSched {
     const int4* subs;
@@ -907,12 +909,13 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
     sm.Ss = sm.Cn + S::MF * S::N;
     const int nP = hdr->nP, npool = cp.T * nP;
     const bool use_ckpt = sched == TT_SCHED_STEAL_L2;
-    int phase = 0, vk = 1;   // scheduler state (thread 0)
+    int phase = 0, vk = 1;   // scheduler state (the scheduling thread, kSchedTid)
     int cur_t = -1, cur_i2 = -1;   // column of the B now in (or on its way to) the B tile
     int cur_cid = -1;              // chunk whose C tile is in shared memory
     int mb = 0;
     bool staged = false;
-    if (tid == 0) M.task[0] = fwd_next(fs, hdr, sched, npool, phase, vk);
+    constexpr int kSchedTid = 32;   // the thread that runs the scheduler (state in its registers)
+    if (tid == kSchedTid) M.task[0] = fwd_next(fs, hdr, sched, npool, phase, vk);
     __syncthreads();
     int q = M.task[0];
     while (q != -1) {
@@ -920,7 +923,7 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
             fwd_pool<S>(cp, -2 - q, nP, uid_at_pos, offsets, hdr, rowbuf, out, status, &M.flag, &pr_wait);
             ++pr_tasks;
             __syncthreads();
-            if (tid == 0) M.task[0] = fwd_next(fs, hdr, sched, npool, phase, vk);
+            if (tid == kSchedTid) M.task[0] = fwd_next(fs, hdr, sched, npool, phase, vk);
             __syncthreads();
             q = M.task[0];
             staged = false;
@@ -938,11 +941,12 @@ k3_fwd_kernel(CoreParams cp, int sched, const K* __restrict__ uniq_keys,
                 cp_async_commit();   // the row keys alone
             }
         }
-        if (tid == 0) M.task[1] = fwd_next(fs, hdr, sched, npool, phase, vk);   // used after the C step
         cp_async_wait_all();   // the subtask's A/B rows and row keys (usually prefetched long ago)
         fence_async_smem();    // A/B tiles: read by the tensor cores after the barrier
         __syncthreads();
         const int nrows = M.re[mb] - M.rb[mb];
+        // the next task, read after the C step's barriers (the queue atomic runs during the C step)
+        if (tid == kSchedTid) M.task[1] = fwd_next(fs, hdr, sched, npool, phase, vk);
         // the first batch of last slices is in flight during the C step (last digits from the keys)
         if (nrows > 0) fwd_issue_batch_keys<S, K>(cp, mb, M, sm, s_keys);
         // the row table; read by the batches, which come after the C step's barriers
