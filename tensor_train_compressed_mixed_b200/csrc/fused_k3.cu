@@ -690,7 +690,8 @@ __device__ void fwd_pool(const CoreParams& cp, int ptask, int nP, const int32_t*
                          int* s_flag, unsigned long long* wait_ns)
 {
     constexpr int D = S::D, LB = D / 4, BPW = 32 / LB;
-    constexpr int kPoolLoads = 16;   // row gathers in flight per lane
+    // row gathers in flight per lane (measured: 24 is best at rank 32, 16 at rank 64)
+    constexpr int kPoolLoads = S::R == 32 ? 24 : 16;
     const int t = ptask / nP, jb = ptask % nP;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     TT_PH_START();

@@ -50,6 +50,10 @@ __global__ void __launch_bounds__(256) k_make_keys(KeyParams kp, const int64_t* 
         if (s_off[j + 1] < s_off[j]) raise_error(status, TT_ERR_OFFSETS, (int)min64(g0 + j, INT32_MAX));
     const int64_t lo = s_off[0], hi = s_off[nb];
     const uint64_t rmask = (uint64_t(1) << kp.ibits) - 1;
+    // the block's bags span at most two tables when B >= 256: one division per block
+    const int t0 = (int)(g0 / kp.B);
+    const int64_t g_next = (int64_t)(t0 + 1) * kp.B;   // first bag of the next table
+    const bool two_max = kp.B >= kBagsPerBlock;
     for (int64_t l = lo + threadIdx.x; l < hi; l += blockDim.x) {
         // bag = last j with s_off[j] <= l (upper bound - 1), clamped to [0, nb)
         int a = 0, b = nb;  // invariant: s_off[a] <= l < s_off[b] when monotone
@@ -58,7 +62,7 @@ __global__ void __launch_bounds__(256) k_make_keys(KeyParams kp, const int64_t* 
             if (s_off[m] <= l) a = m; else b = m;
         }
         const int64_t g = g0 + a;
-        const int t = (int)(g / kp.B);
+        const int t = two_max ? t0 + (g >= g_next ? 1 : 0) : (int)(g / kp.B);
         int64_t row = indices[l];
         if (row < 0 || row >= (int64_t)kp.nrows[t]) {
             raise_error(status, TT_ERR_INDEX_RANGE, (int)min64(l, INT32_MAX));
