@@ -352,11 +352,16 @@ struct FwdMeta {   // shared-memory metadata of a subtask (double buffered)
     RowTable rows;
 };
 
-// Index of the prefix (0..cnt-1) holding the chunk's distinct row number kq.
-__device__ __forceinline__ int prefix_of(const int* ucum, int cnt, int kq)
+// Index of the prefix (0..cnt-1) holding the chunk's distinct row number kq. Every prefix has at
+// least one row, so the first rows ucum[0..cnt) strictly increase and the index is the number of
+// prefixes after the first that start at or before kq: counted with independent loads (ucum has
+// N1 = slots + 1 entries).
+template <int N1>
+__device__ __forceinline__ int prefix_of(const int (&ucum)[N1], int cnt, int kq)
 {
     int j = 0;
-    while (j + 1 < cnt && ucum[j + 1] <= kq) ++j;
+#pragma unroll
+    for (int i = 1; i < N1 - 1; ++i) j += (i < cnt && ucum[i] <= kq) ? 1 : 0;
     return j;
 }
 
@@ -364,8 +369,8 @@ __device__ __forceinline__ int prefix_of(const int* ucum, int cnt, int kq)
 // id, the prefix slot and the last digit, computed once by all threads from the staged keys
 // (which must have landed and be visible).  Batches inside the table then need no per-batch
 // metadata pass.
-template <typename K>
-__device__ __forceinline__ void build_rows(RowTable& rt, int mb, const int* ucum, const int* u0, int cnt, int total,
+template <typename K, int N1>
+__device__ __forceinline__ void build_rows(RowTable& rt, int mb, const int (&ucum)[N1], const int* u0, int cnt, int total,
                                            const K* keys, int ibits, uint32_t n3, int nthreads, int base = 0)
 {
     const int n = min(total - base, kKeyCap);
