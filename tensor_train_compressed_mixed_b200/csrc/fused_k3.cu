@@ -72,6 +72,8 @@ constexpr int kNB = kPoolBags;    // bags per pooling task
 constexpr int kHChunk = 256;      // sorted lookups per upstream-sum warp
 constexpr int kSpinLimit = 1 << 22;
 constexpr int kKeyCap = 256;      // distinct rows per chunk whose keys are staged with the chunk
+constexpr int kKeyCapB = 512;     // the same for a chunk of the tensor-core backward (not split into
+                                  // subtasks, so longer; rows past the cap read their keys directly)
 
 template <int D1_, int D2_, int D3_, int R_>
 struct S3 {
@@ -334,10 +336,12 @@ struct FwdSmem {
     float* Ss;   // [FBUF][NUF][SU] last slices of a batch of distinct rows
 };
 
-// Per chunk buffer, for the chunk's first kKeyCap distinct rows: row id, prefix slot, last digit.
-struct RowTable {
-    int u[2][kKeyCap], p[2][kKeyCap], i3[2][kKeyCap];
+// Per chunk buffer, for the chunk's first CAP distinct rows: row id, prefix slot, last digit.
+template <int CAP>
+struct RowTableT {
+    int u[2][CAP], p[2][CAP], i3[2][CAP];
 };
+using RowTable = RowTableT<kKeyCap>;
 
 template <class S>
 struct FwdMeta {   // shared-memory metadata of a subtask (double buffered)
@@ -369,17 +373,17 @@ __device__ __forceinline__ int prefix_of(const int (&ucum)[N1], int cnt, int kq)
 // id, the prefix slot and the last digit, computed once by all threads from the staged keys
 // (which must have landed and be visible).  Batches inside the table then need no per-batch
 // metadata pass.
-template <typename K, int N1>
-__device__ __forceinline__ void build_rows(RowTable& rt, int mb, const int (&ucum)[N1], const int* u0, int cnt, int total,
+template <typename K, int N1, int CAP>
+__device__ __forceinline__ void build_rows(RowTableT<CAP>& rt, int mb, const int (&ucum)[N1], const int* u0, int cnt, int total,
                                            const K* keys, int ibits, uint32_t n3, int nthreads, int base = 0)
 {
-    const int n = min(total - base, kKeyCap);
+    const int n = min(total - base, CAP);
     for (int i = threadIdx.x; i < n; i += nthreads) {
         const int kq = base + i;
         const int j = prefix_of(ucum, cnt, kq);
         rt.u[mb][i] = u0[j] + (kq - ucum[j]);
         rt.p[mb][i] = j;
-        rt.i3[mb][i] = (int)(key_row(keys[mb * kKeyCap + i], ibits) % n3);
+        rt.i3[mb][i] = (int)(key_row(keys[mb * CAP + i], ibits) % n3);
     }
 }
 // Rows k0 .. k0 + nb of chunk buffer mb: the row table when it covers them, else the batch's own
@@ -1821,12 +1825,12 @@ struct BwdMeta2 {
     int i1[2][kMPB2];
     int cnt[2];
     int task;
-    RowTable rows;
+    RowTableT<kKeyCapB> rows;
     int4 rec[2][kMPB2];   // the next chunk's per-group records, prefetched
 };
 
 // chunk metadata into buffer mb (ends with a barrier), then asynchronous copies of the keys of
-// its first kKeyCap distinct rows into keys[mb] (they join the caller's next commit group)
+// its first kKeyCapB distinct rows into keys[mb] (they join the caller's next commit group)
 template <typename K>
 __device__ __forceinline__ void bwd2_meta(const int4* recs, int j0, int ccount, int mb, const K* __restrict__ uniq_keys,
                                           BwdMeta2& M, K* keys)
@@ -1851,10 +1855,10 @@ __device__ __forceinline__ void bwd2_meta(const int4* recs, int j0, int ccount, 
         if (tid == 0) M.cnt[mb] = cnt;
     }
     __syncthreads();
-    const int nk = min(M.ucum[mb][kMPB2], kKeyCap);
+    const int nk = min(M.ucum[mb][kMPB2], kKeyCapB);
     for (int kq = tid; kq < nk; kq += (int)blockDim.x) {
         const int j = prefix_of(M.ucum[mb], cnt, kq);
-        cp_async_key(keys + mb * kKeyCap + kq, uniq_keys + M.u0[mb][j] + (kq - M.ucum[mb][j]));
+        cp_async_key(keys + mb * kKeyCapB + kq, uniq_keys + M.u0[mb][j] + (kq - M.ucum[mb][j]));
     }
 }
 
@@ -1913,7 +1917,7 @@ __device__ __forceinline__ void warp_row_load2(const CoreParams& cp, int t, int 
 {
     constexpr int R = 64, D3 = 8, D = 128;
     const int lane = threadIdx.x & 31;
-    if (kq < kKeyCap) {
+    if (kq < kKeyCapB) {
         w.u = M.rows.u[mb][kq];
         w.j = M.rows.p[mb][kq];
         w.i3 = M.rows.i3[mb][kq];
@@ -2034,7 +2038,7 @@ k3_bwd_tc2_kernel(CoreParams cp, GradPtrs gp, PlanParams pp, const K* __restrict
     static_assert(TDA + DAQ * R <= 2 * N, "tensor-memory columns");
     extern __shared__ __align__(16) float smem_f[];
     __shared__ BwdMeta2 M;
-    __shared__ __align__(16) K s_keys[2 * kKeyCap];
+    __shared__ __align__(16) K s_keys[2 * kKeyCapB];
     __shared__ __align__(8) uint64_t s_mbar;
     __shared__ __align__(8) uint64_t s_mbar2;   // a chunk's dA and dB products, committed by three threads
     __shared__ __align__(8) uint64_t s_mbar3;   // the second half of a chunk's C^T product
