@@ -174,14 +174,16 @@ def test_split_training_many_chunks_per_column():
 
 @pytest.mark.parametrize("precision_name,tol", [("TT_PREC_FP32_SPLIT_TC", FP32_TOL), ("TT_PREC_BF16_TC", BF16_TOL)])
 def test_rank64_training_chunks_beyond_row_table(precision_name, tol):
-    """One column group of 20 prefixes with 40 last-digit values each, nearly every row
-    looked up: the first 16-prefix chunk holds more distinct rows than the per-chunk row
-    table (256), so rows past it take the path that reads their keys from the sorted
-    distinct keys (forward and backward)."""
+    """One column group of 20 prefixes with 64 last-digit values each, nearly every row
+    looked up: the first 16-prefix chunk holds about 1000 distinct rows, more than the
+    backward's per-chunk row table (512), so its later rows take the path that reads their
+    keys from the sorted distinct keys; the forward splits the chunk into subtasks of at most
+    256 rows, each with its own table."""
     from tensor_train_compressed_mixed_b200 import abi
-    w = random_workload(962, (4, 4, 8), (1, 64, 64, 1), [(20, 1, 40)], batch=200,
+    w = random_workload(962, (4, 4, 8), (1, 64, 64, 1), [(20, 1, 64)], batch=300,
                         pooling={"kind": "uniform", "lo": 10, "hi": 30}, with_grad=True)
-    assert len(np.unique(w.indices)) > 256 + 100
+    rows = np.unique(w.indices)
+    assert len(rows[rows // 64 < 16]) > 512 + 100   # distinct rows of the first chunk
     _, out, grads, new = gpu_train_step(w, options=_opts(getattr(abi, precision_name)), lr=0.01)
     assert output_err(out, oracle.workload_forward(w), w.dim) <= tol
     want = oracle.workload_backward(w)
